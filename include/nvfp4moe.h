@@ -1,0 +1,263 @@
+/*
+ * nvfp4moe.h -- C ABI of the NVFP4 block-scaled Mixture-of-Experts library
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The library implements the MoE FFN hot path that the pages "Peering into the
+ * CUTLASS Kernel Cache", "Peering into the CUTLASS Kernel", "Peering into the
+ * CUTLASS Kernel Scheduler" and "Peering into the CUTLASS SharedStorage" turn
+ * on: an FP4 block-scaled grouped GEMM in which each expert's weight matrix
+ * multiplies only the 16-256 tokens routed to it.
+ *
+ * Data format (NVFP4). Elements are E2M1 4-bit codes, two per byte, the even
+ * element of each pair in the low nibble; every 16 consecutive elements along K
+ * share one E4M3 block scale byte; each tensor carries one FP32 global scale
+ * ("Peering into the CUTLASS SharedStorage", Input Knowledge Required, item 3;
+ * "Peering into the CUTLASS Kernel Cache", Knowledge Required, last item). The
+ * stored global scale is the dequantisation multiplier g_dec = amax / (6*448);
+ * a value decodes as E2M1(code) * E4M3(scale) * g_dec.
+ *
+ * Conventions for every call:
+ *  - Ownership: the caller owns every buffer. The library never allocates or
+ *    frees device memory. Buffers marked "device" must be device (or managed)
+ *    memory of the current device; sizes are in elements unless stated.
+ *  - Streams: every call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream). No call synchronises with the host except
+ *    nvfp4_get_device_status().
+ *  - Errors: argument, alignment, shape and capability problems are reported
+ *    synchronously, before anything is launched. Launch failures map to
+ *    NVFP4_ERR_CUDA. Problems only visible on the device (expert ids out of
+ *    range, inconsistent expert offsets, a pipeline wait that ran out) are
+ *    latched in a device status word read by nvfp4_get_device_status().
+ *  - Layouts: matrices are row-major. GEMM operands are K-major: activations
+ *    [rows, K], weights [N, K] per expert (like nn.Linear), so a packed row is
+ *    K/2 bytes and a row of block scales is K/16 bytes.
+ *  - BF16 tensors are passed as uint16_t bit patterns.
+ */
+#ifndef NVFP4MOE_H
+#define NVFP4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t. */
+typedef struct CUstream_st* nvfp4_stream_t;
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,       /* null pointer, negative or zero size, bad enum */
+    NVFP4_ERR_MISALIGNED = 2,        /* a pointer is not 16-byte aligned */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 3, /* K, N, E, k outside what the kernels implement */
+    NVFP4_ERR_WORKSPACE = 4,         /* workspace missing or smaller than required */
+    NVFP4_ERR_SMEM_BUDGET = 5,       /* the device cannot give the kernel its shared memory */
+    NVFP4_ERR_CUDA = 6,              /* a CUDA runtime call or launch failed */
+    NVFP4_ERR_DEVICE_TIMEOUT = 7,    /* (device) a bounded pipeline wait ran out */
+    NVFP4_ERR_DEVICE_INPUT = 8       /* (device) expert id out of range, duplicate id in a
+                                        token's top-k, or inconsistent expert offsets */
+} nvfp4_status;
+
+typedef enum { NVFP4_EPI_NONE = 0, NVFP4_EPI_SWIGLU = 1 } nvfp4_epilogue;
+
+/* Block-scale layouts.
+ * NVFP4_SF_ROWMAJOR: sf[r * (K/16) + b] is the scale of elements [16b, 16b+16) of row r.
+ * NVFP4_SF_MMA_TILED: the same bytes permuted for the tensor-core scale path. Rows
+ *   are grouped in 128-row blocks and K in 64-element steps (4 scales); each
+ *   (row block rb, step kc) pair is a 512-byte atom at ((rb * (K/64)) + kc) * 512,
+ *   and inside it the scale of row r, block b sits at
+ *   (r % 32) * 16 + ((r % 128) / 32) * 4 + (b % 4).
+ *   Requires rows % 128 == 0 and K % 64 == 0. Weights are stored this way. */
+typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1 } nvfp4_sf_layout;
+
+/* ------------------------------------------------------------------------ */
+/* nvfp4_quantize: BF16 -> packed E2M1 codes + E4M3 block scales + FP32      */
+/* global scale, for one tensor X [rows, K].                                 */
+/*                                                                           */
+/* Computes (format of "Peering into the CUTLASS SharedStorage", Input       */
+/* Knowledge Required, item 3), with IEEE FP32 round-to-nearest-even steps:  */
+/*   amax = max|x|; g_enc = 2688/amax, g_dec = amax/2688 (both 1 if amax=0); */
+/*   if global_scale_in != NULL it is g_dec and g_enc = 1/g_dec (no amax);   */
+/*   per 16-block: S = E4M3_satfinite((amax_b / 6) * g_enc);                 */
+/*   S == 0 -> codes +0, else code = E2M1_satfinite(x * (g_enc / S)), the    */
+/*   sign kept on zero.                                                      */
+/* Arguments:                                                                */
+/*   x                [rows, K] BF16 bits, device, 16-byte aligned           */
+/*   rows, K          rows >= 1, K % 16 == 0 (MMA_TILED: rows % 128 == 0,    */
+/*                    K % 64 == 0)                                           */
+/*   global_scale_in  device FP32 scalar or NULL (dynamic amax)             */
+/*   q                [rows, K/2] bytes, device, 8-byte aligned              */
+/*   sf               rows*K/16 bytes, device, in `layout`                   */
+/*   global_scale_out device FP32 scalar receiving g_dec (may equal         */
+/*                    global_scale_in)                                       */
+/*   ws, ws_bytes     device scratch of nvfp4_quantize_workspace_size() bytes*/
+/*                    (the per-block amax partials); NULL/0 allowed when     */
+/*                    global_scale_in is given                               */
+/* ------------------------------------------------------------------------ */
+NVFP4_API size_t nvfp4_quantize_workspace_size(int64_t rows, int64_t K);
+NVFP4_API nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t K, const float* global_scale_in,
+                            uint8_t* q, uint8_t* sf, float* global_scale_out, nvfp4_sf_layout layout,
+                            void* ws, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* moe_permute: group routed (token, slot) pairs by expert and gather the    */
+/* quantised activation rows into expert order ("Peering into the CUTLASS   */
+/* Kernel Cache", Knowledge Required: each expert's weight matrix multiplies */
+/* the subset of tokens routed to it).                                       */
+/*   expert_offsets[e] = number of pairs routed to experts < e; [E] = T*k.   */
+/*   Inside expert e, pairs are ordered by token t ascending, then slot j.   */
+/*   perm_src[p] = source token of permuted row p;                           */
+/*   inv_perm[t*k + j] = permuted row of pair (t, j);                        */
+/*   q_perm[p] = q[perm_src[p]] (K/2 bytes), sf_perm[p] = sf[perm_src[p]]    */
+/*   (K/16 bytes, row-major scales).                                         */
+/* Arguments: topk_ids [T, k] int32 (device) with ids in [0, E), distinct   */
+/*   within a token (violations latch NVFP4_ERR_DEVICE_INPUT); 1 <= T,       */
+/*   1 <= k <= 32, 1 <= E <= 1024, T*k < 2^31; K % 256 == 0; q [T, K/2],    */
+/*   sf [T, K/16] row-major; outputs q_perm [T*k, K/2], sf_perm [T*k, K/16], */
+/*   expert_offsets [E+1], perm_src [T*k], inv_perm [T*k]; all device,       */
+/*   16-byte aligned. ws of moe_permute_workspace_size() bytes.              */
+/* ------------------------------------------------------------------------ */
+NVFP4_API size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E);
+NVFP4_API nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
+                         const uint8_t* q, const uint8_t* sf, int64_t K,
+                         uint8_t* q_perm, uint8_t* sf_perm, int32_t* expert_offsets,
+                         int32_t* perm_src, int32_t* inv_perm,
+                         void* ws, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* moe_grouped_gemm_nvfp4: one launch for every expert's FP4 block-scaled    */
+/* GEMM ("Peering into the CUTLASS Kernel Cache": TMA warp-specialised       */
+/* grouped GEMM; "Peering into the CUTLASS Kernel Scheduler": producer /     */
+/* MMA / epilogue warp roles).                                               */
+/* For expert e and activation rows m in [off[e], off[e+1]):                 */
+/*   acc[m, n] = sum_k A(m,k) W_e(n,k)   (block-scaled E2M1 x E2M1, FP32)    */
+/*   alpha_e   = a_gscale[0] * w_gscale[e]                                   */
+/*   NONE:   out[m, n] = BF16(alpha_e * acc[m, n]),            out [rows, N] */
+/*   SWIGLU: out[m, n] = BF16(silu(alpha_e acc[m, n]) * alpha_e acc[m, N/2+n])*/
+/*           (rows [0, N/2) of each W_e are the gate, [N/2, N) the up        */
+/*           projection),                                     out [rows, N/2]*/
+/* Arguments:                                                                */
+/*   a_q [max_rows, K/2], a_sf [max_rows, K/16] row-major, a_gscale scalar   */
+/*   w_q [E, N, K/2], w_sf [E, N, K/16] in NVFP4_SF_MMA_TILED layout (per    */
+/*   expert slice, i.e. the [E*N, K] matrix tiled), w_gscale [E]             */
+/*   expert_offsets [E+1] (device; non-decreasing, off[0] >= 0,              */
+/*   off[E] <= max_rows, else NVFP4_ERR_DEVICE_INPUT is latched and the      */
+/*   offending experts are skipped)                                          */
+/*   Shapes: 1 <= E <= 1024, N % 256 == 0, K % 256 == 0, max_rows >= 0.      */
+/*   All pointers device, 16-byte aligned. Rows outside every expert's range */
+/*   are not written.                                                        */
+/* ------------------------------------------------------------------------ */
+NVFP4_API nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
+                                    const uint8_t* w_q, const uint8_t* w_sf, const float* w_gscale,
+                                    const int32_t* expert_offsets, int32_t E, int64_t max_rows,
+                                    int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
+                                    nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* moe_unpermute_combine: top-k weighted sum of the expert outputs back in   */
+/* token order -- the final MoE output write of the FINALIZE epilogue       */
+/* ("Peering into the CUTLASS Kernel", Input Knowledge Required, item 5).    */
+/*   out[t, h] = BF16( sum_{j=0..k-1} topk_w[t, j] * y[inv_perm[t*k+j], h] ) */
+/*   accumulated in FP32 over j ascending; a negative inv_perm entry is      */
+/*   skipped.                                                                */
+/* Arguments: y [T*k, H] BF16, inv_perm [T*k], topk_w [T, k] FP32, out [T, H]*/
+/*   BF16; all device, 16-byte aligned; H % 8 == 0, 1 <= k <= 32.            */
+/* ------------------------------------------------------------------------ */
+NVFP4_API nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* inv_perm, const float* topk_w,
+                                   int32_t T, int32_t k, int64_t H, uint16_t* out,
+                                   nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* moe_layer_nvfp4: the whole MoE FFN in one call, every step in this        */
+/* library's kernels, in this order: quantize(x) -> moe_permute ->           */
+/* grouped GEMM gate/up (SWIGLU, N = 2I, K = H) -> quantize(h) -> grouped   */
+/* GEMM down (NONE, N = H, K = I) -> moe_unpermute_combine.                  */
+/* Arguments: x [T, H] BF16, topk_ids [T, k], topk_w [T, k];                 */
+/*   w13_q [E, 2I, H/2], w13_sf (MMA_TILED), w13_gscale [E];                 */
+/*   w2_q [E, H, I/2], w2_sf (MMA_TILED), w2_gscale [E]; out [T, H] BF16.    */
+/*   H % 256 == 0, I % 128 == 0 (2I % 256 == 0 and I % 256 == 0 for the down */
+/*   GEMM's K), plus the limits of the calls above. ws of                    */
+/*   moe_layer_workspace_size() bytes holds every intermediate; its layout   */
+/*   is reported by moe_layer_workspace_layout().                            */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    size_t q_x, sf_x, g_x;                 /* quantised x [T, H/2], [T, H/16], scalar */
+    size_t q_perm, sf_perm;                /* [T*k, H/2], [T*k, H/16] */
+    size_t offsets, perm_src, inv_perm;    /* [E+1], [T*k], [T*k] int32 */
+    size_t h;                              /* [T*k, I] BF16 */
+    size_t q_h, sf_h, g_h;                 /* [T*k, I/2], [T*k, I/16], scalar */
+    size_t y;                              /* [T*k, H] BF16 */
+    size_t scratch;                        /* quantize / permute scratch */
+    size_t total;
+} nvfp4_layer_workspace;
+
+NVFP4_API nvfp4_status moe_layer_workspace_layout(int32_t T, int32_t k, int32_t E, int64_t H, int64_t I,
+                                        nvfp4_layer_workspace* layout);
+NVFP4_API size_t moe_layer_workspace_size(int32_t T, int32_t k, int32_t E, int64_t H, int64_t I);
+NVFP4_API nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_ids, const float* topk_w,
+                             int32_t T, int32_t k, int32_t E, int64_t H, int64_t I,
+                             const uint8_t* w13_q, const uint8_t* w13_sf, const float* w13_gscale,
+                             const uint8_t* w2_q, const uint8_t* w2_sf, const float* w2_gscale,
+                             uint16_t* out, void* ws, size_t ws_bytes, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Capability and pipeline plan of the grouped GEMM.                         */
+/* The launch succeeds iff nvfp4_can_implement() returns NVFP4_OK for the    */
+/* current device ("Peering into the CUTLASS SharedStorage", Why This        */
+/* Message Was Written: initialize() failed after can_implement() passed --  */
+/* this check is the same one the launcher performs, so they cannot          */
+/* disagree).                                                                */
+/* Per-stage transaction bytes follow the mainloop accounting of that page's */
+/* Message excerpt: bytes of the A tile plus its scales, plus bytes of the B */
+/* tile plus its scales.                                                     */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    int32_t tile_weight_rows;    /* weight rows (GEMM N) per tile: 256 */
+    int32_t tile_tokens_max;     /* activation rows (GEMM M) per tile, at most */
+    int32_t stage_k;             /* K elements per pipeline stage */
+    int32_t stages;              /* pipeline depth */
+    int32_t stage_bytes_weights; /* packed weight bytes per stage */
+    int32_t stage_bytes_weight_sf;
+    int32_t stage_bytes_act_max; /* packed activation bytes per stage at tile_tokens_max */
+    int32_t stage_bytes_act_sf;  /* activation scale bytes staged per stage */
+    int32_t smem_bytes;          /* dynamic shared memory per CTA */
+    int32_t tmem_columns;        /* tensor-memory columns allocated per CTA */
+    int32_t threads;             /* threads per CTA */
+} nvfp4_gemm_plan;
+
+NVFP4_API nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan);
+/* Expect-tx bytes one stage's TMA and bulk copies deliver for a tile of `tokens` rows. */
+NVFP4_API int64_t nvfp4_gemm_stage_tx_bytes(int32_t tokens);
+/* Pure host check against a given opt-in shared-memory budget (bytes per block). */
+NVFP4_API nvfp4_status nvfp4_can_implement_with_budget(int64_t N, int64_t K, int32_t E, nvfp4_epilogue epi,
+                                             int64_t smem_optin_bytes);
+/* The same check against the current device. */
+NVFP4_API nvfp4_status nvfp4_can_implement(int64_t N, int64_t K, int32_t E, nvfp4_epilogue epi);
+
+/* ------------------------------------------------------------------------ */
+/* Device status and diagnostics.                                            */
+/* ------------------------------------------------------------------------ */
+/* Synchronises `stream`, reads the device status word of the current device,
+ * clears it and returns NVFP4_OK, NVFP4_ERR_DEVICE_TIMEOUT or
+ * NVFP4_ERR_DEVICE_INPUT (timeout wins when both are latched). */
+NVFP4_API nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
+/* Upper bound, in nanoseconds, on any single pipeline wait inside the GEMM
+ * (default 1 s). After it the kernel latches NVFP4_ERR_DEVICE_TIMEOUT, drains
+ * its own copies, frees its tensor memory and returns. */
+NVFP4_API void nvfp4_set_wait_timeout_ns(uint64_t ns);
+NVFP4_API uint64_t nvfp4_get_wait_timeout_ns(void);
+/* Number of kernel launches made by this library in this process. */
+NVFP4_API uint64_t nvfp4_launch_count(void);
+NVFP4_API const char* nvfp4_status_string(nvfp4_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4MOE_H */

@@ -1,0 +1,331 @@
+"""NVFP4 block-scaled Mixture-of-Experts hot path for B200 (sm_100a).
+
+A thin Python binding over the C ABI in ``include/nvfp4moe.h`` (library
+``lib/libnvfp4moe.so``, built by ``build.py``). Every function here only
+marshals torch tensors into pointers, sizes and the current CUDA stream; all
+arithmetic runs in the library's CUDA kernels. PyTorch supplies device memory,
+streams and workspaces. There is no CPU fallback: without the built library or
+without a CUDA device the calls raise.
+
+Calls (same names as the C ABI):
+  quantize            -> nvfp4_quantize
+  permute             -> moe_permute
+  grouped_gemm        -> moe_grouped_gemm_nvfp4
+  unpermute_combine   -> moe_unpermute_combine
+  moe_layer           -> moe_layer_nvfp4
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libnvfp4moe.so")
+
+STATUS = {
+    0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_MISALIGNED", 3: "NVFP4_ERR_UNSUPPORTED_SHAPE",
+    4: "NVFP4_ERR_WORKSPACE", 5: "NVFP4_ERR_SMEM_BUDGET", 6: "NVFP4_ERR_CUDA", 7: "NVFP4_ERR_DEVICE_TIMEOUT",
+    8: "NVFP4_ERR_DEVICE_INPUT",
+}
+OK = 0
+EPI_NONE, EPI_SWIGLU = 0, 1
+SF_ROWMAJOR, SF_MMA_TILED = 0, 1
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+class LayerWorkspace(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "q_x", "sf_x", "g_x", "q_perm", "sf_perm", "offsets", "perm_src", "inv_perm", "h", "q_h", "sf_h", "g_h",
+        "y", "scratch", "total")]
+
+
+class GemmPlan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "tile_weight_rows", "tile_tokens_max", "stage_k", "stages", "stage_bytes_weights", "stage_bytes_weight_sf",
+        "stage_bytes_act_max", "stage_bytes_act_sf", "smem_bytes", "tmem_columns", "threads")]
+
+
+_lib = None
+
+
+def lib():
+    """Load the CUDA library (fails loudly when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m nvfp4_block_scaled_09_b200.build` "
+                              "(or __graft_entry__.build()) first")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        st = ctypes.c_int
+        L.nvfp4_quantize_workspace_size.argtypes = [i64, i64]
+        L.nvfp4_quantize_workspace_size.restype = sz
+        L.nvfp4_quantize.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int, P, sz, P]
+        L.nvfp4_quantize.restype = st
+        L.moe_permute_workspace_size.argtypes = [i32, i32, i32]
+        L.moe_permute_workspace_size.restype = sz
+        L.moe_permute.argtypes = [P, i32, i32, i32, P, P, i64, P, P, P, P, P, P, sz, P]
+        L.moe_permute.restype = st
+        L.moe_grouped_gemm_nvfp4.argtypes = [P, P, P, P, P, P, P, i32, i64, i64, i64, ctypes.c_int, P, P]
+        L.moe_grouped_gemm_nvfp4.restype = st
+        L.moe_unpermute_combine.argtypes = [P, P, P, i32, i32, i64, P, P]
+        L.moe_unpermute_combine.restype = st
+        L.moe_layer_workspace_layout.argtypes = [i32, i32, i32, i64, i64, ctypes.POINTER(LayerWorkspace)]
+        L.moe_layer_workspace_layout.restype = st
+        L.moe_layer_workspace_size.argtypes = [i32, i32, i32, i64, i64]
+        L.moe_layer_workspace_size.restype = sz
+        L.moe_layer_nvfp4.argtypes = [P, P, P, i32, i32, i32, i64, i64, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_layer_nvfp4.restype = st
+        L.nvfp4_gemm_get_plan.argtypes = [ctypes.POINTER(GemmPlan)]
+        L.nvfp4_gemm_get_plan.restype = st
+        L.nvfp4_gemm_stage_tx_bytes.argtypes = [i32]
+        L.nvfp4_gemm_stage_tx_bytes.restype = i64
+        L.nvfp4_can_implement_with_budget.argtypes = [i64, i64, i32, ctypes.c_int, i64]
+        L.nvfp4_can_implement_with_budget.restype = st
+        L.nvfp4_can_implement.argtypes = [i64, i64, i32, ctypes.c_int]
+        L.nvfp4_can_implement.restype = st
+        L.nvfp4_get_device_status.argtypes = [P]
+        L.nvfp4_get_device_status.restype = st
+        L.nvfp4_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+        L.nvfp4_set_wait_timeout_ns.restype = None
+        L.nvfp4_get_wait_timeout_ns.restype = ctypes.c_uint64
+        L.nvfp4_launch_count.restype = ctypes.c_uint64
+        L.nvfp4_status_string.argtypes = [ctypes.c_int]
+        L.nvfp4_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise NVFP4Error(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("nvfp4 calls take CUDA tensors only (no CPU fallback)")
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype != torch.bfloat16:
+        raise TypeError("expected a bfloat16 tensor")
+    return t.contiguous()
+
+
+# ----------------------------------------------------------------------------- quantize
+
+def quantize_workspace_size(rows: int, K: int) -> int:
+    return int(lib().nvfp4_quantize_workspace_size(rows, K))
+
+
+def quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None, layout: int = SF_ROWMAJOR,
+             q: torch.Tensor | None = None, sf: torch.Tensor | None = None, g: torch.Tensor | None = None,
+             ws: torch.Tensor | None = None, stream=None):
+    """x [rows, K] bf16 -> (q uint8 [rows, K/2], sf uint8 [rows*K/16], g float32 [1] = g_dec)."""
+    _require_cuda(x, global_scale)
+    x = _bits(x)
+    rows, K = x.shape
+    dev = x.device
+    q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else q
+    sf = torch.empty((rows, K // 16), dtype=torch.uint8, device=dev) if sf is None else sf
+    g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else g
+    if ws is None and global_scale is None:
+        ws = torch.empty(max(quantize_workspace_size(rows, K), 16), dtype=torch.uint8, device=dev)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().nvfp4_quantize(_ptr(x), rows, K, _ptr(global_scale), _ptr(q), _ptr(sf), _ptr(g), layout,
+                                _ptr(ws), nbytes, _stream(stream)), "nvfp4_quantize")
+    return q, sf, g
+
+
+def prepare_expert_weights(w: torch.Tensor, stream=None):
+    """Weights [E, N, K] bf16 -> (q [E, N, K/2], sf [E, N, K/16] MMA-tiled, g [E]) with one global
+    scale per expert matrix. One-time preparation, one quantize call per expert."""
+    _require_cuda(w)
+    E, N, K = w.shape
+    q = torch.empty((E, N, K // 2), dtype=torch.uint8, device=w.device)
+    sf = torch.empty((E, N, K // 16), dtype=torch.uint8, device=w.device)
+    g = torch.empty(E, dtype=torch.float32, device=w.device)
+    ws = torch.empty(max(quantize_workspace_size(N, K), 16), dtype=torch.uint8, device=w.device)
+    for e in range(E):
+        quantize(w[e], layout=SF_MMA_TILED, q=q[e], sf=sf[e], g=g[e:e + 1], ws=ws, stream=stream)
+    return q, sf, g
+
+
+# ----------------------------------------------------------------------------- permute
+
+def permute_workspace_size(T: int, k: int, E: int) -> int:
+    return int(lib().moe_permute_workspace_size(T, k, E))
+
+
+@dataclass
+class Permuted:
+    q_perm: torch.Tensor
+    sf_perm: torch.Tensor
+    offsets: torch.Tensor
+    perm_src: torch.Tensor
+    inv_perm: torch.Tensor
+
+
+def permute(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_experts: int, ws=None,
+            stream=None) -> Permuted:
+    _require_cuda(topk_ids, q, sf)
+    if topk_ids.dtype != torch.int32:
+        raise TypeError("topk_ids must be int32")
+    topk_ids = topk_ids.contiguous()
+    T, k = topk_ids.shape
+    K = q.shape[1] * 2
+    R = T * k
+    dev = q.device
+    out = Permuted(
+        q_perm=torch.empty((R, K // 2), dtype=torch.uint8, device=dev),
+        sf_perm=torch.empty((R, K // 16), dtype=torch.uint8, device=dev),
+        offsets=torch.empty(num_experts + 1, dtype=torch.int32, device=dev),
+        perm_src=torch.empty(R, dtype=torch.int32, device=dev),
+        inv_perm=torch.empty(R, dtype=torch.int32, device=dev),
+    )
+    if ws is None:
+        ws = torch.empty(max(permute_workspace_size(T, k, num_experts), 16), dtype=torch.uint8, device=dev)
+    _check(lib().moe_permute(_ptr(topk_ids), T, k, num_experts, _ptr(q), _ptr(sf), K, _ptr(out.q_perm),
+                             _ptr(out.sf_perm), _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm), _ptr(ws),
+                             ws.numel(), _stream(stream)), "moe_permute")
+    return out
+
+
+# ----------------------------------------------------------------------------- grouped GEMM
+
+def grouped_gemm(a_q, a_sf, a_g, w_q, w_sf, w_g, offsets, N: int, K: int, swiglu: bool, out=None, stream=None):
+    """Per-expert NVFP4 GEMM. Returns bf16 [rows, N] (or [rows, N/2] with SwiGLU)."""
+    _require_cuda(a_q, a_sf, a_g, w_q, w_sf, w_g, offsets)
+    rows = a_q.shape[0]
+    E = offsets.numel() - 1
+    nout = N // 2 if swiglu else N
+    if out is None:
+        out = torch.empty((rows, nout), dtype=torch.bfloat16, device=a_q.device)
+    _check(lib().moe_grouped_gemm_nvfp4(_ptr(a_q), _ptr(a_sf), _ptr(a_g), _ptr(w_q), _ptr(w_sf), _ptr(w_g),
+                                        _ptr(offsets), E, rows, N, K, EPI_SWIGLU if swiglu else EPI_NONE, _ptr(out),
+                                        _stream(stream)), "moe_grouped_gemm_nvfp4")
+    return out
+
+
+def can_implement(N: int, K: int, E: int, swiglu: bool, smem_budget: int | None = None) -> int:
+    epi = EPI_SWIGLU if swiglu else EPI_NONE
+    if smem_budget is None:
+        return int(lib().nvfp4_can_implement(N, K, E, epi))
+    return int(lib().nvfp4_can_implement_with_budget(N, K, E, epi, smem_budget))
+
+
+def gemm_plan() -> dict:
+    p = GemmPlan()
+    _check(lib().nvfp4_gemm_get_plan(ctypes.byref(p)), "nvfp4_gemm_get_plan")
+    return {n: getattr(p, n) for n, _ in GemmPlan._fields_}
+
+
+def gemm_stage_tx_bytes(tokens: int) -> int:
+    return int(lib().nvfp4_gemm_stage_tx_bytes(tokens))
+
+
+# ----------------------------------------------------------------------------- combine
+
+def unpermute_combine(y: torch.Tensor, inv_perm: torch.Tensor, topk_w: torch.Tensor, out=None, stream=None):
+    _require_cuda(y, inv_perm, topk_w)
+    T, k = topk_w.shape
+    H = y.shape[1]
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
+    _check(lib().moe_unpermute_combine(_ptr(y.contiguous()), _ptr(inv_perm), _ptr(topk_w.contiguous()), T, k, H,
+                                       _ptr(out), _stream(stream)), "moe_unpermute_combine")
+    return out
+
+
+# ----------------------------------------------------------------------------- layer
+
+@dataclass
+class MoEWeights:
+    w13_q: torch.Tensor     # [E, 2I, H/2]
+    w13_sf: torch.Tensor    # [E, 2I, H/16] MMA-tiled
+    w13_g: torch.Tensor     # [E]
+    w2_q: torch.Tensor      # [E, H, I/2]
+    w2_sf: torch.Tensor     # [E, H, I/16] MMA-tiled
+    w2_g: torch.Tensor      # [E]
+
+    @property
+    def num_experts(self) -> int:
+        return self.w13_q.shape[0]
+
+    @property
+    def hidden(self) -> int:
+        return self.w13_q.shape[2] * 2
+
+    @property
+    def intermediate(self) -> int:
+        return self.w13_q.shape[1] // 2
+
+
+def layer_workspace_layout(T: int, k: int, E: int, H: int, I: int) -> dict:
+    L = LayerWorkspace()
+    _check(lib().moe_layer_workspace_layout(T, k, E, H, I, ctypes.byref(L)), "moe_layer_workspace_layout")
+    return {n: getattr(L, n) for n, _ in LayerWorkspace._fields_}
+
+
+def layer_workspace(T: int, k: int, E: int, H: int, I: int, device="cuda") -> torch.Tensor:
+    n = int(lib().moe_layer_workspace_size(T, k, E, H, I))
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def moe_layer(x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor, w: MoEWeights, ws=None, out=None,
+              stream=None):
+    """Whole MoE FFN: quantize -> permute -> gate/up GEMM + SwiGLU -> quantize -> down GEMM -> combine."""
+    _require_cuda(x, topk_ids, topk_w)
+    x = _bits(x)
+    T, H = x.shape
+    k = topk_ids.shape[1]
+    E, I = w.num_experts, w.intermediate
+    if ws is None:
+        ws = layer_workspace(T, k, E, H, I, x.device)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    _check(lib().moe_layer_nvfp4(_ptr(x), _ptr(topk_ids.contiguous()), _ptr(topk_w.contiguous()), T, k, E, H, I,
+                                 _ptr(w.w13_q), _ptr(w.w13_sf), _ptr(w.w13_g), _ptr(w.w2_q), _ptr(w.w2_sf),
+                                 _ptr(w.w2_g), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "moe_layer_nvfp4")
+    return out
+
+
+# ----------------------------------------------------------------------------- diagnostics
+
+def device_status(stream=None) -> int:
+    """Synchronise, read and clear the device status word (returns a status code)."""
+    return int(lib().nvfp4_get_device_status(_stream(stream)))
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    lib().nvfp4_set_wait_timeout_ns(int(ns))
+
+
+def get_wait_timeout_ns() -> int:
+    return int(lib().nvfp4_get_wait_timeout_ns())
+
+
+def launch_count() -> int:
+    return int(lib().nvfp4_launch_count())
+
+
+def status_string(status: int) -> str:
+    return lib().nvfp4_status_string(int(status)).decode()

@@ -1,0 +1,183 @@
+// api.cu -- host side of the C ABI: device registry, status word, launch
+// accounting, status strings and the whole-layer orchestration.
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+
+// One status word per device context; kernels latch error bits into it.
+__device__ uint32_t g_nvfp4_device_status;
+
+namespace nvfp4 {
+
+static std::atomic<uint64_t> g_launches{0};
+static std::atomic<uint64_t> g_timeout_ns{1000000000ull};
+
+struct DeviceInfo {
+    bool ready = false;
+    int sm_count = 0;
+    int smem_optin = 0;
+    uint32_t* status = nullptr;
+};
+
+constexpr int kMaxDevices = 64;
+static DeviceInfo g_devices[kMaxDevices];
+static std::mutex g_mutex;
+
+static DeviceInfo* device_info() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& di = g_devices[d];
+    if (!di.ready) {
+        if (cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, d) != cudaSuccess) return nullptr;
+        if (cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, d) != cudaSuccess)
+            return nullptr;
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_nvfp4_device_status) != cudaSuccess) return nullptr;
+        di.status = static_cast<uint32_t*>(p);
+        di.ready = true;
+    }
+    return &di;
+}
+
+uint32_t* status_word_ptr() {
+    DeviceInfo* di = device_info();
+    return di ? di->status : nullptr;
+}
+uint64_t wait_timeout_ns() { return g_timeout_ns.load(); }
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n); }
+int device_sm_count() {
+    DeviceInfo* di = device_info();
+    return di ? di->sm_count : 1;
+}
+int device_smem_optin() {
+    DeviceInfo* di = device_info();
+    return di ? di->smem_optin : -1;
+}
+nvfp4_status check_launch() { return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" const char* nvfp4_status_string(nvfp4_status s) {
+    switch (s) {
+        case NVFP4_OK: return "NVFP4_OK";
+        case NVFP4_ERR_INVALID_ARG: return "NVFP4_ERR_INVALID_ARG";
+        case NVFP4_ERR_MISALIGNED: return "NVFP4_ERR_MISALIGNED";
+        case NVFP4_ERR_UNSUPPORTED_SHAPE: return "NVFP4_ERR_UNSUPPORTED_SHAPE";
+        case NVFP4_ERR_WORKSPACE: return "NVFP4_ERR_WORKSPACE";
+        case NVFP4_ERR_SMEM_BUDGET: return "NVFP4_ERR_SMEM_BUDGET";
+        case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
+        case NVFP4_ERR_DEVICE_TIMEOUT: return "NVFP4_ERR_DEVICE_TIMEOUT";
+        case NVFP4_ERR_DEVICE_INPUT: return "NVFP4_ERR_DEVICE_INPUT";
+    }
+    return "NVFP4_ERR_UNKNOWN";
+}
+
+extern "C" void nvfp4_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns == 0 ? 1 : ns); }
+extern "C" uint64_t nvfp4_get_wait_timeout_ns(void) { return g_timeout_ns.load(); }
+extern "C" uint64_t nvfp4_launch_count(void) { return g_launches.load(); }
+
+extern "C" nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    DeviceInfo* di = device_info();
+    if (!di) return NVFP4_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, di->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return NVFP4_ERR_CUDA;
+    const uint32_t zero = 0;
+    if (cudaMemcpy(di->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (v & kStatusTimeout) return NVFP4_ERR_DEVICE_TIMEOUT;
+    if (v & kStatusBadInput) return NVFP4_ERR_DEVICE_INPUT;
+    return NVFP4_OK;
+}
+
+extern "C" nvfp4_status moe_layer_workspace_layout(int32_t T, int32_t k, int32_t E, int64_t H, int64_t I,
+                                                   nvfp4_layer_workspace* L) {
+    if (!L || T <= 0 || k <= 0 || E <= 0 || H <= 0 || I <= 0) return NVFP4_ERR_INVALID_ARG;
+    const size_t A = 256;
+    const size_t R = (size_t)T * (size_t)k;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align_up(o + bytes, A);
+        return at;
+    };
+    L->q_x = take((size_t)T * H / 2);
+    L->sf_x = take((size_t)T * H / 16);
+    L->g_x = take(sizeof(float));
+    L->q_perm = take(R * H / 2);
+    L->sf_perm = take(R * H / 16);
+    L->offsets = take(sizeof(int32_t) * ((size_t)E + 1));
+    L->perm_src = take(sizeof(int32_t) * R);
+    L->inv_perm = take(sizeof(int32_t) * R);
+    L->h = take(R * I * 2);
+    L->q_h = take(R * I / 2);
+    L->sf_h = take(R * I / 16);
+    L->g_h = take(sizeof(float));
+    L->y = take(R * H * 2);
+    size_t scratch = moe_permute_workspace_size(T, k, E);
+    const size_t qx = nvfp4_quantize_workspace_size(T, H), qh = nvfp4_quantize_workspace_size((int64_t)R, I);
+    if (qx > scratch) scratch = qx;
+    if (qh > scratch) scratch = qh;
+    L->scratch = take(scratch);
+    L->total = o;
+    return NVFP4_OK;
+}
+
+extern "C" size_t moe_layer_workspace_size(int32_t T, int32_t k, int32_t E, int64_t H, int64_t I) {
+    nvfp4_layer_workspace L;
+    if (moe_layer_workspace_layout(T, k, E, H, I, &L) != NVFP4_OK) return 0;
+    return L.total;
+}
+
+extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_ids, const float* topk_w, int32_t T,
+                                        int32_t k, int32_t E, int64_t H, int64_t I, const uint8_t* w13_q,
+                                        const uint8_t* w13_sf, const float* w13_gscale, const uint8_t* w2_q,
+                                        const uint8_t* w2_sf, const float* w2_gscale, uint16_t* out, void* ws,
+                                        size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!x || !topk_ids || !topk_w || !w13_q || !w13_sf || !w13_gscale || !w2_q || !w2_sf || !w2_gscale || !out)
+        return NVFP4_ERR_INVALID_ARG;
+    nvfp4_layer_workspace L;
+    nvfp4_status st = moe_layer_workspace_layout(T, k, E, H, I, &L);
+    if (st != NVFP4_OK) return st;
+    if (!ws || ws_bytes < L.total) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_MISALIGNED;
+    if ((st = nvfp4_can_implement(2 * I, H, E, NVFP4_EPI_SWIGLU)) != NVFP4_OK) return st;
+    if ((st = nvfp4_can_implement(H, I, E, NVFP4_EPI_NONE)) != NVFP4_OK) return st;
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    const int64_t R = (int64_t)T * k;
+    uint8_t* q_x = b + L.q_x;
+    uint8_t* sf_x = b + L.sf_x;
+    float* g_x = reinterpret_cast<float*>(b + L.g_x);
+    uint8_t* q_perm = b + L.q_perm;
+    uint8_t* sf_perm = b + L.sf_perm;
+    int32_t* off = reinterpret_cast<int32_t*>(b + L.offsets);
+    int32_t* perm_src = reinterpret_cast<int32_t*>(b + L.perm_src);
+    int32_t* inv_perm = reinterpret_cast<int32_t*>(b + L.inv_perm);
+    uint16_t* h = reinterpret_cast<uint16_t*>(b + L.h);
+    uint8_t* q_h = b + L.q_h;
+    uint8_t* sf_h = b + L.sf_h;
+    float* g_h = reinterpret_cast<float*>(b + L.g_h);
+    uint16_t* y = reinterpret_cast<uint16_t*>(b + L.y);
+    void* scratch = b + L.scratch;
+    const size_t scratch_bytes = L.total - L.scratch;
+
+    if ((st = nvfp4_quantize(x, T, H, nullptr, q_x, sf_x, g_x, NVFP4_SF_ROWMAJOR, scratch, scratch_bytes, stream)))
+        return st;
+    if ((st = moe_permute(topk_ids, T, k, E, q_x, sf_x, H, q_perm, sf_perm, off, perm_src, inv_perm, scratch,
+                          scratch_bytes, stream)))
+        return st;
+    if ((st = moe_grouped_gemm_nvfp4(q_perm, sf_perm, g_x, w13_q, w13_sf, w13_gscale, off, E, R, 2 * I, H,
+                                     NVFP4_EPI_SWIGLU, h, stream)))
+        return st;
+    if ((st = nvfp4_quantize(h, R, I, nullptr, q_h, sf_h, g_h, NVFP4_SF_ROWMAJOR, scratch, scratch_bytes, stream)))
+        return st;
+    if ((st = moe_grouped_gemm_nvfp4(q_h, sf_h, g_h, w2_q, w2_sf, w2_gscale, off, E, R, H, I, NVFP4_EPI_NONE, y,
+                                     stream)))
+        return st;
+    return moe_unpermute_combine(y, inv_perm, topk_w, T, k, H, out, stream);
+}

@@ -1,0 +1,568 @@
+// grouped_gemm.cu -- NVFP4 block-scaled MoE grouped GEMM on 5th-generation
+// tensor cores (tcgen05, sm_100a).
+//
+// What it computes: for every expert e and activation row m routed to it,
+//   out[m, n] = epilogue( (g_A * g_W[e]) * sum_k A(m,k) W_e(n,k) )
+// with E2M1 operands and one E4M3 scale per 16 K-elements on each side, the
+// FP4 MoE grouped GEMM of "Peering into the CUTLASS Kernel Cache" (one launch
+// over all experts, TMA warp-specialised) with the fused global-scale, SwiGLU
+// and BF16 epilogue.
+//
+// Design (chosen for B200, not the SM120 tiles the pages analyse):
+//  * Swap-AB orientation. Experts see 16-256 rows, so the 128-row MMA M side
+//    holds weight rows and the activation rows ride on the MMA N side
+//    (16..64, in steps of 16, picked per tile on the device). Every weight byte
+//    is read once per (expert, row tile); decode is a pure weight stream.
+//  * Tile = 2 x 128 weight rows x up to 64 activation rows, K stage = 256.
+//    SWIGLU pairs gate rows [n0, n0+128) with up rows [N/2+n0, ...) so both
+//    accumulators of one output column sit in the same TMEM lane; NONE covers
+//    256 consecutive output columns.
+//  * Warp roles ("Peering into the CUTLASS Kernel Scheduler", The Discovery:
+//    explicit warp-specialised schedules that give A loads, B loads, MMA and
+//    epilogue their own warps): warp 0 issues TMA tiles of weights and
+//    activations plus bulk copies of the weights' pre-tiled scales; warp 1
+//    gathers the activation scales (row-major) into the tensor-core scale
+//    layout with cp.async; warp 2 owns tensor memory and issues tcgen05.cp +
+//    tcgen05.mma; warps 4-7 drain the FP32 accumulators from TMEM, apply the
+//    global scales / SwiGLU and store BF16.
+//  * Stage accounting: the expected transaction bytes of a stage are the A
+//    tile bytes plus its scale bytes plus the B tile bytes ("Peering into the
+//    CUTLASS SharedStorage", The Message: MK bytes + NK bytes per stage); the
+//    B scales arrive through their own barrier.
+//  * Shared memory: 4 stages x 46 KB + scheduler tables, checked against the
+//    device's opt-in limit before launch (the same predicate
+//    nvfp4_can_implement() reports, so a passing check never fails to launch).
+//  * Persistent CTAs (one per SM) walk (expert, column tile, row tile) work
+//    items read from device-resident expert offsets; no host synchronisation.
+//    Two TMEM accumulator buffers let the epilogue of one tile overlap the
+//    main loop of the next.
+//  * Every wait is bounded (%globaltimer); on expiry the kernel latches
+//    NVFP4_ERR_DEVICE_TIMEOUT, drains its in-flight copies and MMAs, frees
+//    tensor memory and returns.
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace gg {
+
+constexpr int kBM = 128;                         // weight rows per MMA (tcgen05 M)
+constexpr int kNumA = 2;                         // weight row blocks per tile
+constexpr int kBK = 256;                         // K elements per stage
+constexpr int kRowBytes = kBK / 2;               // packed bytes per row per stage (one 128-byte swizzle row)
+constexpr int kBNMax = 64;                       // activation rows per tile (tcgen05 N), at most
+constexpr int kBNStep = 16;                      // N granularity = activation TMA box rows
+constexpr int kStages = 4;
+constexpr int kKSteps = kBK / 64;                // MMA K-steps per stage (K = 64 per MMA)
+constexpr int kABlockBytes = kBM * kRowBytes;    // 16 KB
+constexpr int kBBytes = kBNMax * kRowBytes;      // 8 KB
+constexpr int kSFAtomBytes = 512;                // 128 rows x 4 scales
+constexpr int kSFStageBytes = kKSteps * kSFAtomBytes;
+constexpr int kOffA0 = 0;
+constexpr int kOffA1 = kABlockBytes;
+constexpr int kOffB = 2 * kABlockBytes;
+constexpr int kOffSFA0 = kOffB + kBBytes;
+constexpr int kOffSFA1 = kOffSFA0 + kSFStageBytes;
+constexpr int kOffSFB = kOffSFA1 + kSFStageBytes;
+constexpr int kStageBytes = kOffSFB + kSFStageBytes;   // 47104 (46 x 1024)
+constexpr int kMaxE = 1024;
+constexpr int kThreads = 256;
+constexpr int kSFDelay = 2;                      // cp.async groups kept in flight by the scale gatherer
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCols = kBNMax;                       // columns per accumulator
+constexpr uint32_t kTmemSFA = 2 * kNumA * kAccCols;         // 256: 2 buffers x 2 accumulators before it
+constexpr uint32_t kTmemSFB = kTmemSFA + kNumA * 4 * kKSteps;  // 288
+
+struct Shared {
+    uint64_t full_tma[kStages];
+    uint64_t full_sf[kStages];
+    uint64_t empty[kStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int32_t total_tiles;
+    int32_t off[kMaxE + 1];
+    int32_t tile_start[kMaxE + 1];
+};
+
+constexpr size_t kSmemBytes = 1024 /* alignment slack */ + (size_t)kStages * kStageBytes + sizeof(Shared);
+
+static_assert(kStageBytes % 1024 == 0, "stage buffers must keep 1024-byte swizzle alignment");
+static_assert(kSFDelay < kStages, "scale gatherer may not hold more stages than the ring has");
+
+struct Params {
+    const uint8_t* a_sf;
+    const float* a_gscale;
+    const uint8_t* w_sf;
+    const float* w_gscale;
+    const int32_t* offsets;
+    uint16_t* out;
+    int32_t E;
+    int64_t max_rows;
+    int64_t N;
+    int64_t K;
+    int32_t swiglu;
+    DeviceCtl ctl;
+};
+
+struct Tile {
+    int32_t e, nt, mt, row0, rows, bn;
+};
+
+__device__ __forceinline__ void decode_tile(const Shared& sh, int32_t E, int32_t n_col_tiles, int32_t w, Tile& t) {
+    int32_t lo = 0, hi = E;  // tile_start[lo] <= w < tile_start[hi]
+    while (hi - lo > 1) {
+        const int32_t mid = (lo + hi) >> 1;
+        if (sh.tile_start[mid] <= w) lo = mid;
+        else hi = mid;
+    }
+    const int32_t M = sh.off[lo + 1] - sh.off[lo];
+    const int32_t mtiles = (M + kBNMax - 1) / kBNMax;
+    const int32_t local = w - sh.tile_start[lo];
+    t.e = lo;
+    t.nt = local / mtiles;
+    t.mt = local - t.nt * mtiles;
+    t.row0 = sh.off[lo] + t.mt * kBNMax;
+    t.rows = min(kBNMax, M - t.mt * kBNMax);
+    t.bn = (t.rows + kBNStep - 1) / kBNStep * kBNStep;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, const DeviceCtl& ctl) {
+    bool ok = mbar_wait_bounded(bar, parity, abort, ctl);
+    return __all_sync(0xFFFFFFFFu, ok);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
+                        const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    Shared& sh = *reinterpret_cast<Shared*>(smem + (size_t)kStages * kStageBytes);
+    volatile int* abort = &sh.abort;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int32_t E = p.E;
+    const int32_t n_col_tiles = (int32_t)(p.swiglu ? (p.N / 2) / kBM : p.N / (kNumA * kBM));
+
+    // ---- scheduler tables: expert offsets and the first work item of each expert ----
+    for (int i = tid; i <= E; i += kThreads) sh.off[i] = __ldg(p.offsets + i);
+    if (tid == 0) {
+        sh.abort = 0;
+        for (int s = 0; s < kStages; s++) {
+            mbar_init(&sh.full_tma[s], 1);
+            mbar_init(&sh.full_sf[s], 1);
+            mbar_init(&sh.empty[s], 1);
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(&sh.acc_full[b], 1);
+            mbar_init(&sh.acc_empty[b], 4);
+        }
+        mbar_init(&sh.drain, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    {
+        // Each thread sums the tiles of 4 consecutive experts, then a block-wide exclusive scan.
+        const int e0 = tid * 4;
+        int32_t cnt[4];
+        int32_t local = 0;
+        bool bad = false;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int e = e0 + i;
+            cnt[i] = 0;
+            if (e < E) {
+                const int32_t a = sh.off[e], b = sh.off[e + 1];
+                if (a < 0 || b < a || (int64_t)b > p.max_rows) {
+                    bad = true;  // inconsistent offsets: skip this expert
+                } else {
+                    cnt[i] = ((b - a + kBNMax - 1) / kBNMax) * n_col_tiles;
+                }
+            }
+            local += cnt[i];
+        }
+        if (bad) atomicOr(p.ctl.status, kStatusBadInput);
+        int32_t incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        __shared__ int32_t warp_tot[kThreads / 32];
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        int32_t before = 0;
+        for (int w2 = 0; w2 < warp; w2++) before += warp_tot[w2];
+        int32_t run = before + incl - local;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int e = e0 + i;
+            if (e < E) sh.tile_start[e] = run;
+            run += cnt[i];
+        }
+        if (tid == kThreads - 1) {
+            sh.total_tiles = before + incl;
+            sh.tile_start[E] = before + incl;
+        }
+    }
+    // ---- tensor memory ----
+    if (warp == 2) {
+        tmem_alloc(&sh.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    const int32_t total = sh.total_tiles;
+    const int32_t ksteps_total = (int32_t)(p.K / kBK);
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        uint32_t issued_parity[kStages];
+        bool issued[kStages];
+#pragma unroll
+        for (int s = 0; s < kStages; s++) issued[s] = false, issued_parity[s] = 0;
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_a = l2_policy_evict_last();
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
+                Tile t;
+                decode_tile(sh, E, n_col_tiles, w, t);
+                int64_t r0, r1;
+                if (p.swiglu) {
+                    r0 = (int64_t)t.nt * kBM;
+                    r1 = p.N / 2 + (int64_t)t.nt * kBM;
+                } else {
+                    r0 = (int64_t)t.nt * (kNumA * kBM);
+                    r1 = r0 + kBM;
+                }
+                const int64_t wr0 = (int64_t)t.e * p.N + r0, wr1 = (int64_t)t.e * p.N + r1;
+                const uint8_t* sfa0 = p.w_sf + (wr0 / kBM) * (p.K / 64) * kSFAtomBytes;
+                const uint8_t* sfa1 = p.w_sf + (wr1 / kBM) * (p.K / 64) * kSFAtomBytes;
+                const uint32_t tx = (uint32_t)(kNumA * (kABlockBytes + kSFStageBytes) + t.bn * kRowBytes);
+                for (int32_t kt = 0; kt < ksteps_total; kt++) {
+                    if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
+                    uint8_t* sb = stages + (size_t)stage * kStageBytes;
+                    uint64_t* bar = &sh.full_tma[stage];
+                    mbar_arrive_expect_tx(bar, tx);
+                    const int32_t kx = kt * kRowBytes;
+                    tma_load_2d(sb + kOffA0, &tm_w, kx, (int32_t)wr0, bar, pol_w);
+                    tma_load_2d(sb + kOffA1, &tm_w, kx, (int32_t)wr1, bar, pol_w);
+                    for (int32_t i = 0; i < t.bn / kBNStep; i++)
+                        tma_load_2d(sb + kOffB + i * kBNStep * kRowBytes, &tm_a, kx, t.row0 + i * kBNStep, bar, pol_a);
+                    bulk_load(sb + kOffSFA0, sfa0 + (size_t)kt * kSFStageBytes, kSFStageBytes, bar, pol_w);
+                    bulk_load(sb + kOffSFA1, sfa1 + (size_t)kt * kSFStageBytes, kSFStageBytes, bar, pol_w);
+                    issued[stage] = true;
+                    issued_parity[stage] = phase;
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok || *abort) {
+                // Abort path: let every copy already issued land before the CTA can exit.
+                for (int s = 0; s < kStages; s++)
+                    if (issued[s]) mbar_wait_drain(&sh.full_tma[s], issued_parity[s], 200000000ull);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ================= activation-scale gatherer =================
+        // Row-major scales [rows, K/16] -> per K-step 512-byte atoms where the
+        // scale word of activation row n sits at (n % 32) * 16 + (n / 32) * 4.
+        uint32_t stage = 0, phase = 0;
+        uint32_t pend[kSFDelay + 1];
+        int npend = 0;
+        bool ok = true;
+        const int64_t sf_row = p.K / 16;
+        for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            Tile t;
+            decode_tile(sh, E, n_col_tiles, w, t);
+            for (int32_t kt = 0; kt < ksteps_total; kt++) {
+                if (!warp_wait(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
+                uint8_t* dst_base = stages + (size_t)stage * kStageBytes + kOffSFB;
+                for (int i = lane; i < 4 * t.bn; i += 32) {
+                    const int n = i >> 2, kc = i & 3;
+                    const int64_t grow = (int64_t)t.row0 + n;
+                    const bool in = grow < p.max_rows;
+                    const uint8_t* src = in ? p.a_sf + grow * sf_row + (int64_t)kt * 16 + kc * 4 : p.a_sf;
+                    cp_async_4(dst_base + kc * kSFAtomBytes + (n & 31) * 16 + (n >> 5) * 4, src, in ? 4u : 0u);
+                }
+                cp_async_commit();
+                pend[npend++] = stage;
+                if (npend > kSFDelay) {
+                    cp_async_wait<kSFDelay>();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sh.full_sf[pend[0]]);
+                    for (int j = 0; j + 1 < npend; j++) pend[j] = pend[j + 1];
+                    npend--;
+                }
+                if (++stage == kStages) { stage = 0; phase ^= 1u; }
+            }
+        }
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (ok && lane == 0)
+            for (int j = 0; j < npend; j++) mbar_arrive(&sh.full_sf[pend[j]]);
+        __syncwarp();
+    } else if (warp == 2) {
+        // ================= MMA issuer =================
+        // Instruction descriptor: E2M1 x E2M1 (format 1), both K-major, UE4M3
+        // scales, M = 128 (bits 24-28 hold M >> 4), N in bits 17-22 (N >> 3).
+        const uint32_t idesc_base = (1u << 7) | (1u << 10) | ((uint32_t)(kBM >> 4) << 24);
+        uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
+        bool ok = true;
+        for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            Tile t;
+            decode_tile(sh, E, n_col_tiles, w, t);
+            const uint32_t idesc = idesc_base | ((uint32_t)(t.bn >> 3) << 17);
+            if (!warp_wait(&sh.acc_empty[abuf], aphase ^ 1u, abort, p.ctl)) { ok = false; break; }
+            tc_fence_after();
+            for (int32_t kt = 0; kt < ksteps_total; kt++) {
+                if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl) ||
+                    !warp_wait(&sh.full_sf[stage], phase, abort, p.ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t sb = smem_u32(stages + (size_t)stage * kStageBytes);
+#pragma unroll
+                    for (int kc = 0; kc < kKSteps; kc++) {
+                        tmem_cp_32x128b_x4(tmem + kTmemSFA + 4 * kc,
+                                           make_smem_desc(sb + kOffSFA0 + kc * kSFAtomBytes, 0, 128, 0));
+                        tmem_cp_32x128b_x4(tmem + kTmemSFA + 4 * kKSteps + 4 * kc,
+                                           make_smem_desc(sb + kOffSFA1 + kc * kSFAtomBytes, 0, 128, 0));
+                        tmem_cp_32x128b_x4(tmem + kTmemSFB + 4 * kc,
+                                           make_smem_desc(sb + kOffSFB + kc * kSFAtomBytes, 0, 128, 0));
+                    }
+#pragma unroll
+                    for (int kc = 0; kc < kKSteps; kc++) {
+                        const uint64_t bdesc = make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2);
+                        const uint32_t acc = (kt | kc) != 0;
+#pragma unroll
+                        for (int a = 0; a < kNumA; a++) {
+                            const uint64_t adesc = make_smem_desc(sb + a * kABlockBytes + kc * 32, 16, 1024, 2);
+                            mma_mxf4nvf4(tmem + abuf * (kNumA * kAccCols) + a * kAccCols, adesc, bdesc, idesc,
+                                         tmem + kTmemSFA + a * 4 * kKSteps + 4 * kc, tmem + kTmemSFB + 4 * kc, acc);
+                        }
+                    }
+                    tc_commit(&sh.empty[stage]);
+                }
+                __syncwarp();
+                if (++stage == kStages) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            if (lane == 0) tc_commit(&sh.acc_full[abuf]);
+            __syncwarp();
+            if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
+        }
+        if (!ok || *abort) {
+            // Abort path: wait for every MMA issued so far before tensor memory is freed.
+            if (lane == 0) {
+                tc_commit(&sh.drain);
+                mbar_wait_drain(&sh.drain, 0, 200000000ull);
+            }
+            __syncwarp();
+        }
+    } else if (warp >= 4) {
+        // ================= epilogue =================
+        const int quad = warp & 3;              // TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;         // accumulator row = weight row within a block
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        const float a_g = __ldg(p.a_gscale);
+        uint32_t abuf = 0, aphase = 0;
+        for (int32_t w = blockIdx.x; w < total; w += gridDim.x) {
+            Tile t;
+            decode_tile(sh, E, n_col_tiles, w, t);
+            if (!warp_wait(&sh.acc_full[abuf], aphase, abort, p.ctl)) break;
+            tc_fence_after();
+            float v0[kBNMax], v1[kBNMax];
+            const uint32_t cbase = tmem + lane_base + abuf * (kNumA * kAccCols);
+#pragma unroll
+            for (int c = 0; c < kBNMax / 16; c++) {
+                if (c * 16 < t.bn) {
+                    float tmp[16];
+                    tmem_ld_32x32b_x16(cbase + c * 16, tmp);
+#pragma unroll
+                    for (int i = 0; i < 16; i++) v0[c * 16 + i] = tmp[i];
+                    tmem_ld_32x32b_x16(cbase + kAccCols + c * 16, tmp);
+#pragma unroll
+                    for (int i = 0; i < 16; i++) v1[c * 16 + i] = tmp[i];
+                }
+            }
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.acc_empty[abuf]);
+            if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
+
+            const float alpha = a_g * __ldg(p.w_gscale + t.e);
+            if (p.swiglu) {
+                const int64_t ldo = p.N / 2;
+                uint16_t* o = p.out + (int64_t)t.row0 * ldo + (int64_t)t.nt * kBM + r;
+#pragma unroll
+                for (int n = 0; n < kBNMax; n++) {
+                    if (n < t.rows) {
+                        const float g = alpha * v0[n], u = alpha * v1[n];
+                        const float h = g / (1.0f + expf(-g)) * u;
+                        o[(int64_t)n * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                    }
+                }
+            } else {
+                const int64_t ldo = p.N;
+                uint16_t* o = p.out + (int64_t)t.row0 * ldo + (int64_t)t.nt * (kNumA * kBM) + r;
+#pragma unroll
+                for (int n = 0; n < kBNMax; n++) {
+                    if (n < t.rows) {
+                        o[(int64_t)n * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v0[n]));
+                        o[(int64_t)n * ldo + kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v1[n]));
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- teardown: every role has drained its own asynchronous work ----
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace gg
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 2-D byte tensor [rows, row_bytes] with 128-byte swizzled boxes of box_rows x 128 bytes.
+static bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, uint32_t box_rows) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {128u, box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+extern "C" nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan) {
+    if (!plan) return NVFP4_ERR_INVALID_ARG;
+    plan->tile_weight_rows = gg::kNumA * gg::kBM;
+    plan->tile_tokens_max = gg::kBNMax;
+    plan->stage_k = gg::kBK;
+    plan->stages = gg::kStages;
+    plan->stage_bytes_weights = gg::kNumA * gg::kABlockBytes;
+    plan->stage_bytes_weight_sf = gg::kNumA * gg::kSFStageBytes;
+    plan->stage_bytes_act_max = gg::kBBytes;
+    plan->stage_bytes_act_sf = gg::kSFStageBytes;
+    plan->smem_bytes = (int32_t)gg::kSmemBytes;
+    plan->tmem_columns = (int32_t)gg::kTmemCols;
+    plan->threads = gg::kThreads;
+    return NVFP4_OK;
+}
+
+extern "C" int64_t nvfp4_gemm_stage_tx_bytes(int32_t tokens) {
+    if (tokens <= 0 || tokens > gg::kBNMax) return -1;
+    const int64_t bn = (tokens + gg::kBNStep - 1) / gg::kBNStep * gg::kBNStep;
+    // MK part: weight tiles + their scales; NK part: activation tile (scales come via cp.async).
+    return (int64_t)gg::kNumA * (gg::kABlockBytes + gg::kSFStageBytes) + bn * gg::kRowBytes;
+}
+
+extern "C" nvfp4_status nvfp4_can_implement_with_budget(int64_t N, int64_t K, int32_t E, nvfp4_epilogue epi,
+                                                        int64_t smem_optin_bytes) {
+    if (epi != NVFP4_EPI_NONE && epi != NVFP4_EPI_SWIGLU) return NVFP4_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0 || E <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (E > gg::kMaxE || N % (gg::kNumA * gg::kBM) != 0 || K % gg::kBK != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if ((int64_t)E * N > INT32_MAX || K / 2 > INT32_MAX) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (smem_optin_bytes < (int64_t)gg::kSmemBytes) return NVFP4_ERR_SMEM_BUDGET;
+    return NVFP4_OK;
+}
+
+extern "C" nvfp4_status nvfp4_can_implement(int64_t N, int64_t K, int32_t E, nvfp4_epilogue epi) {
+    const int optin = device_smem_optin();
+    if (optin < 0) return NVFP4_ERR_CUDA;
+    return nvfp4_can_implement_with_budget(N, K, E, epi, optin);
+}
+
+extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
+                                               const uint8_t* w_q, const uint8_t* w_sf, const float* w_gscale,
+                                               const int32_t* expert_offsets, int32_t E, int64_t max_rows,
+                                               int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
+                                               nvfp4_stream_t stream) {
+    if (!a_q || !a_sf || !a_gscale || !w_q || !w_sf || !w_gscale || !expert_offsets || !out)
+        return NVFP4_ERR_INVALID_ARG;
+    if (max_rows < 0 || max_rows > INT32_MAX) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_q) || !aligned16(a_sf) || !aligned16(w_q) || !aligned16(w_sf) || !aligned16(out) ||
+        ((uintptr_t)a_gscale & 3u) || ((uintptr_t)w_gscale & 3u) || ((uintptr_t)expert_offsets & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    const int optin = device_smem_optin();
+    if (optin < 0) return NVFP4_ERR_CUDA;
+    nvfp4_status st = nvfp4_can_implement_with_budget(N, K, E, epi, optin);
+    if (st != NVFP4_OK) return st;
+    if (max_rows == 0) return NVFP4_OK;
+    uint32_t* status = status_word_ptr();
+    if (!status) return NVFP4_ERR_CUDA;
+
+    CUtensorMap tm_w, tm_a;
+    if (!encode_rows_map(&tm_w, w_q, (int64_t)E * N, K / 2, gg::kBM)) return NVFP4_ERR_CUDA;
+    if (!encode_rows_map(&tm_a, a_q, max_rows, K / 2, gg::kBNStep)) return NVFP4_ERR_CUDA;
+
+    static int configured_device = -1;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (configured_device != dev) {
+        if (cudaFuncSetAttribute(gg::grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gg::kSmemBytes) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        configured_device = dev;
+    }
+    gg::Params prm;
+    prm.a_sf = a_sf;
+    prm.a_gscale = a_gscale;
+    prm.w_sf = w_sf;
+    prm.w_gscale = w_gscale;
+    prm.offsets = expert_offsets;
+    prm.out = out;
+    prm.E = E;
+    prm.max_rows = max_rows;
+    prm.N = N;
+    prm.K = K;
+    prm.swiglu = epi == NVFP4_EPI_SWIGLU ? 1 : 0;
+    prm.ctl.status = status;
+    prm.ctl.timeout_ns = wait_timeout_ns();
+    const int grid = device_sm_count();
+    gg::grouped_gemm_kernel<<<grid, gg::kThreads, gg::kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(
+        tm_w, tm_a, prm);
+    count_launch();
+    return check_launch();
+}

@@ -1,0 +1,188 @@
+// permute.cu -- routing gather: group (token, slot) pairs by expert, stable in
+// (t ascending, j ascending), and copy the quantised activation rows into
+// expert order ("Peering into the CUTLASS Kernel Cache", Knowledge Required:
+// each expert's weights multiply only the subset of tokens routed to it).
+//
+// Deterministic counting sort, no atomics on the output order:
+//   1. count:  CTA c counts, per expert, the pairs of its 256 tokens.
+//   2. scan:   one CTA turns the per-chunk counts into expert offsets and into
+//              the first output row of every (chunk, expert) pair.
+//   3. rank:   CTA c marks, per expert, which of its tokens route there (one
+//              bit per token); a pair's rank inside its expert is the number of
+//              marked earlier tokens (popcount), so positions follow token
+//              order. A token lists each expert at most once, so slot order
+//              inside a token never decides a rank.
+//   4. gather: one warp per output row copies K/2 code bytes and K/16 scale
+//              bytes with 16-byte vector loads and stores.
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int kTok = 256;           // tokens per chunk (one thread each)
+constexpr int kMaxE = 1024;
+constexpr int kWordsPerExpert = kTok / 32;
+
+__global__ void __launch_bounds__(kTok) permute_count_kernel(const int32_t* __restrict__ ids, int32_t T, int32_t k,
+                                                               int32_t E, int32_t* __restrict__ counts,
+                                                               uint32_t* status) {
+    __shared__ int32_t hist[kMaxE];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    const int32_t t = blockIdx.x * kTok + threadIdx.x;
+    if (t < T) {
+        for (int j = 0; j < k; j++) {
+            const int32_t e = ids[(int64_t)t * k + j];
+            if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+            else atomicOr(status, kStatusBadInput);
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+// One CTA of kMaxE threads: thread e owns expert e.
+__global__ void __launch_bounds__(kMaxE) permute_scan_kernel(int32_t* __restrict__ counts, int32_t nchunks,
+                                                               int32_t E, int32_t* __restrict__ offsets) {
+    __shared__ int32_t warp_sums[kMaxE / 32];
+    const int e = threadIdx.x;
+    int32_t total = 0;
+    if (e < E)
+        for (int c = 0; c < nchunks; c++) total += counts[(int64_t)c * E + e];
+    // exclusive scan of `total` over e
+    const int lane = e & 31, warp = e >> 5;
+    int32_t incl = total;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int32_t s = warp_sums[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t v = __shfl_up_sync(0xFFFFFFFFu, s, o);
+            if (lane >= o) s += v;
+        }
+        warp_sums[lane] = s;  // inclusive over warps
+    }
+    __syncthreads();
+    const int32_t excl = incl - total + (warp > 0 ? warp_sums[warp - 1] : 0);
+    if (e < E) {
+        offsets[e] = excl;
+        if (e == E - 1) offsets[E] = excl + total;
+        int32_t run = excl;  // first output row of (chunk c, expert e)
+        for (int c = 0; c < nchunks; c++) {
+            const int32_t n = counts[(int64_t)c * E + e];
+            counts[(int64_t)c * E + e] = run;
+            run += n;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kTok) permute_rank_kernel(const int32_t* __restrict__ ids, int32_t T, int32_t k,
+                                                              int32_t E, const int32_t* __restrict__ base,
+                                                              int32_t* __restrict__ perm_src,
+                                                              int32_t* __restrict__ inv_perm, uint32_t* status) {
+    extern __shared__ uint32_t bits[];  // [E][kWordsPerExpert]
+    for (int i = threadIdx.x; i < E * kWordsPerExpert; i += blockDim.x) bits[i] = 0u;
+    __syncthreads();
+    const int tl = threadIdx.x;
+    const int32_t t = blockIdx.x * kTok + tl;
+    const uint32_t my_bit = 1u << (tl & 31);
+    const int my_word = tl >> 5;
+    if (t < T) {
+        for (int j = 0; j < k; j++) {
+            const int32_t e = ids[(int64_t)t * k + j];
+            if (e >= 0 && e < E) {
+                const uint32_t old = atomicOr(&bits[e * kWordsPerExpert + my_word], my_bit);
+                if (old & my_bit) atomicOr(status, kStatusBadInput);  // expert listed twice by one token
+            }
+        }
+    }
+    __syncthreads();
+    if (t < T) {
+        for (int j = 0; j < k; j++) {
+            const int32_t e = ids[(int64_t)t * k + j];
+            int32_t pos = -1;
+            if (e >= 0 && e < E) {
+                const uint32_t* row = bits + e * kWordsPerExpert;
+                int32_t rank = 0;
+                for (int w = 0; w < my_word; w++) rank += __popc(row[w]);
+                rank += __popc(row[my_word] & (my_bit - 1u));
+                pos = base[(int64_t)blockIdx.x * E + e] + rank;
+                perm_src[pos] = t;
+            }
+            inv_perm[(int64_t)t * k + j] = pos;
+        }
+    }
+}
+
+// One warp per output row; rows whose source index is invalid become zeros.
+__global__ void __launch_bounds__(256) permute_gather_kernel(const uint4* __restrict__ q, const uint4* __restrict__ sf,
+                                                             int64_t qvec, int64_t sfvec,
+                                                             const int32_t* __restrict__ perm_src, int32_t T,
+                                                             int64_t R, uint4* __restrict__ q_perm,
+                                                             uint4* __restrict__ sf_perm) {
+    const int64_t p = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (p >= R) return;
+    const int lane = threadIdx.x & 31;
+    const int32_t src = perm_src[p];
+    const bool ok = src >= 0 && src < T;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    const uint4* qs = q + (int64_t)(ok ? src : 0) * qvec;
+    uint4* qd = q_perm + p * qvec;
+    for (int64_t i = lane; i < qvec; i += 32) qd[i] = ok ? __ldg(qs + i) : zero;
+    const uint4* ss = sf + (int64_t)(ok ? src : 0) * sfvec;
+    uint4* sd = sf_perm + p * sfvec;
+    for (int64_t i = lane; i < sfvec; i += 32) sd[i] = ok ? __ldg(ss + i) : zero;
+}
+
+}  // namespace
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+static inline int32_t permute_chunks(int32_t T) { return (T + kTok - 1) / kTok; }
+
+extern "C" size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E) {
+    (void)k;
+    if (T <= 0 || E <= 0) return 0;
+    return (size_t)permute_chunks(T) * (size_t)E * sizeof(int32_t);
+}
+
+extern "C" nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E, const uint8_t* q,
+                                    const uint8_t* sf, int64_t K, uint8_t* q_perm, uint8_t* sf_perm,
+                                    int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm, void* ws,
+                                    size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!topk_ids || !q || !sf || !q_perm || !sf_perm || !expert_offsets || !perm_src || !inv_perm)
+        return NVFP4_ERR_INVALID_ARG;
+    if (T <= 0 || k <= 0 || E <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (k > 32 || E > kMaxE || (int64_t)T * k >= (int64_t)1 << 31 || K % 256 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(topk_ids) || !aligned16(q) || !aligned16(sf) || !aligned16(q_perm) || !aligned16(sf_perm) ||
+        !aligned16(expert_offsets) || !aligned16(perm_src) || !aligned16(inv_perm))
+        return NVFP4_ERR_MISALIGNED;
+    const size_t need = moe_permute_workspace_size(T, k, E);
+    if (!ws || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_MISALIGNED;
+    uint32_t* status = status_word_ptr();
+    if (!status) return NVFP4_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int32_t nchunks = permute_chunks(T);
+    int32_t* counts = static_cast<int32_t*>(ws);
+    const int64_t R = (int64_t)T * k;
+
+    permute_count_kernel<<<nchunks, kTok, 0, s>>>(topk_ids, T, k, E, counts, status);
+    permute_scan_kernel<<<1, kMaxE, 0, s>>>(counts, nchunks, E, expert_offsets);
+    const size_t rank_smem = (size_t)E * kWordsPerExpert * sizeof(uint32_t);
+    permute_rank_kernel<<<nchunks, kTok, rank_smem, s>>>(topk_ids, T, k, E, counts, perm_src, inv_perm, status);
+    const int64_t gblocks = (R + 7) / 8;
+    permute_gather_kernel<<<(unsigned)gblocks, 256, 0, s>>>(
+        reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(sf), K / 32, K / 256, perm_src, T, R,
+        reinterpret_cast<uint4*>(q_perm), reinterpret_cast<uint4*>(sf_perm));
+    count_launch(4);
+    return check_launch();
+}

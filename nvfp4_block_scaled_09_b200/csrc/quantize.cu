@@ -1,0 +1,230 @@
+// quantize.cu -- BF16 -> NVFP4 (packed E2M1 codes, E4M3 block scales, FP32
+// global scale) for one tensor.
+//
+// Format: two FP4 values per byte and one FP8 scale per 16 elements ("Peering
+// into the CUTLASS SharedStorage", Input Knowledge Required, item 3). The
+// global scale maps the tensor amax onto 6 * 448 (E2M1 max times E4M3 max) and
+// is stored as the dequantisation multiplier g_dec = amax / 2688.
+//
+// Two memory-bound passes, no tensor cores:
+//   1. amax_partial_kernel: grid-stride, 16-byte loads, packed 16-bit integer
+//      max of |bf16| bit patterns (finite BF16 magnitudes order like their
+//      bits), one partial per CTA.
+//   2. quantize_kernel: every CTA folds the partials into the tensor amax (a
+//      few KB from L2), then each thread turns one 16-element block (32 bytes
+//      in) into 8 code bytes and one scale byte with the hardware satfinite
+//      round-to-nearest-even conversions.
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMaxPartials = 8 * 148;
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Largest |x| over a packed pair of BF16 values, kept packed (two u16 lanes).
+__device__ __forceinline__ uint32_t absmax_pair(uint32_t acc, uint32_t w) { return __vmaxu2(acc, w & 0x7FFF7FFFu); }
+
+__device__ __forceinline__ uint32_t fold_pair(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
+
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+__global__ void __launch_bounds__(kThreads) amax_partial_kernel(const uint4* __restrict__ x, int64_t nvec,
+                                                                 uint32_t* __restrict__ partial) {
+    uint32_t m = 0;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += stride) {
+        uint4 v = __ldg(x + i);  // default caching: the quantiser reads x again right after
+        m = absmax_pair(m, v.x);
+        m = absmax_pair(m, v.y);
+        m = absmax_pair(m, v.z);
+        m = absmax_pair(m, v.w);
+    }
+    m = warp_max_u32(fold_pair(m));
+    __shared__ uint32_t s_warp[kThreads / 32];
+    if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        uint32_t v = threadIdx.x < kThreads / 32 ? s_warp[threadIdx.x] : 0u;
+        v = warp_max_u32(v);
+        if (threadIdx.x == 0) partial[blockIdx.x] = v;
+    }
+}
+
+// FP32 -> E4M3, round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint32_t f32_to_e4m3_satfinite(float s) {
+    uint16_t pair;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(0.0f), "f"(s));
+    return pair & 0xFFu;
+}
+
+// Non-negative finite E4M3 byte -> FP32 (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+    if (e == 0) return (float)m * 0.001953125f;  // m * 2^-9, exact
+    return __uint_as_float(((e + 120u) << 23) | (m << 20));  // (1 + m/8) * 2^(e-7)
+}
+
+// Four FP32 values -> four E2M1 pairs packed little-endian: value 2i in the low nibble of byte i.
+__device__ __forceinline__ uint32_t f32x8_to_e2m1x8(const float (&y)[8]) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+    return out;
+}
+
+struct GlobalScale {
+    float enc, dec;
+};
+
+__device__ __forceinline__ GlobalScale global_scale(float amax, const float* gdec_in) {
+    GlobalScale g;
+    if (gdec_in != nullptr) {
+        g.dec = *gdec_in;
+        g.enc = __fdiv_rn(1.0f, g.dec);
+    } else if (amax == 0.0f) {
+        g.enc = 1.0f;
+        g.dec = 1.0f;
+    } else {
+        g.enc = __fdiv_rn(2688.0f, amax);
+        g.dec = __fdiv_rn(amax, 2688.0f);
+    }
+    return g;
+}
+
+template <bool kTiled>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, int64_t rows, int64_t K,
+                                                            const float* __restrict__ gdec_in,
+                                                            const uint32_t* __restrict__ partial, int npartial,
+                                                            uint2* __restrict__ q, uint8_t* __restrict__ sf,
+                                                            float* __restrict__ gdec_out) {
+    __shared__ float s_genc;
+    if (threadIdx.x < 32) {
+        float amax = 0.0f;
+        if (gdec_in == nullptr) {
+            uint32_t m = 0;
+            for (int i = threadIdx.x; i < npartial; i += 32) m = max(m, partial[i]);
+            m = warp_max_u32(m);
+            amax = bf16_bits_to_f32(m);
+        }
+        const GlobalScale g = global_scale(amax, gdec_in);
+        if (threadIdx.x == 0) {
+            s_genc = g.enc;
+            if (blockIdx.x == 0) *gdec_out = g.dec;
+        }
+    }
+    __syncthreads();
+    const float g_enc = s_genc;
+    const int64_t blocks_per_row = K >> 4;
+    const int64_t nblk = rows * blocks_per_row;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
+        const uint4 v0 = __ldcs(x + 2 * b);
+        const uint4 v1 = __ldcs(x + 2 * b + 1);
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 8; i++) m = absmax_pair(m, w[i]);
+        const float amax_b = bf16_bits_to_f32(fold_pair(m));
+        const float s = __fmul_rn(__fdiv_rn(amax_b, 6.0f), g_enc);
+        const uint32_t S = f32_to_e4m3_satfinite(s);
+        const float sfv = e4m3_to_f32(S);
+        uint2 packed = make_uint2(0u, 0u);
+        if (sfv != 0.0f) {
+            const float f = __fdiv_rn(g_enc, sfv);
+            float y[8];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                y[2 * i] = __fmul_rn(bf16_bits_to_f32(w[i] & 0xFFFFu), f);
+                y[2 * i + 1] = __fmul_rn(bf16_bits_to_f32(w[i] >> 16), f);
+            }
+            packed.x = f32x8_to_e2m1x8(y);
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                y[2 * i] = __fmul_rn(bf16_bits_to_f32(w[4 + i] & 0xFFFFu), f);
+                y[2 * i + 1] = __fmul_rn(bf16_bits_to_f32(w[4 + i] >> 16), f);
+            }
+            packed.y = f32x8_to_e2m1x8(y);
+        }
+        q[b] = packed;
+        int64_t sf_off;
+        if (kTiled) {
+            const int64_t r = b / blocks_per_row, kb = b - r * blocks_per_row;
+            const int64_t atom = (r >> 7) * (K >> 6) + (kb >> 2);
+            sf_off = atom * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
+        } else {
+            sf_off = b;
+        }
+        sf[sf_off] = (uint8_t)S;
+    }
+}
+
+}  // namespace
+
+static int amax_grid(int64_t nvec) {
+    int64_t g = (nvec + kThreads * 4 - 1) / (kThreads * 4);
+    if (g < 1) g = 1;
+    if (g > kMaxPartials) g = kMaxPartials;
+    return (int)g;
+}
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" size_t nvfp4_quantize_workspace_size(int64_t rows, int64_t K) {
+    if (rows <= 0 || K <= 0) return 0;
+    return (size_t)amax_grid(rows * K / 8) * sizeof(uint32_t);
+}
+
+extern "C" nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t K, const float* global_scale_in,
+                                       uint8_t* q, uint8_t* sf, float* global_scale_out, nvfp4_sf_layout layout,
+                                       void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!x || !q || !sf || !global_scale_out) return NVFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_MMA_TILED) return NVFP4_ERR_INVALID_ARG;
+    if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (layout == NVFP4_SF_MMA_TILED && (rows % 128 != 0 || K % 64 != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned8(q)) return NVFP4_ERR_MISALIGNED;
+    if (((uintptr_t)global_scale_out & 3u) || (global_scale_in && ((uintptr_t)global_scale_in & 3u)))
+        return NVFP4_ERR_MISALIGNED;
+    const int64_t nvec = rows * K / 8;
+    const int grid_a = amax_grid(nvec);
+    if (global_scale_in == nullptr) {
+        if (!ws || ws_bytes < (size_t)grid_a * sizeof(uint32_t)) return NVFP4_ERR_WORKSPACE;
+        if ((uintptr_t)ws & 3u) return NVFP4_ERR_MISALIGNED;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* partial = static_cast<uint32_t*>(ws);
+    if (global_scale_in == nullptr) {
+        amax_partial_kernel<<<grid_a, kThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), nvec, partial);
+        count_launch();
+    }
+    const int64_t nblk = rows * K / 16;
+    int64_t grid_q = (nblk + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)device_sm_count() * 16;
+    if (grid_q > cap) grid_q = cap;
+    if (grid_q < 1) grid_q = 1;
+    if (layout == NVFP4_SF_MMA_TILED)
+        quantize_kernel<true><<<(int)grid_q, kThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), rows, K,
+                                                               global_scale_in, partial, grid_a,
+                                                               reinterpret_cast<uint2*>(q), sf, global_scale_out);
+    else
+        quantize_kernel<false><<<(int)grid_q, kThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), rows, K,
+                                                                global_scale_in, partial, grid_a,
+                                                                reinterpret_cast<uint2*>(q), sf, global_scale_out);
+    count_launch();
+    return check_launch();
+}

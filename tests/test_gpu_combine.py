@@ -1,0 +1,38 @@
+"""moe_unpermute_combine on the GPU against the oracle (FP64 sum, BF16-rounded)."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_09_b200 as nv
+import oracle
+import workloads
+from tests.helpers import compare_bf16, gpu_bf16, host, host_bits, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+@pytest.mark.parametrize("T,E,k,H", [(1, 4, 1, 8), (37, 8, 4, 256), (512, 256, 8, 6144), (1024, 256, 8, 6144)])
+def test_combine_parity(T, E, k, H):
+    ids, w = workloads.routing(T, E, k, "uniform", seed=T)
+    _, _, inv = oracle.permute(ids, E)
+    y = workloads.random_bf16_bits((T * k, H), seed=T + 1)
+    out = nv.unpermute_combine(gpu_bf16(y), torch.from_numpy(inv).cuda(), torch.from_numpy(w).cuda())
+    ref = oracle.bf16_round(oracle.combine(y, inv, w))
+    stats = compare_bf16(host_bits(out), ref, "combine")
+    assert stats["exact_frac"] > 0.99
+
+
+def test_one_hot_weights_select_rows_exactly():
+    T, E, k, H = 16, 8, 4, 64
+    ids, _ = workloads.routing(T, E, k, "uniform", seed=3)
+    _, _, inv = oracle.permute(ids, E)
+    y = workloads.random_bf16_bits((T * k, H), seed=4)
+    w = np.zeros((T, k), dtype=np.float32)
+    w[:, 1] = 1.0
+    out = nv.unpermute_combine(gpu_bf16(y), torch.from_numpy(inv).cuda(), torch.from_numpy(w).cuda())
+    assert np.array_equal(host_bits(out), y[inv.reshape(T, k)[:, 1]])

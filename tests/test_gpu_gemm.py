@@ -1,0 +1,205 @@
+"""moe_grouped_gemm_nvfp4 on the GPU against the oracle.
+
+Teacher-forced: the oracle consumes the GPU's own quantised operands (whose
+quantisation is itself checked bit-exact against the oracle), computes the
+block-scaled dot products in FP64, and the BF16-rounded result is the
+reference. Small cases are compared element by element; the full-size cases
+(dense 8192^3, the decode layer's two GEMMs) on sampled outputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_09_b200 as nv
+import oracle
+import workloads
+from tests.helpers import compare_bf16, gpu_bf16, host, host_bits, require_gpu, untile_sf
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def make_case(rows, N, K, seed, a_std=1.0, w_std=0.02):
+    """Quantised activations [sum(rows), K] and per-expert weights [E, N, K] on the GPU."""
+    E = len(rows)
+    R = int(sum(rows))
+    a_bits = workloads.random_bf16_bits((max(R, 1), K), seed=seed, std=a_std)
+    a_q, a_sf, a_g = nv.quantize(gpu_bf16(a_bits))
+    w = workloads.normal_bf16((E, N, K), w_std, seed, workloads.TAG_W13, device="cuda")
+    w_q, w_sf, w_g = nv.prepare_expert_weights(w)
+    off = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
+    torch.cuda.synchronize()
+    # the GPU's operands are the oracle's operands: check their quantisation first
+    oq, osf, og = oracle.quantize(a_bits)
+    assert np.array_equal(host(a_q), oq) and np.array_equal(host(a_sf), osf) and host(a_g)[0] == og
+    return dict(a_q=a_q, a_sf=a_sf, a_g=a_g, w_q=w_q, w_sf=w_sf, w_g=w_g, off=torch.from_numpy(off).cuda(),
+                off_np=off, w=w, E=E, R=R, N=N, K=K)
+
+
+def oracle_operands(c, experts=None):
+    """Host copies of the GPU operands (weight scales un-tiled to row-major)."""
+    E, N, K = c["E"], c["N"], c["K"]
+    sel = range(E) if experts is None else experts
+    w_q = np.stack([host(c["w_q"][e]) for e in sel])
+    w_sf = np.stack([untile_sf(host(c["w_sf"][e]), N, K) for e in sel])
+    w_g = host(c["w_g"])[list(sel)]
+    return w_q, w_sf, w_g
+
+
+def check_weights_quantised_like_oracle(c, experts):
+    for e in experts:
+        wq, wsf, wg = oracle.quantize(host_bits(c["w"][e]))
+        assert np.array_equal(host(c["w_q"][e]), wq)
+        assert np.array_equal(untile_sf(host(c["w_sf"][e]), c["N"], c["K"]), wsf)
+        assert host(c["w_g"])[e] == wg
+
+
+def run_full(rows, N, K, swiglu, seed):
+    c = make_case(rows, N, K, seed)
+    out = nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["w_q"], c["w_sf"], c["w_g"], c["off"], N, K, swiglu)
+    assert nv.device_status() == 0
+    check_weights_quantised_like_oracle(c, range(min(c["E"], 3)))
+    w_q, w_sf, w_g = oracle_operands(c)
+    ref = oracle.grouped_gemm(host(c["a_q"]), host(c["a_sf"]), host(c["a_g"])[0], w_q, w_sf, w_g, c["off_np"],
+                              N, K, swiglu)
+    got = host_bits(out)[: c["R"]]
+    return compare_bf16(got, oracle.bf16_round(ref), f"gemm rows={rows} N={N} K={K} swiglu={swiglu}")
+
+
+def test_tiny_config():
+    # 4 experts x 16 rows, K = N = 256, plain epilogue
+    stats = run_full([16, 16, 16, 16], 256, 256, False, seed=0)
+    assert stats["exact_frac"] > 0.97
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
+def test_ragged_experts_and_row_tiles(swiglu):
+    # empty expert, 1 row, a partial 16-row step, exactly one 64-row tile, 64+1, several tiles
+    run_full([0, 1, 17, 64, 65, 130], 512, 512, swiglu, seed=1)
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
+def test_deeper_k_and_wider_n(swiglu):
+    run_full([5, 40, 200], 768, 2048, swiglu, seed=2)
+
+
+def test_rows_outside_experts_untouched():
+    c = make_case([10, 0, 20], 256, 256, seed=3)
+    R = c["R"]
+    out = torch.full((R + 8, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    # offsets cover only rows [0, 30); rows 30.. must keep their canary
+    nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["w_q"], c["w_sf"], c["w_g"], c["off"], 256, 256, False,
+                    out=out)
+    assert nv.device_status() == 0
+    assert torch.all(out[R:] == 7.0)
+
+
+def test_bad_offsets_latch_status_and_skip():
+    c = make_case([16, 16], 256, 256, seed=4)
+    bad = torch.tensor([0, 20, 10], dtype=torch.int32, device="cuda")   # decreasing
+    nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["w_q"], c["w_sf"], c["w_g"], bad, 256, 256, False)
+    assert nv.device_status() == 8
+
+
+def sampled_check(a_q, a_sf, a_g, c_w, off_np, N, K, swiglu, out, experts, n_cols=64, seed=0):
+    """Compare the GPU output against the oracle at every row of `experts` x n_cols random columns."""
+    rng = np.random.default_rng(seed)
+    nout = N // 2 if swiglu else N
+    w_q, w_sf, w_g = c_w(experts)
+    rows_l, cols_l, sub_off = [], [], [0]
+    a_rows = []
+    for i, e in enumerate(experts):
+        r0, r1 = int(off_np[e]), int(off_np[e + 1])
+        a_rows.extend(range(r0, r1))
+        sub_off.append(sub_off[-1] + (r1 - r0))
+    a_rows = np.array(a_rows, dtype=np.int64)
+    cols = rng.choice(nout, size=min(n_cols, nout), replace=False)
+    rr, cc = np.meshgrid(np.arange(a_rows.size), cols, indexing="ij")
+    rr, cc = rr.ravel(), cc.ravel()
+    aq = host(a_q)[a_rows]
+    asf = host(a_sf)[a_rows]
+    ref = oracle.grouped_gemm_at(aq, asf, float(host(a_g)[0]), w_q, w_sf, w_g, np.array(sub_off, np.int32), N, K,
+                                 swiglu, rr, cc)
+    got = host_bits(out)[a_rows[rr], cc]
+    return compare_bf16(got, oracle.bf16_round(ref), f"sampled N={N} K={K} swiglu={swiglu}")
+
+
+def test_dense_8192_sampled():
+    M = N = K = 8192
+    a_bits_t = workloads.normal_bf16((M, K), 1.0, 0, workloads.TAG_A, device="cuda")
+    a_q, a_sf, a_g = nv.quantize(a_bits_t)
+    b = workloads.normal_bf16((1, N, K), 0.02, 0, workloads.TAG_B, device="cuda")
+    w_q, w_sf, w_g = nv.prepare_expert_weights(b)
+    off = torch.tensor([0, M], dtype=torch.int32, device="cuda")
+    out = nv.grouped_gemm(a_q, a_sf, a_g, w_q, w_sf, w_g, off, N, K, False)
+    assert nv.device_status() == 0
+    # quantisation of a sample of A rows against the oracle
+    oq, osf, og = oracle.quantize(host_bits(a_bits_t[:256]), float(host(a_g)[0]))
+    assert np.array_equal(host(a_q[:256]), oq) and np.array_equal(host(a_sf[:256]), osf)
+    rng = np.random.default_rng(5)
+    rows = np.sort(rng.choice(M, size=48, replace=False))
+    cols = rng.choice(N, size=48, replace=False)
+    rr, cc = np.meshgrid(rows, cols, indexing="ij")
+    rr, cc = rr.ravel(), cc.ravel()
+    wq = host(w_q)
+    wsf = untile_sf(host(w_sf[0]), N, K)[None]
+    ref = oracle.grouped_gemm_at(host(a_q), host(a_sf), float(host(a_g)[0]), wq, wsf, host(w_g),
+                                 np.array([0, M], np.int32), N, K, False, rr, cc)
+    compare_bf16(host_bits(out)[rr, cc], oracle.bf16_round(ref), "dense 8192")
+
+
+@pytest.mark.parametrize("name", ["moe_decode_t512", "moe_zipf_t1024"])
+def test_moe_layer_gemms_full_size_sampled(name):
+    cfg = workloads.CONFIGS[name]
+    T, H, I, E, k = cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"]
+    ids, _ = workloads.config_routing(name)
+    off_np, src, _ = oracle.permute(ids, E)
+    R = T * k
+    # activations already in expert order (permute is tested on its own)
+    a = workloads.normal_bf16((R, H), 1.0, 0, workloads.TAG_X, device="cuda")
+    a_q, a_sf, a_g = nv.quantize(a)
+    w13 = [None] * E
+    w13_q = torch.empty((E, 2 * I, H // 2), dtype=torch.uint8, device="cuda")
+    w13_sf = torch.empty((E, 2 * I, H // 16), dtype=torch.uint8, device="cuda")
+    w13_g = torch.empty(E, dtype=torch.float32, device="cuda")
+    for e in range(E):
+        w = workloads.normal_bf16((2 * I, H), 0.02, 0, workloads.TAG_W13, e, device="cuda")
+        nv.quantize(w, layout=nv.SF_MMA_TILED, q=w13_q[e], sf=w13_sf[e], g=w13_g[e:e + 1])
+        if e < 2:
+            w13[e] = host_bits(w)
+    off = torch.from_numpy(off_np).cuda()
+    h = nv.grouped_gemm(a_q, a_sf, a_g, w13_q, w13_sf, w13_g, off, 2 * I, H, True)
+    assert nv.device_status() == 0
+    for e in range(2):
+        wq, wsf, wg = oracle.quantize(w13[e])
+        assert np.array_equal(host(w13_q[e]), wq) and np.array_equal(untile_sf(host(w13_sf[e]), 2 * I, H), wsf)
+    counts = np.diff(off_np)
+    experts = [int(np.argmax(counts)), int(np.argmin(np.where(counts > 0, counts, 1 << 30))), 0, E - 1]
+    experts = sorted(set(e for e in experts if counts[e] > 0))
+
+    def w13_host(sel):
+        return (np.stack([host(w13_q[e]) for e in sel]),
+                np.stack([untile_sf(host(w13_sf[e]), 2 * I, H) for e in sel]), host(w13_g)[sel])
+
+    sampled_check(a_q, a_sf, a_g, w13_host, off_np, 2 * I, H, True, h, experts, n_cols=32)
+
+    # down projection on the GPU's own h
+    hq, hsf, hg = nv.quantize(h)
+    w2_q = torch.empty((E, H, I // 2), dtype=torch.uint8, device="cuda")
+    w2_sf = torch.empty((E, H, I // 16), dtype=torch.uint8, device="cuda")
+    w2_g = torch.empty(E, dtype=torch.float32, device="cuda")
+    for e in range(E):
+        w = workloads.normal_bf16((H, I), 0.02, 0, workloads.TAG_W2, e, device="cuda")
+        nv.quantize(w, layout=nv.SF_MMA_TILED, q=w2_q[e], sf=w2_sf[e], g=w2_g[e:e + 1])
+    y = nv.grouped_gemm(hq, hsf, hg, w2_q, w2_sf, w2_g, off, H, I, False)
+    assert nv.device_status() == 0
+
+    def w2_host(sel):
+        return (np.stack([host(w2_q[e]) for e in sel]),
+                np.stack([untile_sf(host(w2_sf[e]), H, I) for e in sel]), host(w2_g)[sel])
+
+    sampled_check(hq, hsf, hg, w2_host, off_np, H, I, False, y, experts, n_cols=32, seed=1)

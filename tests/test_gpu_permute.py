@@ -1,0 +1,57 @@
+"""moe_permute on the GPU against the oracle: offsets, indices and gathered
+bytes bit-exact, for every routing pattern of the workloads."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_09_b200 as nv
+import oracle
+import workloads
+from tests.helpers import host, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def run(ids, E, K, seed=0):
+    T = ids.shape[0]
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, 256, size=(T, K // 2), dtype=np.uint8)
+    sf = rng.integers(0, 256, size=(T, K // 16), dtype=np.uint8)
+    out = nv.permute(torch.from_numpy(ids).cuda(), torch.from_numpy(q).cuda(), torch.from_numpy(sf).cuda(), E)
+    assert nv.device_status() == 0
+    off, src, inv = oracle.permute(ids, E)
+    assert np.array_equal(host(out.offsets), off)
+    assert np.array_equal(host(out.perm_src), src)
+    assert np.array_equal(host(out.inv_perm), inv)
+    assert np.array_equal(host(out.q_perm), oracle.gather_rows(q, src))
+    assert np.array_equal(host(out.sf_perm), oracle.gather_rows(sf, src))
+
+
+@pytest.mark.parametrize("name", ["moe_decode_t512", "moe_zipf_t1024", "moe_prefill_t8192"])
+def test_workload_routing(name):
+    ids, _ = workloads.config_routing(name)
+    run(ids, 256, 6144 if name != "moe_prefill_t8192" else 256)
+
+
+@pytest.mark.parametrize("T,E,k,kind", [(1, 4, 1, "uniform"), (37, 5, 3, "uniform"), (300, 1024, 8, "zipf"),
+                                        (257, 64, 16, "uniform"), (513, 3, 2, "zipf")])
+def test_ragged_shapes(T, E, k, kind):
+    ids, _ = workloads.routing(T, E, k, kind, seed=T)
+    run(ids, E, 256, seed=T)
+
+
+def test_invalid_and_duplicate_ids_latch_status():
+    ids = np.array([[0, 1], [2, 7]], dtype=np.int32)       # 7 >= E
+    q = torch.zeros((2, 128), dtype=torch.uint8, device="cuda")
+    sf = torch.zeros((2, 16), dtype=torch.uint8, device="cuda")
+    nv.permute(torch.from_numpy(ids).cuda(), q, sf, 4)
+    assert nv.device_status() == 8
+    ids = np.array([[1, 1], [2, 3]], dtype=np.int32)       # expert listed twice by token 0
+    nv.permute(torch.from_numpy(ids).cuda(), q, sf, 4)
+    assert nv.device_status() == 8
+    assert nv.device_status() == 0                          # reading clears the word

@@ -1,0 +1,87 @@
+"""The C-ABI library builds, loads and exports every call the header declares;
+host-side checks (capability predicate, pipeline plan, stage byte accounting,
+status strings) run without a GPU."""
+import ctypes
+
+import pytest
+
+import nvfp4_block_scaled_09_b200 as nv
+from nvfp4_block_scaled_09_b200 import build as nvbuild
+from tests.helpers import header_symbols
+
+
+@pytest.fixture(scope="module")
+def L():
+    nvbuild.build()
+    return nv.lib()
+
+
+def test_every_header_symbol_is_exported(L):
+    syms = header_symbols()
+    assert len(syms) >= 18, syms
+    for s in syms:
+        assert hasattr(L, s), f"{s} declared in include/nvfp4moe.h but not exported"
+
+
+def test_status_strings(L):
+    for code, name in nv.STATUS.items():
+        assert nv.status_string(code) == name
+
+
+def test_can_implement_shapes_and_budget(L):
+    big = 232448  # B200 opt-in shared memory per block
+    plan = nv.gemm_plan()
+    assert plan["smem_bytes"] <= big
+    assert nv.can_implement(4096, 6144, 256, True, big) == 0
+    assert nv.can_implement(6144, 2048, 256, False, big) == 0
+    assert nv.can_implement(8192, 8192, 1, False, big) == 0
+    assert nv.can_implement(256, 256, 4, False, big) == 0
+    assert nv.can_implement(4096 + 128, 6144, 256, True, big) == 3
+    assert nv.can_implement(4096, 6144 + 128, 256, True, big) == 3
+    assert nv.can_implement(4096, 6144, 1025, True, big) == 3
+    assert nv.can_implement(0, 6144, 8, True, big) == 1
+    # a budget below the kernel's shared memory is refused before any launch
+    assert nv.can_implement(4096, 6144, 256, True, plan["smem_bytes"] - 1) == 5
+    assert nv.can_implement(4096, 6144, 256, True, 101376) == 5     # an SM120-sized budget
+
+
+def test_stage_transaction_bytes_are_tile_sums(L):
+    # Per stage: (A tile bits + A scale bits) + (B tile bits), in bytes, for
+    # packed E2M1 (4 bits) and one 8-bit scale per 16 elements.
+    plan = nv.gemm_plan()
+    bk = plan["stage_k"]
+    wrows = plan["tile_weight_rows"]
+    a_bits = wrows * bk * 4
+    sfa_bits = wrows * (bk // 16) * 8
+    for tokens in (1, 15, 16, 17, 32, 48, 64):
+        bn = -(-tokens // 16) * 16
+        b_bits = bn * bk * 4
+        assert nv.gemm_stage_tx_bytes(tokens) == (a_bits + sfa_bits + b_bits) // 8
+    assert nv.gemm_stage_tx_bytes(0) == -1
+    assert nv.gemm_stage_tx_bytes(plan["tile_tokens_max"] + 1) == -1
+    # the ring fits the shared-memory budget it claims
+    stage = plan["stage_bytes_weights"] + plan["stage_bytes_weight_sf"] + plan["stage_bytes_act_max"] + \
+        plan["stage_bytes_act_sf"]
+    assert plan["stages"] * stage <= plan["smem_bytes"]
+    assert plan["tmem_columns"] in (32, 64, 128, 256, 512)
+
+
+def test_layer_workspace_layout_is_disjoint_and_aligned(L):
+    lay = nv.layer_workspace_layout(512, 8, 256, 6144, 2048)
+    names = [n for n in lay if n != "total"]
+    offs = sorted(lay[n] for n in names)
+    assert all(o % 256 == 0 for o in offs)
+    assert len(set(offs)) == len(offs)
+    R = 512 * 8
+    assert lay["q_perm"] - lay["g_x"] >= 4 and lay["sf_perm"] - lay["q_perm"] >= R * 6144 // 2
+    assert lay["total"] >= lay["scratch"]
+
+
+def test_invalid_arguments_rejected_before_any_cuda_call(L):
+    # Null pointers and bad shapes return synchronously (no device needed).
+    assert L.nvfp4_quantize(None, 4, 32, None, None, None, None, 0, None, 0, None) == 1
+    assert L.moe_unpermute_combine(None, None, None, 1, 1, 8, None, None) == 1
+    p = ctypes.c_void_p(16)
+    assert L.moe_unpermute_combine(p, p, p, 1, 1, 12, p, None) == 3     # H % 8 != 0
+    assert L.moe_permute(p, 4, 8, 2000, p, p, 256, p, p, p, p, p, p, 1 << 20, None) == 3  # E > 1024
+    assert L.moe_permute(p, 4, 8, 8, p, p, 256, p, p, p, p, p, None, 0, None) == 4       # no workspace
