@@ -165,10 +165,12 @@ NVFP4_API nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t*
 /* token order -- the final MoE output write of the FINALIZE epilogue       */
 /* ("Peering into the CUTLASS Kernel", Input Knowledge Required, item 5).    */
 /*   out[t, h] = BF16( sum_{j=0..k-1} topk_w[t, j] * y[inv_perm[t*k+j], h] ) */
-/*   accumulated in FP32 over j ascending; a negative inv_perm entry is      */
-/*   skipped.                                                                */
+/*   accumulated in FP64 over j ascending (each FP32 x BF16 product is exact */
+/*   in FP64) and rounded once to BF16 (nearest even); a negative inv_perm   */
+/*   entry is skipped.                                                       */
 /* Arguments: y [T*k, H] BF16, inv_perm [T*k], topk_w [T, k] FP32, out [T, H]*/
-/*   BF16; all device, 16-byte aligned; H % 8 == 0, 1 <= k <= 32.            */
+/*   BF16; y and out 16-byte aligned, inv_perm and topk_w 4-byte aligned;   */
+/*   all device; H % 8 == 0, 1 <= k <= 32, 1 <= T <= 65535.                  */
 /* ------------------------------------------------------------------------ */
 NVFP4_API nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* inv_perm, const float* topk_w,
                                    int32_t T, int32_t k, int64_t H, uint16_t* out,

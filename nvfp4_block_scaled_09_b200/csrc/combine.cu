@@ -5,7 +5,12 @@
 //   out[t, :] = BF16( sum_{j ascending} w[t, j] * y[inv_perm[t*k + j], :] )
 //
 // Memory bound (reads k rows of y per token, writes one row): each thread owns
-// 8 consecutive columns (16-byte loads and stores), FP32 accumulation.
+// 8 consecutive columns (16-byte loads and stores). The sum is accumulated in
+// FP64: a product of an FP32 weight and a BF16 value has at most 32
+// significant bits, so every product is exact and the only roundings are the
+// FP64 additions and one final rounding to BF16 (through round-to-odd FP32,
+// which keeps that single rounding correct). FP64 costs nothing here: the
+// kernel moves 2 bytes per FMA.
 #include "common.cuh"
 
 namespace nvfp4 {
@@ -14,14 +19,21 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kColsPerThread = 8;
 
-__device__ __forceinline__ void acc_bf16x2(float& a0, float& a1, uint32_t w, float s) {
-    a0 = fmaf(s, __uint_as_float(w << 16), a0);
-    a1 = fmaf(s, __uint_as_float(w & 0xFFFF0000u), a1);
+__device__ __forceinline__ void acc_bf16x2(double& a0, double& a1, uint32_t w, double s) {
+    a0 = fma(s, (double)__uint_as_float(w << 16), a0);
+    a1 = fma(s, (double)__uint_as_float(w & 0xFFFF0000u), a1);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&v);
+// FP64 -> BF16, round to nearest even, in effect a single rounding: truncate to
+// FP32, mark inexactness in the last bit (round-to-odd), then round to BF16.
+__device__ __forceinline__ uint32_t f64_to_bf16_bits(double d) {
+    float f = __double2float_rz(d);
+    if ((double)f != d) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(double lo, double hi) {
+    return f64_to_bf16_bits(lo) | (f64_to_bf16_bits(hi) << 16);
 }
 
 __global__ void __launch_bounds__(kThreads) combine_kernel(const uint4* __restrict__ y,
@@ -31,13 +43,13 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const uint4* __restri
     const int64_t t = blockIdx.y;
     const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;  // 16-byte column group
     if (c >= hvec) return;
-    float a[kColsPerThread];
+    double a[kColsPerThread];
 #pragma unroll
-    for (int i = 0; i < kColsPerThread; i++) a[i] = 0.0f;
+    for (int i = 0; i < kColsPerThread; i++) a[i] = 0.0;
     for (int j = 0; j < k; j++) {
         const int32_t p = __ldg(inv_perm + t * k + j);
         if (p < 0) continue;
-        const float s = __ldg(w + t * k + j);
+        const double s = (double)__ldg(w + t * k + j);
         const uint4 v = __ldcs(y + (int64_t)p * hvec + c);
         acc_bf16x2(a[0], a[1], v.x, s);
         acc_bf16x2(a[2], a[3], v.y, s);

@@ -67,13 +67,13 @@ def run_full(rows, N, K, swiglu, seed):
     ref = oracle.grouped_gemm(host(c["a_q"]), host(c["a_sf"]), host(c["a_g"])[0], w_q, w_sf, w_g, c["off_np"],
                               N, K, swiglu)
     got = host_bits(out)[: c["R"]]
-    return compare_bf16(got, oracle.bf16_round(ref), f"gemm rows={rows} N={N} K={K} swiglu={swiglu}")
+    return compare_bf16(got, oracle.bf16_round(ref), f"gemm rows={rows} N={N} K={K} swiglu={swiglu}", exact=ref)
 
 
 def test_tiny_config():
     # 4 experts x 16 rows, K = N = 256, plain epilogue
     stats = run_full([16, 16, 16, 16], 256, 256, False, seed=0)
-    assert stats["exact_frac"] > 0.97
+    assert stats["exact_frac"] > 0.95
 
 
 @pytest.mark.parametrize("swiglu", [False, True])
@@ -125,7 +125,7 @@ def sampled_check(a_q, a_sf, a_g, c_w, off_np, N, K, swiglu, out, experts, n_col
     ref = oracle.grouped_gemm_at(aq, asf, float(host(a_g)[0]), w_q, w_sf, w_g, np.array(sub_off, np.int32), N, K,
                                  swiglu, rr, cc)
     got = host_bits(out)[a_rows[rr], cc]
-    return compare_bf16(got, oracle.bf16_round(ref), f"sampled N={N} K={K} swiglu={swiglu}")
+    return compare_bf16(got, oracle.bf16_round(ref), f"sampled N={N} K={K} swiglu={swiglu}", exact=ref)
 
 
 def test_dense_8192_sampled():
@@ -149,7 +149,7 @@ def test_dense_8192_sampled():
     wsf = untile_sf(host(w_sf[0]), N, K)[None]
     ref = oracle.grouped_gemm_at(host(a_q), host(a_sf), float(host(a_g)[0]), wq, wsf, host(w_g),
                                  np.array([0, M], np.int32), N, K, False, rr, cc)
-    compare_bf16(host_bits(out)[rr, cc], oracle.bf16_round(ref), "dense 8192")
+    compare_bf16(host_bits(out)[rr, cc], oracle.bf16_round(ref), "dense 8192", exact=ref)
 
 
 @pytest.mark.parametrize("name", ["moe_decode_t512", "moe_zipf_t1024"])
