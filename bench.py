@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    # size overrides, used to make small cases of a workload for profiler captures
+    ap.add_argument("--tokens", type=int, default=None)
+    ap.add_argument("--experts", type=int, default=None)
     return ap.parse_args()
 
 
@@ -398,6 +401,10 @@ def cpu_baseline(cfg, seed):
 def main():
     args = parse()
     cfg = dict(workloads.CONFIGS[args.config])
+    if args.tokens:
+        cfg["T"] = args.tokens
+    if args.experts:
+        cfg["E"] = args.experts
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -467,10 +474,12 @@ def main():
         "ms_per_step": max_ms / K,
         "higher_is_better": True,
         "scaling": "weak",
-        "vs_baseline": value / PAGES_DECODE_TFLOPS if args.config == "moe_decode_t512" else None,
+        "vs_baseline": (value / PAGES_DECODE_TFLOPS
+                        if args.config == "moe_decode_t512" and not (args.tokens or args.experts) else None),
         "dtype": "nvfp4 (e2m1 x e2m1, fp32 accumulate)",
         "data": "synthetic",
-        "config": {"workload": args.config, "tokens": cfg["T"], "hidden": cfg["H"], "intermediate": cfg["I"],
+        "config": {"workload": args.config if not (args.tokens or args.experts) else
+                   f"{args.config} resized to T={cfg['T']} E={cfg['E']}", "tokens": cfg["T"], "hidden": cfg["H"], "intermediate": cfg["I"],
                    "experts": cfg["E"], "top_k": cfg["k"], "routing": cfg["routing"],
                    "rows_per_expert": {"min": int(rows.min()), "mean": float(rows.mean()), "max": int(rows.max()),
                                        "empty": int(np.sum(rows == 0))},
@@ -491,7 +500,7 @@ def main():
         "e2e": e2e,
         "cpu_baseline": cb,
     }
-    if args.config == "moe_decode_t512":
+    if line["vs_baseline"] is not None:
         line["vs_baseline_basis"] = ("0.8 TFLOPS: per-expert FP4 grouped GEMM at ~16 tokens/expert on RTX PRO "
                                      "6000 (SM120), quoted by the pages as context")
     print(json.dumps(line))

@@ -132,6 +132,32 @@ NVFP4_API nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k
                          void* ws, size_t ws_bytes, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* moe_permute_noalloc: moe_permute without a caller workspace. No passage   */
+/* of the pages corresponds to it; it exists for callers that cannot hand    */
+/* the library any device memory of their own -- code running where         */
+/* cudaMalloc is not allowed (inside a CUDA stream capture, on a real-time   */
+/* path that forbids allocation, or in a host framework that owns every     */
+/* device byte through a fixed pool it does not expose).                    */
+/* Same arguments, results and errors as moe_permute, minus ws / ws_bytes.  */
+/* Its per-(token chunk, expert) count table lives in a fixed array of      */
+/* NVFP4_PERMUTE_NOALLOC_SCRATCH_ENTRIES int32 (256 KiB) in the library's   */
+/* own device memory, which every GPU that loads the library holds until    */
+/* the process exits. Shapes with ceil(T/256) * E above that limit return   */
+/* NVFP4_ERR_UNSUPPORTED_SHAPE before anything is launched.                  */
+/* The first call on a device looks up the array's device address (with    */
+/* that device current); make that first call before any stream capture.   */
+/* All calls share the one array and leave their counts in it; every entry  */
+/* a call reads is written earlier in the same call, so nothing needs       */
+/* clearing, but calls whose kernels overlap on the GPU (different streams  */
+/* without ordering) race on the array and give wrong results.              */
+/* ------------------------------------------------------------------------ */
+#define NVFP4_PERMUTE_NOALLOC_SCRATCH_ENTRIES 65536
+NVFP4_API nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
+                                 const uint8_t* q, const uint8_t* sf, int64_t K,
+                                 uint8_t* q_perm, uint8_t* sf_perm, int32_t* expert_offsets,
+                                 int32_t* perm_src, int32_t* inv_perm, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* moe_grouped_gemm_nvfp4: one launch for every expert's FP4 block-scaled    */
 /* GEMM ("Peering into the CUTLASS Kernel Cache": TMA warp-specialised       */
 /* grouped GEMM; "Peering into the CUTLASS Kernel Scheduler": producer /     */

@@ -74,6 +74,8 @@ def lib():
         L.moe_permute_workspace_size.restype = sz
         L.moe_permute.argtypes = [P, i32, i32, i32, P, P, i64, P, P, P, P, P, P, sz, P]
         L.moe_permute.restype = st
+        L.moe_permute_noalloc.argtypes = [P, i32, i32, i32, P, P, i64, P, P, P, P, P, P]
+        L.moe_permute_noalloc.restype = st
         L.moe_grouped_gemm_nvfp4.argtypes = [P, P, P, P, P, P, P, i32, i64, i64, i64, ctypes.c_int, P, P]
         L.moe_grouped_gemm_nvfp4.restype = st
         L.moe_unpermute_combine.argtypes = [P, P, P, i32, i32, i64, P, P]
@@ -206,6 +208,31 @@ def permute(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_exper
     _check(lib().moe_permute(_ptr(topk_ids), T, k, num_experts, _ptr(q), _ptr(sf), K, _ptr(out.q_perm),
                              _ptr(out.sf_perm), _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm), _ptr(ws),
                              ws.numel(), _stream(stream)), "moe_permute")
+    return out
+
+
+def permute_noalloc(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_experts: int,
+                    stream=None) -> Permuted:
+    """moe_permute without a workspace: the library's own fixed device array holds the count table
+    (for callers that cannot allocate device memory; see moe_permute_noalloc in the header)."""
+    _require_cuda(topk_ids, q, sf)
+    if topk_ids.dtype != torch.int32:
+        raise TypeError("topk_ids must be int32")
+    topk_ids = topk_ids.contiguous()
+    T, k = topk_ids.shape
+    K = q.shape[1] * 2
+    R = T * k
+    dev = q.device
+    out = Permuted(
+        q_perm=torch.empty((R, K // 2), dtype=torch.uint8, device=dev),
+        sf_perm=torch.empty((R, K // 16), dtype=torch.uint8, device=dev),
+        offsets=torch.empty(num_experts + 1, dtype=torch.int32, device=dev),
+        perm_src=torch.empty(R, dtype=torch.int32, device=dev),
+        inv_perm=torch.empty(R, dtype=torch.int32, device=dev),
+    )
+    _check(lib().moe_permute_noalloc(_ptr(topk_ids), T, k, num_experts, _ptr(q), _ptr(sf), K, _ptr(out.q_perm),
+                                     _ptr(out.sf_perm), _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm),
+                                     _stream(stream)), "moe_permute_noalloc")
     return out
 
 

@@ -14,6 +14,8 @@
 //              inside a token never decides a rank.
 //   4. gather: one warp per output row copies K/2 code bytes and K/16 scale
 //              bytes with 16-byte vector loads and stores.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace nvfp4 {
@@ -181,6 +183,64 @@ extern "C" nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t 
     permute_rank_kernel<<<nchunks, kTok, rank_smem, s>>>(topk_ids, T, k, E, counts, perm_src, inv_perm, status);
     const int64_t gblocks = (R + 7) / 8;
     permute_gather_kernel<<<(unsigned)gblocks, 256, 0, s>>>(
+        reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(sf), K / 32, K / 256, perm_src, T, R,
+        reinterpret_cast<uint4*>(q_perm), reinterpret_cast<uint4*>(sf_perm));
+    count_launch(4);
+    return check_launch();
+}
+
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: the same four kernels, with the count table in a fixed
+// file-scope device array instead of a caller workspace (for callers that
+// cannot allocate device memory). Host code must not pass the array's name to
+// a kernel: on the host it is only a stand-in symbol, so its device address is
+// looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) int32_t g_permute_noalloc_scratch[NVFP4_PERMUTE_NOALLOC_SCRATCH_ENTRIES];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+int32_t* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array on the current device, or nullptr.
+int32_t* noalloc_scratch_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        int32_t* p = nullptr;
+        if (cudaGetSymbolAddress((void**)&p, g_permute_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = p;
+    }
+    return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
+                                            const uint8_t* q, const uint8_t* sf, int64_t K, uint8_t* q_perm,
+                                            uint8_t* sf_perm, int32_t* expert_offsets, int32_t* perm_src,
+                                            int32_t* inv_perm, nvfp4_stream_t stream) {
+    if (!topk_ids || !q || !sf || !q_perm || !sf_perm || !expert_offsets || !perm_src || !inv_perm)
+        return NVFP4_ERR_INVALID_ARG;
+    if (T <= 0 || k <= 0 || E <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (k > 32 || E > kMaxE || (int64_t)T * k >= (int64_t)1 << 31 || K % 256 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const int32_t nchunks = permute_chunks(T);
+    if ((int64_t)nchunks * E > NVFP4_PERMUTE_NOALLOC_SCRATCH_ENTRIES) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(topk_ids) || !aligned16(q) || !aligned16(sf) || !aligned16(q_perm) || !aligned16(sf_perm) ||
+        !aligned16(expert_offsets) || !aligned16(perm_src) || !aligned16(inv_perm))
+        return NVFP4_ERR_MISALIGNED;
+    int32_t* counts = noalloc_scratch_ptr();
+    uint32_t* status = status_word_ptr();
+    if (!counts || !status) return NVFP4_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t R = (int64_t)T * k;
+    permute_count_kernel<<<nchunks, kTok, 0, s>>>(topk_ids, T, k, E, counts, status);
+    permute_scan_kernel<<<1, kMaxE, 0, s>>>(counts, nchunks, E, expert_offsets);
+    const size_t rank_smem = (size_t)E * kWordsPerExpert * sizeof(uint32_t);
+    permute_rank_kernel<<<nchunks, kTok, rank_smem, s>>>(topk_ids, T, k, E, counts, perm_src, inv_perm, status);
+    permute_gather_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(
         reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(sf), K / 32, K / 256, perm_src, T, R,
         reinterpret_cast<uint4*>(q_perm), reinterpret_cast<uint4*>(sf_perm));
     count_launch(4);
