@@ -45,8 +45,8 @@ PAGES_DECODE_TFLOPS = 0.8   # per-expert FP4 grouped GEMM at ~16 tokens/expert, 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", default="moe_decode_t512", choices=[n for n in workloads.CONFIGS if n != "tiny"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
@@ -189,21 +189,23 @@ class MoEBench:
         c = self.cfg
         E, H, I = c["E"], c["H"], c["I"]
         d = self.dev
-        w13_q = torch.empty((E, 2 * I, H // 2), dtype=torch.uint8, device=d)
-        w13_sf = torch.empty((E, 2 * I, H // 16), dtype=torch.uint8, device=d)
-        w13_g = torch.empty(E, dtype=torch.float32, device=d)
-        w2_q = torch.empty((E, H, I // 2), dtype=torch.uint8, device=d)
-        w2_sf = torch.empty((E, H, I // 16), dtype=torch.uint8, device=d)
-        w2_g = torch.empty(E, dtype=torch.float32, device=d)
-        ws = torch.empty(max(nv.quantize_workspace_size(2 * I, H), nv.quantize_workspace_size(H, I)),
-                         dtype=torch.uint8, device=d)
-        for e in range(E):
-            w = workloads.normal_bf16((2 * I, H), 0.02, seed, workloads.TAG_W13, e, device=d)
-            nv.quantize(w, layout=nv.SF_MMA_TILED, q=w13_q[e], sf=w13_sf[e], g=w13_g[e:e + 1], ws=ws)
-            w = workloads.normal_bf16((H, I), 0.02, seed, workloads.TAG_W2, e, device=d)
-            nv.quantize(w, layout=nv.SF_MMA_TILED, q=w2_q[e], sf=w2_sf[e], g=w2_g[e:e + 1], ws=ws)
+
+        def build(N, K, tag):
+            packed = torch.empty((E, N * (K // 2 + K // 16)), dtype=torch.uint8, device=d)
+            g = torch.empty(E, dtype=torch.float32, device=d)
+            q = torch.empty((N, K // 2), dtype=torch.uint8, device=d)
+            sf = torch.empty((N, K // 16), dtype=torch.uint8, device=d)
+            ws = torch.empty(max(nv.quantize_workspace_size(N, K), 16), dtype=torch.uint8, device=d)
+            for e in range(E):
+                w = workloads.normal_bf16((N, K), 0.02, seed, tag, e, device=d)
+                nv.quantize(w, q=q, sf=sf, g=g[e:e + 1], ws=ws)
+                nv.pack_weights(q, sf, out=packed[e])
+            return nv.PackedWeights(packed, g, E, N, K)
+
+        w13 = build(2 * I, H, workloads.TAG_W13)
+        w2 = build(H, I, workloads.TAG_W2)
         torch.cuda.synchronize()
-        return nv.MoEWeights(w13_q, w13_sf, w13_g, w2_q, w2_sf, w2_g)
+        return nv.MoEWeights(w13, w2)
 
     def step(self, ev=None):
         """One layer through the C ABI, stage by stage (the same sequence moe_layer_nvfp4 runs), with
@@ -234,14 +236,14 @@ class MoEBench:
                             P(b + lay["perm_src"]), P(b + lay["inv_perm"]), scratch, sbytes, s)
         rec(2)
         st |= L.moe_grouped_gemm_nvfp4(P(b + lay["q_perm"]), P(b + lay["sf_perm"]), P(b + lay["g_x"]),
-                                       P(W.w13_q.data_ptr()), P(W.w13_sf.data_ptr()), P(W.w13_g.data_ptr()),
+                                       P(W.w13.packed.data_ptr()), P(W.w13.gscale.data_ptr()),
                                        P(b + lay["offsets"]), E, R, 2 * I, H, 1, P(b + lay["h"]), s)
         rec(3)
         st |= L.nvfp4_quantize(P(b + lay["h"]), R, I, None, P(b + lay["q_h"]), P(b + lay["sf_h"]),
                                P(b + lay["g_h"]), 0, scratch, sbytes, s)
         rec(4)
         st |= L.moe_grouped_gemm_nvfp4(P(b + lay["q_h"]), P(b + lay["sf_h"]), P(b + lay["g_h"]),
-                                       P(W.w2_q.data_ptr()), P(W.w2_sf.data_ptr()), P(W.w2_g.data_ptr()),
+                                       P(W.w2.packed.data_ptr()), P(W.w2.gscale.data_ptr()),
                                        P(b + lay["offsets"]), E, R, H, I, 0, P(b + lay["y"]), s)
         rec(5)
         st |= L.moe_unpermute_combine(P(b + lay["y"]), P(b + lay["inv_perm"]), P(self.w.data_ptr()), T, k, H,
@@ -396,6 +398,122 @@ def cpu_baseline(cfg, seed):
             "sample": desc, "seconds": dt}
 
 
+# ----------------------------------------------------------------------------- dense 8192^3
+
+def oracle_dense_sample(M, N, K, seed, budget_s):
+    """Oracle GEMM on a bounded sample of rows of the dense problem (quantise A's sampled rows + GEMM)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    w_q = rng.integers(0, 256, size=(1, N, K // 2), dtype=np.uint8)
+    w_sf = rng.integers(0x20, 0x40, size=(1, N, K // 16), dtype=np.uint8)
+    t0 = time.perf_counter()
+    rows = 0
+    flops = 0.0
+    while time.perf_counter() - t0 < budget_s:
+        a = workloads.random_bf16_bits((8, K), seed=seed + rows, tag=workloads.TAG_A)
+        aq, asf, ag = oracle.quantize(a)
+        oracle.grouped_gemm(aq, asf, ag, w_q, w_sf, np.ones(1, np.float32), np.array([0, 8], np.int32), N, K, False)
+        rows += 8
+        flops += 2.0 * 8 * N * K
+    dt = time.perf_counter() - t0
+    return flops, dt, f"oracle dense GEMM on {rows} of {M} rows (FP64, {oracle.num_threads()} threads)"
+
+
+def main_dense(args, cfg, metric, world, rank, local_rank):
+    M, N, K = cfg["M"], cfg["N"], cfg["K"]
+    if args.impl == "reference":
+        raise AssertionError("unreachable")
+    import torch
+    import torch.distributed as dist
+    import nvfp4_block_scaled_09_b200 as nv
+    from nvfp4_block_scaled_09_b200 import build as nvbuild
+    nvbuild.build()
+    if world > 1:
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    a = workloads.normal_bf16((M, K), 1.0, args.seed + 7919 * rank, workloads.TAG_A, device=dev)
+    b = workloads.normal_bf16((1, N, K), 0.02, args.seed, workloads.TAG_B, device=dev)
+    pw = nv.prepare_expert_weights(b)
+    del b
+    a_q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    a_sf = torch.empty((M, K // 16), dtype=torch.uint8, device=dev)
+    a_g = torch.empty(1, dtype=torch.float32, device=dev)
+    qws = torch.empty(nv.quantize_workspace_size(M, K), dtype=torch.uint8, device=dev)
+    c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    off = torch.tensor([0, M], dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # larger than the 126 MB L2
+
+    def step(e0=None, e1=None, e2=None):
+        if e0 is not None:
+            e0.record()
+        nv.quantize(a, q=a_q, sf=a_sf, g=a_g, ws=qws)
+        if e1 is not None:
+            e1.record()
+        nv.grouped_gemm(a_q, a_sf, a_g, pw, off, False, out=c)
+        if e2 is not None:
+            e2.record()
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    assert nv.device_status() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.4)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    l0 = nv.launch_count()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)                      # evict A, B and C from L2 between steps (not timed)
+        step(*evs[i])
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches = nv.launch_count() - l0
+    clk = clocks.stop() if clocks else None
+    step_ms = sum(e[0].elapsed_time(e[2]) for e in evs)
+    gemm_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    K_steps = args.steps
+    flops = 2.0 * M * N * K
+    value = world * flops * K_steps / (float(t.item()) * 1e-3) / 1e12
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    achieved = flops / (gemm_ms * 1e-3) / 1e12
+    cb = None
+    if world == 1 and not args.no_cpu_baseline:
+        f, dt, desc = oracle_dense_sample(M, N, K, args.seed, 10.0)
+        import oracle
+        cb = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+              "sample": desc}
+    line = {
+        "metric": metric, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K_steps,
+        "warmup": args.warmup, "ms_per_step": float(t.item()) / K_steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": "dense", "M": M, "N": N, "K": K,
+                   "l2": "flushed between steps (256 MB write, outside the timed events)",
+                   "step": "quantize(A) + GEMM with B quantised once beforehand"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": achieved / fp4_peak, "traffic": None, "kernel": "grouped_gemm_kernel (E=1)",
+                     "peak_source": peaks["source"] + " bf16 x 4 (nominal FP4/BF16 ratio)",
+                     "avg_launch_ms": gemm_ms},
+        "clocks": clk, "gpu_launches": int(launches), "e2e": None, "cpu_baseline": cb,
+    }
+    print(json.dumps(line))
+    return 0
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -410,6 +528,28 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     metric = "NVFP4 MoE grouped-GEMM TFLOPS and HBM GB/s at 16-256 tokens/expert"
 
+    if args.impl == "reference" and cfg["kind"] == "dense":
+        if rank != 0:
+            return 0
+        import oracle
+        tot_f = tot_t = 0.0
+        desc = ""
+        budget = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+        for i in range(args.warmup + args.steps):
+            f, dt, desc = oracle_dense_sample(cfg["M"], cfg["N"], cfg["K"], args.seed, budget)
+            if i >= args.warmup:
+                tot_f += f
+                tot_t += dt
+        v = tot_f / tot_t / 1e12
+        print(json.dumps({"impl": "reference", "metric": metric, "value": v, "unit": "TFLOP/s",
+                          "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+                          "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": {"workload": "dense", "M": cfg["M"], "N": cfg["N"], "K": cfg["K"]},
+                          "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                                           "kind": "oracle", "sample": desc},
+                          "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return 0
     if args.impl == "reference":
         if rank != 0:
             return 0
@@ -435,9 +575,8 @@ def main():
         print(json.dumps(line))
         return 0
 
-    if cfg["kind"] != "moe":
-        raise SystemExit("bench.py times the MoE layer workloads (moe_decode_t512, moe_zipf_t1024, "
-                         "moe_prefill_t8192); the dense GEMM is covered by the tests")
+    if cfg["kind"] == "dense":
+        return main_dense(args, cfg, metric, world, rank, local_rank)
     import torch
     import torch.distributed as dist
     if world > 1:

@@ -74,7 +74,7 @@ typedef enum { NVFP4_EPI_NONE = 0, NVFP4_EPI_SWIGLU = 1 } nvfp4_epilogue;
  *   (row block rb, step kc) pair is a 512-byte atom at ((rb * (K/64)) + kc) * 512,
  *   and inside it the scale of row r, block b sits at
  *   (r % 32) * 16 + ((r % 128) / 32) * 4 + (b % 4).
- *   Requires rows % 128 == 0 and K % 64 == 0. Weights are stored this way. */
+ *   Requires rows % 128 == 0 and K % 64 == 0. */
 typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1 } nvfp4_sf_layout;
 
 /* ------------------------------------------------------------------------ */
@@ -171,8 +171,9 @@ NVFP4_API nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, i
 /*           projection),                                     out [rows, N/2]*/
 /* Arguments:                                                                */
 /*   a_q [max_rows, K/2], a_sf [max_rows, K/16] row-major, a_gscale scalar   */
-/*   w_q [E, N, K/2], w_sf [E, N, K/16] in NVFP4_SF_MMA_TILED layout (per    */
-/*   expert slice, i.e. the [E*N, K] matrix tiled), w_gscale [E]             */
+/*   w_packed: the weights [E, N, K] packed by nvfp4_pack_weights() as one   */
+/*     [E*N, K] matrix (nvfp4_packed_weight_bytes(E*N, K) bytes);           */
+/*     w_gscale [E]                                                          */
 /*   expert_offsets [E+1] (device; non-decreasing, off[0] >= 0,              */
 /*   off[E] <= max_rows, else NVFP4_ERR_DEVICE_INPUT is latched and the      */
 /*   offending experts are skipped)                                          */
@@ -181,10 +182,27 @@ NVFP4_API nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, i
 /*   are not written.                                                        */
 /* ------------------------------------------------------------------------ */
 NVFP4_API nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
-                                    const uint8_t* w_q, const uint8_t* w_sf, const float* w_gscale,
+                                    const uint8_t* w_packed, const float* w_gscale,
                                     const int32_t* expert_offsets, int32_t E, int64_t max_rows,
                                     int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
                                     nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* nvfp4_pack_weights: one-time packing of a quantised weight matrix         */
+/* [rows, K] (codes q [rows, K/2], row-major scales sf [rows, K/16]) into   */
+/* the tiles the grouped GEMM streams. Tile (rb, kt) = rows [128 rb, +128) x */
+/* K [256 kt, +256) is 18432 contiguous bytes at (rb*(K/256) + kt) * 18432:  */
+/*   [0, 16384): code bytes, row r at r*128, its 16-byte piece c (K bytes    */
+/*   16c..16c+15 of the tile row) at (c XOR (r % 8)) * 16 (the 128-byte      */
+/*   swizzle the tensor core reads);                                         */
+/*   [16384, 18432): scales, K step kc (64 elements) at kc*512, row r's 4    */
+/*   scale bytes of that step at (r % 32)*16 + (r / 32)*4.                   */
+/* rows % 128 == 0, K % 256 == 0; all pointers device, 16-byte aligned;      */
+/* packed holds nvfp4_packed_weight_bytes(rows, K) bytes (= rows*(K/2+K/16)).*/
+/* ------------------------------------------------------------------------ */
+NVFP4_API size_t nvfp4_packed_weight_bytes(int64_t rows, int64_t K);
+NVFP4_API nvfp4_status nvfp4_pack_weights(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t K,
+                                uint8_t* packed, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* moe_unpermute_combine: top-k weighted sum of the expert outputs back in   */
@@ -208,8 +226,9 @@ NVFP4_API nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* i
 /* grouped GEMM gate/up (SWIGLU, N = 2I, K = H) -> quantize(h) -> grouped   */
 /* GEMM down (NONE, N = H, K = I) -> moe_unpermute_combine.                  */
 /* Arguments: x [T, H] BF16, topk_ids [T, k], topk_w [T, k];                 */
-/*   w13_q [E, 2I, H/2], w13_sf (MMA_TILED), w13_gscale [E];                 */
-/*   w2_q [E, H, I/2], w2_sf (MMA_TILED), w2_gscale [E]; out [T, H] BF16.    */
+/*   w13_packed (W13 [E, 2I, H] packed as an [E*2I, H] matrix), w13_gscale   */
+/*   [E]; w2_packed (W2 [E, H, I] packed as [E*H, I]), w2_gscale [E];        */
+/*   out [T, H] BF16.                                                        */
 /*   H % 256 == 0, I % 128 == 0 (2I % 256 == 0 and I % 256 == 0 for the down */
 /*   GEMM's K), plus the limits of the calls above. ws of                    */
 /*   moe_layer_workspace_size() bytes holds every intermediate; its layout   */
@@ -231,8 +250,8 @@ NVFP4_API nvfp4_status moe_layer_workspace_layout(int32_t T, int32_t k, int32_t 
 NVFP4_API size_t moe_layer_workspace_size(int32_t T, int32_t k, int32_t E, int64_t H, int64_t I);
 NVFP4_API nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_ids, const float* topk_w,
                              int32_t T, int32_t k, int32_t E, int64_t H, int64_t I,
-                             const uint8_t* w13_q, const uint8_t* w13_sf, const float* w13_gscale,
-                             const uint8_t* w2_q, const uint8_t* w2_sf, const float* w2_gscale,
+                             const uint8_t* w13_packed, const float* w13_gscale,
+                             const uint8_t* w2_packed, const float* w2_gscale,
                              uint16_t* out, void* ws, size_t ws_bytes, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */

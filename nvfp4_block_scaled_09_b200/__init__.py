@@ -11,6 +11,7 @@ Calls (same names as the C ABI):
   quantize            -> nvfp4_quantize
   permute             -> moe_permute
   grouped_gemm        -> moe_grouped_gemm_nvfp4
+  pack_weights        -> nvfp4_pack_weights
   unpermute_combine   -> moe_unpermute_combine
   moe_layer           -> moe_layer_nvfp4
 """
@@ -76,7 +77,7 @@ def lib():
         L.moe_permute.restype = st
         L.moe_permute_noalloc.argtypes = [P, i32, i32, i32, P, P, i64, P, P, P, P, P, P]
         L.moe_permute_noalloc.restype = st
-        L.moe_grouped_gemm_nvfp4.argtypes = [P, P, P, P, P, P, P, i32, i64, i64, i64, ctypes.c_int, P, P]
+        L.moe_grouped_gemm_nvfp4.argtypes = [P, P, P, P, P, P, i32, i64, i64, i64, ctypes.c_int, P, P]
         L.moe_grouped_gemm_nvfp4.restype = st
         L.moe_unpermute_combine.argtypes = [P, P, P, i32, i32, i64, P, P]
         L.moe_unpermute_combine.restype = st
@@ -84,7 +85,11 @@ def lib():
         L.moe_layer_workspace_layout.restype = st
         L.moe_layer_workspace_size.argtypes = [i32, i32, i32, i64, i64]
         L.moe_layer_workspace_size.restype = sz
-        L.moe_layer_nvfp4.argtypes = [P, P, P, i32, i32, i32, i64, i64, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_layer_nvfp4.argtypes = [P, P, P, i32, i32, i32, i64, i64, P, P, P, P, P, P, sz, P]
+        L.nvfp4_packed_weight_bytes.argtypes = [i64, i64]
+        L.nvfp4_packed_weight_bytes.restype = sz
+        L.nvfp4_pack_weights.argtypes = [P, P, i64, i64, P, P]
+        L.nvfp4_pack_weights.restype = st
         L.moe_layer_nvfp4.restype = st
         L.nvfp4_gemm_get_plan.argtypes = [ctypes.POINTER(GemmPlan)]
         L.nvfp4_gemm_get_plan.restype = st
@@ -157,18 +162,52 @@ def quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None, layout: 
     return q, sf, g
 
 
-def prepare_expert_weights(w: torch.Tensor, stream=None):
-    """Weights [E, N, K] bf16 -> (q [E, N, K/2], sf [E, N, K/16] MMA-tiled, g [E]) with one global
-    scale per expert matrix. One-time preparation, one quantize call per expert."""
+def packed_weight_bytes(rows: int, K: int) -> int:
+    return int(lib().nvfp4_packed_weight_bytes(rows, K))
+
+
+def pack_weights(q: torch.Tensor, sf: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Quantised weights (codes [rows, K/2], row-major scales [rows, K/16]) -> the GEMM's packed tiles."""
+    _require_cuda(q, sf)
+    rows, half = q.shape[-2], q.shape[-1]
+    rows = q.numel() // half
+    K = half * 2
+    if out is None:
+        out = torch.empty(packed_weight_bytes(rows, K), dtype=torch.uint8, device=q.device)
+    _check(lib().nvfp4_pack_weights(_ptr(q), _ptr(sf), rows, K, _ptr(out), _stream(stream)), "nvfp4_pack_weights")
+    return out
+
+
+@dataclass
+class PackedWeights:
+    packed: torch.Tensor          # [E, N*(K/2 + K/16)] bytes, packed tiles
+    gscale: torch.Tensor          # [E] FP32 global scales (dequantisation multipliers)
+    E: int
+    N: int
+    K: int
+    q: torch.Tensor | None = None   # row-major codes [E, N, K/2] (kept only on request)
+    sf: torch.Tensor | None = None  # row-major scales [E, N, K/16] (kept only on request)
+
+
+def prepare_expert_weights(w: torch.Tensor, keep_rowmajor: bool = False, stream=None) -> PackedWeights:
+    """Weights [E, N, K] bf16 -> packed NVFP4 tiles with one global scale per expert matrix.
+    One-time preparation: quantise each expert (row-major), then pack."""
     _require_cuda(w)
     E, N, K = w.shape
-    q = torch.empty((E, N, K // 2), dtype=torch.uint8, device=w.device)
-    sf = torch.empty((E, N, K // 16), dtype=torch.uint8, device=w.device)
-    g = torch.empty(E, dtype=torch.float32, device=w.device)
-    ws = torch.empty(max(quantize_workspace_size(N, K), 16), dtype=torch.uint8, device=w.device)
+    dev = w.device
+    packed = torch.empty((E, N * (K // 2 + K // 16)), dtype=torch.uint8, device=dev)
+    g = torch.empty(E, dtype=torch.float32, device=dev)
+    qk = torch.empty((E, N, K // 2), dtype=torch.uint8, device=dev) if keep_rowmajor else None
+    sk = torch.empty((E, N, K // 16), dtype=torch.uint8, device=dev) if keep_rowmajor else None
+    qt = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    st = torch.empty((N, K // 16), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(quantize_workspace_size(N, K), 16), dtype=torch.uint8, device=dev)
     for e in range(E):
-        quantize(w[e], layout=SF_MMA_TILED, q=q[e], sf=sf[e], g=g[e:e + 1], ws=ws, stream=stream)
-    return q, sf, g
+        q_e = qk[e] if keep_rowmajor else qt
+        s_e = sk[e] if keep_rowmajor else st
+        quantize(w[e], q=q_e, sf=s_e, g=g[e:e + 1], ws=ws, stream=stream)
+        pack_weights(q_e, s_e, out=packed[e], stream=stream)
+    return PackedWeights(packed, g, E, N, K, qk, sk)
 
 
 # ----------------------------------------------------------------------------- permute
@@ -238,15 +277,16 @@ def permute_noalloc(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, n
 
 # ----------------------------------------------------------------------------- grouped GEMM
 
-def grouped_gemm(a_q, a_sf, a_g, w_q, w_sf, w_g, offsets, N: int, K: int, swiglu: bool, out=None, stream=None):
+def grouped_gemm(a_q, a_sf, a_g, w: PackedWeights, offsets, swiglu: bool, out=None, stream=None):
     """Per-expert NVFP4 GEMM. Returns bf16 [rows, N] (or [rows, N/2] with SwiGLU)."""
-    _require_cuda(a_q, a_sf, a_g, w_q, w_sf, w_g, offsets)
+    _require_cuda(a_q, a_sf, a_g, w.packed, w.gscale, offsets)
     rows = a_q.shape[0]
     E = offsets.numel() - 1
+    N, K = w.N, w.K
     nout = N // 2 if swiglu else N
     if out is None:
         out = torch.empty((rows, nout), dtype=torch.bfloat16, device=a_q.device)
-    _check(lib().moe_grouped_gemm_nvfp4(_ptr(a_q), _ptr(a_sf), _ptr(a_g), _ptr(w_q), _ptr(w_sf), _ptr(w_g),
+    _check(lib().moe_grouped_gemm_nvfp4(_ptr(a_q), _ptr(a_sf), _ptr(a_g), _ptr(w.packed), _ptr(w.gscale),
                                         _ptr(offsets), E, rows, N, K, EPI_SWIGLU if swiglu else EPI_NONE, _ptr(out),
                                         _stream(stream)), "moe_grouped_gemm_nvfp4")
     return out
@@ -286,24 +326,20 @@ def unpermute_combine(y: torch.Tensor, inv_perm: torch.Tensor, topk_w: torch.Ten
 
 @dataclass
 class MoEWeights:
-    w13_q: torch.Tensor     # [E, 2I, H/2]
-    w13_sf: torch.Tensor    # [E, 2I, H/16] MMA-tiled
-    w13_g: torch.Tensor     # [E]
-    w2_q: torch.Tensor      # [E, H, I/2]
-    w2_sf: torch.Tensor     # [E, H, I/16] MMA-tiled
-    w2_g: torch.Tensor      # [E]
+    w13: PackedWeights   # gate/up [E, 2I, H]
+    w2: PackedWeights    # down [E, H, I]
 
     @property
     def num_experts(self) -> int:
-        return self.w13_q.shape[0]
+        return self.w13.E
 
     @property
     def hidden(self) -> int:
-        return self.w13_q.shape[2] * 2
+        return self.w13.K
 
     @property
     def intermediate(self) -> int:
-        return self.w13_q.shape[1] // 2
+        return self.w13.N // 2
 
 
 def layer_workspace_layout(T: int, k: int, E: int, H: int, I: int) -> dict:
@@ -330,8 +366,8 @@ def moe_layer(x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor, w: 
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
     _check(lib().moe_layer_nvfp4(_ptr(x), _ptr(topk_ids.contiguous()), _ptr(topk_w.contiguous()), T, k, E, H, I,
-                                 _ptr(w.w13_q), _ptr(w.w13_sf), _ptr(w.w13_g), _ptr(w.w2_q), _ptr(w.w2_sf),
-                                 _ptr(w.w2_g), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "moe_layer_nvfp4")
+                                 _ptr(w.w13.packed), _ptr(w.w13.gscale), _ptr(w.w2.packed), _ptr(w.w2.gscale),
+                                 _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "moe_layer_nvfp4")
     return out
 
 

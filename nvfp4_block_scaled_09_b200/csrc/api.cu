@@ -135,11 +135,10 @@ extern "C" size_t moe_layer_workspace_size(int32_t T, int32_t k, int32_t E, int6
 }
 
 extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_ids, const float* topk_w, int32_t T,
-                                        int32_t k, int32_t E, int64_t H, int64_t I, const uint8_t* w13_q,
-                                        const uint8_t* w13_sf, const float* w13_gscale, const uint8_t* w2_q,
-                                        const uint8_t* w2_sf, const float* w2_gscale, uint16_t* out, void* ws,
-                                        size_t ws_bytes, nvfp4_stream_t stream) {
-    if (!x || !topk_ids || !topk_w || !w13_q || !w13_sf || !w13_gscale || !w2_q || !w2_sf || !w2_gscale || !out)
+                                        int32_t k, int32_t E, int64_t H, int64_t I, const uint8_t* w13_packed,
+                                        const float* w13_gscale, const uint8_t* w2_packed, const float* w2_gscale,
+                                        uint16_t* out, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!x || !topk_ids || !topk_w || !w13_packed || !w13_gscale || !w2_packed || !w2_gscale || !out)
         return NVFP4_ERR_INVALID_ARG;
     nvfp4_layer_workspace L;
     nvfp4_status st = moe_layer_workspace_layout(T, k, E, H, I, &L);
@@ -171,12 +170,12 @@ extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_i
     if ((st = moe_permute(topk_ids, T, k, E, q_x, sf_x, H, q_perm, sf_perm, off, perm_src, inv_perm, scratch,
                           scratch_bytes, stream)))
         return st;
-    if ((st = moe_grouped_gemm_nvfp4(q_perm, sf_perm, g_x, w13_q, w13_sf, w13_gscale, off, E, R, 2 * I, H,
+    if ((st = moe_grouped_gemm_nvfp4(q_perm, sf_perm, g_x, w13_packed, w13_gscale, off, E, R, 2 * I, H,
                                      NVFP4_EPI_SWIGLU, h, stream)))
         return st;
     if ((st = nvfp4_quantize(h, R, I, nullptr, q_h, sf_h, g_h, NVFP4_SF_ROWMAJOR, scratch, scratch_bytes, stream)))
         return st;
-    if ((st = moe_grouped_gemm_nvfp4(q_h, sf_h, g_h, w2_q, w2_sf, w2_gscale, off, E, R, H, I, NVFP4_EPI_NONE, y,
+    if ((st = moe_grouped_gemm_nvfp4(q_h, sf_h, g_h, w2_packed, w2_gscale, off, E, R, H, I, NVFP4_EPI_NONE, y,
                                      stream)))
         return st;
     return moe_unpermute_combine(y, inv_perm, topk_w, T, k, H, out, stream);

@@ -17,10 +17,15 @@
 //    SWIGLU pairs gate rows [n0, n0+128) with up rows [N/2+n0, ...) so both
 //    accumulators of one output column sit in the same TMEM lane; NONE covers
 //    256 consecutive output columns.
+//  * Weights arrive pre-packed (pack.cu): every 128-row x 256-K tile with its
+//    scales is one contiguous 18 KB chunk already in the shared-memory image the
+//    tensor core reads, so a weight stage is two contiguous bulk copies (the
+//    weight stream is what decode is bound by, and contiguous pieces stream
+//    ~15% faster from HBM than strided 2-D tiles).
 //  * Warp roles ("Peering into the CUTLASS Kernel Scheduler", The Discovery:
 //    explicit warp-specialised schedules that give A loads, B loads, MMA and
-//    epilogue their own warps): warp 0 issues TMA tiles of weights and
-//    activations plus bulk copies of the weights' pre-tiled scales; warp 1
+//    epilogue their own warps): warp 0 issues the weight bulk copies and the
+//    TMA tiles of activations; warp 1
 //    gathers the activation scales (row-major) into the tensor-core scale
 //    layout with cp.async; warp 2 owns tensor memory and issues tcgen05.cp +
 //    tcgen05.mma; warps 4-7 drain the FP32 accumulators from TMEM, apply the
@@ -56,12 +61,14 @@ constexpr int kABlockBytes = kBM * kRowBytes;    // 16 KB
 constexpr int kBBytes = kBNMax * kRowBytes;      // 8 KB
 constexpr int kSFAtomBytes = 512;                // 128 rows x 4 scales
 constexpr int kSFStageBytes = kKSteps * kSFAtomBytes;
+constexpr int kPackedTileBytes = kABlockBytes + kSFStageBytes;  // one packed weight tile (codes + scales)
+// Stage layout: [A0 codes | A0 scales][A1 codes | A1 scales][B codes][B scales]
 constexpr int kOffA0 = 0;
-constexpr int kOffA1 = kABlockBytes;
-constexpr int kOffB = 2 * kABlockBytes;
-constexpr int kOffSFA0 = kOffB + kBBytes;
-constexpr int kOffSFA1 = kOffSFA0 + kSFStageBytes;
-constexpr int kOffSFB = kOffSFA1 + kSFStageBytes;
+constexpr int kOffSFA0 = kABlockBytes;
+constexpr int kOffA1 = kPackedTileBytes;
+constexpr int kOffSFA1 = kOffA1 + kABlockBytes;
+constexpr int kOffB = 2 * kPackedTileBytes;
+constexpr int kOffSFB = kOffB + kBBytes;
 constexpr int kStageBytes = kOffSFB + kSFStageBytes;   // 47104 (46 x 1024)
 constexpr int kMaxE = 1024;
 constexpr int kThreads = 256;
@@ -89,12 +96,13 @@ struct Shared {
 constexpr size_t kSmemBytes = 1024 /* alignment slack */ + (size_t)kStages * kStageBytes + sizeof(Shared);
 
 static_assert(kStageBytes % 1024 == 0, "stage buffers must keep 1024-byte swizzle alignment");
+static_assert(kOffA1 % 1024 == 0 && kOffB % 1024 == 0, "swizzled operand tiles must start on 1024 bytes");
 static_assert(kSFDelay < kStages, "scale gatherer may not hold more stages than the ring has");
 
 struct Params {
     const uint8_t* a_sf;
     const float* a_gscale;
-    const uint8_t* w_sf;
+    const uint8_t* w_packed;
     const float* w_gscale;
     const int32_t* offsets;
     uint16_t* out;
@@ -134,8 +142,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
-                        const Params p) {
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
@@ -228,7 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int s = 0; s < kStages; s++) issued[s] = false, issued_parity[s] = 0;
         if (lane == 0) {
-            const uint64_t pol_w = l2_policy_evict_first();
+            // Weights read by one row tile only are streamed past L2; experts with
+            // several row tiles re-read theirs from L2 (their tiles run back to back).
+            const uint64_t pol_w_once = l2_policy_evict_first();
+            const uint64_t pol_w_reuse = l2_policy_evict_normal();
             const uint64_t pol_a = l2_policy_evict_last();
             uint32_t stage = 0, phase = 0;
             bool ok = true;
@@ -244,21 +254,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     r1 = r0 + kBM;
                 }
                 const int64_t wr0 = (int64_t)t.e * p.N + r0, wr1 = (int64_t)t.e * p.N + r1;
-                const uint8_t* sfa0 = p.w_sf + (wr0 / kBM) * (p.K / 64) * kSFAtomBytes;
-                const uint8_t* sfa1 = p.w_sf + (wr1 / kBM) * (p.K / 64) * kSFAtomBytes;
-                const uint32_t tx = (uint32_t)(kNumA * (kABlockBytes + kSFStageBytes) + t.bn * kRowBytes);
+                const uint8_t* wp0 = p.w_packed + (wr0 / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
+                const uint8_t* wp1 = p.w_packed + (wr1 / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
+                const bool reuse = (sh.off[t.e + 1] - sh.off[t.e]) > kBNMax;
+                const uint64_t pol_w = reuse ? pol_w_reuse : pol_w_once;
+                const uint32_t tx = (uint32_t)(kNumA * kPackedTileBytes + t.bn * kRowBytes);
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
                     if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
                     uint8_t* sb = stages + (size_t)stage * kStageBytes;
                     uint64_t* bar = &sh.full_tma[stage];
                     mbar_arrive_expect_tx(bar, tx);
                     const int32_t kx = kt * kRowBytes;
-                    tma_load_2d(sb + kOffA0, &tm_w, kx, (int32_t)wr0, bar, pol_w);
-                    tma_load_2d(sb + kOffA1, &tm_w, kx, (int32_t)wr1, bar, pol_w);
+                    bulk_load(sb + kOffA0, wp0 + (size_t)kt * kPackedTileBytes, kPackedTileBytes, bar, pol_w);
+                    bulk_load(sb + kOffA1, wp1 + (size_t)kt * kPackedTileBytes, kPackedTileBytes, bar, pol_w);
                     for (int32_t i = 0; i < t.bn / kBNStep; i++)
                         tma_load_2d(sb + kOffB + i * kBNStep * kRowBytes, &tm_a, kx, t.row0 + i * kBNStep, bar, pol_a);
-                    bulk_load(sb + kOffSFA0, sfa0 + (size_t)kt * kSFStageBytes, kSFStageBytes, bar, pol_w);
-                    bulk_load(sb + kOffSFA1, sfa1 + (size_t)kt * kSFStageBytes, kSFStageBytes, bar, pol_w);
                     issued[stage] = true;
                     issued_parity[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -349,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t acc = (kt | kc) != 0;
 #pragma unroll
                         for (int a = 0; a < kNumA; a++) {
-                            const uint64_t adesc = make_smem_desc(sb + a * kABlockBytes + kc * 32, 16, 1024, 2);
+                            const uint64_t adesc = make_smem_desc(sb + a * kPackedTileBytes + kc * 32, 16, 1024, 2);
                             mma_mxf4nvf4(tmem + abuf * (kNumA * kAccCols) + a * kAccCols, adesc, bdesc, idesc,
                                          tmem + kTmemSFA + a * 4 * kKSteps + 4 * kc, tmem + kTmemSFB + 4 * kc, acc);
                         }
@@ -481,7 +491,7 @@ extern "C" nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan) {
     plan->tile_tokens_max = gg::kBNMax;
     plan->stage_k = gg::kBK;
     plan->stages = gg::kStages;
-    plan->stage_bytes_weights = gg::kNumA * gg::kABlockBytes;
+    plan->stage_bytes_weights = gg::kNumA * gg::kABlockBytes;   // arrives with its scales in one packed tile
     plan->stage_bytes_weight_sf = gg::kNumA * gg::kSFStageBytes;
     plan->stage_bytes_act_max = gg::kBBytes;
     plan->stage_bytes_act_sf = gg::kSFStageBytes;
@@ -494,8 +504,9 @@ extern "C" nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan) {
 extern "C" int64_t nvfp4_gemm_stage_tx_bytes(int32_t tokens) {
     if (tokens <= 0 || tokens > gg::kBNMax) return -1;
     const int64_t bn = (tokens + gg::kBNStep - 1) / gg::kBNStep * gg::kBNStep;
-    // MK part: weight tiles + their scales; NK part: activation tile (scales come via cp.async).
-    return (int64_t)gg::kNumA * (gg::kABlockBytes + gg::kSFStageBytes) + bn * gg::kRowBytes;
+    // MK part: weight tiles + their scales (packed together); NK part: activation tile (its scales come
+    // through cp.async on their own barrier).
+    return (int64_t)gg::kNumA * gg::kPackedTileBytes + bn * gg::kRowBytes;
 }
 
 extern "C" nvfp4_status nvfp4_can_implement_with_budget(int64_t N, int64_t K, int32_t E, nvfp4_epilogue epi,
@@ -515,14 +526,14 @@ extern "C" nvfp4_status nvfp4_can_implement(int64_t N, int64_t K, int32_t E, nvf
 }
 
 extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
-                                               const uint8_t* w_q, const uint8_t* w_sf, const float* w_gscale,
+                                               const uint8_t* w_packed, const float* w_gscale,
                                                const int32_t* expert_offsets, int32_t E, int64_t max_rows,
                                                int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
                                                nvfp4_stream_t stream) {
-    if (!a_q || !a_sf || !a_gscale || !w_q || !w_sf || !w_gscale || !expert_offsets || !out)
+    if (!a_q || !a_sf || !a_gscale || !w_packed || !w_gscale || !expert_offsets || !out)
         return NVFP4_ERR_INVALID_ARG;
     if (max_rows < 0 || max_rows > INT32_MAX) return NVFP4_ERR_INVALID_ARG;
-    if (!aligned16(a_q) || !aligned16(a_sf) || !aligned16(w_q) || !aligned16(w_sf) || !aligned16(out) ||
+    if (!aligned16(a_q) || !aligned16(a_sf) || !aligned16(w_packed) || !aligned16(out) ||
         ((uintptr_t)a_gscale & 3u) || ((uintptr_t)w_gscale & 3u) || ((uintptr_t)expert_offsets & 3u))
         return NVFP4_ERR_MISALIGNED;
     const int optin = device_smem_optin();
@@ -533,8 +544,7 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
     uint32_t* status = status_word_ptr();
     if (!status) return NVFP4_ERR_CUDA;
 
-    CUtensorMap tm_w, tm_a;
-    if (!encode_rows_map(&tm_w, w_q, (int64_t)E * N, K / 2, gg::kBM)) return NVFP4_ERR_CUDA;
+    CUtensorMap tm_a;
     if (!encode_rows_map(&tm_a, a_q, max_rows, K / 2, gg::kBNStep)) return NVFP4_ERR_CUDA;
 
     static int configured_device = -1;
@@ -549,7 +559,7 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
     gg::Params prm;
     prm.a_sf = a_sf;
     prm.a_gscale = a_gscale;
-    prm.w_sf = w_sf;
+    prm.w_packed = w_packed;
     prm.w_gscale = w_gscale;
     prm.offsets = expert_offsets;
     prm.out = out;
@@ -561,8 +571,8 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     const int grid = device_sm_count();
-    gg::grouped_gemm_kernel<<<grid, gg::kThreads, gg::kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(
-        tm_w, tm_a, prm);
+    gg::grouped_gemm_kernel<<<grid, gg::kThreads, gg::kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(tm_a,
+                                                                                                             prm);
     count_launch();
     return check_launch();
 }

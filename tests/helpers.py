@@ -104,3 +104,23 @@ def require_gpu():
         pytest.fail("GPU tests need a CUDA device (run them with -m gpu on a B200)")
     from nvfp4_block_scaled_09_b200 import build as nvbuild
     nvbuild.build()
+
+
+def unpack_weights(packed, rows, K):
+    """Packed weight tiles (layout of nvfp4_pack_weights in the header) -> (codes [rows, K/2],
+    row-major scales [rows, K/16])."""
+    flat = np.ascontiguousarray(packed).reshape(-1)
+    kt_n = K // 256
+    tiles = flat.reshape(rows // 128, kt_n, 18432)
+    codes = tiles[:, :, :16384].reshape(rows // 128, kt_n, 128, 8, 16)      # [rb, kt, r, swizzled piece, byte]
+    r = np.arange(128)[:, None]
+    c = np.arange(8)[None, :]
+    logical = codes[:, :, r, c ^ (r & 7), :]                                  # [rb, kt, r, c, byte]
+    q = logical.transpose(0, 2, 1, 3, 4).reshape(rows, K // 2)
+    sc = tiles[:, :, 16384:].reshape(rows // 128, kt_n, 4, 512)               # [rb, kt, kc, atom]
+    rr = np.arange(128)[:, None]
+    j = np.arange(4)[None, :]
+    off = (rr % 32) * 16 + (rr // 32) * 4 + j                                  # [r, j]
+    s = sc[:, :, :, off]                                                       # [rb, kt, kc, r, j]
+    sf = s.transpose(0, 3, 1, 2, 4).reshape(rows, K // 16)
+    return q, sf

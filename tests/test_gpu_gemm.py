@@ -13,7 +13,7 @@ import torch
 import nvfp4_block_scaled_09_b200 as nv
 import oracle
 import workloads
-from tests.helpers import compare_bf16, gpu_bf16, host, host_bits, require_gpu, untile_sf
+from tests.helpers import compare_bf16, gpu_bf16, host, host_bits, require_gpu, unpack_weights
 
 pytestmark = pytest.mark.gpu
 
@@ -24,45 +24,44 @@ def _gpu():
 
 
 def make_case(rows, N, K, seed, a_std=1.0, w_std=0.02):
-    """Quantised activations [sum(rows), K] and per-expert weights [E, N, K] on the GPU."""
+    """Quantised activations [sum(rows), K] and packed per-expert weights [E, N, K] on the GPU."""
     E = len(rows)
     R = int(sum(rows))
     a_bits = workloads.random_bf16_bits((max(R, 1), K), seed=seed, std=a_std)
     a_q, a_sf, a_g = nv.quantize(gpu_bf16(a_bits))
     w = workloads.normal_bf16((E, N, K), w_std, seed, workloads.TAG_W13, device="cuda")
-    w_q, w_sf, w_g = nv.prepare_expert_weights(w)
+    pw = nv.prepare_expert_weights(w, keep_rowmajor=True)
     off = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
     torch.cuda.synchronize()
     # the GPU's operands are the oracle's operands: check their quantisation first
     oq, osf, og = oracle.quantize(a_bits)
     assert np.array_equal(host(a_q), oq) and np.array_equal(host(a_sf), osf) and host(a_g)[0] == og
-    return dict(a_q=a_q, a_sf=a_sf, a_g=a_g, w_q=w_q, w_sf=w_sf, w_g=w_g, off=torch.from_numpy(off).cuda(),
-                off_np=off, w=w, E=E, R=R, N=N, K=K)
+    return dict(a_q=a_q, a_sf=a_sf, a_g=a_g, pw=pw, off=torch.from_numpy(off).cuda(), off_np=off, w=w, E=E, R=R,
+                N=N, K=K)
 
 
-def oracle_operands(c, experts=None):
-    """Host copies of the GPU operands (weight scales un-tiled to row-major)."""
-    E, N, K = c["E"], c["N"], c["K"]
-    sel = range(E) if experts is None else experts
-    w_q = np.stack([host(c["w_q"][e]) for e in sel])
-    w_sf = np.stack([untile_sf(host(c["w_sf"][e]), N, K) for e in sel])
-    w_g = host(c["w_g"])[list(sel)]
-    return w_q, w_sf, w_g
+def oracle_operands(c):
+    """Host copies of the GPU's row-major weight codes / scales / global scales."""
+    pw = c["pw"]
+    return host(pw.q), host(pw.sf), host(pw.gscale)
 
 
-def check_weights_quantised_like_oracle(c, experts):
+def check_weights_quantised_and_packed(c, experts):
+    pw = c["pw"]
     for e in experts:
         wq, wsf, wg = oracle.quantize(host_bits(c["w"][e]))
-        assert np.array_equal(host(c["w_q"][e]), wq)
-        assert np.array_equal(untile_sf(host(c["w_sf"][e]), c["N"], c["K"]), wsf)
-        assert host(c["w_g"])[e] == wg
+        assert np.array_equal(host(pw.q[e]), wq)
+        assert np.array_equal(host(pw.sf[e]), wsf)
+        assert host(pw.gscale)[e] == wg
+        uq, usf = unpack_weights(host(pw.packed[e]), c["N"], c["K"])
+        assert np.array_equal(uq, wq) and np.array_equal(usf, wsf)
 
 
 def run_full(rows, N, K, swiglu, seed):
     c = make_case(rows, N, K, seed)
-    out = nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["w_q"], c["w_sf"], c["w_g"], c["off"], N, K, swiglu)
+    out = nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["pw"], c["off"], swiglu)
     assert nv.device_status() == 0
-    check_weights_quantised_like_oracle(c, range(min(c["E"], 3)))
+    check_weights_quantised_and_packed(c, range(min(c["E"], 3)))
     w_q, w_sf, w_g = oracle_operands(c)
     ref = oracle.grouped_gemm(host(c["a_q"]), host(c["a_sf"]), host(c["a_g"])[0], w_q, w_sf, w_g, c["off_np"],
                               N, K, swiglu)
@@ -92,8 +91,7 @@ def test_rows_outside_experts_untouched():
     R = c["R"]
     out = torch.full((R + 8, 256), 7.0, dtype=torch.bfloat16, device="cuda")
     # offsets cover only rows [0, 30); rows 30.. must keep their canary
-    nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["w_q"], c["w_sf"], c["w_g"], c["off"], 256, 256, False,
-                    out=out)
+    nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["pw"], c["off"], False, out=out)
     assert nv.device_status() == 0
     assert torch.all(out[R:] == 7.0)
 
@@ -101,7 +99,7 @@ def test_rows_outside_experts_untouched():
 def test_bad_offsets_latch_status_and_skip():
     c = make_case([16, 16], 256, 256, seed=4)
     bad = torch.tensor([0, 20, 10], dtype=torch.int32, device="cuda")   # decreasing
-    nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["w_q"], c["w_sf"], c["w_g"], bad, 256, 256, False)
+    nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["pw"], bad, False)
     assert nv.device_status() == 8
 
 
@@ -133,73 +131,74 @@ def test_dense_8192_sampled():
     a_bits_t = workloads.normal_bf16((M, K), 1.0, 0, workloads.TAG_A, device="cuda")
     a_q, a_sf, a_g = nv.quantize(a_bits_t)
     b = workloads.normal_bf16((1, N, K), 0.02, 0, workloads.TAG_B, device="cuda")
-    w_q, w_sf, w_g = nv.prepare_expert_weights(b)
+    pw = nv.prepare_expert_weights(b, keep_rowmajor=True)
     off = torch.tensor([0, M], dtype=torch.int32, device="cuda")
-    out = nv.grouped_gemm(a_q, a_sf, a_g, w_q, w_sf, w_g, off, N, K, False)
+    out = nv.grouped_gemm(a_q, a_sf, a_g, pw, off, False)
     assert nv.device_status() == 0
     # quantisation of a sample of A rows against the oracle
     oq, osf, og = oracle.quantize(host_bits(a_bits_t[:256]), float(host(a_g)[0]))
     assert np.array_equal(host(a_q[:256]), oq) and np.array_equal(host(a_sf[:256]), osf)
+    uq, usf = unpack_weights(host(pw.packed[0]), N, K)
+    assert np.array_equal(uq, host(pw.q[0])) and np.array_equal(usf, host(pw.sf[0]))
     rng = np.random.default_rng(5)
     rows = np.sort(rng.choice(M, size=48, replace=False))
     cols = rng.choice(N, size=48, replace=False)
     rr, cc = np.meshgrid(rows, cols, indexing="ij")
     rr, cc = rr.ravel(), cc.ravel()
-    wq = host(w_q)
-    wsf = untile_sf(host(w_sf[0]), N, K)[None]
-    ref = oracle.grouped_gemm_at(host(a_q), host(a_sf), float(host(a_g)[0]), wq, wsf, host(w_g),
-                                 np.array([0, M], np.int32), N, K, False, rr, cc)
+    ref = oracle.grouped_gemm_at(host(a_q), host(a_sf), float(host(a_g)[0]), host(pw.q), host(pw.sf),
+                                 host(pw.gscale), np.array([0, M], np.int32), N, K, False, rr, cc)
     compare_bf16(host_bits(out)[rr, cc], oracle.bf16_round(ref), "dense 8192", exact=ref)
 
 
-@pytest.mark.parametrize("name", ["moe_decode_t512", "moe_zipf_t1024"])
+def build_layer_weights(E, N, K, tag, keep):
+    """Packed weights of a full-size layer, generated and packed expert by expert; row-major copies (host)
+    are kept for the experts in `keep`."""
+    packed = torch.empty((E, N * (K // 2 + K // 16)), dtype=torch.uint8, device="cuda")
+    g = torch.empty(E, dtype=torch.float32, device="cuda")
+    qt = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+    st = torch.empty((N, K // 16), dtype=torch.uint8, device="cuda")
+    kept = {}
+    for e in range(E):
+        w = workloads.normal_bf16((N, K), 0.02, 0, tag, e, device="cuda")
+        nv.quantize(w, q=qt, sf=st, g=g[e:e + 1])
+        nv.pack_weights(qt, st, out=packed[e])
+        if e in keep:
+            kept[e] = (host_bits(w), host(qt), host(st))
+    return nv.PackedWeights(packed, g, E, N, K), kept
+
+
+@pytest.mark.parametrize("name", ["moe_decode_t512", "moe_zipf_t1024", "moe_prefill_t8192"])
 def test_moe_layer_gemms_full_size_sampled(name):
     cfg = workloads.CONFIGS[name]
     T, H, I, E, k = cfg["T"], cfg["H"], cfg["I"], cfg["E"], cfg["k"]
     ids, _ = workloads.config_routing(name)
     off_np, src, _ = oracle.permute(ids, E)
     R = T * k
-    # activations already in expert order (permute is tested on its own)
-    a = workloads.normal_bf16((R, H), 1.0, 0, workloads.TAG_X, device="cuda")
-    a_q, a_sf, a_g = nv.quantize(a)
-    w13 = [None] * E
-    w13_q = torch.empty((E, 2 * I, H // 2), dtype=torch.uint8, device="cuda")
-    w13_sf = torch.empty((E, 2 * I, H // 16), dtype=torch.uint8, device="cuda")
-    w13_g = torch.empty(E, dtype=torch.float32, device="cuda")
-    for e in range(E):
-        w = workloads.normal_bf16((2 * I, H), 0.02, 0, workloads.TAG_W13, e, device="cuda")
-        nv.quantize(w, layout=nv.SF_MMA_TILED, q=w13_q[e], sf=w13_sf[e], g=w13_g[e:e + 1])
-        if e < 2:
-            w13[e] = host_bits(w)
-    off = torch.from_numpy(off_np).cuda()
-    h = nv.grouped_gemm(a_q, a_sf, a_g, w13_q, w13_sf, w13_g, off, 2 * I, H, True)
-    assert nv.device_status() == 0
-    for e in range(2):
-        wq, wsf, wg = oracle.quantize(w13[e])
-        assert np.array_equal(host(w13_q[e]), wq) and np.array_equal(untile_sf(host(w13_sf[e]), 2 * I, H), wsf)
     counts = np.diff(off_np)
     experts = [int(np.argmax(counts)), int(np.argmin(np.where(counts > 0, counts, 1 << 30))), 0, E - 1]
     experts = sorted(set(e for e in experts if counts[e] > 0))
+    # activations already in expert order (permute is tested on its own)
+    a = workloads.normal_bf16((R, H), 1.0, 0, workloads.TAG_X, device="cuda")
+    a_q, a_sf, a_g = nv.quantize(a)
+    w13, kept13 = build_layer_weights(E, 2 * I, H, workloads.TAG_W13, set(experts))
+    off = torch.from_numpy(off_np).cuda()
+    h = nv.grouped_gemm(a_q, a_sf, a_g, w13, off, True)
+    assert nv.device_status() == 0
+    for e in experts[:2]:
+        wq, wsf, wg = oracle.quantize(kept13[e][0])
+        assert np.array_equal(kept13[e][1], wq) and np.array_equal(kept13[e][2], wsf)
+        uq, usf = unpack_weights(host(w13.packed[e]), 2 * I, H)
+        assert np.array_equal(uq, wq) and np.array_equal(usf, wsf)
 
-    def w13_host(sel):
-        return (np.stack([host(w13_q[e]) for e in sel]),
-                np.stack([untile_sf(host(w13_sf[e]), 2 * I, H) for e in sel]), host(w13_g)[sel])
+    def host_w(kept, gs):
+        return lambda sel: (np.stack([kept[e][1] for e in sel]), np.stack([kept[e][2] for e in sel]),
+                            host(gs)[sel])
 
-    sampled_check(a_q, a_sf, a_g, w13_host, off_np, 2 * I, H, True, h, experts, n_cols=32)
+    sampled_check(a_q, a_sf, a_g, host_w(kept13, w13.gscale), off_np, 2 * I, H, True, h, experts, n_cols=32)
 
     # down projection on the GPU's own h
     hq, hsf, hg = nv.quantize(h)
-    w2_q = torch.empty((E, H, I // 2), dtype=torch.uint8, device="cuda")
-    w2_sf = torch.empty((E, H, I // 16), dtype=torch.uint8, device="cuda")
-    w2_g = torch.empty(E, dtype=torch.float32, device="cuda")
-    for e in range(E):
-        w = workloads.normal_bf16((H, I), 0.02, 0, workloads.TAG_W2, e, device="cuda")
-        nv.quantize(w, layout=nv.SF_MMA_TILED, q=w2_q[e], sf=w2_sf[e], g=w2_g[e:e + 1])
-    y = nv.grouped_gemm(hq, hsf, hg, w2_q, w2_sf, w2_g, off, H, I, False)
+    w2, kept2 = build_layer_weights(E, H, I, workloads.TAG_W2, set(experts))
+    y = nv.grouped_gemm(hq, hsf, hg, w2, off, False)
     assert nv.device_status() == 0
-
-    def w2_host(sel):
-        return (np.stack([host(w2_q[e]) for e in sel]),
-                np.stack([untile_sf(host(w2_sf[e]), H, I) for e in sel]), host(w2_g)[sel])
-
-    sampled_check(hq, hsf, hg, w2_host, off_np, H, I, False, y, experts, n_cols=32, seed=1)
+    sampled_check(hq, hsf, hg, host_w(kept2, w2.gscale), off_np, H, I, False, y, experts, n_cols=32, seed=1)
