@@ -26,10 +26,13 @@
 //    explicit warp-specialised schedules that give A loads, B loads, MMA and
 //    epilogue their own warps): warp 0 issues the weight bulk copies and the
 //    TMA tiles of activations; warp 1
-//    gathers the activation scales (row-major) into the tensor-core scale
-//    layout with cp.async; warp 2 owns tensor memory and issues tcgen05.cp +
-//    tcgen05.mma; warps 4-7 drain the FP32 accumulators from TMEM, apply the
-//    global scales / SwiGLU and store BF16.
+//    gathers the activation scales (row-major) into shared memory with
+//    cp.async; warps 8-11 (one per TMEM lane quadrant) store every stage's
+//    scales into a per-stage TMEM ring with tcgen05.st; warp 2 owns tensor
+//    memory and issues only tcgen05.mma (scale copies issued on the MMA pipe
+//    serialise with the MMAs; measured, this halved the decode stream rate);
+//    warps 4-7 drain the FP32 accumulators from TMEM, apply the global scales /
+//    SwiGLU and store BF16.
 //  * Stage accounting: the expected transaction bytes of a stage are the A
 //    tile bytes plus its scale bytes plus the B tile bytes ("Peering into the
 //    CUTLASS SharedStorage", The Message: MK bytes + NK bytes per stage); the
@@ -71,17 +74,21 @@ constexpr int kOffB = 2 * kPackedTileBytes;
 constexpr int kOffSFB = kOffB + kBBytes;
 constexpr int kStageBytes = kOffSFB + kSFStageBytes;   // 47104 (46 x 1024)
 constexpr int kMaxE = 1024;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kSFDelay = 2;                      // cp.async groups kept in flight by the scale gatherer
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = kBNMax;                       // columns per accumulator
-constexpr uint32_t kTmemSFA = 2 * kNumA * kAccCols;         // 256: 2 buffers x 2 accumulators before it
-constexpr uint32_t kTmemSFB = kTmemSFA + kNumA * 4 * kKSteps;  // 288
+// Scale factors live in a TMEM ring, one 48-column slot per pipeline stage:
+// [SFA block 0: 16][SFA block 1: 16][SFB: 16], after the 2 x 2 accumulators.
+constexpr uint32_t kTmemSFRing = 2 * kNumA * kAccCols;            // 256
+constexpr uint32_t kTmemSFSlot = (kNumA + 1) * 4 * kKSteps;       // 48
+static_assert(kTmemSFRing + kStages * kTmemSFSlot <= kTmemCols, "TMEM budget");
 
 struct Shared {
     uint64_t full_tma[kStages];
     uint64_t full_sf[kStages];
+    uint64_t sf_ready[kStages];
     uint64_t empty[kStages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
@@ -162,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; s++) {
             mbar_init(&sh.full_tma[s], 1);
             mbar_init(&sh.full_sf[s], 1);
+            mbar_init(&sh.sf_ready[s], 4);
             mbar_init(&sh.empty[s], 1);
         }
         for (int b = 0; b < 2; b++) {
@@ -337,22 +345,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             for (int32_t kt = 0; kt < ksteps_total; kt++) {
                 if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl) ||
-                    !warp_wait(&sh.full_sf[stage], phase, abort, p.ctl)) {
+                    !warp_wait(&sh.sf_ready[stage], phase, abort, p.ctl)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t sb = smem_u32(stages + (size_t)stage * kStageBytes);
-#pragma unroll
-                    for (int kc = 0; kc < kKSteps; kc++) {
-                        tmem_cp_32x128b_x4(tmem + kTmemSFA + 4 * kc,
-                                           make_smem_desc(sb + kOffSFA0 + kc * kSFAtomBytes, 0, 128, 0));
-                        tmem_cp_32x128b_x4(tmem + kTmemSFA + 4 * kKSteps + 4 * kc,
-                                           make_smem_desc(sb + kOffSFA1 + kc * kSFAtomBytes, 0, 128, 0));
-                        tmem_cp_32x128b_x4(tmem + kTmemSFB + 4 * kc,
-                                           make_smem_desc(sb + kOffSFB + kc * kSFAtomBytes, 0, 128, 0));
-                    }
+                    const uint32_t sf = tmem + kTmemSFRing + stage * kTmemSFSlot;
 #pragma unroll
                     for (int kc = 0; kc < kKSteps; kc++) {
                         const uint64_t bdesc = make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2);
@@ -361,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int a = 0; a < kNumA; a++) {
                             const uint64_t adesc = make_smem_desc(sb + a * kPackedTileBytes + kc * 32, 16, 1024, 2);
                             mma_mxf4nvf4(tmem + abuf * (kNumA * kAccCols) + a * kAccCols, adesc, bdesc, idesc,
-                                         tmem + kTmemSFA + a * 4 * kKSteps + 4 * kc, tmem + kTmemSFB + 4 * kc, acc);
+                                         sf + a * 4 * kKSteps + 4 * kc, sf + kNumA * 4 * kKSteps + 4 * kc, acc);
                         }
                     }
                     tc_commit(&sh.empty[stage]);
@@ -382,6 +382,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
         }
+    } else if (warp >= 8) {
+        // ================= scale writers =================
+        // Warp 8 + q owns TMEM lane quadrant q. For each stage it reads the
+        // scales from shared memory and stores them into that stage's TMEM ring
+        // slot with tcgen05.st, so the MMA warp issues nothing but MMAs (a
+        // tcgen05.cp on the MMA pipe serialises with the MMAs around it).
+        // MMA reads: row m of a weight block at lane m, column base + 4 kc + m/32;
+        // activation row n at lane n % 32 of every quadrant, column base + 4 kc + n/32.
+        const int quad = warp & 3;
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
+        for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            for (int32_t kt = 0; kt < ksteps_total; kt++) {
+                if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl) ||
+                    !warp_wait(&sh.full_sf[stage], phase, abort, p.ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint8_t* sb = stages + (size_t)stage * kStageBytes;
+                const uint32_t slot = tmem + lane_addr + kTmemSFRing + stage * kTmemSFSlot;
+                uint32_t word[kKSteps], v[16];
+#pragma unroll
+                for (int a = 0; a < kNumA; a++) {
+                    const uint8_t* src = sb + (a ? kOffSFA1 : kOffSFA0) + lane * 16 + quad * 4;
+#pragma unroll
+                    for (int kc = 0; kc < kKSteps; kc++)
+                        word[kc] = *reinterpret_cast<const uint32_t*>(src + kc * kSFAtomBytes);
+#pragma unroll
+                    for (int j = 0; j < 16; j++) v[j] = ((j & 3) == quad) ? word[j >> 2] : 0u;
+                    tmem_st_32x32b_x16(slot + a * 4 * kKSteps, v);
+                }
+#pragma unroll
+                for (int kc = 0; kc < kKSteps; kc++) {
+                    const uint8_t* src = sb + kOffSFB + kc * kSFAtomBytes + lane * 16;
+                    v[4 * kc + 0] = *reinterpret_cast<const uint32_t*>(src);      // activation row lane
+                    v[4 * kc + 1] = *reinterpret_cast<const uint32_t*>(src + 4);  // activation row 32 + lane
+                    v[4 * kc + 2] = 0u;
+                    v[4 * kc + 3] = 0u;
+                }
+                tmem_st_32x32b_x16(slot + kNumA * 4 * kKSteps, v);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.sf_ready[stage]);
+                if (++stage == kStages) { stage = 0; phase ^= 1u; }
+            }
+        }
     } else if (warp >= 4) {
         // ================= epilogue =================
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
@@ -394,49 +443,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             decode_tile(sh, E, n_col_tiles, w, t);
             if (!warp_wait(&sh.acc_full[abuf], aphase, abort, p.ctl)) break;
             tc_fence_after();
-            float v0[kBNMax], v1[kBNMax];
             const uint32_t cbase = tmem + lane_base + abuf * (kNumA * kAccCols);
+            const float alpha = a_g * __ldg(p.w_gscale + t.e);
+            for (int c = 0; c * 16 < t.bn; c++) {
+                float v0[16], v1[16];
+                tmem_ld_32x32b_x16(cbase + c * 16, v0);
+                tmem_ld_32x32b_x16(cbase + kAccCols + c * 16, v1);
+                tmem_ld_wait();
+                const int nrows = min(16, t.rows - c * 16);
+                if (p.swiglu) {
+                    const int64_t ldo = p.N / 2;
+                    uint16_t* o = p.out + ((int64_t)t.row0 + c * 16) * ldo + (int64_t)t.nt * kBM + r;
 #pragma unroll
-            for (int c = 0; c < kBNMax / 16; c++) {
-                if (c * 16 < t.bn) {
-                    float tmp[16];
-                    tmem_ld_32x32b_x16(cbase + c * 16, tmp);
+                    for (int i = 0; i < 16; i++) {
+                        if (i < nrows) {
+                            const float g = alpha * v0[i], u = alpha * v1[i];
+                            const float h = g / (1.0f + expf(-g)) * u;
+                            o[(int64_t)i * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                        }
+                    }
+                } else {
+                    const int64_t ldo = p.N;
+                    uint16_t* o = p.out + ((int64_t)t.row0 + c * 16) * ldo + (int64_t)t.nt * (kNumA * kBM) + r;
 #pragma unroll
-                    for (int i = 0; i < 16; i++) v0[c * 16 + i] = tmp[i];
-                    tmem_ld_32x32b_x16(cbase + kAccCols + c * 16, tmp);
-#pragma unroll
-                    for (int i = 0; i < 16; i++) v1[c * 16 + i] = tmp[i];
+                    for (int i = 0; i < 16; i++) {
+                        if (i < nrows) {
+                            o[(int64_t)i * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v0[i]));
+                            o[(int64_t)i * ldo + kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v1[i]));
+                        }
+                    }
                 }
             }
-            tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.acc_empty[abuf]);
             if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
-
-            const float alpha = a_g * __ldg(p.w_gscale + t.e);
-            if (p.swiglu) {
-                const int64_t ldo = p.N / 2;
-                uint16_t* o = p.out + (int64_t)t.row0 * ldo + (int64_t)t.nt * kBM + r;
-#pragma unroll
-                for (int n = 0; n < kBNMax; n++) {
-                    if (n < t.rows) {
-                        const float g = alpha * v0[n], u = alpha * v1[n];
-                        const float h = g / (1.0f + expf(-g)) * u;
-                        o[(int64_t)n * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
-                    }
-                }
-            } else {
-                const int64_t ldo = p.N;
-                uint16_t* o = p.out + (int64_t)t.row0 * ldo + (int64_t)t.nt * (kNumA * kBM) + r;
-#pragma unroll
-                for (int n = 0; n < kBNMax; n++) {
-                    if (n < t.rows) {
-                        o[(int64_t)n * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v0[n]));
-                        o[(int64_t)n * ldo + kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v1[n]));
-                    }
-                }
-            }
         }
     }
 
