@@ -265,7 +265,7 @@ NVFP4_API nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_id
 /* Message excerpt: bytes of the A tile plus its scales, plus bytes of the B */
 /* tile plus its scales.                                                     */
 /* ------------------------------------------------------------------------ */
-typedef struct {
+typedef struct {                 /* fields up to `threads` describe the narrow (decode) tile shape */
     int32_t tile_weight_rows;    /* weight rows (GEMM N) per tile: 256 */
     int32_t tile_tokens_max;     /* activation rows (GEMM M) per tile, at most */
     int32_t stage_k;             /* K elements per pipeline stage */
@@ -277,11 +277,19 @@ typedef struct {
     int32_t smem_bytes;          /* dynamic shared memory per CTA */
     int32_t tmem_columns;        /* tensor-memory columns allocated per CTA */
     int32_t threads;             /* threads per CTA */
+    /* The wide tile shape, used when the experts average at least
+     * wide_min_avg_rows rows (max_rows >= wide_min_avg_rows * E): up to
+     * wide_tile_tokens_max activation rows per tile, one accumulator buffer. */
+    int32_t wide_tile_tokens_max;
+    int32_t wide_stage_bytes_act_max;
+    int32_t wide_smem_bytes;
+    int32_t wide_min_avg_rows;
 } nvfp4_gemm_plan;
 
 NVFP4_API nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan);
-/* Expect-tx bytes one stage's TMA and bulk copies deliver for a tile of `tokens` rows. */
-NVFP4_API int64_t nvfp4_gemm_stage_tx_bytes(int32_t tokens);
+/* Expect-tx bytes one stage's TMA and bulk copies deliver for a tile of `tokens` rows
+ * (wide != 0: the wide tile shape). -1 when tokens is outside [1, tile maximum]. */
+NVFP4_API int64_t nvfp4_gemm_stage_tx_bytes(int32_t tokens, int32_t wide);
 /* Pure host check against a given opt-in shared-memory budget (bytes per block). */
 NVFP4_API nvfp4_status nvfp4_can_implement_with_budget(int64_t N, int64_t K, int32_t E, nvfp4_epilogue epi,
                                              int64_t smem_optin_bytes);

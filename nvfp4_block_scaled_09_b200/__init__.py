@@ -51,7 +51,8 @@ class LayerWorkspace(ctypes.Structure):
 class GemmPlan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "tile_weight_rows", "tile_tokens_max", "stage_k", "stages", "stage_bytes_weights", "stage_bytes_weight_sf",
-        "stage_bytes_act_max", "stage_bytes_act_sf", "smem_bytes", "tmem_columns", "threads")]
+        "stage_bytes_act_max", "stage_bytes_act_sf", "smem_bytes", "tmem_columns", "threads",
+        "wide_tile_tokens_max", "wide_stage_bytes_act_max", "wide_smem_bytes", "wide_min_avg_rows")]
 
 
 _lib = None
@@ -93,7 +94,7 @@ def lib():
         L.moe_layer_nvfp4.restype = st
         L.nvfp4_gemm_get_plan.argtypes = [ctypes.POINTER(GemmPlan)]
         L.nvfp4_gemm_get_plan.restype = st
-        L.nvfp4_gemm_stage_tx_bytes.argtypes = [i32]
+        L.nvfp4_gemm_stage_tx_bytes.argtypes = [i32, i32]
         L.nvfp4_gemm_stage_tx_bytes.restype = i64
         L.nvfp4_can_implement_with_budget.argtypes = [i64, i64, i32, ctypes.c_int, i64]
         L.nvfp4_can_implement_with_budget.restype = st
@@ -305,8 +306,8 @@ def gemm_plan() -> dict:
     return {n: getattr(p, n) for n, _ in GemmPlan._fields_}
 
 
-def gemm_stage_tx_bytes(tokens: int) -> int:
-    return int(lib().nvfp4_gemm_stage_tx_bytes(tokens))
+def gemm_stage_tx_bytes(tokens: int, wide: bool = False) -> int:
+    return int(lib().nvfp4_gemm_stage_tx_bytes(tokens, 1 if wide else 0))
 
 
 # ----------------------------------------------------------------------------- combine

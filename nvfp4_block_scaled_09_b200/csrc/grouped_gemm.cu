@@ -25,9 +25,8 @@
 //  * Warp roles ("Peering into the CUTLASS Kernel Scheduler", The Discovery:
 //    explicit warp-specialised schedules that give A loads, B loads, MMA and
 //    epilogue their own warps): warp 0 issues the weight bulk copies and the
-//    TMA tiles of activations; warp 1
-//    gathers the activation scales (row-major) into shared memory with
-//    cp.async; warps 8-11 (one per TMEM lane quadrant) store every stage's
+//    TMA tiles of activations and of their row-major scales; warps 8-11 (one
+//    per TMEM lane quadrant) store every stage's
 //    scales into a per-stage TMEM ring with tcgen05.st; warp 2 owns tensor
 //    memory and issues only tcgen05.mma (scale copies issued on the MMA pipe
 //    serialise with the MMAs; measured, this halved the decode stream rate);
@@ -35,9 +34,11 @@
 //    SwiGLU and store BF16.
 //  * Stage accounting: the expected transaction bytes of a stage are the A
 //    tile bytes plus its scale bytes plus the B tile bytes ("Peering into the
-//    CUTLASS SharedStorage", The Message: MK bytes + NK bytes per stage); the
-//    B scales arrive through their own barrier.
-//  * Shared memory: 4 stages x 46 KB + scheduler tables, checked against the
+//    CUTLASS SharedStorage", The Message: MK bytes + NK bytes per stage): two
+//    packed weight tiles (codes + scales), the activation tile and one box of
+//    its scales.
+//  * Shared memory: 4 stages x 46 KB (narrow) or 54 KB (wide) + scheduler
+//    tables, checked against the
 //    device's opt-in limit before launch (the same predicate
 //    nvfp4_can_implement() reports, so a passing check never fails to launch).
 //  * Persistent CTAs (one per SM) walk (expert, column tile, row tile) work
@@ -56,12 +57,10 @@ constexpr int kBM = 128;                         // weight rows per MMA (tcgen05
 constexpr int kNumA = 2;                         // weight row blocks per tile
 constexpr int kBK = 256;                         // K elements per stage
 constexpr int kRowBytes = kBK / 2;               // packed bytes per row per stage (one 128-byte swizzle row)
-constexpr int kBNMax = 64;                       // activation rows per tile (tcgen05 N), at most
 constexpr int kBNStep = 16;                      // N granularity = activation TMA box rows
 constexpr int kStages = 4;
 constexpr int kKSteps = kBK / 64;                // MMA K-steps per stage (K = 64 per MMA)
 constexpr int kABlockBytes = kBM * kRowBytes;    // 16 KB
-constexpr int kBBytes = kBNMax * kRowBytes;      // 8 KB
 constexpr int kSFAtomBytes = 512;                // 128 rows x 4 scales
 constexpr int kSFStageBytes = kKSteps * kSFAtomBytes;
 constexpr int kPackedTileBytes = kABlockBytes + kSFStageBytes;  // one packed weight tile (codes + scales)
@@ -71,23 +70,13 @@ constexpr int kOffSFA0 = kABlockBytes;
 constexpr int kOffA1 = kPackedTileBytes;
 constexpr int kOffSFA1 = kOffA1 + kABlockBytes;
 constexpr int kOffB = 2 * kPackedTileBytes;
-constexpr int kOffSFB = kOffB + kBBytes;
-constexpr int kStageBytes = kOffSFB + kSFStageBytes;   // 47104 (46 x 1024)
 constexpr int kMaxE = 1024;
 constexpr int kThreads = 384;
-constexpr int kSFDelay = 2;                      // cp.async groups kept in flight by the scale gatherer
-
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCols = kBNMax;                       // columns per accumulator
-// Scale factors live in a TMEM ring, one 48-column slot per pipeline stage:
-// [SFA block 0: 16][SFA block 1: 16][SFB: 16], after the 2 x 2 accumulators.
-constexpr uint32_t kTmemSFRing = 2 * kNumA * kAccCols;            // 256
-constexpr uint32_t kTmemSFSlot = (kNumA + 1) * 4 * kKSteps;       // 48
-static_assert(kTmemSFRing + kStages * kTmemSFSlot <= kTmemCols, "TMEM budget");
+constexpr int kSmemLimit = 232448;               // B200 opt-in shared memory per block
 
 struct Shared {
     uint64_t full_tma[kStages];
-    uint64_t full_sf[kStages];
     uint64_t sf_ready[kStages];
     uint64_t empty[kStages];
     uint64_t acc_full[2];
@@ -100,11 +89,35 @@ struct Shared {
     int32_t tile_start[kMaxE + 1];
 };
 
-constexpr size_t kSmemBytes = 1024 /* alignment slack */ + (size_t)kStages * kStageBytes + sizeof(Shared);
+// Two tile shapes share one kernel body:
+//  - narrow (decode): up to 64 activation rows per tile, two TMEM accumulator
+//    buffers so the epilogue of one tile overlaps the main loop of the next;
+//  - wide (prefill, dense): up to 128 activation rows per tile -- N = 128 MMAs
+//    cost the same ~50 ns as N = 64 ones on B200, so the tensor rate doubles and
+//    the activation re-reads from L2 halve -- with one accumulator buffer (two
+//    128-column accumulators plus the scale ring fill the 512 TMEM columns).
+template <int BN_MAX, int ACC_BUFS>
+struct Cfg {
+    static constexpr int kBNMax = BN_MAX;
+    static constexpr int kAccBufs = ACC_BUFS;
+    static constexpr int kBBytes = BN_MAX * kRowBytes;
+    static constexpr int kOffSFB = kOffB + kBBytes;
+    static constexpr int kStageBytes = kOffSFB + kSFStageBytes;
+    static constexpr uint32_t kAccCols = BN_MAX;
+    // Scale factors live in a TMEM ring, one 48-column slot per pipeline stage:
+    // [SFA block 0: 16][SFA block 1: 16][SFB: 16], after the accumulators.
+    static constexpr uint32_t kTmemSFRing = ACC_BUFS * kNumA * kAccCols;
+    static constexpr uint32_t kTmemSFSlot = (kNumA + 1) * 4 * kKSteps;
+    static constexpr size_t kSmemBytes = 1024 /* alignment slack */ + (size_t)kStages * kStageBytes + sizeof(Shared);
+    static_assert(BN_MAX % kBNStep == 0 && BN_MAX <= 128, "one scale atom covers at most 128 activation rows");
+    static_assert(kTmemSFRing + kStages * kTmemSFSlot <= kTmemCols, "TMEM budget");
+    static_assert(kStageBytes % 1024 == 0, "stage buffers must keep 1024-byte swizzle alignment");
+    static_assert(kSmemBytes + 256 <= (size_t)kSmemLimit, "shared memory budget (dynamic + static)");
+};
+using Narrow = Cfg<64, 2>;
+using Wide = Cfg<128, 1>;
 
-static_assert(kStageBytes % 1024 == 0, "stage buffers must keep 1024-byte swizzle alignment");
 static_assert(kOffA1 % 1024 == 0 && kOffB % 1024 == 0, "swizzled operand tiles must start on 1024 bytes");
-static_assert(kSFDelay < kStages, "scale gatherer may not hold more stages than the ring has");
 
 struct Params {
     const uint8_t* a_sf;
@@ -125,6 +138,7 @@ struct Tile {
     int32_t e, nt, mt, row0, rows, bn;
 };
 
+template <int kBNMax>
 __device__ __forceinline__ void decode_tile(const Shared& sh, int32_t E, int32_t n_col_tiles, int32_t w, Tile& t) {
     int32_t lo = 0, hi = E;  // tile_start[lo] <= w < tile_start[hi]
     while (hi - lo > 1) {
@@ -148,8 +162,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
+template <class C>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const Params p) {
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_sf,
+                        const Params p) {
+    constexpr int kBNMax = C::kBNMax;
+    constexpr int kOffSFB = C::kOffSFB;
+    constexpr int kStageBytes = C::kStageBytes;
+    constexpr uint32_t kAccCols = C::kAccCols;
+    constexpr uint32_t kTmemSFRing = C::kTmemSFRing;
+    constexpr uint32_t kTmemSFSlot = C::kTmemSFSlot;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
@@ -168,7 +190,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         sh.abort = 0;
         for (int s = 0; s < kStages; s++) {
             mbar_init(&sh.full_tma[s], 1);
-            mbar_init(&sh.full_sf[s], 1);
             mbar_init(&sh.sf_ready[s], 4);
             mbar_init(&sh.empty[s], 1);
         }
@@ -252,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
                 Tile t;
-                decode_tile(sh, E, n_col_tiles, w, t);
+                decode_tile<kBNMax>(sh, E, n_col_tiles, w, t);
                 int64_t r0, r1;
                 if (p.swiglu) {
                     r0 = (int64_t)t.nt * kBM;
@@ -266,7 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint8_t* wp1 = p.w_packed + (wr1 / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
                 const bool reuse = (sh.off[t.e + 1] - sh.off[t.e]) > kBNMax;
                 const uint64_t pol_w = reuse ? pol_w_reuse : pol_w_once;
-                const uint32_t tx = (uint32_t)(kNumA * kPackedTileBytes + t.bn * kRowBytes);
+                // MK part: two packed weight tiles (codes + scales); NK part: the activation
+                // tile and one box of its row-major scales (kBNMax rows x 16 bytes).
+                const uint32_t tx = (uint32_t)(kNumA * kPackedTileBytes + t.bn * kRowBytes + kBNMax * 16);
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
                     if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
                     uint8_t* sb = stages + (size_t)stage * kStageBytes;
@@ -277,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bulk_load(sb + kOffA1, wp1 + (size_t)kt * kPackedTileBytes, kPackedTileBytes, bar, pol_w);
                     for (int32_t i = 0; i < t.bn / kBNStep; i++)
                         tma_load_2d(sb + kOffB + i * kBNStep * kRowBytes, &tm_a, kx, t.row0 + i * kBNStep, bar, pol_a);
+                    tma_load_2d(sb + kOffSFB, &tm_sf, kt * 16, t.row0, bar, pol_a);
                     issued[stage] = true;
                     issued_parity[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -289,47 +313,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ================= activation-scale gatherer =================
-        // Row-major scales [rows, K/16] -> per K-step 512-byte atoms where the
-        // scale word of activation row n sits at (n % 32) * 16 + (n / 32) * 4.
-        uint32_t stage = 0, phase = 0;
-        uint32_t pend[kSFDelay + 1];
-        int npend = 0;
-        bool ok = true;
-        const int64_t sf_row = p.K / 16;
-        for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
-            Tile t;
-            decode_tile(sh, E, n_col_tiles, w, t);
-            for (int32_t kt = 0; kt < ksteps_total; kt++) {
-                if (!warp_wait(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
-                uint8_t* dst_base = stages + (size_t)stage * kStageBytes + kOffSFB;
-                for (int i = lane; i < 4 * t.bn; i += 32) {
-                    const int n = i >> 2, kc = i & 3;
-                    const int64_t grow = (int64_t)t.row0 + n;
-                    const bool in = grow < p.max_rows;
-                    const uint8_t* src = in ? p.a_sf + grow * sf_row + (int64_t)kt * 16 + kc * 4 : p.a_sf;
-                    cp_async_4(dst_base + kc * kSFAtomBytes + (n & 31) * 16 + (n >> 5) * 4, src, in ? 4u : 0u);
-                }
-                cp_async_commit();
-                pend[npend++] = stage;
-                if (npend > kSFDelay) {
-                    cp_async_wait<kSFDelay>();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sh.full_sf[pend[0]]);
-                    for (int j = 0; j + 1 < npend; j++) pend[j] = pend[j + 1];
-                    npend--;
-                }
-                if (++stage == kStages) { stage = 0; phase ^= 1u; }
-            }
-        }
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (ok && lane == 0)
-            for (int j = 0; j < npend; j++) mbar_arrive(&sh.full_sf[pend[j]]);
-        __syncwarp();
     } else if (warp == 2) {
         // ================= MMA issuer =================
         // Instruction descriptor: E2M1 x E2M1 (format 1), both K-major, UE4M3
@@ -339,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
             Tile t;
-            decode_tile(sh, E, n_col_tiles, w, t);
+            decode_tile<kBNMax>(sh, E, n_col_tiles, w, t);
             const uint32_t idesc = idesc_base | ((uint32_t)(t.bn >> 3) << 17);
             if (!warp_wait(&sh.acc_empty[abuf], aphase ^ 1u, abort, p.ctl)) { ok = false; break; }
             tc_fence_after();
@@ -372,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             if (lane == 0) tc_commit(&sh.acc_full[abuf]);
             __syncwarp();
-            if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
+            if (++abuf == (uint32_t)C::kAccBufs) { abuf = 0; aphase ^= 1u; }
         }
         if (!ok || *abort) {
             // Abort path: wait for every MMA issued so far before tensor memory is freed.
@@ -390,14 +373,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tcgen05.cp on the MMA pipe serialises with the MMAs around it).
         // MMA reads: row m of a weight block at lane m, column base + 4 kc + m/32;
         // activation row n at lane n % 32 of every quadrant, column base + 4 kc + n/32.
+        // Activation scales arrive by TMA as [rows][16 bytes] (row-major, one stage).
         const int quad = warp & 3;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         uint32_t stage = 0, phase = 0;
         bool ok = true;
         for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
             for (int32_t kt = 0; kt < ksteps_total; kt++) {
-                if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl) ||
-                    !warp_wait(&sh.full_sf[stage], phase, abort, p.ctl)) {
+                if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl)) {
                     ok = false;
                     break;
                 }
@@ -417,11 +400,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
 #pragma unroll
                 for (int kc = 0; kc < kKSteps; kc++) {
-                    const uint8_t* src = sb + kOffSFB + kc * kSFAtomBytes + lane * 16;
-                    v[4 * kc + 0] = *reinterpret_cast<const uint32_t*>(src);      // activation row lane
-                    v[4 * kc + 1] = *reinterpret_cast<const uint32_t*>(src + 4);  // activation row 32 + lane
-                    v[4 * kc + 2] = 0u;
-                    v[4 * kc + 3] = 0u;
+#pragma unroll
+                    for (int g = 0; g < 4; g++)   // activation row 32 g + lane: 16 scale bytes per row in smem
+                        v[4 * kc + g] = g * 32 < kBNMax
+                                            ? *reinterpret_cast<const uint32_t*>(sb + kOffSFB + (32 * g + lane) * 16 + 4 * kc)
+                                            : 0u;
                 }
                 tmem_st_32x32b_x16(slot + kNumA * 4 * kKSteps, v);
                 tmem_st_wait();
@@ -440,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t abuf = 0, aphase = 0;
         for (int32_t w = blockIdx.x; w < total; w += gridDim.x) {
             Tile t;
-            decode_tile(sh, E, n_col_tiles, w, t);
+            decode_tile<kBNMax>(sh, E, n_col_tiles, w, t);
             if (!warp_wait(&sh.acc_full[abuf], aphase, abort, p.ctl)) break;
             tc_fence_after();
             const uint32_t cbase = tmem + lane_base + abuf * (kNumA * kAccCols);
@@ -477,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.acc_empty[abuf]);
-            if (++abuf == 2) { abuf = 0; aphase ^= 1u; }
+            if (++abuf == (uint32_t)C::kAccBufs) { abuf = 0; aphase ^= 1u; }
         }
     }
 
@@ -512,42 +495,53 @@ static EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// 2-D byte tensor [rows, row_bytes] with 128-byte swizzled boxes of box_rows x 128 bytes.
-static bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, uint32_t box_rows) {
+// 2-D byte tensor [rows, row_bytes] loaded in boxes of box_rows x box_bytes (128-byte swizzle when
+// box_bytes is 128, none otherwise); rows past the end read as zeros.
+static bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, uint32_t box_rows,
+                            uint32_t box_bytes) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    cuuint32_t box[2] = {128u, box_rows};
+    cuuint32_t box[2] = {box_bytes, box_rows};
     cuuint32_t estr[2] = {1u, 1u};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+
+// Experts averaging at least this many rows use the wide tile shape.
+static constexpr int64_t kWideMinAvgRows = 96;
 
 extern "C" nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan) {
     if (!plan) return NVFP4_ERR_INVALID_ARG;
     plan->tile_weight_rows = gg::kNumA * gg::kBM;
-    plan->tile_tokens_max = gg::kBNMax;
+    plan->tile_tokens_max = gg::Narrow::kBNMax;
     plan->stage_k = gg::kBK;
     plan->stages = gg::kStages;
     plan->stage_bytes_weights = gg::kNumA * gg::kABlockBytes;   // arrives with its scales in one packed tile
     plan->stage_bytes_weight_sf = gg::kNumA * gg::kSFStageBytes;
-    plan->stage_bytes_act_max = gg::kBBytes;
+    plan->stage_bytes_act_max = gg::Narrow::kBBytes;
     plan->stage_bytes_act_sf = gg::kSFStageBytes;
-    plan->smem_bytes = (int32_t)gg::kSmemBytes;
+    plan->smem_bytes = (int32_t)gg::Narrow::kSmemBytes;
     plan->tmem_columns = (int32_t)gg::kTmemCols;
     plan->threads = gg::kThreads;
+    plan->wide_tile_tokens_max = gg::Wide::kBNMax;
+    plan->wide_stage_bytes_act_max = gg::Wide::kBBytes;
+    plan->wide_smem_bytes = (int32_t)gg::Wide::kSmemBytes;
+    plan->wide_min_avg_rows = (int32_t)kWideMinAvgRows;
     return NVFP4_OK;
 }
 
-extern "C" int64_t nvfp4_gemm_stage_tx_bytes(int32_t tokens) {
-    if (tokens <= 0 || tokens > gg::kBNMax) return -1;
+extern "C" int64_t nvfp4_gemm_stage_tx_bytes(int32_t tokens, int32_t wide) {
+    const int64_t bn_max = wide ? gg::Wide::kBNMax : gg::Narrow::kBNMax;
+    if (tokens <= 0 || tokens > bn_max) return -1;
     const int64_t bn = (tokens + gg::kBNStep - 1) / gg::kBNStep * gg::kBNStep;
-    // MK part: weight tiles + their scales (packed together); NK part: activation tile (its scales come
-    // through cp.async on their own barrier).
-    return (int64_t)gg::kNumA * gg::kPackedTileBytes + bn * gg::kRowBytes;
+    // MK part: the two weight tiles with their scales (packed together); NK part: the activation
+    // tile plus one TMA box of its scales (bn_max rows x 16 bytes).
+    return (int64_t)gg::kNumA * gg::kPackedTileBytes + bn * gg::kRowBytes + bn_max * 16;
 }
 
 extern "C" nvfp4_status nvfp4_can_implement_with_budget(int64_t N, int64_t K, int32_t E, nvfp4_epilogue epi,
@@ -556,7 +550,10 @@ extern "C" nvfp4_status nvfp4_can_implement_with_budget(int64_t N, int64_t K, in
     if (N <= 0 || K <= 0 || E <= 0) return NVFP4_ERR_INVALID_ARG;
     if (E > gg::kMaxE || N % (gg::kNumA * gg::kBM) != 0 || K % gg::kBK != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if ((int64_t)E * N > INT32_MAX || K / 2 > INT32_MAX) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (smem_optin_bytes < (int64_t)gg::kSmemBytes) return NVFP4_ERR_SMEM_BUDGET;
+    // both tile shapes must fit: the launcher picks one from the rows per expert
+    const int64_t need = (int64_t)(gg::Wide::kSmemBytes > gg::Narrow::kSmemBytes ? gg::Wide::kSmemBytes
+                                                                                  : gg::Narrow::kSmemBytes);
+    if (smem_optin_bytes < need) return NVFP4_ERR_SMEM_BUDGET;
     return NVFP4_OK;
 }
 
@@ -564,6 +561,24 @@ extern "C" nvfp4_status nvfp4_can_implement(int64_t N, int64_t K, int32_t E, nvf
     const int optin = device_smem_optin();
     if (optin < 0) return NVFP4_ERR_CUDA;
     return nvfp4_can_implement_with_budget(N, K, E, epi, optin);
+}
+
+template <class C>
+static nvfp4_status launch_variant(const CUtensorMap& tm_a, const uint8_t* a_sf, const gg::Params& prm,
+                                   cudaStream_t s) {
+    static bool configured[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(gg::grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        configured[dev] = true;
+    }
+    CUtensorMap tm_sf;  // one stage of activation scales: kBNMax rows x 16 bytes
+    if (!encode_rows_map(&tm_sf, a_sf, prm.max_rows, prm.K / 16, C::kBNMax, 16)) return NVFP4_ERR_CUDA;
+    gg::grouped_gemm_kernel<C><<<device_sm_count(), gg::kThreads, C::kSmemBytes, s>>>(tm_a, tm_sf, prm);
+    return NVFP4_OK;
 }
 
 extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
@@ -586,17 +601,8 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
     if (!status) return NVFP4_ERR_CUDA;
 
     CUtensorMap tm_a;
-    if (!encode_rows_map(&tm_a, a_q, max_rows, K / 2, gg::kBNStep)) return NVFP4_ERR_CUDA;
+    if (!encode_rows_map(&tm_a, a_q, max_rows, K / 2, gg::kBNStep, 128)) return NVFP4_ERR_CUDA;
 
-    static int configured_device = -1;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
-    if (configured_device != dev) {
-        if (cudaFuncSetAttribute(gg::grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gg::kSmemBytes) != cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        configured_device = dev;
-    }
     gg::Params prm;
     prm.a_sf = a_sf;
     prm.a_gscale = a_gscale;
@@ -611,9 +617,11 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
     prm.swiglu = epi == NVFP4_EPI_SWIGLU ? 1 : 0;
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
-    const int grid = device_sm_count();
-    gg::grouped_gemm_kernel<<<grid, gg::kThreads, gg::kSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(tm_a,
-                                                                                                             prm);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool wide = max_rows >= kWideMinAvgRows * (int64_t)E;
+    const nvfp4_status ls =
+        wide ? launch_variant<gg::Wide>(tm_a, a_sf, prm, s) : launch_variant<gg::Narrow>(tm_a, a_sf, prm, s);
+    if (ls != NVFP4_OK) return ls;
     count_launch();
     return check_launch();
 }

@@ -82,6 +82,12 @@ def test_ragged_experts_and_row_tiles(swiglu):
 
 
 @pytest.mark.parametrize("swiglu", [False, True])
+def test_wide_tiles_ragged(swiglu):
+    # experts averaging >= 96 rows take the 128-row tile shape: empty, partial, exact, 128 + 1, several tiles
+    run_full([0, 100, 128, 129, 300, 17], 512, 768, swiglu, seed=6)
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
 def test_deeper_k_and_wider_n(swiglu):
     run_full([5, 40, 200], 768, 2048, swiglu, seed=2)
 

@@ -40,29 +40,36 @@ def test_can_implement_shapes_and_budget(L):
     assert nv.can_implement(4096, 6144 + 128, 256, True, big) == 3
     assert nv.can_implement(4096, 6144, 1025, True, big) == 3
     assert nv.can_implement(0, 6144, 8, True, big) == 1
-    # a budget below the kernel's shared memory is refused before any launch
-    assert nv.can_implement(4096, 6144, 256, True, plan["smem_bytes"] - 1) == 5
+    # a budget below either tile shape's shared memory is refused before any launch
+    assert nv.can_implement(4096, 6144, 256, True, max(plan["smem_bytes"], plan["wide_smem_bytes"]) - 1) == 5
     assert nv.can_implement(4096, 6144, 256, True, 101376) == 5     # an SM120-sized budget
 
 
 def test_stage_transaction_bytes_are_tile_sums(L):
-    # Per stage: (A tile bits + A scale bits) + (B tile bits), in bytes, for
-    # packed E2M1 (4 bits) and one 8-bit scale per 16 elements.
+    # Per stage: (A tile bits + A scale bits) + (B tile bits + B scale bits), in bytes, for
+    # packed E2M1 (4 bits) and one 8-bit scale per 16 elements. The B scales travel as one
+    # box covering the tile shape's maximum row count.
     plan = nv.gemm_plan()
     bk = plan["stage_k"]
     wrows = plan["tile_weight_rows"]
     a_bits = wrows * bk * 4
     sfa_bits = wrows * (bk // 16) * 8
-    for tokens in (1, 15, 16, 17, 32, 48, 64):
-        bn = -(-tokens // 16) * 16
-        b_bits = bn * bk * 4
-        assert nv.gemm_stage_tx_bytes(tokens) == (a_bits + sfa_bits + b_bits) // 8
-    assert nv.gemm_stage_tx_bytes(0) == -1
-    assert nv.gemm_stage_tx_bytes(plan["tile_tokens_max"] + 1) == -1
-    # the ring fits the shared-memory budget it claims
-    stage = plan["stage_bytes_weights"] + plan["stage_bytes_weight_sf"] + plan["stage_bytes_act_max"] + \
-        plan["stage_bytes_act_sf"]
-    assert plan["stages"] * stage <= plan["smem_bytes"]
+    for wide, bn_max in ((False, plan["tile_tokens_max"]), (True, plan["wide_tile_tokens_max"])):
+        sfb_bits = bn_max * (bk // 16) * 8
+        for tokens in (1, 15, 16, 17, 32, 48, 64, 65, 100, 128):
+            if tokens > bn_max:
+                assert nv.gemm_stage_tx_bytes(tokens, wide) == -1
+                continue
+            bn = -(-tokens // 16) * 16
+            b_bits = bn * bk * 4
+            assert nv.gemm_stage_tx_bytes(tokens, wide) == (a_bits + sfa_bits + b_bits + sfb_bits) // 8
+        assert nv.gemm_stage_tx_bytes(0, wide) == -1
+    assert plan["wide_tile_tokens_max"] > plan["tile_tokens_max"]
+    # the rings fit the shared-memory budgets they claim
+    for act, smem in ((plan["stage_bytes_act_max"], plan["smem_bytes"]),
+                      (plan["wide_stage_bytes_act_max"], plan["wide_smem_bytes"])):
+        stage = plan["stage_bytes_weights"] + plan["stage_bytes_weight_sf"] + act + plan["stage_bytes_act_sf"]
+        assert plan["stages"] * stage <= smem <= 232448
     assert plan["tmem_columns"] in (32, 64, 128, 256, 512)
 
 
