@@ -70,6 +70,37 @@ def load_peaks():
 
 FP4_PER_BF16 = 4.0  # nominal dense ratio (9 PF FP4 / 2.25 PF BF16)
 
+GEMM_SOURCES = ("nvfp4_block_scaled_09_b200/csrc/grouped_gemm.cu", "nvfp4_block_scaled_09_b200/csrc/common.cuh")
+
+
+def gemm_source_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(config: str):
+    """DRAM bytes per gate/up GEMM launch from the committed ncu summary of this workload, or None when
+    there is none or the GEMM sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{config}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    if fields.get("source_sha256") != gemm_source_sha256():
+        return None
+    try:
+        return int(fields["gate_up_dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
 
 # ----------------------------------------------------------------------------- work accounting
 
@@ -628,7 +659,7 @@ def main():
         "stage_ms": {"quantize_x": stage_ms[0], "permute": stage_ms[1], "gemm_gate_up": stage_ms[2],
                      "quantize_h": stage_ms[3], "gemm_down": stage_ms[4], "combine": stage_ms[5]},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(args.config),
                      "kernel": "grouped_gemm_kernel, gate/up + SwiGLU", "peak_source": peaks["source"],
                      "algorithmic_bytes": g1b, "avg_launch_ms": stage_ms[2]},
         "roofline_down": {"bound": "hbm", "achieved": g2b / gemm2_s / 1e9, "peak": peaks["hbm_gbs"],

@@ -308,6 +308,12 @@ NVFP4_API nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
  * its own copies, frees its tensor memory and returns. */
 NVFP4_API void nvfp4_set_wait_timeout_ns(uint64_t ns);
 NVFP4_API uint64_t nvfp4_get_wait_timeout_ns(void);
+/* Test hook for the failure-detection test only; 0 (the default) on every
+ * normal call. Bit 0: the grouped GEMM's producer warp issues no loads, so each
+ * consumer's bounded wait runs out after the wait timeout and the kernel
+ * latches NVFP4_ERR_DEVICE_TIMEOUT and returns (nothing is in flight, the
+ * context stays usable). Other bits are ignored. */
+NVFP4_API void nvfp4_debug_set_flags(uint32_t flags);
 /* Number of kernel launches made by this library in this process. */
 NVFP4_API uint64_t nvfp4_launch_count(void);
 NVFP4_API const char* nvfp4_status_string(nvfp4_status status);

@@ -106,6 +106,8 @@ def lib():
         L.nvfp4_set_wait_timeout_ns.restype = None
         L.nvfp4_get_wait_timeout_ns.restype = ctypes.c_uint64
         L.nvfp4_launch_count.restype = ctypes.c_uint64
+        L.nvfp4_debug_set_flags.argtypes = [ctypes.c_uint32]
+        L.nvfp4_debug_set_flags.restype = None
         L.nvfp4_status_string.argtypes = [ctypes.c_int]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -385,6 +387,11 @@ def set_wait_timeout_ns(ns: int) -> None:
 
 def get_wait_timeout_ns() -> int:
     return int(lib().nvfp4_get_wait_timeout_ns())
+
+
+def debug_set_flags(flags: int) -> None:
+    """Test hook (see nvfp4_debug_set_flags in the header)."""
+    lib().nvfp4_debug_set_flags(int(flags))
 
 
 def launch_count() -> int:

@@ -12,6 +12,7 @@ namespace nvfp4 {
 
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<uint64_t> g_timeout_ns{1000000000ull};
+static std::atomic<uint32_t> g_debug_flags{0};
 
 struct DeviceInfo {
     bool ready = false;
@@ -46,6 +47,7 @@ uint32_t* status_word_ptr() {
     return di ? di->status : nullptr;
 }
 uint64_t wait_timeout_ns() { return g_timeout_ns.load(); }
+uint32_t debug_flags() { return g_debug_flags.load(); }
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n); }
 int device_sm_count() {
     DeviceInfo* di = device_info();
@@ -80,6 +82,7 @@ extern "C" const char* nvfp4_status_string(nvfp4_status s) {
 
 extern "C" void nvfp4_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns == 0 ? 1 : ns); }
 extern "C" uint64_t nvfp4_get_wait_timeout_ns(void) { return g_timeout_ns.load(); }
+extern "C" void nvfp4_debug_set_flags(uint32_t flags) { g_debug_flags.store(flags & kCtlStallProducer); }
 extern "C" uint64_t nvfp4_launch_count(void) { return g_launches.load(); }
 
 extern "C" nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream) {

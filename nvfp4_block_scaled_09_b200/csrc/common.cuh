@@ -19,14 +19,19 @@ namespace nvfp4 {
 constexpr uint32_t kStatusTimeout = 1u;
 constexpr uint32_t kStatusBadInput = 2u;
 
+// Test-only behaviour flags (nvfp4_debug_set_flags); 0 on every normal launch.
+constexpr uint32_t kCtlStallProducer = 1u;   // GEMM producer issues no loads: every consumer wait runs out
+
 struct DeviceCtl {
     uint32_t* status;      // device status word (global memory)
     uint64_t timeout_ns;   // bound on one pipeline wait
+    uint32_t flags;        // kCtl* test flags
 };
 
 // Host-side registry (api.cu).
 uint32_t* status_word_ptr();          // nullptr on failure
 uint64_t wait_timeout_ns();
+uint32_t debug_flags();
 void count_launch(int n = 1);
 int device_sm_count();
 int device_smem_optin();

@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool issued[kStages];
 #pragma unroll
         for (int s = 0; s < kStages; s++) issued[s] = false, issued_parity[s] = 0;
-        if (lane == 0) {
+        if (lane == 0 && !(p.ctl.flags & kCtlStallProducer)) {
             // Weights read by one row tile only are streamed past L2; experts with
             // several row tiles re-read theirs from L2 (their tiles run back to back).
             const uint64_t pol_w_once = l2_policy_evict_first();
@@ -617,6 +617,7 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
     prm.swiglu = epi == NVFP4_EPI_SWIGLU ? 1 : 0;
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
+    prm.ctl.flags = debug_flags();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool wide = max_rows >= kWideMinAvgRows * (int64_t)E;
     const nvfp4_status ls =
