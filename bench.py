@@ -50,12 +50,20 @@ def parse():
     ap.add_argument("--config", default="moe_decode_t512", choices=[n for n in workloads.CONFIGS if n != "tiny"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--ref-seconds", type=float, default=None,
+                    help="CPU seconds per reference-arm step (default: 120 s spread over warm-up + steps, at most 30)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     # size overrides, used to make small cases of a workload for profiler captures
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--experts", type=int, default=None)
     return ap.parse_args()
+
+
+def ref_budget(args) -> float:
+    if args.ref_seconds is not None:
+        return max(0.05, float(args.ref_seconds))
+    return min(30.0, max(1.0, 120.0 / max(1, args.steps + args.warmup)))
 
 
 def load_peaks():
@@ -71,6 +79,22 @@ def load_peaks():
 FP4_PER_BF16 = 4.0  # nominal dense ratio (9 PF FP4 / 2.25 PF BF16)
 
 GEMM_SOURCES = ("nvfp4_block_scaled_09_b200/csrc/grouped_gemm.cu", "nvfp4_block_scaled_09_b200/csrc/common.cuh")
+
+
+def replica_seed(seed: int, rank: int) -> int:
+    """Each rank is an independent replica: its own token batch and routing (weights are shared)."""
+    return int(seed) + 7919 * int(rank)
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Max of a per-rank measurement over all ranks (the bench's timing rule); identity at world 1."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def gemm_source_sha256() -> str:
@@ -203,11 +227,11 @@ class MoEBench:
         T, k, H, I, E = cfg["T"], cfg["k"], cfg["H"], cfg["I"], cfg["E"]
         self.dev = device
         # Each rank is a replica: its own tokens and routing, the same weights.
-        ids, w = workloads.routing(T, E, k, cfg["routing"], seed + 7919 * rank, cfg.get("zipf_s", 1.1),
+        ids, w = workloads.routing(T, E, k, cfg["routing"], replica_seed(seed, rank), cfg.get("zipf_s", 1.1),
                                    cfg.get("zero_experts", 0))
         self.ids_np, self.w_np = ids, w
         self.counts = moe_counts(cfg, ids)
-        self.x = workloads.normal_bf16((T, H), 1.0, seed + 7919 * rank, workloads.TAG_X, device=device)
+        self.x = workloads.normal_bf16((T, H), 1.0, replica_seed(seed, rank), workloads.TAG_X, device=device)
         self.ids = torch.from_numpy(ids).to(device)
         self.w = torch.from_numpy(w).to(device)
         self.weights = self._weights(seed)
@@ -331,10 +355,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         for j in range(nev - 1):
             stage_ms[j] += evs[i][j].elapsed_time(evs[i][j + 1])
     stage_ms /= K
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, world, dev)
     st = nv.device_status()
     if st != 0:
         raise RuntimeError(f"device status {nv.status_string(st)} after the timed region")
@@ -365,14 +386,12 @@ def run_ours(args, cfg, rank, world, local_rank):
             out_h.copy_(bench.out, non_blocking=True)
         e1.record()
         barrier()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         f1, f2 = moe_flops(cfg)
-        e2e = {"value": world * (f1 + f2) * K / (float(te.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": world * (f1 + f2) * K / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(x_h.numel() * 2 + ids_h.numel() * 4 + w_h.numel() * 4),
                "d2h_bytes_per_step": int(out_h.numel() * 2), "api": "moe_layer_nvfp4",
-               "ms_per_step": float(te.item()) / K}
+               "ms_per_step": e2e_ms / K}
     return bench, max_ms, stage_ms, launches, clk, e2e
 
 
@@ -463,7 +482,7 @@ def main_dense(args, cfg, metric, world, rank, local_rank):
         dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank))
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    a = workloads.normal_bf16((M, K), 1.0, args.seed + 7919 * rank, workloads.TAG_A, device=dev)
+    a = workloads.normal_bf16((M, K), 1.0, replica_seed(args.seed, rank), workloads.TAG_A, device=dev)
     b = workloads.normal_bf16((1, N, K), 0.02, args.seed, workloads.TAG_B, device=dev)
     pw = nv.prepare_expert_weights(b)
     del b
@@ -509,15 +528,14 @@ def main_dense(args, cfg, metric, world, rank, local_rank):
     clk = clocks.stop() if clocks else None
     step_ms = sum(e[0].elapsed_time(e[2]) for e in evs)
     gemm_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+    max_step_ms = max_over_ranks(step_ms, world, dev)
     if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.destroy_process_group()
     if rank != 0:
         return 0
     K_steps = args.steps
     flops = 2.0 * M * N * K
-    value = world * flops * K_steps / (float(t.item()) * 1e-3) / 1e12
+    value = world * flops * K_steps / (max_step_ms * 1e-3) / 1e12
     peaks = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
     achieved = flops / (gemm_ms * 1e-3) / 1e12
@@ -529,7 +547,7 @@ def main_dense(args, cfg, metric, world, rank, local_rank):
               "sample": desc}
     line = {
         "metric": metric, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K_steps,
-        "warmup": args.warmup, "ms_per_step": float(t.item()) / K_steps, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": max_step_ms / K_steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, fp32 accumulate)",
         "data": "synthetic",
         "config": {"workload": "dense", "M": M, "N": N, "K": K,
@@ -565,7 +583,7 @@ def main():
         import oracle
         tot_f = tot_t = 0.0
         desc = ""
-        budget = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+        budget = ref_budget(args)
         for i in range(args.warmup + args.steps):
             f, dt, desc = oracle_dense_sample(cfg["M"], cfg["N"], cfg["K"], args.seed, budget)
             if i >= args.warmup:
@@ -586,7 +604,7 @@ def main():
             return 0
         import oracle
         K, W = args.steps, args.warmup
-        budget = max(1.0, 120.0 / max(1, K + W))
+        budget = ref_budget(args)
         for _ in range(W):
             oracle_sample(cfg, args.seed, budget_s=budget)
         tot_f, tot_t = 0.0, 0.0
