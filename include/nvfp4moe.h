@@ -284,6 +284,12 @@ typedef struct {                 /* fields up to `threads` describe the narrow (
     int32_t wide_stage_bytes_act_max;
     int32_t wide_smem_bytes;
     int32_t wide_min_avg_rows;
+    /* The CTA-pair tile (two SMs, tcgen05 cta_group::2: 256 weight rows x up to
+     * pair_tile_tokens_max activation rows), used when the experts average at
+     * least pair_min_avg_rows rows. */
+    int32_t pair_tile_tokens_max;
+    int32_t pair_smem_bytes;
+    int32_t pair_min_avg_rows;
 } nvfp4_gemm_plan;
 
 NVFP4_API nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan);

@@ -52,7 +52,8 @@ class GemmPlan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "tile_weight_rows", "tile_tokens_max", "stage_k", "stages", "stage_bytes_weights", "stage_bytes_weight_sf",
         "stage_bytes_act_max", "stage_bytes_act_sf", "smem_bytes", "tmem_columns", "threads",
-        "wide_tile_tokens_max", "wide_stage_bytes_act_max", "wide_smem_bytes", "wide_min_avg_rows")]
+        "wide_tile_tokens_max", "wide_stage_bytes_act_max", "wide_smem_bytes", "wide_min_avg_rows",
+        "pair_tile_tokens_max", "pair_smem_bytes", "pair_min_avg_rows")]
 
 
 _lib = None

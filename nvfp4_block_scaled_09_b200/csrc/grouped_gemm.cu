@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 16; i++) {
                         if (i < nrows) {
                             const float g = alpha * v0[i], u = alpha * v1[i];
-                            const float h = g / (1.0f + expf(-g)) * u;
+                            const float h = swiglu_f32(g, u);
                             o[(int64_t)i * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
                         }
                     }
@@ -512,8 +512,10 @@ static bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int6
     return r == CUDA_SUCCESS;
 }
 
-// Experts averaging at least this many rows use the wide tile shape.
+// Experts averaging at least this many rows use the wide tile shape, at least
+// kPairMinAvgRows the CTA-pair kernel (grouped_gemm_pair.cu).
 static constexpr int64_t kWideMinAvgRows = 96;
+static constexpr int64_t kPairMinAvgRows = 192;
 
 extern "C" nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan) {
     if (!plan) return NVFP4_ERR_INVALID_ARG;
@@ -532,6 +534,9 @@ extern "C" nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan) {
     plan->wide_stage_bytes_act_max = gg::Wide::kBBytes;
     plan->wide_smem_bytes = (int32_t)gg::Wide::kSmemBytes;
     plan->wide_min_avg_rows = (int32_t)kWideMinAvgRows;
+    plan->pair_tile_tokens_max = pair_gemm_tokens_max();
+    plan->pair_smem_bytes = (int32_t)pair_gemm_smem_bytes();
+    plan->pair_min_avg_rows = (int32_t)kPairMinAvgRows;
     return NVFP4_OK;
 }
 
@@ -551,8 +556,9 @@ extern "C" nvfp4_status nvfp4_can_implement_with_budget(int64_t N, int64_t K, in
     if (E > gg::kMaxE || N % (gg::kNumA * gg::kBM) != 0 || K % gg::kBK != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if ((int64_t)E * N > INT32_MAX || K / 2 > INT32_MAX) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     // both tile shapes must fit: the launcher picks one from the rows per expert
-    const int64_t need = (int64_t)(gg::Wide::kSmemBytes > gg::Narrow::kSmemBytes ? gg::Wide::kSmemBytes
-                                                                                  : gg::Narrow::kSmemBytes);
+    int64_t need = (int64_t)(gg::Wide::kSmemBytes > gg::Narrow::kSmemBytes ? gg::Wide::kSmemBytes
+                                                                            : gg::Narrow::kSmemBytes);
+    if ((int64_t)pair_gemm_smem_bytes() > need) need = (int64_t)pair_gemm_smem_bytes();
     if (smem_optin_bytes < need) return NVFP4_ERR_SMEM_BUDGET;
     return NVFP4_OK;
 }
@@ -619,6 +625,16 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (max_rows >= kPairMinAvgRows * (int64_t)E) {
+        CUtensorMap tm_sf;  // one stage of activation scales for a whole pair tile: 256 rows x 16 bytes
+        if (!encode_rows_map(&tm_sf, a_sf, max_rows, K / 16, (uint32_t)pair_gemm_tokens_max(), 16))
+            return NVFP4_ERR_CUDA;
+        CUtensorMap tm_a_full;  // one CTA's half of a full pair tile: 128 rows x 128 bytes
+        if (!encode_rows_map(&tm_a_full, a_q, max_rows, K / 2, (uint32_t)pair_gemm_tokens_max() / 2, 128))
+            return NVFP4_ERR_CUDA;
+        return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_sf, a_sf, a_gscale, w_packed, w_gscale, expert_offsets, E, max_rows,
+                                        N, K, prm.swiglu, out, s, status);
+    }
     const bool wide = max_rows >= kWideMinAvgRows * (int64_t)E;
     const nvfp4_status ls =
         wide ? launch_variant<gg::Wide>(tm_a, a_sf, prm, s) : launch_variant<gg::Narrow>(tm_a, a_sf, prm, s);

@@ -1,0 +1,515 @@
+// grouped_gemm_pair.cu -- the grouped NVFP4 GEMM on CTA pairs (tcgen05
+// cta_group::2) for experts with many rows (prefill) and dense GEMMs.
+//
+// Same computation as grouped_gemm.cu. A cluster of two CTAs on neighbouring
+// SMs shares one tile of 256 weight rows x up to 256 activation rows: each CTA
+// loads its own 128 weight rows and half of the activation rows, and the even
+// CTA issues M = 256 MMAs that read both CTAs' shared memory. Per SM this
+// halves the bytes moved per FLOP against a one-SM 256 x 128 tile (each SM
+// fetches 128 + 128 rows per K step for a 128 x 256 output), and the N = 256
+// MMA runs ~30% faster per FLOP than two N = 128 ones -- the two limits
+// (L2 -> SM traffic, MMA time) of the one-SM wide tile on prefill and dense.
+//
+// SwiGLU: CTA r covers output columns [n0 + 64r, +64). Its 128 A rows interleave
+// the gate and up rows 16 at a time (lanes 32q..32q+15: gate rows n0+64r+16q+j,
+// lanes 32q+16..32q+31: the matching up rows), so one warp reads both halves of
+// its 16 output columns and pairs them with a lane shuffle.
+//
+// Synchronisation uses no multicast: the peer's scale-writer and epilogue warps
+// arrive on the even CTA's barriers through cluster addresses (mapa), and the
+// even CTA's MMA completions are committed to each CTA's barrier separately.
+// Every wait is bounded as in the one-SM kernel; a cluster barrier guards the
+// release of tensor memory.
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace gp {
+
+constexpr int kBM = 128;                          // weight rows per CTA (MMA M = 256 per pair)
+constexpr int kBK = 256;                          // K elements per stage
+constexpr int kRowBytes = kBK / 2;
+constexpr int kKSteps = kBK / 64;
+constexpr int kBNMax = 256;                       // activation rows per pair tile (MMA N)
+constexpr int kBNStep = 32;                       // N granularity: each CTA holds a multiple of 16 rows
+constexpr int kBoxRows = 16;                      // activation TMA box rows
+constexpr int kStages = 5;
+constexpr int kPackedTileBytes = 18432;           // packed weight tile: 16 KB codes + 2 KB scales
+constexpr int kCodeBytes = 16384;
+constexpr int kTileSFBytes = 2048;
+constexpr int kOffA = 0;                          // 128 weight rows x 128 B (SwiGLU: gate half | up half)
+constexpr int kOffSFA = kCodeBytes;               // scales of one packed tile (SwiGLU: gate tile's, then up tile's)
+constexpr int kOffB = kOffSFA + 2 * kTileSFBytes;  // this CTA's half of the activation rows
+constexpr int kOffSFB = kOffB + (kBNMax / 2) * kRowBytes;  // row-major scales of all kBNMax rows
+constexpr int kStageBytes = kOffSFB + kBNMax * 16;         // 40960
+constexpr int kThreads = 512;                     // warps: 0 loads, 2 MMA, 4-7 + 12-15 epilogue, 8-11 scales
+constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant, alternating 32-token chunks
+constexpr int kMaxE = 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCols = kBNMax;             // one 128-lane x 256-column accumulator per CTA
+constexpr uint32_t kSFSlot = 4 * kKSteps + 8 * kKSteps;  // SFA: 4 columns per K step, SFB: 8 (256 rows)
+constexpr uint32_t kTmemSFRing = kAccCols;
+static_assert(kTmemSFRing + kStages * kSFSlot <= kTmemCols, "TMEM budget");
+static_assert(kStageBytes % 1024 == 0 && kOffB % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+
+struct Shared {
+    alignas(16) uint16_t ostage[kEpiWarps][32 * 32];  // epilogue: one 32-token x 32-column BF16 block per warp
+    uint64_t full_tma[kStages];   // this CTA's loads of the stage landed
+    uint64_t sf_ready[kStages];   // even CTA: both CTAs' scales are in TMEM (8 warp arrivals)
+    uint64_t empty[kStages];      // the pair's MMAs of the stage completed (commit from the even CTA)
+    uint64_t acc_full;            // the pair's MMAs of the tile completed
+    uint64_t acc_empty;           // even CTA: both CTAs' epilogues drained TMEM (2 x kEpiWarps arrivals)
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int32_t total_tiles;
+    int32_t off[kMaxE + 1];
+    int32_t tile_start[kMaxE + 1];
+};
+
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Shared);
+static_assert(kSmemBytes + 256 <= 232448, "shared memory budget");
+
+struct Params {
+    const uint8_t* a_sf;
+    const float* a_gscale;
+    const uint8_t* w_packed;
+    const float* w_gscale;
+    const int32_t* offsets;
+    uint16_t* out;
+    int32_t E;
+    int64_t max_rows;
+    int64_t N;
+    int64_t K;
+    int32_t swiglu;
+    DeviceCtl ctl;
+};
+
+struct Tile {
+    int32_t e, nt, mt, row0, rows, bn;
+};
+
+__device__ __forceinline__ void decode_tile(const Shared& sh, int32_t E, int32_t w, Tile& t) {
+    int32_t lo = 0, hi = E;  // tile_start[lo] <= w < tile_start[hi]
+    while (hi - lo > 1) {
+        const int32_t mid = (lo + hi) >> 1;
+        if (sh.tile_start[mid] <= w) lo = mid;
+        else hi = mid;
+    }
+    const int32_t M = sh.off[lo + 1] - sh.off[lo];
+    const int32_t mtiles = (M + kBNMax - 1) / kBNMax;
+    const int32_t local = w - sh.tile_start[lo];
+    t.e = lo;
+    t.nt = local / mtiles;
+    t.mt = local - t.nt * mtiles;
+    t.row0 = sh.off[lo] + t.mt * kBNMax;
+    t.rows = min(kBNMax, M - t.mt * kBNMax);
+    t.bn = (t.rows + kBNStep - 1) / kBNStep * kBNStep;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, const DeviceCtl& ctl) {
+    bool ok = mbar_wait_bounded(bar, parity, abort, ctl);
+    return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// Arrive on barrier `bar` of the even CTA (locally when this is the even CTA).
+__device__ __forceinline__ void arrive_on_leader(uint64_t* bar, uint32_t rank) {
+    if (rank == 0) mbar_arrive(bar);
+    else mbar_arrive_cluster(cluster_smem_addr(bar, 0));
+}
+
+// Expert offsets and the first work item of each expert (every CTA builds its own copy).
+__device__ __forceinline__ void build_schedule(Shared& sh, const Params& p, int32_t n_col_tiles) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int32_t E = p.E;
+    const int e0 = tid * 4;
+    int32_t cnt[4];
+    int32_t local = 0;
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const int e = e0 + i;
+        cnt[i] = 0;
+        if (e < E) {
+            const int32_t a = sh.off[e], b = sh.off[e + 1];
+            if (a < 0 || b < a || (int64_t)b > p.max_rows) bad = true;  // inconsistent offsets: skip the expert
+            else cnt[i] = ((b - a + kBNMax - 1) / kBNMax) * n_col_tiles;
+        }
+        local += cnt[i];
+    }
+    if (bad) atomicOr(p.ctl.status, kStatusBadInput);
+    int32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    __shared__ int32_t warp_tot[kThreads / 32];
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int32_t before = 0;
+    for (int w2 = 0; w2 < warp; w2++) before += warp_tot[w2];
+    int32_t run = before + incl - local;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const int e = e0 + i;
+        if (e < E) sh.tile_start[e] = run;
+        run += cnt[i];
+    }
+    if (tid == kThreads - 1) {
+        sh.total_tiles = before + incl;
+        sh.tile_start[E] = before + incl;
+    }
+}
+
+}  // namespace gp
+}  // namespace nvfp4
+
+namespace nvfp4 {
+namespace gp {
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_full,
+                             const __grid_constant__ CUtensorMap tm_sf, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    Shared& sh = *reinterpret_cast<Shared*>(smem + (size_t)kStages * kStageBytes);
+    volatile int* abort = &sh.abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const uint32_t pair = cluster_id_x(), npairs = num_clusters_x();
+    const int32_t E = p.E;
+    const int32_t n_col_tiles = (int32_t)(p.swiglu ? (p.N / 2) / kBM : p.N / (2 * kBM));
+    const int32_t ksteps_total = (int32_t)(p.K / kBK);
+
+    for (int i = tid; i <= E; i += kThreads) sh.off[i] = __ldg(p.offsets + i);
+    if (tid == 0) {
+        sh.abort = 0;
+        for (int s = 0; s < kStages; s++) {
+            mbar_init(&sh.full_tma[s], 1);
+            mbar_init(&sh.sf_ready[s], 8);
+            mbar_init(&sh.empty[s], 1);
+        }
+        mbar_init(&sh.acc_full, 1);
+        mbar_init(&sh.acc_empty, 2 * kEpiWarps);
+        mbar_init(&sh.drain, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    build_schedule(sh, p, n_col_tiles);
+    if (warp == 2) {
+        tmem_alloc_pair(&sh.tmem_base, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrival
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    const int32_t total = sh.total_tiles;
+
+    if (warp == 0) {
+        // ================= loads of this CTA's halves =================
+        uint32_t issued_parity[kStages];
+        bool issued[kStages];
+#pragma unroll
+        for (int s = 0; s < kStages; s++) issued[s] = false, issued_parity[s] = 0;
+        if (lane == 0 && !(p.ctl.flags & kCtlStallProducer)) {
+            const uint64_t pol_w = l2_policy_evict_normal();
+            const uint64_t pol_a = l2_policy_evict_last();
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int32_t w = pair; w < total && ok; w += npairs) {
+                Tile t;
+                decode_tile(sh, E, w, t);
+                // weight rows of this CTA, as (packed tile base, byte offset of the first row's codes)
+                const uint8_t* g_tile;   // NONE: the whole 128-row tile; SWIGLU: the gate tile
+                const uint8_t* u_tile = nullptr;
+                uint32_t half = 0;
+                if (p.swiglu) {
+                    const int64_t gate_base = (int64_t)t.e * p.N + (int64_t)t.nt * kBM;
+                    g_tile = p.w_packed + (gate_base / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
+                    u_tile = p.w_packed + ((gate_base + p.N / 2) / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
+                    half = rank * 64;
+                } else {
+                    const int64_t base = (int64_t)t.e * p.N + (int64_t)t.nt * 2 * kBM + rank * kBM;
+                    g_tile = p.w_packed + (base / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
+                }
+                const int32_t my_rows = t.bn / 2;
+                const int32_t my_row0 = t.row0 + (int32_t)rank * my_rows;
+                const uint32_t a_bytes = p.swiglu ? 2u * (kCodeBytes / 2 + kTileSFBytes) : (uint32_t)kPackedTileBytes;
+                const uint32_t tx = a_bytes + (uint32_t)my_rows * kRowBytes + kBNMax * 16;
+                for (int32_t kt = 0; kt < ksteps_total; kt++) {
+                    if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
+                    uint8_t* sb = stages + (size_t)stage * kStageBytes;
+                    uint64_t* bar = &sh.full_tma[stage];
+                    mbar_arrive_expect_tx(bar, tx);
+                    const size_t ko = (size_t)kt * kPackedTileBytes;
+                    if (p.swiglu) {
+                        // 16-row slabs (2 KB, whole swizzle atoms): gate slab q -> A rows 32q.., up slab q -> 32q+16..
+#pragma unroll
+                        for (int q = 0; q < 4; q++) {
+                            const size_t src = ko + (size_t)(half + 16 * q) * kRowBytes;
+                            bulk_load(sb + kOffA + 32 * q * kRowBytes, g_tile + src, 16 * kRowBytes, bar, pol_w);
+                            bulk_load(sb + kOffA + (32 * q + 16) * kRowBytes, u_tile + src, 16 * kRowBytes, bar, pol_w);
+                        }
+                        bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
+                        bulk_load(sb + kOffSFA + kTileSFBytes, u_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
+                    } else {
+                        bulk_load(sb + kOffA, g_tile + ko, kPackedTileBytes, bar, pol_w);
+                    }
+                    if (my_rows == kBNMax / 2) {
+                        tma_load_2d(sb + kOffB, &tm_a_full, kt * kRowBytes, my_row0, bar, pol_a);
+                    } else {
+                        for (int32_t i = 0; i < my_rows / kBoxRows; i++)
+                            tma_load_2d(sb + kOffB + i * kBoxRows * kRowBytes, &tm_a, kt * kRowBytes,
+                                        my_row0 + i * kBoxRows, bar, pol_a);
+                    }
+                    tma_load_2d(sb + kOffSFB, &tm_sf, kt * 16, t.row0, bar, pol_a);
+                    issued[stage] = true;
+                    issued_parity[stage] = phase;
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok || *abort) {
+                for (int s = 0; s < kStages; s++)
+                    if (issued[s]) mbar_wait_drain(&sh.full_tma[s], issued_parity[s], 200000000ull);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 8 && warp < 12) {
+        // ================= scale writers (one per TMEM lane quadrant) =================
+        // SFA: the weight row of lane m at column slot + 4 kc + m/32. SFB: activation row n (all
+        // kBNMax rows, both CTAs) at lane n % 32 of every quadrant, column slot + 16 + 8 kc + n/32.
+        const int quad = warp & 3;
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        // row of this lane inside its packed tile, and that tile's scale atom in the stage
+        const int tile_row = p.swiglu ? (int)rank * 64 + quad * 16 + (lane & 15) : quad * 32 + lane;
+        const uint32_t sfa_off = kOffSFA + ((p.swiglu && lane >= 16) ? kTileSFBytes : 0) + (tile_row & 31) * 16 +
+                                 (tile_row >> 5) * 4;
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
+        for (int32_t w = pair; w < total && ok; w += npairs) {
+            for (int32_t kt = 0; kt < ksteps_total; kt++) {
+                if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl)) { ok = false; break; }
+                tc_fence_after();
+                const uint8_t* sb = stages + (size_t)stage * kStageBytes;
+                const uint32_t slot = tmem + lane_addr + kTmemSFRing + stage * kSFSlot;
+                uint32_t v16[16];
+#pragma unroll
+                for (int kc = 0; kc < kKSteps; kc++) {
+                    const uint32_t word = *reinterpret_cast<const uint32_t*>(sb + sfa_off + kc * 512);
+#pragma unroll
+                    for (int q = 0; q < 4; q++) v16[4 * kc + q] = (q == quad) ? word : 0u;
+                }
+                tmem_st_32x32b_x16(slot, v16);
+                uint32_t v32[32];
+#pragma unroll
+                for (int g = 0; g < 8; g++) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(sb + kOffSFB + (32 * g + lane) * 16);
+                    v32[g] = x.x;
+                    v32[8 + g] = x.y;
+                    v32[16 + g] = x.z;
+                    v32[24 + g] = x.w;
+                }
+                tmem_st_32x32b_x32(slot + 16, v32);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) arrive_on_leader(&sh.sf_ready[stage], rank);
+                if (++stage == kStages) { stage = 0; phase ^= 1u; }
+            }
+        }
+    } else if (warp == 2) {
+        // ================= MMA issuer (even CTA) =================
+        if (rank == 0) {
+            const uint32_t idesc_base = (1u << 7) | (1u << 10) | ((uint32_t)((2 * kBM) >> 4) << 24);
+            const uint32_t peer_empty0 = cluster_smem_addr(&sh.empty[0], 1);
+            const uint32_t own_empty0 = cluster_smem_addr(&sh.empty[0], 0);
+            uint32_t stage = 0, phase = 0, aphase = 0;
+            bool ok = true;
+            for (int32_t w = pair; w < total && ok; w += npairs) {
+                Tile t;
+                decode_tile(sh, E, w, t);
+                const uint32_t idesc = idesc_base | ((uint32_t)(t.bn >> 3) << 17);
+                if (!warp_wait(&sh.acc_empty, aphase ^ 1u, abort, p.ctl)) { ok = false; break; }
+                tc_fence_after();
+                for (int32_t kt = 0; kt < ksteps_total; kt++) {
+                    if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl) ||
+                        !warp_wait(&sh.sf_ready[stage], phase, abort, p.ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t sb = smem_u32(stages + (size_t)stage * kStageBytes);
+                        const uint32_t sf = tmem + kTmemSFRing + stage * kSFSlot;
+#pragma unroll
+                        for (int kc = 0; kc < kKSteps; kc++) {
+                            mma_mxf4nvf4_pair(tmem, make_smem_desc(sb + kOffA + kc * 32, 16, 1024, 2),
+                                              make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2), idesc,
+                                              sf + 4 * kc, sf + 16 + 8 * kc, (kt | kc) != 0);
+                        }
+                        tc_commit_pair(own_empty0 + stage * 8);
+                        tc_commit_pair(peer_empty0 + stage * 8);
+                    }
+                    __syncwarp();
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                if (lane == 0) {
+                    tc_commit_pair(cluster_smem_addr(&sh.acc_full, 0));
+                    tc_commit_pair(cluster_smem_addr(&sh.acc_full, 1));
+                }
+                __syncwarp();
+                aphase ^= 1u;
+            }
+            if (!ok || *abort) {
+                if (lane == 0) {
+                    tc_commit_pair(cluster_smem_addr(&sh.drain, 0));
+                    mbar_wait_drain(&sh.drain, 0, 200000000ull);
+                }
+                __syncwarp();
+            }
+        }
+    } else if (warp >= 4) {  // warps 4-7 and 12-15
+        // ================= epilogue (both CTAs) =================
+        // TMEM lane = A row of this CTA, column = token of the tile. Per 32-token chunk each warp
+        // converts its 32 lanes to BF16 in a private shared block and writes 16-byte row pieces.
+        const int quad = warp & 3;
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        const int half = warp >= 12 ? 1 : 0;  // this warp takes the chunks c with c % 2 == half
+        uint16_t* stg = sh.ostage[half * 4 + quad];
+        const bool up_lane = lane >= 16;
+        const float a_g = __ldg(p.a_gscale);
+        uint32_t aphase = 0;
+        for (int32_t w = pair; w < total; w += npairs) {
+            Tile t;
+            decode_tile(sh, E, w, t);
+            if (!warp_wait(&sh.acc_full, aphase, abort, p.ctl)) break;
+            tc_fence_after();
+            const float alpha = a_g * __ldg(p.w_gscale + t.e);
+            for (int c = half; c * 32 < t.bn; c += 2) {
+                float v[32];
+                tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v);
+                tmem_ld_wait();
+                const int nrows = min(32, t.rows - c * 32);
+                const int64_t r0 = (int64_t)t.row0 + c * 32;
+                if (p.swiglu) {
+                    // lane l < 16 holds gate, lane l + 16 up, of output column 16 quad + l; lane l
+                    // produces the even tokens, lane l + 16 the odd ones
+#pragma unroll
+                    for (int j = 0; j < 16; j++) {
+                        const float send = up_lane ? v[2 * j] : v[2 * j + 1];
+                        const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
+                        const float g = alpha * (up_lane ? recv : v[2 * j]);
+                        const float u = alpha * (up_lane ? v[2 * j + 1] : recv);
+                        const float h = swiglu_f32(g, u);
+                        stg[(2 * j + (up_lane ? 1 : 0)) * 16 + (lane & 15)] =
+                            __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                    }
+                    __syncwarp();
+                    const int64_t ldo = p.N / 2;
+                    const int64_t col = (int64_t)t.nt * kBM + rank * 64 + quad * 16 + 8 * (lane & 1);
+#pragma unroll
+                    for (int it = 0; it < 2; it++) {
+                        const int r = (lane >> 1) + 16 * it;
+                        if (r < nrows)
+                            *reinterpret_cast<uint4*>(p.out + (r0 + r) * ldo + col) =
+                                *reinterpret_cast<const uint4*>(stg + r * 16 + 8 * (lane & 1));
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; i++) stg[i * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i]));
+                    __syncwarp();
+                    const int64_t ldo = p.N;
+                    const int64_t col = (int64_t)t.nt * 2 * kBM + rank * kBM + quad * 32 + 8 * (lane & 3);
+#pragma unroll
+                    for (int it = 0; it < 4; it++) {
+                        const int r = (lane >> 2) + 8 * it;
+                        if (r < nrows)
+                            *reinterpret_cast<uint4*>(p.out + (r0 + r) * ldo + col) =
+                                *reinterpret_cast<const uint4*>(stg + r * 32 + 8 * (lane & 3));
+                    }
+                }
+                __syncwarp();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_on_leader(&sh.acc_empty, rank);
+            aphase ^= 1u;
+        }
+    }
+
+    // ---- teardown: both CTAs have drained their own work; then the pair frees its TMEM ----
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc_pair(tmem, kTmemCols);
+}
+
+}  // namespace gp
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+namespace nvfp4 {
+
+size_t pair_gemm_smem_bytes() { return gp::kSmemBytes; }
+int pair_gemm_tokens_max() { return gp::kBNMax; }
+
+// Launches the pair kernel; the caller validated every argument (same contract as the one-SM kernel).
+nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full, const CUtensorMap& tm_sf,
+                                      const uint8_t* a_sf,
+                                      const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
+                                      const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
+                                      int swiglu, uint16_t* out, cudaStream_t s, uint32_t* status) {
+    static bool configured[64] = {};
+    static int grid_for[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(gp::grouped_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gp::kSmemBytes) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        // as many pairs as can be resident at once (persistent grid)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)device_sm_count() / 2 * 2);
+        cfg.blockDim = dim3(gp::kThreads);
+        cfg.dynamicSmemBytes = gp::kSmemBytes;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, gp::grouped_gemm_pair_kernel, &cfg) != cudaSuccess ||
+            clusters <= 0)
+            return NVFP4_ERR_SMEM_BUDGET;
+        grid_for[dev] = 2 * clusters < device_sm_count() ? 2 * clusters : device_sm_count() / 2 * 2;
+        configured[dev] = true;
+    }
+    gp::Params prm;
+    prm.a_sf = a_sf;
+    prm.a_gscale = a_gscale;
+    prm.w_packed = w_packed;
+    prm.w_gscale = w_gscale;
+    prm.offsets = offsets;
+    prm.out = out;
+    prm.E = E;
+    prm.max_rows = max_rows;
+    prm.N = N;
+    prm.K = K;
+    prm.swiglu = swiglu;
+    prm.ctl.status = status;
+    prm.ctl.timeout_ns = wait_timeout_ns();
+    prm.ctl.flags = debug_flags();
+    gp::grouped_gemm_pair_kernel<<<grid_for[dev], gp::kThreads, gp::kSmemBytes, s>>>(tm_a, tm_a_full, tm_sf, prm);
+    count_launch();
+    return check_launch();
+}
+
+}  // namespace nvfp4

@@ -88,6 +88,13 @@ def test_wide_tiles_ragged(swiglu):
 
 
 @pytest.mark.parametrize("swiglu", [False, True])
+def test_pair_tiles_ragged(swiglu):
+    # experts averaging >= 192 rows run on CTA pairs (256 weight rows x up to 256 activation rows):
+    # empty, partial, exact, 256 + 1, two tiles, a small expert
+    run_full([0, 200, 256, 257, 500, 40], 512, 768, swiglu, seed=7)
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
 def test_deeper_k_and_wider_n(swiglu):
     run_full([5, 40, 200], 768, 2048, swiglu, seed=2)
 

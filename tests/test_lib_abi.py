@@ -41,7 +41,10 @@ def test_can_implement_shapes_and_budget(L):
     assert nv.can_implement(4096, 6144, 1025, True, big) == 3
     assert nv.can_implement(0, 6144, 8, True, big) == 1
     # a budget below either tile shape's shared memory is refused before any launch
-    assert nv.can_implement(4096, 6144, 256, True, max(plan["smem_bytes"], plan["wide_smem_bytes"]) - 1) == 5
+    need = max(plan["smem_bytes"], plan["wide_smem_bytes"], plan["pair_smem_bytes"])
+    assert need <= big
+    assert nv.can_implement(4096, 6144, 256, True, need - 1) == 5
+    assert plan["pair_min_avg_rows"] > plan["wide_min_avg_rows"] and plan["pair_tile_tokens_max"] == 256
     assert nv.can_implement(4096, 6144, 256, True, 101376) == 5     # an SM120-sized budget
 
 
