@@ -512,6 +512,42 @@ static bool encode_rows_map(CUtensorMap* m, const void* base, int64_t rows, int6
     return r == CUDA_SUCCESS;
 }
 
+// 2-D BF16 output [rows, cols] stored in boxes of 32 rows x box_cols columns (no swizzle).
+static bool encode_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, uint32_t box_cols) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {box_cols, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Packed SwiGLU weights [E, N, K] viewed as 5-D bytes for the CTA-pair kernel: {128 bytes of a row,
+// 16 rows of a slab, gate/up (the up tile of the same columns lies N/2 rows further), 8 slabs of a
+// packed tile, packed tile index}. A box {128, 16, 2, 4, 1} gathers one CTA's 64 gate rows and the
+// matching 64 up rows, interleaved 16 at a time. Tiles run only over gate tiles plus the ones whose
+// up tile still lies inside the tensor, so no box can leave the allocation.
+static bool encode_swiglu_weights_map(CUtensorMap* m, const void* w_packed, int32_t E, int64_t N, int64_t K) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    const int64_t ksteps = K / 256;
+    const int64_t tile_bytes = 18432;
+    const int64_t up_stride = (N / 2 / 128) * ksteps * tile_bytes;
+    const int64_t tiles = ((int64_t)E * N - N / 2) / 128 * ksteps;
+    cuuint64_t dims[5] = {128u, 16u, 2u, 8u, (cuuint64_t)tiles};
+    cuuint64_t strides[4] = {128u, (cuuint64_t)up_stride, 2048u, (cuuint64_t)tile_bytes};
+    cuuint32_t box[5] = {128u, 16u, 2u, 4u, 1u};
+    cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(w_packed), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Experts averaging at least this many rows use the wide tile shape, at least
 // kPairMinAvgRows the CTA-pair kernel (grouped_gemm_pair.cu).
 static constexpr int64_t kWideMinAvgRows = 96;
@@ -632,7 +668,13 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
         CUtensorMap tm_a_full;  // one CTA's half of a full pair tile: 128 rows x 128 bytes
         if (!encode_rows_map(&tm_a_full, a_q, max_rows, K / 2, (uint32_t)pair_gemm_tokens_max() / 2, 128))
             return NVFP4_ERR_CUDA;
-        return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_sf, a_sf, a_gscale, w_packed, w_gscale, expert_offsets, E, max_rows,
+        CUtensorMap tm_out;  // one epilogue warp's 32-token block of the output
+        const int64_t out_cols = prm.swiglu ? N / 2 : N;
+        if (!encode_out_map(&tm_out, out, max_rows, out_cols, (uint32_t)pair_gemm_store_cols(prm.swiglu)))
+            return NVFP4_ERR_CUDA;
+        CUtensorMap tm_wsw = tm_a;  // SWIGLU: interleaved gate/up weight slabs (unused otherwise)
+        if (prm.swiglu && !encode_swiglu_weights_map(&tm_wsw, w_packed, E, N, K)) return NVFP4_ERR_CUDA;
+        return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_sf, tm_out, tm_wsw, a_sf, a_gscale, w_packed, w_gscale, expert_offsets, E, max_rows,
                                         N, K, prm.swiglu, out, s, status);
     }
     const bool wide = max_rows >= kWideMinAvgRows * (int64_t)E;

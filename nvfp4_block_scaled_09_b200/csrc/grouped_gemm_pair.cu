@@ -36,7 +36,7 @@ constexpr int kStages = 5;
 constexpr int kPackedTileBytes = 18432;           // packed weight tile: 16 KB codes + 2 KB scales
 constexpr int kCodeBytes = 16384;
 constexpr int kTileSFBytes = 2048;
-constexpr int kOffA = 0;                          // 128 weight rows x 128 B (SwiGLU: gate half | up half)
+constexpr int kOffA = 0;                          // 128 weight rows x 128 B (SwiGLU: gate/up slabs of 16 rows, interleaved)
 constexpr int kOffSFA = kCodeBytes;               // scales of one packed tile (SwiGLU: gate tile's, then up tile's)
 constexpr int kOffB = kOffSFA + 2 * kTileSFBytes;  // this CTA's half of the activation rows
 constexpr int kOffSFB = kOffB + (kBNMax / 2) * kRowBytes;  // row-major scales of all kBNMax rows
@@ -169,7 +169,8 @@ namespace gp {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_full,
-                             const __grid_constant__ CUtensorMap tm_sf, const Params p) {
+                             const __grid_constant__ CUtensorMap tm_sf, const __grid_constant__ CUtensorMap tm_out,
+                             const __grid_constant__ CUtensorMap tm_wsw, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
@@ -226,11 +227,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint8_t* g_tile;   // NONE: the whole 128-row tile; SWIGLU: the gate tile
                 const uint8_t* u_tile = nullptr;
                 uint32_t half = 0;
+                int32_t sw_tile0 = 0;    // SWIGLU: packed-tile index of the gate tile at K step 0
                 if (p.swiglu) {
                     const int64_t gate_base = (int64_t)t.e * p.N + (int64_t)t.nt * kBM;
                     g_tile = p.w_packed + (gate_base / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
                     u_tile = p.w_packed + ((gate_base + p.N / 2) / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
                     half = rank * 64;
+                    sw_tile0 = (int32_t)((gate_base / kBM) * ksteps_total);
                 } else {
                     const int64_t base = (int64_t)t.e * p.N + (int64_t)t.nt * 2 * kBM + rank * kBM;
                     g_tile = p.w_packed + (base / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
@@ -246,13 +249,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(bar, tx);
                     const size_t ko = (size_t)kt * kPackedTileBytes;
                     if (p.swiglu) {
-                        // 16-row slabs (2 KB, whole swizzle atoms): gate slab q -> A rows 32q.., up slab q -> 32q+16..
-#pragma unroll
-                        for (int q = 0; q < 4; q++) {
-                            const size_t src = ko + (size_t)(half + 16 * q) * kRowBytes;
-                            bulk_load(sb + kOffA + 32 * q * kRowBytes, g_tile + src, 16 * kRowBytes, bar, pol_w);
-                            bulk_load(sb + kOffA + (32 * q + 16) * kRowBytes, u_tile + src, 16 * kRowBytes, bar, pol_w);
-                        }
+                        // 16-row slabs (2 KB, whole swizzle atoms) of this CTA's half: gate slab q -> A rows
+                        // 32q.., up slab q -> 32q+16.. (one box: bytes x rows x gate/up x slab x tile)
+                        tma_load_5d(sb + kOffA, &tm_wsw, 0, 0, 0, (int32_t)(half / 16), sw_tile0 + kt, bar, pol_w);
                         bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
                         bulk_load(sb + kOffSFA + kTileSFBytes, u_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
                     } else {
@@ -394,7 +393,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v);
                 tmem_ld_wait();
                 const int nrows = min(32, t.rows - c * 32);
-                const int64_t r0 = (int64_t)t.row0 + c * 32;
+                const int32_t r0 = t.row0 + c * 32;
+                // the previous chunk's tensor store has finished reading the staging block
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+                int32_t col;      // first output column of this warp's block
+                int lane_cols;    // lanes per 16-byte row piece in the direct-store path: 2 (SwiGLU) or 4
                 if (p.swiglu) {
                     // lane l < 16 holds gate, lane l + 16 up, of output column 16 quad + l; lane l
                     // produces the even tokens, lane l + 16 the odd ones
@@ -408,37 +412,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         stg[(2 * j + (up_lane ? 1 : 0)) * 16 + (lane & 15)] =
                             __bfloat16_as_ushort(__float2bfloat16_rn(h));
                     }
-                    __syncwarp();
-                    const int64_t ldo = p.N / 2;
-                    const int64_t col = (int64_t)t.nt * kBM + rank * 64 + quad * 16 + 8 * (lane & 1);
-#pragma unroll
-                    for (int it = 0; it < 2; it++) {
-                        const int r = (lane >> 1) + 16 * it;
-                        if (r < nrows)
-                            *reinterpret_cast<uint4*>(p.out + (r0 + r) * ldo + col) =
-                                *reinterpret_cast<const uint4*>(stg + r * 16 + 8 * (lane & 1));
-                    }
+                    col = t.nt * kBM + (int32_t)rank * 64 + quad * 16;
+                    lane_cols = 2;
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; i++) stg[i * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i]));
-                    __syncwarp();
-                    const int64_t ldo = p.N;
-                    const int64_t col = (int64_t)t.nt * 2 * kBM + rank * kBM + quad * 32 + 8 * (lane & 3);
-#pragma unroll
-                    for (int it = 0; it < 4; it++) {
-                        const int r = (lane >> 2) + 8 * it;
-                        if (r < nrows)
-                            *reinterpret_cast<uint4*>(p.out + (r0 + r) * ldo + col) =
-                                *reinterpret_cast<const uint4*>(stg + r * 32 + 8 * (lane & 3));
-                    }
+                    col = t.nt * 2 * kBM + (int32_t)rank * kBM + quad * 32;
+                    lane_cols = 4;
                 }
-                __syncwarp();
+                if (nrows == 32) {
+                    // a whole chunk of the expert: one asynchronous tensor store of the block
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tm_out, stg, col, r0);
+                        bulk_commit_group();
+                    }
+                } else {
+                    // the expert's last, partial chunk: rows past its end belong to the next expert
+                    __syncwarp();
+                    const int64_t ldo = p.swiglu ? p.N / 2 : p.N;
+                    const int row_elems = 8 * lane_cols;
+                    const int rows_per_pass = 32 / lane_cols;
+                    for (int r = lane / lane_cols; r < nrows; r += rows_per_pass) {
+                        const int piece = 8 * (lane % lane_cols);
+                        *reinterpret_cast<uint4*>(p.out + (int64_t)(r0 + r) * ldo + col + piece) =
+                            *reinterpret_cast<const uint4*>(stg + r * row_elems + piece);
+                    }
+                    __syncwarp();
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) arrive_on_leader(&sh.acc_empty, rank);
             aphase ^= 1u;
         }
+        if (lane == 0) bulk_wait_group0();  // this warp's tensor stores completed
+        __syncwarp();
     }
 
     // ---- teardown: both CTAs have drained their own work; then the pair frees its TMEM ----
@@ -458,10 +468,11 @@ namespace nvfp4 {
 
 size_t pair_gemm_smem_bytes() { return gp::kSmemBytes; }
 int pair_gemm_tokens_max() { return gp::kBNMax; }
+int pair_gemm_store_cols(int swiglu) { return swiglu ? 16 : 32; }  // 32 tokens x this many BF16 columns
 
 // Launches the pair kernel; the caller validated every argument (same contract as the one-SM kernel).
 nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full, const CUtensorMap& tm_sf,
-                                      const uint8_t* a_sf,
+                                      const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const uint8_t* a_sf,
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
                                       int swiglu, uint16_t* out, cudaStream_t s, uint32_t* status) {
@@ -507,7 +518,7 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
-    gp::grouped_gemm_pair_kernel<<<grid_for[dev], gp::kThreads, gp::kSmemBytes, s>>>(tm_a, tm_a_full, tm_sf, prm);
+    gp::grouped_gemm_pair_kernel<<<grid_for[dev], gp::kThreads, gp::kSmemBytes, s>>>(tm_a, tm_a_full, tm_sf, tm_out, tm_wsw, prm);
     count_launch();
     return check_launch();
 }
