@@ -40,6 +40,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const uint4* __restri
                                                            const int32_t* __restrict__ inv_perm,
                                                            const float* __restrict__ w, int32_t k, int64_t hvec,
                                                            uint4* __restrict__ out) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int64_t t = blockIdx.y;
     const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;  // 16-byte column group
     if (c >= hvec) return;
@@ -79,7 +81,7 @@ extern "C" nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* 
         return NVFP4_ERR_MISALIGNED;
     const int64_t hvec = H / kColsPerThread;
     dim3 grid((unsigned)((hvec + kThreads - 1) / kThreads), (unsigned)T);
-    combine_kernel<<<grid, kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+    launch_pdl(combine_kernel, dim3(grid), dim3(kThreads), 0, reinterpret_cast<cudaStream_t>(stream),
         reinterpret_cast<const uint4*>(y), inv_perm, topk_w, k, hvec, reinterpret_cast<uint4*>(out));
     count_launch();
     return check_launch();

@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -45,6 +46,25 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
                                       int swiglu, uint16_t* out, cudaStream_t s, uint32_t* status);
+
+#ifdef __CUDACC__
+// Launch `kernel` on `s` with programmatic stream serialization (see pdl_wait()).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+#endif
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
@@ -121,6 +141,18 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
         if (global_timer_ns() - t0 > budget_ns) return false;
     }
     return true;
+}
+
+// Programmatic dependent launch. Kernels of the layer are launched with launch_pdl(), so a kernel
+// may become resident while the previous one in the stream is still running. pdl_wait() blocks
+// until that kernel -- and, since it waited in turn, every earlier one -- has completed and its
+// writes are visible; every kernel calls it before its first global-memory access (and before any
+// early return, so that no grid can complete ahead of its predecessor). pdl_launch_dependents()
+// lets the next kernel start its prologue; it carries no memory ordering.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 // TMA: 2-D tiled tensor load into shared memory, completion on an mbarrier.

@@ -184,9 +184,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t E = p.E;
     const int32_t n_col_tiles = (int32_t)(p.swiglu ? (p.N / 2) / kBM : p.N / (kNumA * kBM));
 
-    // ---- scheduler tables: expert offsets and the first work item of each expert ----
-    for (int i = tid; i <= E; i += kThreads) sh.off[i] = __ldg(p.offsets + i);
     if (tid == 0) {
+        prefetch_tensormap(&tm_a);
+        prefetch_tensormap(&tm_sf);
         sh.abort = 0;
         for (int s = 0; s < kStages; s++) {
             mbar_init(&sh.full_tma[s], 1);
@@ -200,6 +200,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sh.drain, 1);
         fence_barrier_init();
     }
+    // everything above overlaps the previous kernel; global memory only from here on
+    pdl_launch_dependents();
+    pdl_wait();
+    // ---- scheduler tables: expert offsets and the first work item of each expert ----
+    for (int i = tid; i <= E; i += kThreads) sh.off[i] = __ldg(p.offsets + i);
     __syncthreads();
     {
         // Each thread sums the tiles of 4 consecutive experts, then a block-wide exclusive scan.
@@ -619,7 +624,8 @@ static nvfp4_status launch_variant(const CUtensorMap& tm_a, const uint8_t* a_sf,
     }
     CUtensorMap tm_sf;  // one stage of activation scales: kBNMax rows x 16 bytes
     if (!encode_rows_map(&tm_sf, a_sf, prm.max_rows, prm.K / 16, C::kBNMax, 16)) return NVFP4_ERR_CUDA;
-    gg::grouped_gemm_kernel<C><<<device_sm_count(), gg::kThreads, C::kSmemBytes, s>>>(tm_a, tm_sf, prm);
+    launch_pdl(gg::grouped_gemm_kernel<C>, dim3(device_sm_count()), dim3(gg::kThreads), C::kSmemBytes, s, tm_a, tm_sf,
+               prm);
     return NVFP4_OK;
 }
 

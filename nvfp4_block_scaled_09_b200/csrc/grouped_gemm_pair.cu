@@ -183,8 +183,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int32_t n_col_tiles = (int32_t)(p.swiglu ? (p.N / 2) / kBM : p.N / (2 * kBM));
     const int32_t ksteps_total = (int32_t)(p.K / kBK);
 
-    for (int i = tid; i <= E; i += kThreads) sh.off[i] = __ldg(p.offsets + i);
     if (tid == 0) {
+        prefetch_tensormap(&tm_a);
+        prefetch_tensormap(&tm_a_full);
+        prefetch_tensormap(&tm_sf);
+        prefetch_tensormap(&tm_out);
+        if (p.swiglu) prefetch_tensormap(&tm_wsw);
         sh.abort = 0;
         for (int s = 0; s < kStages; s++) {
             mbar_init(&sh.full_tma[s], 1);
@@ -196,6 +200,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_init(&sh.drain, 1);
         fence_barrier_init();
     }
+    // everything above overlaps the previous kernel; global memory only from here on
+    pdl_launch_dependents();
+    pdl_wait();
+    for (int i = tid; i <= E; i += kThreads) sh.off[i] = __ldg(p.offsets + i);
     __syncthreads();
     build_schedule(sh, p, n_col_tiles);
     if (warp == 2) {
@@ -518,7 +526,8 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
-    gp::grouped_gemm_pair_kernel<<<grid_for[dev], gp::kThreads, gp::kSmemBytes, s>>>(tm_a, tm_a_full, tm_sf, tm_out, tm_wsw, prm);
+    launch_pdl(gp::grouped_gemm_pair_kernel, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes, s, tm_a, tm_a_full,
+               tm_sf, tm_out, tm_wsw, prm);
     count_launch();
     return check_launch();
 }

@@ -28,6 +28,8 @@ constexpr int kWordsPerExpert = kTok / 32;
 __global__ void __launch_bounds__(kTok) permute_count_kernel(const int32_t* __restrict__ ids, int32_t T, int32_t k,
                                                                int32_t E, int32_t* __restrict__ counts,
                                                                uint32_t* status) {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ int32_t hist[kMaxE];
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
@@ -46,6 +48,8 @@ __global__ void __launch_bounds__(kTok) permute_count_kernel(const int32_t* __re
 // One CTA of kMaxE threads: thread e owns expert e.
 __global__ void __launch_bounds__(kMaxE) permute_scan_kernel(int32_t* __restrict__ counts, int32_t nchunks,
                                                                int32_t E, int32_t* __restrict__ offsets) {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ int32_t warp_sums[kMaxE / 32];
     const int e = threadIdx.x;
     int32_t total = 0;
@@ -88,6 +92,8 @@ __global__ void __launch_bounds__(kTok) permute_rank_kernel(const int32_t* __res
                                                               int32_t E, const int32_t* __restrict__ base,
                                                               int32_t* __restrict__ perm_src,
                                                               int32_t* __restrict__ inv_perm, uint32_t* status) {
+    pdl_launch_dependents();
+    pdl_wait();
     extern __shared__ uint32_t bits[];  // [E][kWordsPerExpert]
     for (int i = threadIdx.x; i < E * kWordsPerExpert; i += blockDim.x) bits[i] = 0u;
     __syncthreads();
@@ -128,6 +134,8 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(const uint4* __rest
                                                              const int32_t* __restrict__ perm_src, int32_t T,
                                                              int64_t R, uint4* __restrict__ q_perm,
                                                              uint4* __restrict__ sf_perm) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int64_t p = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (p >= R) return;
     const int lane = threadIdx.x & 31;
@@ -177,12 +185,12 @@ extern "C" nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t 
     int32_t* counts = static_cast<int32_t*>(ws);
     const int64_t R = (int64_t)T * k;
 
-    permute_count_kernel<<<nchunks, kTok, 0, s>>>(topk_ids, T, k, E, counts, status);
-    permute_scan_kernel<<<1, kMaxE, 0, s>>>(counts, nchunks, E, expert_offsets);
+    launch_pdl(permute_count_kernel, dim3(nchunks), dim3(kTok), 0, s, topk_ids, T, k, E, counts, status);
+    launch_pdl(permute_scan_kernel, dim3(1), dim3(kMaxE), 0, s, counts, nchunks, E, expert_offsets);
     const size_t rank_smem = (size_t)E * kWordsPerExpert * sizeof(uint32_t);
-    permute_rank_kernel<<<nchunks, kTok, rank_smem, s>>>(topk_ids, T, k, E, counts, perm_src, inv_perm, status);
+    launch_pdl(permute_rank_kernel, dim3(nchunks), dim3(kTok), rank_smem, s, topk_ids, T, k, E, counts, perm_src, inv_perm, status);
     const int64_t gblocks = (R + 7) / 8;
-    permute_gather_kernel<<<(unsigned)gblocks, 256, 0, s>>>(
+    launch_pdl(permute_gather_kernel, dim3((unsigned)gblocks), dim3(256), 0, s,
         reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(sf), K / 32, K / 256, perm_src, T, R,
         reinterpret_cast<uint4*>(q_perm), reinterpret_cast<uint4*>(sf_perm));
     count_launch(4);
@@ -236,11 +244,11 @@ extern "C" nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, 
     if (!counts || !status) return NVFP4_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int64_t R = (int64_t)T * k;
-    permute_count_kernel<<<nchunks, kTok, 0, s>>>(topk_ids, T, k, E, counts, status);
-    permute_scan_kernel<<<1, kMaxE, 0, s>>>(counts, nchunks, E, expert_offsets);
+    launch_pdl(permute_count_kernel, dim3(nchunks), dim3(kTok), 0, s, topk_ids, T, k, E, counts, status);
+    launch_pdl(permute_scan_kernel, dim3(1), dim3(kMaxE), 0, s, counts, nchunks, E, expert_offsets);
     const size_t rank_smem = (size_t)E * kWordsPerExpert * sizeof(uint32_t);
-    permute_rank_kernel<<<nchunks, kTok, rank_smem, s>>>(topk_ids, T, k, E, counts, perm_src, inv_perm, status);
-    permute_gather_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(
+    launch_pdl(permute_rank_kernel, dim3(nchunks), dim3(kTok), rank_smem, s, topk_ids, T, k, E, counts, perm_src, inv_perm, status);
+    launch_pdl(permute_gather_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, s,
         reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(sf), K / 32, K / 256, perm_src, T, R,
         reinterpret_cast<uint4*>(q_perm), reinterpret_cast<uint4*>(sf_perm));
     count_launch(4);

@@ -37,6 +37,8 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
 
 __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const uint4* __restrict__ x, int64_t nvec,
                                                                  uint32_t* __restrict__ partial) {
+    pdl_launch_dependents();
+    pdl_wait();
     uint32_t m = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += stride) {
@@ -110,6 +112,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
                                                             const uint32_t* __restrict__ partial, int npartial,
                                                             uint2* __restrict__ q, uint8_t* __restrict__ sf,
                                                             float* __restrict__ gdec_out) {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ float s_genc;
     if (threadIdx.x < 32) {
         float amax = 0.0f;
@@ -209,7 +213,7 @@ extern "C" nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint32_t* partial = static_cast<uint32_t*>(ws);
     if (global_scale_in == nullptr) {
-        amax_partial_kernel<<<grid_a, kThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), nvec, partial);
+        launch_pdl(amax_partial_kernel, dim3(grid_a), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x), nvec, partial);
         count_launch();
     }
     const int64_t nblk = rows * K / 16;
@@ -218,11 +222,11 @@ extern "C" nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t 
     if (grid_q > cap) grid_q = cap;
     if (grid_q < 1) grid_q = 1;
     if (layout == NVFP4_SF_MMA_TILED)
-        quantize_kernel<true><<<(int)grid_q, kThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), rows, K,
+        launch_pdl(quantize_kernel<true>, dim3((int)grid_q), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x), rows, K,
                                                                global_scale_in, partial, grid_a,
                                                                reinterpret_cast<uint2*>(q), sf, global_scale_out);
     else
-        quantize_kernel<false><<<(int)grid_q, kThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), rows, K,
+        launch_pdl(quantize_kernel<false>, dim3((int)grid_q), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x), rows, K,
                                                                 global_scale_in, partial, grid_a,
                                                                 reinterpret_cast<uint2*>(q), sf, global_scale_out);
     count_launch();
