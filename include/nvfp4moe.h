@@ -106,6 +106,17 @@ NVFP4_API nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t K
                             uint8_t* q, uint8_t* sf, float* global_scale_out, nvfp4_sf_layout layout,
                             void* ws, size_t ws_bytes, nvfp4_stream_t stream);
 
+/* nvfp4_quantize_from_amax: nvfp4_quantize with a dynamic global scale whose */
+/* amax is already known (amax_bits: device uint32 holding max |x| as the    */
+/* BF16 bit pattern in its low 16 bits, e.g. written by                      */
+/* moe_grouped_gemm_nvfp4_amax). Identical output to nvfp4_quantize(x, ...,  */
+/* global_scale_in = NULL, ...) for the same amax; one pass over x, no       */
+/* workspace. Same shape, layout and alignment rules; amax_bits 4-byte       */
+/* aligned.                                                                  */
+NVFP4_API nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows, int64_t K, const uint32_t* amax_bits,
+                                      uint8_t* q, uint8_t* sf, float* global_scale_out, nvfp4_sf_layout layout,
+                                      nvfp4_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* moe_permute: group routed (token, slot) pairs by expert and gather the    */
 /* quantised activation rows into expert order ("Peering into the CUTLASS   */
@@ -187,6 +198,20 @@ NVFP4_API nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t*
                                     int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
                                     nvfp4_stream_t stream);
 
+/* moe_grouped_gemm_nvfp4_amax: the same GEMM, and also the amax of its      */
+/* output for the next quantisation (nvfp4_quantize_from_amax), so that step */
+/* needs no separate pass over out.                                          */
+/*   out_amax: device uint32, 4-byte aligned, or NULL (= the call above).    */
+/*   The kernel raises *out_amax (atomic max) to max |out| over every stored */
+/*   element, as the BF16 bit pattern of |out| in the low 16 bits; the       */
+/*   caller sets it to 0 before the call. Same value as the amax pass of     */
+/*   nvfp4_quantize on out (NaN sorts above +inf in both).                   */
+NVFP4_API nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
+                                         const uint8_t* w_packed, const float* w_gscale,
+                                         const int32_t* expert_offsets, int32_t E, int64_t max_rows,
+                                         int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
+                                         uint32_t* out_amax, nvfp4_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* nvfp4_pack_weights: one-time packing of a quantised weight matrix         */
 /* [rows, K] (codes q [rows, K/2], row-major scales sf [rows, K/16]) into   */
@@ -223,8 +248,10 @@ NVFP4_API nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* i
 /* ------------------------------------------------------------------------ */
 /* moe_layer_nvfp4: the whole MoE FFN in one call, every step in this        */
 /* library's kernels, in this order: quantize(x) -> moe_permute ->           */
-/* grouped GEMM gate/up (SWIGLU, N = 2I, K = H) -> quantize(h) -> grouped   */
-/* GEMM down (NONE, N = H, K = I) -> moe_unpermute_combine.                  */
+/* grouped GEMM gate/up (SWIGLU, N = 2I, K = H, amax of h as a side output)  */
+/* -> quantize(h) from that amax -> grouped GEMM down (NONE, N = H, K = I)   */
+/* -> moe_unpermute_combine. Results equal the four calls above run one by   */
+/* one (nvfp4_quantize of h with a dynamic scale).                           */
 /* Arguments: x [T, H] BF16, topk_ids [T, k], topk_w [T, k];                 */
 /*   w13_packed (W13 [E, 2I, H] packed as an [E*2I, H] matrix), w13_gscale   */
 /*   [E]; w2_packed (W2 [E, H, I] packed as [E*H, I]), w2_gscale [E];        */
@@ -240,6 +267,7 @@ typedef struct {
     size_t offsets, perm_src, inv_perm;    /* [E+1], [T*k], [T*k] int32 */
     size_t h;                              /* [T*k, I] BF16 */
     size_t q_h, sf_h, g_h;                 /* [T*k, I/2], [T*k, I/16], scalar */
+    size_t amax_h;                         /* uint32: max |h| (BF16 bits), from the gate/up GEMM */
     size_t y;                              /* [T*k, H] BF16 */
     size_t scratch;                        /* quantize / permute scratch */
     size_t total;

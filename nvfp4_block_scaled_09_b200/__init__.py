@@ -10,7 +10,8 @@ without a CUDA device the calls raise.
 Calls (same names as the C ABI):
   quantize            -> nvfp4_quantize
   permute             -> moe_permute
-  grouped_gemm        -> moe_grouped_gemm_nvfp4
+  grouped_gemm        -> moe_grouped_gemm_nvfp4 (moe_grouped_gemm_nvfp4_amax with amax_out)
+  quantize_from_amax  -> nvfp4_quantize_from_amax
   pack_weights        -> nvfp4_pack_weights
   unpermute_combine   -> moe_unpermute_combine
   moe_layer           -> moe_layer_nvfp4
@@ -45,7 +46,7 @@ class NVFP4Error(RuntimeError):
 class LayerWorkspace(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "q_x", "sf_x", "g_x", "q_perm", "sf_perm", "offsets", "perm_src", "inv_perm", "h", "q_h", "sf_h", "g_h",
-        "y", "scratch", "total")]
+        "amax_h", "y", "scratch", "total")]
 
 
 class GemmPlan(ctypes.Structure):
@@ -81,6 +82,10 @@ def lib():
         L.moe_permute_noalloc.restype = st
         L.moe_grouped_gemm_nvfp4.argtypes = [P, P, P, P, P, P, i32, i64, i64, i64, ctypes.c_int, P, P]
         L.moe_grouped_gemm_nvfp4.restype = st
+        L.moe_grouped_gemm_nvfp4_amax.argtypes = [P, P, P, P, P, P, i32, i64, i64, i64, ctypes.c_int, P, P, P]
+        L.moe_grouped_gemm_nvfp4_amax.restype = st
+        L.nvfp4_quantize_from_amax.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int, P]
+        L.nvfp4_quantize_from_amax.restype = st
         L.moe_unpermute_combine.argtypes = [P, P, P, i32, i32, i64, P, P]
         L.moe_unpermute_combine.restype = st
         L.moe_layer_workspace_layout.argtypes = [i32, i32, i32, i64, i64, ctypes.POINTER(LayerWorkspace)]
@@ -163,6 +168,23 @@ def quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None, layout: 
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib().nvfp4_quantize(_ptr(x), rows, K, _ptr(global_scale), _ptr(q), _ptr(sf), _ptr(g), layout,
                                 _ptr(ws), nbytes, _stream(stream)), "nvfp4_quantize")
+    return q, sf, g
+
+
+def quantize_from_amax(x: torch.Tensor, amax_bits: torch.Tensor, layout: int = SF_ROWMAJOR,
+                       q: torch.Tensor | None = None, sf: torch.Tensor | None = None, g: torch.Tensor | None = None,
+                       stream=None):
+    """quantize() with a dynamic global scale from a known amax: amax_bits is a device int32 [1] holding max |x|
+    as BF16 bits (e.g. the amax_out of grouped_gemm)."""
+    _require_cuda(x, amax_bits)
+    x = _bits(x)
+    rows, K = x.shape
+    dev = x.device
+    q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else q
+    sf = torch.empty((rows, K // 16), dtype=torch.uint8, device=dev) if sf is None else sf
+    g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else g
+    _check(lib().nvfp4_quantize_from_amax(_ptr(x), rows, K, _ptr(amax_bits), _ptr(q), _ptr(sf), _ptr(g), layout,
+                                          _stream(stream)), "nvfp4_quantize_from_amax")
     return q, sf, g
 
 
@@ -281,18 +303,19 @@ def permute_noalloc(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, n
 
 # ----------------------------------------------------------------------------- grouped GEMM
 
-def grouped_gemm(a_q, a_sf, a_g, w: PackedWeights, offsets, swiglu: bool, out=None, stream=None):
-    """Per-expert NVFP4 GEMM. Returns bf16 [rows, N] (or [rows, N/2] with SwiGLU)."""
-    _require_cuda(a_q, a_sf, a_g, w.packed, w.gscale, offsets)
+def grouped_gemm(a_q, a_sf, a_g, w: PackedWeights, offsets, swiglu: bool, out=None, stream=None, amax_out=None):
+    """Per-expert NVFP4 GEMM. Returns bf16 [rows, N] (or [rows, N/2] with SwiGLU). With amax_out (device int32
+    [1], zeroed by the caller) the kernel also raises it to max |out| as BF16 bits."""
+    _require_cuda(a_q, a_sf, a_g, w.packed, w.gscale, offsets, amax_out)
     rows = a_q.shape[0]
     E = offsets.numel() - 1
     N, K = w.N, w.K
     nout = N // 2 if swiglu else N
     if out is None:
         out = torch.empty((rows, nout), dtype=torch.bfloat16, device=a_q.device)
-    _check(lib().moe_grouped_gemm_nvfp4(_ptr(a_q), _ptr(a_sf), _ptr(a_g), _ptr(w.packed), _ptr(w.gscale),
-                                        _ptr(offsets), E, rows, N, K, EPI_SWIGLU if swiglu else EPI_NONE, _ptr(out),
-                                        _stream(stream)), "moe_grouped_gemm_nvfp4")
+    _check(lib().moe_grouped_gemm_nvfp4_amax(_ptr(a_q), _ptr(a_sf), _ptr(a_g), _ptr(w.packed), _ptr(w.gscale),
+                                             _ptr(offsets), E, rows, N, K, EPI_SWIGLU if swiglu else EPI_NONE,
+                                             _ptr(out), _ptr(amax_out), _stream(stream)), "moe_grouped_gemm_nvfp4_amax")
     return out
 
 

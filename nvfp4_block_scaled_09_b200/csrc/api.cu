@@ -121,6 +121,7 @@ extern "C" nvfp4_status moe_layer_workspace_layout(int32_t T, int32_t k, int32_t
     L->q_h = take(R * I / 2);
     L->sf_h = take(R * I / 16);
     L->g_h = take(sizeof(float));
+    L->amax_h = take(sizeof(uint32_t));
     L->y = take(R * H * 2);
     size_t scratch = moe_permute_workspace_size(T, k, E);
     const size_t qx = nvfp4_quantize_workspace_size(T, H), qh = nvfp4_quantize_workspace_size((int64_t)R, I);
@@ -164,20 +165,24 @@ extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_i
     uint8_t* q_h = b + L.q_h;
     uint8_t* sf_h = b + L.sf_h;
     float* g_h = reinterpret_cast<float*>(b + L.g_h);
+    uint32_t* amax_h = reinterpret_cast<uint32_t*>(b + L.amax_h);
     uint16_t* y = reinterpret_cast<uint16_t*>(b + L.y);
     void* scratch = b + L.scratch;
     const size_t scratch_bytes = L.total - L.scratch;
 
+    // the gate/up GEMM raises amax_h; it starts from 0 (before the first kernel, so that every kernel
+    // boundary after it keeps its programmatic launch)
+    if (cudaMemsetAsync(amax_h, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
     if ((st = nvfp4_quantize(x, T, H, nullptr, q_x, sf_x, g_x, NVFP4_SF_ROWMAJOR, scratch, scratch_bytes, stream)))
         return st;
     if ((st = moe_permute(topk_ids, T, k, E, q_x, sf_x, H, q_perm, sf_perm, off, perm_src, inv_perm, scratch,
                           scratch_bytes, stream)))
         return st;
-    if ((st = moe_grouped_gemm_nvfp4(q_perm, sf_perm, g_x, w13_packed, w13_gscale, off, E, R, 2 * I, H,
-                                     NVFP4_EPI_SWIGLU, h, stream)))
+    if ((st = moe_grouped_gemm_nvfp4_amax(q_perm, sf_perm, g_x, w13_packed, w13_gscale, off, E, R, 2 * I, H,
+                                          NVFP4_EPI_SWIGLU, h, amax_h, stream)))
         return st;
-    if ((st = nvfp4_quantize(h, R, I, nullptr, q_h, sf_h, g_h, NVFP4_SF_ROWMAJOR, scratch, scratch_bytes, stream)))
-        return st;
+    if ((st = nvfp4_quantize_from_amax(h, R, I, amax_h, q_h, sf_h, g_h, NVFP4_SF_ROWMAJOR, stream))) return st;
     if ((st = moe_grouped_gemm_nvfp4(q_h, sf_h, g_h, w2_packed, w2_gscale, off, E, R, H, I, NVFP4_EPI_NONE, y,
                                      stream)))
         return st;

@@ -45,7 +45,8 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
                                       const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const uint8_t* a_sf,
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
-                                      int swiglu, uint16_t* out, cudaStream_t s, uint32_t* status);
+                                      int swiglu, uint16_t* out, uint32_t* out_amax, cudaStream_t s,
+                                      uint32_t* status);
 
 #ifdef __CUDACC__
 // Launch `kernel` on `s` with programmatic stream serialization (see pdl_wait()).

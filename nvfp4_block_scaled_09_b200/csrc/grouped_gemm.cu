@@ -58,7 +58,7 @@ constexpr int kNumA = 2;                         // weight row blocks per tile
 constexpr int kBK = 256;                         // K elements per stage
 constexpr int kRowBytes = kBK / 2;               // packed bytes per row per stage (one 128-byte swizzle row)
 constexpr int kBNStep = 16;                      // N granularity = activation TMA box rows
-constexpr int kStages = 4;
+constexpr int kMaxStages = 4;                    // barrier arrays are sized for the deepest shape
 constexpr int kKSteps = kBK / 64;                // MMA K-steps per stage (K = 64 per MMA)
 constexpr int kABlockBytes = kBM * kRowBytes;    // 16 KB
 constexpr int kSFAtomBytes = 512;                // 128 rows x 4 scales
@@ -76,9 +76,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemLimit = 232448;               // B200 opt-in shared memory per block
 
 struct Shared {
-    uint64_t full_tma[kStages];
-    uint64_t sf_ready[kStages];
-    uint64_t empty[kStages];
+    uint64_t full_tma[kMaxStages];
+    uint64_t sf_ready[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
@@ -96,8 +96,9 @@ struct Shared {
 //    cost the same ~50 ns as N = 64 ones on B200, so the tensor rate doubles and
 //    the activation re-reads from L2 halve -- with one accumulator buffer (two
 //    128-column accumulators plus the scale ring fill the 512 TMEM columns).
-template <int BN_MAX, int ACC_BUFS>
+template <int BN_MAX, int ACC_BUFS, int STAGES>
 struct Cfg {
+    static constexpr int kStages = STAGES;
     static constexpr int kBNMax = BN_MAX;
     static constexpr int kAccBufs = ACC_BUFS;
     static constexpr int kBBytes = BN_MAX * kRowBytes;
@@ -110,12 +111,13 @@ struct Cfg {
     static constexpr uint32_t kTmemSFSlot = (kNumA + 1) * 4 * kKSteps;
     static constexpr size_t kSmemBytes = 1024 /* alignment slack */ + (size_t)kStages * kStageBytes + sizeof(Shared);
     static_assert(BN_MAX % kBNStep == 0 && BN_MAX <= 128, "one scale atom covers at most 128 activation rows");
+    static_assert(STAGES >= 2 && STAGES <= kMaxStages, "stage count");
     static_assert(kTmemSFRing + kStages * kTmemSFSlot <= kTmemCols, "TMEM budget");
     static_assert(kStageBytes % 1024 == 0, "stage buffers must keep 1024-byte swizzle alignment");
     static_assert(kSmemBytes + 256 <= (size_t)kSmemLimit, "shared memory budget (dynamic + static)");
 };
-using Narrow = Cfg<64, 2>;
-using Wide = Cfg<128, 1>;
+using Narrow = Cfg<64, 2, 4>;
+using Wide = Cfg<128, 1, 4>;
 
 static_assert(kOffA1 % 1024 == 0 && kOffB % 1024 == 0, "swizzled operand tiles must start on 1024 bytes");
 
@@ -131,6 +133,7 @@ struct Params {
     int64_t N;
     int64_t K;
     int32_t swiglu;
+    uint32_t* amax_out;   // nullable: raised to max |out| (BF16 bits)
     DeviceCtl ctl;
 };
 
@@ -172,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kAccCols = C::kAccCols;
     constexpr uint32_t kTmemSFRing = C::kTmemSFRing;
     constexpr uint32_t kTmemSFSlot = C::kTmemSFSlot;
+    constexpr int kStages = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
@@ -425,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = quad * 32 + lane;         // accumulator row = weight row within a block
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const float a_g = __ldg(p.a_gscale);
+        uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
         uint32_t abuf = 0, aphase = 0;
         for (int32_t w = blockIdx.x; w < total; w += gridDim.x) {
             Tile t;
@@ -447,7 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (i < nrows) {
                             const float g = alpha * v0[i], u = alpha * v1[i];
                             const float h = swiglu_f32(g, u);
-                            o[(int64_t)i * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                            const uint16_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                            amax = max(amax, (uint32_t)(hb & 0x7FFFu));
+                            o[(int64_t)i * ldo] = hb;
                         }
                     }
                 } else {
@@ -456,8 +463,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 16; i++) {
                         if (i < nrows) {
-                            o[(int64_t)i * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v0[i]));
-                            o[(int64_t)i * ldo + kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v1[i]));
+                            const uint16_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v0[i]));
+                            const uint16_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v1[i]));
+                            amax = max(amax, (uint32_t)max(b0 & 0x7FFFu, b1 & 0x7FFFu));
+                            o[(int64_t)i * ldo] = b0;
+                            o[(int64_t)i * ldo + kBM] = b1;
                         }
                     }
                 }
@@ -466,6 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.acc_empty[abuf]);
             if (++abuf == (uint32_t)C::kAccBufs) { abuf = 0; aphase ^= 1u; }
+        }
+        if (p.amax_out != nullptr) {
+            amax = __reduce_max_sync(0xFFFFFFFFu, amax);
+            if (lane == 0 && amax != 0u) atomicMax(p.amax_out, amax);
         }
     }
 
@@ -563,7 +577,7 @@ extern "C" nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan) {
     plan->tile_weight_rows = gg::kNumA * gg::kBM;
     plan->tile_tokens_max = gg::Narrow::kBNMax;
     plan->stage_k = gg::kBK;
-    plan->stages = gg::kStages;
+    plan->stages = gg::Narrow::kStages;
     plan->stage_bytes_weights = gg::kNumA * gg::kABlockBytes;   // arrives with its scales in one packed tile
     plan->stage_bytes_weight_sf = gg::kNumA * gg::kSFStageBytes;
     plan->stage_bytes_act_max = gg::Narrow::kBBytes;
@@ -634,8 +648,18 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
                                                const int32_t* expert_offsets, int32_t E, int64_t max_rows,
                                                int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
                                                nvfp4_stream_t stream) {
+    return moe_grouped_gemm_nvfp4_amax(a_q, a_sf, a_gscale, w_packed, w_gscale, expert_offsets, E, max_rows, N, K,
+                                       epi, out, nullptr, stream);
+}
+
+extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
+                                                    const uint8_t* w_packed, const float* w_gscale,
+                                                    const int32_t* expert_offsets, int32_t E, int64_t max_rows,
+                                                    int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
+                                                    uint32_t* out_amax, nvfp4_stream_t stream) {
     if (!a_q || !a_sf || !a_gscale || !w_packed || !w_gscale || !expert_offsets || !out)
         return NVFP4_ERR_INVALID_ARG;
+    if ((uintptr_t)out_amax & 3u) return NVFP4_ERR_MISALIGNED;
     if (max_rows < 0 || max_rows > INT32_MAX) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(a_q) || !aligned16(a_sf) || !aligned16(w_packed) || !aligned16(out) ||
         ((uintptr_t)a_gscale & 3u) || ((uintptr_t)w_gscale & 3u) || ((uintptr_t)expert_offsets & 3u))
@@ -663,6 +687,7 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
     prm.N = N;
     prm.K = K;
     prm.swiglu = epi == NVFP4_EPI_SWIGLU ? 1 : 0;
+    prm.amax_out = out_amax;
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
@@ -680,8 +705,8 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
             return NVFP4_ERR_CUDA;
         CUtensorMap tm_wsw = tm_a;  // SWIGLU: interleaved gate/up weight slabs (unused otherwise)
         if (prm.swiglu && !encode_swiglu_weights_map(&tm_wsw, w_packed, E, N, K)) return NVFP4_ERR_CUDA;
-        return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_sf, tm_out, tm_wsw, a_sf, a_gscale, w_packed, w_gscale, expert_offsets, E, max_rows,
-                                        N, K, prm.swiglu, out, s, status);
+        return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_sf, tm_out, tm_wsw, a_sf, a_gscale, w_packed, w_gscale,
+                                        expert_offsets, E, max_rows, N, K, prm.swiglu, out, out_amax, s, status);
     }
     const bool wide = max_rows >= kWideMinAvgRows * (int64_t)E;
     const nvfp4_status ls =

@@ -81,6 +81,7 @@ struct Params {
     int64_t N;
     int64_t K;
     int32_t swiglu;
+    uint32_t* amax_out;   // nullable: raised to max |out| (BF16 bits)
     DeviceCtl ctl;
 };
 
@@ -389,6 +390,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint16_t* stg = sh.ostage[half * 4 + quad];
         const bool up_lane = lane >= 16;
         const float a_g = __ldg(p.a_gscale);
+        uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
         uint32_t aphase = 0;
         for (int32_t w = pair; w < total; w += npairs) {
             Tile t;
@@ -417,14 +419,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         const float g = alpha * (up_lane ? recv : v[2 * j]);
                         const float u = alpha * (up_lane ? v[2 * j + 1] : recv);
                         const float h = swiglu_f32(g, u);
-                        stg[(2 * j + (up_lane ? 1 : 0)) * 16 + (lane & 15)] =
-                            __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                        const uint16_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                        if (2 * j + (up_lane ? 1 : 0) < nrows) amax = max(amax, (uint32_t)(hb & 0x7FFFu));
+                        stg[(2 * j + (up_lane ? 1 : 0)) * 16 + (lane & 15)] = hb;
                     }
                     col = t.nt * kBM + (int32_t)rank * 64 + quad * 16;
                     lane_cols = 2;
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 32; i++) stg[i * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i]));
+                    for (int i = 0; i < 32; i++) {
+                        const uint16_t b = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i]));
+                        if (i < nrows) amax = max(amax, (uint32_t)(b & 0x7FFFu));
+                        stg[i * 32 + lane] = b;
+                    }
                     col = t.nt * 2 * kBM + (int32_t)rank * kBM + quad * 32;
                     lane_cols = 4;
                 }
@@ -457,6 +464,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (lane == 0) bulk_wait_group0();  // this warp's tensor stores completed
         __syncwarp();
+        if (p.amax_out != nullptr) {
+            amax = __reduce_max_sync(0xFFFFFFFFu, amax);
+            if (lane == 0 && amax != 0u) atomicMax(p.amax_out, amax);
+        }
     }
 
     // ---- teardown: both CTAs have drained their own work; then the pair frees its TMEM ----
@@ -483,7 +494,8 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
                                       const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const uint8_t* a_sf,
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
-                                      int swiglu, uint16_t* out, cudaStream_t s, uint32_t* status) {
+                                      int swiglu, uint16_t* out, uint32_t* out_amax, cudaStream_t s,
+                                      uint32_t* status) {
     static bool configured[64] = {};
     static int grid_for[64] = {};
     int dev = 0;
@@ -523,6 +535,7 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     prm.N = N;
     prm.K = K;
     prm.swiglu = swiglu;
+    prm.amax_out = out_amax;
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();

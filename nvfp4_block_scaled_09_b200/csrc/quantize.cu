@@ -184,6 +184,23 @@ static int amax_grid(int64_t nvec) {
     return (int)g;
 }
 
+// Second pass: every CTA folds the npartial amax words (BF16 bits) into the tensor amax, then quantises.
+static void launch_quantize(const uint16_t* x, int64_t rows, int64_t K, const float* global_scale_in,
+                            const uint32_t* partial, int npartial, uint8_t* q, uint8_t* sf, float* global_scale_out,
+                            nvfp4_sf_layout layout, cudaStream_t s) {
+    const int64_t nblk = rows * K / 16;
+    int64_t grid_q = (nblk + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)device_sm_count() * 16;
+    if (grid_q > cap) grid_q = cap;
+    if (grid_q < 1) grid_q = 1;
+    if (layout == NVFP4_SF_MMA_TILED)
+        launch_pdl(quantize_kernel<true>, dim3((int)grid_q), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x),
+                   rows, K, global_scale_in, partial, npartial, reinterpret_cast<uint2*>(q), sf, global_scale_out);
+    else
+        launch_pdl(quantize_kernel<false>, dim3((int)grid_q), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x),
+                   rows, K, global_scale_in, partial, npartial, reinterpret_cast<uint2*>(q), sf, global_scale_out);
+}
+
 }  // namespace nvfp4
 
 using namespace nvfp4;
@@ -216,19 +233,23 @@ extern "C" nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t 
         launch_pdl(amax_partial_kernel, dim3(grid_a), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x), nvec, partial);
         count_launch();
     }
-    const int64_t nblk = rows * K / 16;
-    int64_t grid_q = (nblk + kThreads - 1) / kThreads;
-    const int64_t cap = (int64_t)device_sm_count() * 16;
-    if (grid_q > cap) grid_q = cap;
-    if (grid_q < 1) grid_q = 1;
-    if (layout == NVFP4_SF_MMA_TILED)
-        launch_pdl(quantize_kernel<true>, dim3((int)grid_q), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x), rows, K,
-                                                               global_scale_in, partial, grid_a,
-                                                               reinterpret_cast<uint2*>(q), sf, global_scale_out);
-    else
-        launch_pdl(quantize_kernel<false>, dim3((int)grid_q), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x), rows, K,
-                                                                global_scale_in, partial, grid_a,
-                                                                reinterpret_cast<uint2*>(q), sf, global_scale_out);
+    launch_quantize(x, rows, K, global_scale_in, partial, grid_a, q, sf, global_scale_out, layout, s);
+    count_launch();
+    return check_launch();
+}
+
+extern "C" nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows, int64_t K, const uint32_t* amax_bits,
+                                                 uint8_t* q, uint8_t* sf, float* global_scale_out,
+                                                 nvfp4_sf_layout layout, nvfp4_stream_t stream) {
+    if (!x || !q || !sf || !global_scale_out || !amax_bits) return NVFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_MMA_TILED) return NVFP4_ERR_INVALID_ARG;
+    if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (layout == NVFP4_SF_MMA_TILED && (rows % 128 != 0 || K % 64 != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned8(q)) return NVFP4_ERR_MISALIGNED;
+    if (((uintptr_t)global_scale_out & 3u) || ((uintptr_t)amax_bits & 3u)) return NVFP4_ERR_MISALIGNED;
+    launch_quantize(x, rows, K, nullptr, amax_bits, 1, q, sf, global_scale_out, layout,
+                    reinterpret_cast<cudaStream_t>(stream));
     count_launch();
     return check_launch();
 }

@@ -59,8 +59,14 @@ def check_weights_quantised_and_packed(c, experts):
 
 def run_full(rows, N, K, swiglu, seed):
     c = make_case(rows, N, K, seed)
-    out = nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["pw"], c["off"], swiglu)
+    amax = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["pw"], c["off"], swiglu, amax_out=amax)
     assert nv.device_status() == 0
+    # the side output is the max |BF16| over the stored rows only (BF16 bits), i.e. what the amax pass of
+    # quantize() would find on out[:R]
+    got_bits = host_bits(out)[: c["R"]]
+    want = int((got_bits & 0x7FFF).max()) if got_bits.size else 0
+    assert int(host(amax)[0]) == want
     check_weights_quantised_and_packed(c, range(min(c["E"], 3)))
     w_q, w_sf, w_g = oracle_operands(c)
     ref = oracle.grouped_gemm(host(c["a_q"]), host(c["a_sf"]), host(c["a_g"])[0], w_q, w_sf, w_g, c["off_np"],

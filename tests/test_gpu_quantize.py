@@ -86,3 +86,17 @@ def test_rejects_bad_arguments():
     with pytest.raises(nv.NVFP4Error) as e:
         nv.quantize(x, layout=nv.SF_MMA_TILED)
     assert e.value.status == 3
+
+
+@pytest.mark.parametrize("rows,K,std,seed", [(1, 16, 1.0, 10), (96, 2048, 0.5, 11), (300, 512, 3.0, 12)])
+def test_from_amax_equals_dynamic(rows, K, std, seed):
+    # quantize_from_amax with the tensor's own amax (BF16 bits, as the GEMM side output carries it) is the
+    # dynamic-scale quantiser: compared with the oracle bit for bit, and with an all-zero tensor
+    xbits = workloads.random_bf16_bits((rows, K), seed=seed, std=std)
+    for bits in (xbits, np.zeros_like(xbits)):
+        amax = torch.tensor([int((bits & 0x7FFF).max())], dtype=torch.int32, device="cuda")
+        q, sf, g = nv.quantize_from_amax(gpu_bf16(bits), amax)
+        oq, osf, og = oracle.quantize(bits)
+        assert np.float32(host(g)[0]) == og
+        assert np.array_equal(host(sf).reshape(osf.shape), osf)
+        assert np.array_equal(host(q), oq)

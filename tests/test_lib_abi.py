@@ -95,3 +95,6 @@ def test_invalid_arguments_rejected_before_any_cuda_call(L):
     assert L.moe_unpermute_combine(p, p, p, 1, 1, 12, p, None) == 3     # H % 8 != 0
     assert L.moe_permute(p, 4, 8, 2000, p, p, 256, p, p, p, p, p, p, 1 << 20, None) == 3  # E > 1024
     assert L.moe_permute(p, 4, 8, 8, p, p, 256, p, p, p, p, p, None, 0, None) == 4       # no workspace
+    assert L.nvfp4_quantize_from_amax(None, 4, 32, None, None, None, None, 0, None) == 1
+    assert L.nvfp4_quantize_from_amax(p, 4, 32, ctypes.c_void_p(18), p, p, p, 0, None) == 2  # amax word misaligned
+    assert L.moe_grouped_gemm_nvfp4_amax(p, p, p, p, p, p, 1, 16, 256, 256, 0, p, ctypes.c_void_p(18), None) == 2
