@@ -78,7 +78,9 @@ def load_peaks():
 
 FP4_PER_BF16 = 4.0  # nominal dense ratio (9 PF FP4 / 2.25 PF BF16)
 
-GEMM_SOURCES = ("nvfp4_block_scaled_09_b200/csrc/grouped_gemm.cu", "nvfp4_block_scaled_09_b200/csrc/common.cuh")
+# kernel sources a committed ncu traffic figure belongs to (the summary names them; default: all GEMM sources)
+GEMM_SOURCES = ("nvfp4_block_scaled_09_b200/csrc/grouped_gemm.cu", "nvfp4_block_scaled_09_b200/csrc/grouped_gemm_pair.cu",
+                "nvfp4_block_scaled_09_b200/csrc/common.cuh")
 
 
 def replica_seed(seed: int, rank: int) -> int:
@@ -97,10 +99,10 @@ def max_over_ranks(value: float, world: int, device) -> float:
     return float(t.item())
 
 
-def gemm_source_sha256() -> str:
+def gemm_source_sha256(sources=GEMM_SOURCES) -> str:
     import hashlib
     h = hashlib.sha256()
-    for rel in GEMM_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -108,7 +110,7 @@ def gemm_source_sha256() -> str:
 
 def measured_traffic(config: str):
     """DRAM bytes per gate/up GEMM launch from the committed ncu summary of this workload, or None when
-    there is none or the GEMM sources changed since it was taken."""
+    there is none or the kernel sources it names changed since it was taken."""
     path = os.path.join(ROOT, "profiles", f"traffic_{config}.md")
     if not os.path.exists(path):
         return None
@@ -118,7 +120,8 @@ def measured_traffic(config: str):
             if ":" in line and line.startswith("- "):
                 k, v = line[2:].split(":", 1)
                 fields[k.strip()] = v.strip().strip("`")
-    if fields.get("source_sha256") != gemm_source_sha256():
+    sources = tuple(x.strip().strip("`") for x in fields.get("sources", "").split(",") if x.strip()) or GEMM_SOURCES
+    if fields.get("source_sha256") != gemm_source_sha256(sources):
         return None
     try:
         return int(fields["gate_up_dram_bytes_per_launch"])

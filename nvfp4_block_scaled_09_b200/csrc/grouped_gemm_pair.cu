@@ -225,13 +225,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int s = 0; s < kStages; s++) issued[s] = false, issued_parity[s] = 0;
         if (lane == 0 && !(p.ctl.flags & kCtlStallProducer)) {
-            const uint64_t pol_w = l2_policy_evict_normal();
-            const uint64_t pol_a = l2_policy_evict_last();
+            // L2: an expert's activation rows are re-read by each of its column tiles and stay hot on
+            // their own; a weight tile is re-read only by the expert's other row tiles, which run
+            // alongside (row tile fastest), so it is streamed evict-first when the expert has one
+            const uint64_t pol_w_once = l2_policy_evict_first();
+            const uint64_t pol_w_reuse = l2_policy_evict_normal();
+            const uint64_t pol_a = l2_policy_evict_normal();
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             for (int32_t w = pair; w < total && ok; w += npairs) {
                 Tile t;
                 decode_tile(sh, E, w, t);
+                const uint64_t pol_w = (sh.off[t.e + 1] - sh.off[t.e] > kBNMax) ? pol_w_reuse : pol_w_once;
                 // weight rows of this CTA, as (packed tile base, byte offset of the first row's codes)
                 const uint8_t* g_tile;   // NONE: the whole 128-row tile; SWIGLU: the gate tile
                 const uint8_t* u_tile = nullptr;
