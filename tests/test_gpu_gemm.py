@@ -23,11 +23,12 @@ def _gpu():
     require_gpu()
 
 
-def make_case(rows, N, K, seed, a_std=1.0, w_std=0.02):
-    """Quantised activations [sum(rows), K] and packed per-expert weights [E, N, K] on the GPU."""
+def make_case(rows, N, K, seed, a_std=1.0, w_std=0.02, pad_rows=0):
+    """Quantised activations [sum(rows) + pad_rows, K] and packed per-expert weights [E, N, K] on the GPU.
+    The GEMM's max_rows is the activation row count, so padding rows changes the tile shape it picks."""
     E = len(rows)
     R = int(sum(rows))
-    a_bits = workloads.random_bf16_bits((max(R, 1), K), seed=seed, std=a_std)
+    a_bits = workloads.random_bf16_bits((max(R + pad_rows, 1), K), seed=seed, std=a_std)
     a_q, a_sf, a_g = nv.quantize(gpu_bf16(a_bits))
     w = workloads.normal_bf16((E, N, K), w_std, seed, workloads.TAG_W13, device="cuda")
     pw = nv.prepare_expert_weights(w, keep_rowmajor=True)
@@ -57,8 +58,8 @@ def check_weights_quantised_and_packed(c, experts):
         assert np.array_equal(uq, wq) and np.array_equal(usf, wsf)
 
 
-def run_full(rows, N, K, swiglu, seed):
-    c = make_case(rows, N, K, seed)
+def run_full(rows, N, K, swiglu, seed, pad_rows=0):
+    c = make_case(rows, N, K, seed, pad_rows=pad_rows)
     amax = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["pw"], c["off"], swiglu, amax_out=amax)
     assert nv.device_status() == 0
@@ -69,8 +70,9 @@ def run_full(rows, N, K, swiglu, seed):
     assert int(host(amax)[0]) == want
     check_weights_quantised_and_packed(c, range(min(c["E"], 3)))
     w_q, w_sf, w_g = oracle_operands(c)
-    ref = oracle.grouped_gemm(host(c["a_q"]), host(c["a_sf"]), host(c["a_g"])[0], w_q, w_sf, w_g, c["off_np"],
-                              N, K, swiglu)
+    R = c["R"]
+    ref = oracle.grouped_gemm(host(c["a_q"])[:R], host(c["a_sf"])[:R], host(c["a_g"])[0], w_q, w_sf, w_g,
+                              c["off_np"], N, K, swiglu)
     got = host_bits(out)[: c["R"]]
     return compare_bf16(got, oracle.bf16_round(ref), f"gemm rows={rows} N={N} K={K} swiglu={swiglu}", exact=ref)
 
@@ -98,6 +100,42 @@ def test_pair_tiles_ragged(swiglu):
     # experts averaging >= 192 rows run on CTA pairs (256 weight rows x up to 256 activation rows):
     # empty, partial, exact, 256 + 1, two tiles, a small expert
     run_full([0, 200, 256, 257, 500, 40], 512, 768, swiglu, seed=7)
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
+def test_pair_tiles_small_ragged_experts(swiglu):
+    # padding the activations to 192 rows per expert selects the CTA-pair kernel for experts of 1-33 rows:
+    # one-row tiles, a 32-row tile (one full N step), 33 rows (two N steps), an empty expert
+    plan = nv.gemm_plan()
+    rows = [1, 0, 31, 32, 33, 7]
+    pad = plan["pair_min_avg_rows"] * len(rows) - sum(rows)
+    run_full(rows, 512, 512, swiglu, seed=8, pad_rows=pad)
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
+def test_max_experts(swiglu):
+    # E = 1024 (the largest the scheduler takes): 0-3 rows per expert, a third of them empty
+    rng = np.random.default_rng(9)
+    rows = [int(r) for r in rng.integers(0, 4, size=1024)]
+    run_full(rows, 256, 256, swiglu, seed=9)
+
+
+def test_max_experts_pair_tiles():
+    # E = 1024 on the CTA-pair kernel (expert offsets and tile starts of all 1024 experts in shared memory)
+    plan = nv.gemm_plan()
+    rng = np.random.default_rng(10)
+    rows = [int(r) for r in rng.integers(0, 40, size=1024)]
+    run_full(rows, 256, 256, False, seed=10, pad_rows=plan["pair_min_avg_rows"] * 1024 - sum(rows))
+
+
+@pytest.mark.parametrize("pad", [64, 600])   # narrow and CTA-pair tile shapes
+def test_all_experts_empty_writes_nothing(pad):
+    c = make_case([0, 0, 0], 256, 256, seed=11, pad_rows=pad)
+    out = torch.full((pad, 256), 3.0, dtype=torch.bfloat16, device="cuda")
+    amax = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.grouped_gemm(c["a_q"], c["a_sf"], c["a_g"], c["pw"], c["off"], False, out=out, amax_out=amax)
+    assert nv.device_status() == 0
+    assert torch.all(out == 3.0) and int(host(amax)[0]) == 0
 
 
 @pytest.mark.parametrize("swiglu", [False, True])
