@@ -106,6 +106,14 @@ NVFP4_API nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t K
                             uint8_t* q, uint8_t* sf, float* global_scale_out, nvfp4_sf_layout layout,
                             void* ws, size_t ws_bytes, nvfp4_stream_t stream);
 
+/* nvfp4_amax: raises *amax_bits (device uint32, 4-byte aligned; the caller  */
+/* sets it to 0 first) to max |x| over x [rows, K] BF16 (device, 16-byte    */
+/* aligned, K % 8 == 0), as the BF16 bit pattern in the low 16 bits -- the   */
+/* amax nvfp4_quantize derives its dynamic scale from. Several calls (or     */
+/* ranks combining their words with an integer max) accumulate one amax.     */
+NVFP4_API nvfp4_status nvfp4_amax(const uint16_t* x, int64_t rows, int64_t K, uint32_t* amax_bits,
+                        nvfp4_stream_t stream);
+
 /* nvfp4_quantize_from_amax: nvfp4_quantize with a dynamic global scale whose */
 /* amax is already known (amax_bits: device uint32 holding max |x| as the    */
 /* BF16 bit pattern in its low 16 bits, e.g. written by                      */
@@ -239,7 +247,7 @@ NVFP4_API nvfp4_status nvfp4_pack_weights(const uint8_t* q, const uint8_t* sf, i
 /*   entry is skipped.                                                       */
 /* Arguments: y [T*k, H] BF16, inv_perm [T*k], topk_w [T, k] FP32, out [T, H]*/
 /*   BF16; y and out 16-byte aligned, inv_perm and topk_w 4-byte aligned;   */
-/*   all device; H % 8 == 0, 1 <= k <= 32, 1 <= T <= 65535.                  */
+/*   all device; H % 8 == 0, 1 <= k <= 32, T >= 1.                           */
 /* ------------------------------------------------------------------------ */
 NVFP4_API nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* inv_perm, const float* topk_w,
                                    int32_t T, int32_t k, int64_t H, uint16_t* out,

@@ -12,6 +12,7 @@ Calls (same names as the C ABI):
   permute             -> moe_permute
   grouped_gemm        -> moe_grouped_gemm_nvfp4 (moe_grouped_gemm_nvfp4_amax with amax_out)
   quantize_from_amax  -> nvfp4_quantize_from_amax
+  amax                -> nvfp4_amax
   pack_weights        -> nvfp4_pack_weights
   unpermute_combine   -> moe_unpermute_combine
   moe_layer           -> moe_layer_nvfp4
@@ -86,6 +87,8 @@ def lib():
         L.moe_grouped_gemm_nvfp4_amax.restype = st
         L.nvfp4_quantize_from_amax.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int, P]
         L.nvfp4_quantize_from_amax.restype = st
+        L.nvfp4_amax.argtypes = [P, i64, i64, P, P]
+        L.nvfp4_amax.restype = st
         L.moe_unpermute_combine.argtypes = [P, P, P, i32, i32, i64, P, P]
         L.moe_unpermute_combine.restype = st
         L.moe_layer_workspace_layout.argtypes = [i32, i32, i32, i64, i64, ctypes.POINTER(LayerWorkspace)]
@@ -169,6 +172,16 @@ def quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None, layout: 
     _check(lib().nvfp4_quantize(_ptr(x), rows, K, _ptr(global_scale), _ptr(q), _ptr(sf), _ptr(g), layout,
                                 _ptr(ws), nbytes, _stream(stream)), "nvfp4_quantize")
     return q, sf, g
+
+
+def amax(x: torch.Tensor, amax_bits: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Raise amax_bits (device int32 [1], zeroed here when not given) to max |x| as BF16 bits."""
+    _require_cuda(x, amax_bits)
+    x = _bits(x)
+    if amax_bits is None:
+        amax_bits = torch.zeros(1, dtype=torch.int32, device=x.device)
+    _check(lib().nvfp4_amax(_ptr(x), x.shape[0], x.shape[1], _ptr(amax_bits), _stream(stream)), "nvfp4_amax")
+    return amax_bits
 
 
 def quantize_from_amax(x: torch.Tensor, amax_bits: torch.Tensor, layout: int = SF_ROWMAJOR,

@@ -38,32 +38,33 @@ __device__ __forceinline__ uint32_t pack_bf16x2(double lo, double hi) {
 
 __global__ void __launch_bounds__(kThreads) combine_kernel(const uint4* __restrict__ y,
                                                            const int32_t* __restrict__ inv_perm,
-                                                           const float* __restrict__ w, int32_t k, int64_t hvec,
-                                                           uint4* __restrict__ out) {
+                                                           const float* __restrict__ w, int64_t T, int32_t k,
+                                                           int64_t hvec, uint4* __restrict__ out) {
     pdl_launch_dependents();
     pdl_wait();
-    const int64_t t = blockIdx.y;
     const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;  // 16-byte column group
     if (c >= hvec) return;
-    double a[kColsPerThread];
+    for (int64_t t = blockIdx.y; t < T; t += gridDim.y) {
+        double a[kColsPerThread];
 #pragma unroll
-    for (int i = 0; i < kColsPerThread; i++) a[i] = 0.0;
-    for (int j = 0; j < k; j++) {
-        const int32_t p = __ldg(inv_perm + t * k + j);
-        if (p < 0) continue;
-        const double s = (double)__ldg(w + t * k + j);
-        const uint4 v = __ldcs(y + (int64_t)p * hvec + c);
-        acc_bf16x2(a[0], a[1], v.x, s);
-        acc_bf16x2(a[2], a[3], v.y, s);
-        acc_bf16x2(a[4], a[5], v.z, s);
-        acc_bf16x2(a[6], a[7], v.w, s);
+        for (int i = 0; i < kColsPerThread; i++) a[i] = 0.0;
+        for (int j = 0; j < k; j++) {
+            const int32_t p = __ldg(inv_perm + t * k + j);
+            if (p < 0) continue;
+            const double s = (double)__ldg(w + t * k + j);
+            const uint4 v = __ldcs(y + (int64_t)p * hvec + c);
+            acc_bf16x2(a[0], a[1], v.x, s);
+            acc_bf16x2(a[2], a[3], v.y, s);
+            acc_bf16x2(a[4], a[5], v.z, s);
+            acc_bf16x2(a[6], a[7], v.w, s);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(a[0], a[1]);
+        o.y = pack_bf16x2(a[2], a[3]);
+        o.z = pack_bf16x2(a[4], a[5]);
+        o.w = pack_bf16x2(a[6], a[7]);
+        out[t * hvec + c] = o;
     }
-    uint4 o;
-    o.x = pack_bf16x2(a[0], a[1]);
-    o.y = pack_bf16x2(a[2], a[3]);
-    o.z = pack_bf16x2(a[4], a[5]);
-    o.w = pack_bf16x2(a[6], a[7]);
-    out[t * hvec + c] = o;
 }
 
 }  // namespace
@@ -76,13 +77,13 @@ extern "C" nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* 
                                               nvfp4_stream_t stream) {
     if (!y || !inv_perm || !topk_w || !out) return NVFP4_ERR_INVALID_ARG;
     if (T <= 0 || k <= 0 || H <= 0) return NVFP4_ERR_INVALID_ARG;
-    if (k > 32 || H % kColsPerThread != 0 || T > 65535) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (k > 32 || H % kColsPerThread != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(y) || !aligned16(out) || ((uintptr_t)inv_perm & 3u) || ((uintptr_t)topk_w & 3u))
         return NVFP4_ERR_MISALIGNED;
     const int64_t hvec = H / kColsPerThread;
-    dim3 grid((unsigned)((hvec + kThreads - 1) / kThreads), (unsigned)T);
+    dim3 grid((unsigned)((hvec + kThreads - 1) / kThreads), (unsigned)(T < 65535 ? T : 65535));  // tokens loop
     launch_pdl(combine_kernel, dim3(grid), dim3(kThreads), 0, reinterpret_cast<cudaStream_t>(stream),
-        reinterpret_cast<const uint4*>(y), inv_perm, topk_w, k, hvec, reinterpret_cast<uint4*>(out));
+        reinterpret_cast<const uint4*>(y), inv_perm, topk_w, (int64_t)T, k, hvec, reinterpret_cast<uint4*>(out));
     count_launch();
     return check_launch();
 }

@@ -35,6 +35,8 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
     return v;
 }
 
+// kRaise: atomically raise partial[0] to the tensor amax instead of one partial per CTA.
+template <bool kRaise>
 __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const uint4* __restrict__ x, int64_t nvec,
                                                                  uint32_t* __restrict__ partial) {
     pdl_launch_dependents();
@@ -55,7 +57,10 @@ __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const uint4* __r
     if (threadIdx.x < 32) {
         uint32_t v = threadIdx.x < kThreads / 32 ? s_warp[threadIdx.x] : 0u;
         v = warp_max_u32(v);
-        if (threadIdx.x == 0) partial[blockIdx.x] = v;
+        if (threadIdx.x == 0) {
+            if (kRaise) atomicMax(partial, v);
+            else partial[blockIdx.x] = v;
+        }
     }
 }
 
@@ -230,7 +235,7 @@ extern "C" nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint32_t* partial = static_cast<uint32_t*>(ws);
     if (global_scale_in == nullptr) {
-        launch_pdl(amax_partial_kernel, dim3(grid_a), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x), nvec, partial);
+        launch_pdl(amax_partial_kernel<false>, dim3(grid_a), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x), nvec, partial);
         count_launch();
     }
     launch_quantize(x, rows, K, global_scale_in, partial, grid_a, q, sf, global_scale_out, layout, s);
@@ -250,6 +255,19 @@ extern "C" nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows
     if (((uintptr_t)global_scale_out & 3u) || ((uintptr_t)amax_bits & 3u)) return NVFP4_ERR_MISALIGNED;
     launch_quantize(x, rows, K, nullptr, amax_bits, 1, q, sf, global_scale_out, layout,
                     reinterpret_cast<cudaStream_t>(stream));
+    count_launch();
+    return check_launch();
+}
+
+extern "C" nvfp4_status nvfp4_amax(const uint16_t* x, int64_t rows, int64_t K, uint32_t* amax_bits,
+                                   nvfp4_stream_t stream) {
+    if (!x || !amax_bits) return NVFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (K % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || ((uintptr_t)amax_bits & 3u)) return NVFP4_ERR_MISALIGNED;
+    const int64_t nvec = rows * K / 8;
+    launch_pdl(amax_partial_kernel<true>, dim3(amax_grid(nvec)), dim3(kThreads), 0,
+               reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const uint4*>(x), nvec, amax_bits);
     count_launch();
     return check_launch();
 }

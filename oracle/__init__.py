@@ -52,6 +52,7 @@ def lib():
         L.oracle_amax.argtypes = [P, i64]
         L.oracle_amax.restype = f32
         L.oracle_quantize.argtypes = [P, i64, i64, P, P, P, P]
+        L.oracle_quantize_amax.argtypes = [P, i64, i64, f32, P, P, P]
         L.oracle_dequantize.argtypes = [P, P, f32, i64, i64, P]
         L.oracle_permute.argtypes = [P, i32, i32, i32, P, P, P]
         L.oracle_permute.restype = ctypes.c_int
@@ -144,6 +145,20 @@ def quantize(x_bf16: np.ndarray, global_scale=None):
     if global_scale is not None:
         gin = np.array([global_scale], dtype=np.float32)
     lib().oracle_quantize(_p(x), rows, K, _p(gin) if gin is not None else None, _p(q), _p(sf), _p(g))
+    return q, sf, np.float32(g[0])
+
+
+def quantize_with_amax(x_bf16: np.ndarray, amax_value: float):
+    """quantize() of rows that belong to a larger tensor whose amax is amax_value (one global scale per
+    tensor, reading 8): the same steps with the given amax."""
+    x = _u16(x_bf16)
+    rows, K = x.shape
+    if K % 16:
+        raise ValueError("K must be a multiple of 16")
+    q = np.empty((rows, K // 2), dtype=np.uint8)
+    sf = np.empty((rows, K // 16), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    lib().oracle_quantize_amax(_p(x), rows, K, np.float32(amax_value), _p(q), _p(sf), _p(g))
     return q, sf, np.float32(g[0])
 
 

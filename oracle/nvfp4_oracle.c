@@ -201,6 +201,23 @@ void oracle_quantize(const uint16_t* x, int64_t rows, int64_t K, const float* gd
     if (gdec_out) *gdec_out = g_dec;
 }
 
+/* Quantisation with the tensor amax supplied by the caller: the same steps as
+ * oracle_quantize, for a tensor whose rows are spread over several places (one
+ * global scale for the whole tensor: its amax is the max over all parts). */
+void oracle_quantize_amax(const uint16_t* x, int64_t rows, int64_t K, float amax,
+                          uint8_t* q, uint8_t* sf, float* gdec_out) {
+    float g_enc, g_dec;
+    oracle_global_scales(amax, NULL, &g_enc, &g_dec);
+    int64_t nblk = K / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t b = 0; b < nblk; b++) {
+            quantize_block(x + r * K + b * 16, g_enc, q + r * (K / 2) + b * 8, sf + r * nblk + b);
+        }
+    }
+    if (gdec_out) *gdec_out = g_dec;
+}
+
 /* Decoded-value tables, filled from the decode functions above. */
 static double E2M1_VAL[16];
 static double E4M3_VAL[256];

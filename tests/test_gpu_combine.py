@@ -16,7 +16,8 @@ def _gpu():
     require_gpu()
 
 
-@pytest.mark.parametrize("T,E,k,H", [(1, 4, 1, 8), (37, 8, 4, 256), (512, 256, 8, 6144), (1024, 256, 8, 6144)])
+@pytest.mark.parametrize("T,E,k,H", [(1, 4, 1, 8), (37, 8, 4, 256), (512, 256, 8, 6144), (1024, 256, 8, 6144),
+                                     (70000, 16, 2, 16)])   # more tokens than one grid dimension holds
 def test_combine_parity(T, E, k, H):
     ids, w = workloads.routing(T, E, k, "uniform", seed=T)
     _, _, inv = oracle.permute(ids, E)

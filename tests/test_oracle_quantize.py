@@ -105,3 +105,21 @@ def test_static_global_scale_saturates():
     q, sf, g = oracle.quantize(x, global_scale=1.0 / 448.0)   # g_enc = 448: s = 2*448 -> 448 (satfinite)
     assert sf[0, 0] == 0x7E
     assert (q[0, 0] & 0xF) == 0x7                              # y = 12 * 448/448 = 12 -> saturates to 6
+
+
+def test_quantize_with_amax_is_quantize_of_the_whole_tensor():
+    # one global scale per tensor: rows quantised with the tensor's amax equal the tensor's own quantisation,
+    # also when the rows are split into parts (expert-parallel ranks) that each see only their part
+    x = workloads.random_bf16_bits((96, 256), seed=21, std=2.0)
+    q, sf, g = oracle.quantize(x)
+    q1, sf1, g1 = oracle.quantize_with_amax(x, oracle.amax(x))
+    assert np.array_equal(q1, q) and np.array_equal(sf1, sf) and g1 == g
+    a, b = x[:40], x[40:]
+    assert oracle.amax(a) != oracle.amax(b)            # the parts alone would get different scales
+    for part, lo in ((a, 0), (b, 40)):
+        qp, sfp, gp = oracle.quantize_with_amax(part, oracle.amax(x))
+        assert np.array_equal(qp, q[lo: lo + len(part)]) and np.array_equal(sfp, sf[lo: lo + len(part)])
+        assert gp == g
+    # and the part without the tensor's max element has a different scale of its own (not vacuous)
+    small = a if oracle.amax(a) < oracle.amax(x) else b
+    assert oracle.quantize(small)[2] != g
