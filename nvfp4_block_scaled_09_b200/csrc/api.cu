@@ -7,6 +7,10 @@
 
 // One status word per device context; kernels latch error bits into it.
 __device__ uint32_t g_nvfp4_device_status;
+// Work counters of the grouped GEMM's dynamic schedule: launches draw the slots in turn (two words each,
+// left at zero by the launch's last CTA), so GEMMs in flight on different streams use different slots.
+constexpr int kSchedSlots = 64;
+__device__ uint32_t g_nvfp4_sched[2 * kSchedSlots];
 
 namespace nvfp4 {
 
@@ -19,6 +23,8 @@ struct DeviceInfo {
     int sm_count = 0;
     int smem_optin = 0;
     uint32_t* status = nullptr;
+    uint32_t* sched = nullptr;
+    std::atomic<uint32_t> sched_next{0};
 };
 
 constexpr int kMaxDevices = 64;
@@ -37,6 +43,8 @@ static DeviceInfo* device_info() {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_nvfp4_device_status) != cudaSuccess) return nullptr;
         di.status = static_cast<uint32_t*>(p);
+        if (cudaGetSymbolAddress(&p, g_nvfp4_sched) != cudaSuccess) return nullptr;
+        di.sched = static_cast<uint32_t*>(p);
         di.ready = true;
     }
     return &di;
@@ -45,6 +53,11 @@ static DeviceInfo* device_info() {
 uint32_t* status_word_ptr() {
     DeviceInfo* di = device_info();
     return di ? di->status : nullptr;
+}
+uint32_t* sched_counter_slot() {
+    DeviceInfo* di = device_info();
+    if (!di) return nullptr;
+    return di->sched + 2 * (di->sched_next.fetch_add(1u) % kSchedSlots);
 }
 uint64_t wait_timeout_ns() { return g_timeout_ns.load(); }
 uint32_t debug_flags() { return g_debug_flags.load(); }

@@ -31,6 +31,7 @@ struct DeviceCtl {
 
 // Host-side registry (api.cu).
 uint32_t* status_word_ptr();          // nullptr on failure
+uint32_t* sched_counter_slot();       // two zeroed words for one GEMM launch's dynamic schedule (nullptr on failure)
 uint64_t wait_timeout_ns();
 uint32_t debug_flags();
 void count_launch(int n = 1);

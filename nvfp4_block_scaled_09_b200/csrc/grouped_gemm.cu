@@ -75,7 +75,13 @@ constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemLimit = 232448;               // B200 opt-in shared memory per block
 
+constexpr int kTileRing = 4;                     // work items the producer may publish ahead of the slowest role
+constexpr int kTileConsumers = 9;                // MMA warp + 4 scale writers + 4 epilogue warps
+
 struct Shared {
+    uint64_t tq_full[kTileRing];                 // producer published tq[i]
+    uint64_t tq_empty[kTileRing];                // every consumer role read tq[i]
+    int32_t tq[kTileRing];                       // work item index (>= total: no more work)
     uint64_t full_tma[kMaxStages];
     uint64_t sf_ready[kMaxStages];
     uint64_t empty[kMaxStages];
@@ -134,6 +140,7 @@ struct Params {
     int64_t K;
     int32_t swiglu;
     uint32_t* amax_out;   // nullable: raised to max |out| (BF16 bits)
+    uint32_t* sched;      // this launch's work counter [0] and finished-CTA counter [1]; zero at launch
     DeviceCtl ctl;
 };
 
@@ -163,6 +170,18 @@ __device__ __forceinline__ void decode_tile(const Shared& sh, int32_t E, int32_t
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, const DeviceCtl& ctl) {
     bool ok = mbar_wait_bounded(bar, parity, abort, ctl);
     return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// Next work item of this CTA for one consumer role (a whole warp): the producer publishes the items it
+// took from the launch's work counter in a ring of kTileRing entries. False when a wait ran out.
+__device__ __forceinline__ bool next_tile(Shared& sh, uint32_t& qi, uint32_t& qphase, int32_t& w, int lane,
+                                          volatile int* abort, const DeviceCtl& ctl) {
+    if (!warp_wait(&sh.tq_full[qi], qphase, abort, ctl)) return false;
+    w = *reinterpret_cast<volatile int32_t*>(&sh.tq[qi]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.tq_empty[qi]);
+    if (++qi == kTileRing) { qi = 0; qphase ^= 1u; }
+    return true;
 }
 
 template <class C>
@@ -202,6 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sh.acc_empty[b], 4);
         }
         mbar_init(&sh.drain, 1);
+        for (int i = 0; i < kTileRing; i++) {
+            mbar_init(&sh.tq_full[i], 1);
+            mbar_init(&sh.tq_empty[i], kTileConsumers);
+        }
         fence_barrier_init();
     }
     // everything above overlaps the previous kernel; global memory only from here on
@@ -278,9 +301,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_w_once = l2_policy_evict_first();
             const uint64_t pol_w_reuse = l2_policy_evict_normal();
             const uint64_t pol_a = l2_policy_evict_last();
-            uint32_t stage = 0, phase = 0;
+            uint32_t stage = 0, phase = 0, qi = 0, qphase = 0;
             bool ok = true;
-            for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            while (ok) {
+                // dynamic schedule: the next work item of the whole grid, in increasing order, so items
+                // that share a weight tile (row tile fastest) still run side by side, and CTAs that run
+                // ahead take the tail
+                int32_t w = (int32_t)min(atomicAdd(p.sched, 1u), (uint32_t)total);
+                if (!mbar_wait_bounded(&sh.tq_empty[qi], qphase ^ 1u, abort, p.ctl)) { ok = false; break; }
+                *reinterpret_cast<volatile int32_t*>(&sh.tq[qi]) = w;
+                mbar_arrive(&sh.tq_full[qi]);
+                if (++qi == kTileRing) { qi = 0; qphase ^= 1u; }
+                if (w >= total) break;
                 Tile t;
                 decode_tile<kBNMax>(sh, E, n_col_tiles, w, t);
                 int64_t r0, r1;
@@ -327,9 +359,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Instruction descriptor: E2M1 x E2M1 (format 1), both K-major, UE4M3
         // scales, M = 128 (bits 24-28 hold M >> 4), N in bits 17-22 (N >> 3).
         const uint32_t idesc_base = (1u << 7) | (1u << 10) | ((uint32_t)(kBM >> 4) << 24);
-        uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
+        uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0, qi = 0, qphase = 0;
         bool ok = true;
-        for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        while (ok) {
+            int32_t w;
+            if (!next_tile(sh, qi, qphase, w, lane, abort, p.ctl)) { ok = false; break; }
+            if (w >= total) break;
             Tile t;
             decode_tile<kBNMax>(sh, E, n_col_tiles, w, t);
             const uint32_t idesc = idesc_base | ((uint32_t)(t.bn >> 3) << 17);
@@ -385,9 +420,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Activation scales arrive by TMA as [rows][16 bytes] (row-major, one stage).
         const int quad = warp & 3;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        uint32_t stage = 0, phase = 0;
+        uint32_t stage = 0, phase = 0, qi = 0, qphase = 0;
         bool ok = true;
-        for (int32_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        while (ok) {
+            int32_t w;
+            if (!next_tile(sh, qi, qphase, w, lane, abort, p.ctl)) break;
+            if (w >= total) break;
             for (int32_t kt = 0; kt < ksteps_total; kt++) {
                 if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl)) {
                     ok = false;
@@ -430,8 +468,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const float a_g = __ldg(p.a_gscale);
         uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
-        uint32_t abuf = 0, aphase = 0;
-        for (int32_t w = blockIdx.x; w < total; w += gridDim.x) {
+        uint32_t abuf = 0, aphase = 0, qi = 0, qphase = 0;
+        while (true) {
+            int32_t w;
+            if (!next_tile(sh, qi, qphase, w, lane, abort, p.ctl)) break;
+            if (w >= total) break;
             Tile t;
             decode_tile<kBNMax>(sh, E, n_col_tiles, w, t);
             if (!warp_wait(&sh.acc_full[abuf], aphase, abort, p.ctl)) break;
@@ -488,6 +529,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 2) tmem_dealloc(tmem, kTmemCols);
+    // The last CTA to finish (every producer has taken its final item) leaves the counters at zero for
+    // the next launch that draws this slot.
+    if (tid == 0 && atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+        atomicExch(p.sched, 0u);
+        atomicExch(p.sched + 1, 0u);
+    }
 }
 
 }  // namespace gg
@@ -688,6 +735,8 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const ui
     prm.K = K;
     prm.swiglu = epi == NVFP4_EPI_SWIGLU ? 1 : 0;
     prm.amax_out = out_amax;
+    prm.sched = sched_counter_slot();
+    if (!prm.sched) return NVFP4_ERR_CUDA;
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
