@@ -90,8 +90,17 @@ def test_ragged_experts_and_row_tiles(swiglu):
 
 
 @pytest.mark.parametrize("swiglu", [False, True])
+def test_narrow_tiles_several_row_tiles(swiglu):
+    # the same ragged experts plus empty ones, so that the mean stays below the wide-tile threshold and the
+    # 64-row (narrow) tile shape takes experts of 65 and 130 rows in several row tiles
+    rows = [0, 1, 17, 64, 65, 130, 0, 0, 0, 0]
+    assert sum(rows) < nv.gemm_plan()["wide_min_avg_rows"] * len(rows)
+    run_full(rows, 512, 512, swiglu, seed=12)
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
 def test_wide_tiles_ragged(swiglu):
-    # experts averaging >= 96 rows take the 128-row tile shape: empty, partial, exact, 128 + 1, several tiles
+    # experts averaging >= 32 rows take the 128-row tile shape: empty, partial, exact, 128 + 1, several tiles
     run_full([0, 100, 128, 129, 300, 17], 512, 768, swiglu, seed=6)
 
 
