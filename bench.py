@@ -123,8 +123,8 @@ def measured_traffic(config: str):
     sources = tuple(x.strip().strip("`") for x in fields.get("sources", "").split(",") if x.strip()) or GEMM_SOURCES
     if fields.get("source_sha256") != gemm_source_sha256(sources):
         return None
-    try:
-        return int(fields["gate_up_dram_bytes_per_launch"])
+    try:   # the dominant GEMM launch: the gate/up GEMM of a layer, the GEMM of the dense workload
+        return int(fields.get("gate_up_dram_bytes_per_launch") or fields["dram_bytes_per_launch"])
     except (KeyError, ValueError):
         return None
 
@@ -597,7 +597,8 @@ def main_dense(args, cfg, metric, world, rank, local_rank):
                    "l2": "flushed between steps (256 MB write, outside the timed events)",
                    "step": "quantize(A) + GEMM with B quantised once beforehand"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": achieved / fp4_peak, "traffic": None, "kernel": "grouped_gemm_kernel (E=1)",
+                     "frac": achieved / fp4_peak, "traffic": measured_traffic("dense"),
+                     "kernel": "grouped GEMM, E=1 (CTA-pair tiles)",
                      "peak_source": peaks["source"] + " bf16 x 4 (nominal FP4/BF16 ratio)",
                      "avg_launch_ms": gemm_ms},
         "clocks": clk, "gpu_launches": int(launches), "e2e": None, "cpu_baseline": cb,
