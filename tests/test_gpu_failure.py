@@ -44,3 +44,29 @@ def test_stalled_producer_times_out_then_context_recovers():
     ref = oracle.grouped_gemm(host(a_q), host(a_sf), host(a_g)[0], host(pw.q), host(pw.sf), host(pw.gscale),
                               np.array([0, 16, 32], np.int32), 256, 256, False)
     compare_bf16(host_bits(out), oracle.bf16_round(ref), "gemm after a timed-out launch", exact=ref)
+    # every counter slot of the dynamic schedule (the timed-out launch's among them) is clean when drawn
+    # again: 2 x 64 more launches, each equal to the first
+    first = host_bits(out)
+    for _ in range(128):
+        again = nv.grouped_gemm(a_q, a_sf, a_g, pw, off, False)
+    assert nv.device_status() == 0
+    assert np.array_equal(host_bits(again), first)
+
+
+def test_concurrent_launches_on_several_streams():
+    # GEMMs in flight on four streams at once draw different counter slots of the dynamic schedule; each
+    # result equals the serial one bit for bit
+    require_gpu()
+    a_q, a_sf, a_g, pw, off = small_case()
+    ref = host_bits(nv.grouped_gemm(a_q, a_sf, a_g, pw, off, False))
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    outs = []
+    torch.cuda.synchronize()
+    for i in range(48):
+        s = streams[i % 4]
+        with torch.cuda.stream(s):
+            outs.append(nv.grouped_gemm(a_q, a_sf, a_g, pw, off, False, stream=s))
+    torch.cuda.synchronize()
+    assert nv.device_status() == 0
+    for o in outs:
+        assert np.array_equal(host_bits(o), ref)
