@@ -172,6 +172,17 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// The producer: take the next work item of the grid and publish it in the ring. False when a wait ran out.
+__device__ __forceinline__ bool publish_tile(Shared& sh, const Params& p, int32_t total, uint32_t& qi,
+                                             uint32_t& qphase, int32_t& w, volatile int* abort) {
+    w = (int32_t)min(atomicAdd(p.sched, 1u), (uint32_t)total);
+    if (!mbar_wait_bounded(&sh.tq_empty[qi], qphase ^ 1u, abort, p.ctl)) return false;
+    *reinterpret_cast<volatile int32_t*>(&sh.tq[qi]) = w;
+    mbar_arrive(&sh.tq_full[qi]);
+    if (++qi == kTileRing) { qi = 0; qphase ^= 1u; }
+    return true;
+}
+
 // Next work item of this CTA for one consumer role (a whole warp): the producer publishes the items it
 // took from the launch's work counter in a ring of kTileRing entries. False when a wait ran out.
 __device__ __forceinline__ bool next_tile(Shared& sh, uint32_t& qi, uint32_t& qphase, int32_t& w, int lane,
@@ -302,17 +313,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_w_reuse = l2_policy_evict_normal();
             const uint64_t pol_a = l2_policy_evict_last();
             uint32_t stage = 0, phase = 0, qi = 0, qphase = 0;
-            bool ok = true;
-            while (ok) {
-                // dynamic schedule: the next work item of the whole grid, in increasing order, so items
-                // that share a weight tile (row tile fastest) still run side by side, and CTAs that run
-                // ahead take the tail
-                int32_t w = (int32_t)min(atomicAdd(p.sched, 1u), (uint32_t)total);
-                if (!mbar_wait_bounded(&sh.tq_empty[qi], qphase ^ 1u, abort, p.ctl)) { ok = false; break; }
-                *reinterpret_cast<volatile int32_t*>(&sh.tq[qi]) = w;
-                mbar_arrive(&sh.tq_full[qi]);
-                if (++qi == kTileRing) { qi = 0; qphase ^= 1u; }
-                if (w >= total) break;
+            // dynamic schedule: work items of the whole grid in increasing order, so items that share a
+            // weight tile (row tile fastest) still run side by side, and CTAs that run ahead take the
+            // tail. The item after the current one is published before the current one's loads, so the
+            // counter's round trip overlaps the MMAs.
+            int32_t w = total, w_next = total;
+            bool ok = publish_tile(sh, p, total, qi, qphase, w, abort);
+            if (ok && w < total) ok = publish_tile(sh, p, total, qi, qphase, w_next, abort);
+            while (ok && w < total) {
                 Tile t;
                 decode_tile<kBNMax>(sh, E, n_col_tiles, w, t);
                 int64_t r0, r1;
@@ -346,6 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     issued_parity[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
+                if (!ok) break;
+                w = w_next;
+                if (w < total) ok = publish_tile(sh, p, total, qi, qphase, w_next, abort);
             }
             if (!ok || *abort) {
                 // Abort path: let every copy already issued land before the CTA can exit.

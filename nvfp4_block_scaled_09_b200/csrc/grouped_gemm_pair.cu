@@ -51,8 +51,15 @@ constexpr uint32_t kTmemSFRing = kAccCols;
 static_assert(kTmemSFRing + kStages * kSFSlot <= kTmemCols, "TMEM budget");
 static_assert(kStageBytes % 1024 == 0 && kOffB % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 
+constexpr int kTileRing = 4;                      // work items the even CTA may publish ahead
+constexpr int kTileConsumersPerCta = 13;          // even CTA: MMA warp + 4 scale writers + 8 epilogue warps;
+                                                  // odd CTA: its producer + 4 scale writers + 8 epilogue warps
+
 struct Shared {
     alignas(16) uint16_t ostage[kEpiWarps][32 * 32];  // epilogue: one 32-token x 32-column BF16 block per warp
+    uint64_t tq_full[kTileRing];  // the even CTA published tq[i] (in this CTA's copy of the ring)
+    uint64_t tq_empty[kTileRing]; // even CTA: every consumer warp of both CTAs read entry i
+    int32_t tq[kTileRing];        // work item index (>= total: no more work)
     uint64_t full_tma[kStages];   // this CTA's loads of the stage landed
     uint64_t sf_ready[kStages];   // even CTA: both CTAs' scales are in TMEM (8 warp arrivals)
     uint64_t empty[kStages];      // the pair's MMAs of the stage completed (commit from the even CTA)
@@ -82,6 +89,7 @@ struct Params {
     int64_t K;
     int32_t swiglu;
     uint32_t* amax_out;   // nullable: raised to max |out| (BF16 bits)
+    uint32_t* sched;      // this launch's work counter [0] and finished-CTA counter [1]; zero at launch
     DeviceCtl ctl;
 };
 
@@ -116,6 +124,52 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ void arrive_on_leader(uint64_t* bar, uint32_t rank) {
     if (rank == 0) mbar_arrive(bar);
     else mbar_arrive_cluster(cluster_smem_addr(bar, 0));
+}
+
+// ---- the pair's work-item ring -------------------------------------------------------------------
+// The even CTA's producer takes each work item from the launch's counter and writes it into both CTAs'
+// copies of the ring (the odd CTA's through distributed shared memory, released at cluster scope); every
+// consumer warp of both CTAs reports on the even CTA's tq_empty once it has read an entry.
+__device__ __forceinline__ bool tq_wait(Shared& sh, uint32_t qi, uint32_t qphase, uint32_t rank, volatile int* abort,
+                                        const DeviceCtl& ctl) {
+    return rank == 0 ? mbar_wait_bounded(&sh.tq_full[qi], qphase, abort, ctl)
+                     : mbar_wait_bounded_acq_cluster(&sh.tq_full[qi], qphase, abort, ctl);
+}
+__device__ __forceinline__ void tq_release(Shared& sh, uint32_t qi, uint32_t rank) {
+    if (rank == 0) mbar_arrive(&sh.tq_empty[qi]);
+    else mbar_arrive_release_cluster(cluster_smem_addr(&sh.tq_empty[qi], 0));
+}
+// Next work item for a whole consumer warp. False when a wait ran out.
+__device__ __forceinline__ bool next_tile_warp(Shared& sh, uint32_t rank, uint32_t& qi, uint32_t& qphase, int32_t& w,
+                                               int lane, volatile int* abort, const DeviceCtl& ctl) {
+    const bool ok = __all_sync(0xFFFFFFFFu, tq_wait(sh, qi, qphase, rank, abort, ctl));
+    if (!ok) return false;
+    w = *reinterpret_cast<volatile int32_t*>(&sh.tq[qi]);
+    __syncwarp();
+    if (lane == 0) tq_release(sh, qi, rank);
+    if (++qi == kTileRing) { qi = 0; qphase ^= 1u; }
+    return true;
+}
+// Next work item for one thread (the odd CTA's producer).
+__device__ __forceinline__ bool next_tile_thread(Shared& sh, uint32_t rank, uint32_t& qi, uint32_t& qphase,
+                                                 int32_t& w, volatile int* abort, const DeviceCtl& ctl) {
+    if (!tq_wait(sh, qi, qphase, rank, abort, ctl)) return false;
+    w = *reinterpret_cast<volatile int32_t*>(&sh.tq[qi]);
+    tq_release(sh, qi, rank);
+    if (++qi == kTileRing) { qi = 0; qphase ^= 1u; }
+    return true;
+}
+// The even CTA's producer: take the next work item of the grid and publish it to both CTAs.
+__device__ __forceinline__ bool publish_tile(Shared& sh, const Params& p, int32_t total, uint32_t& qi,
+                                             uint32_t& qphase, int32_t& w, volatile int* abort) {
+    w = (int32_t)min(atomicAdd(p.sched, 1u), (uint32_t)total);
+    if (!mbar_wait_bounded_acq_cluster(&sh.tq_empty[qi], qphase ^ 1u, abort, p.ctl)) return false;
+    *reinterpret_cast<volatile int32_t*>(&sh.tq[qi]) = w;
+    st_shared_cluster_u32(cluster_smem_addr(&sh.tq[qi], 1), (uint32_t)w);
+    mbar_arrive(&sh.tq_full[qi]);
+    mbar_arrive_release_cluster(cluster_smem_addr(&sh.tq_full[qi], 1));   // orders the store above
+    if (++qi == kTileRing) { qi = 0; qphase ^= 1u; }
+    return true;
 }
 
 // Expert offsets and the first work item of each expert (every CTA builds its own copy).
@@ -179,7 +233,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     volatile int* abort = &sh.abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
-    const uint32_t pair = cluster_id_x(), npairs = num_clusters_x();
     const int32_t E = p.E;
     const int32_t n_col_tiles = (int32_t)(p.swiglu ? (p.N / 2) / kBM : p.N / (2 * kBM));
     const int32_t ksteps_total = (int32_t)(p.K / kBK);
@@ -199,6 +252,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_init(&sh.acc_full, 1);
         mbar_init(&sh.acc_empty, 2 * kEpiWarps);
         mbar_init(&sh.drain, 1);
+        for (int i = 0; i < kTileRing; i++) {
+            mbar_init(&sh.tq_full[i], 1);
+            mbar_init(&sh.tq_empty[i], 2 * kTileConsumersPerCta);
+        }
         fence_barrier_init();
     }
     // everything above overlaps the previous kernel; global memory only from here on
@@ -231,9 +288,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint64_t pol_w_once = l2_policy_evict_first();
             const uint64_t pol_w_reuse = l2_policy_evict_normal();
             const uint64_t pol_a = l2_policy_evict_normal();
-            uint32_t stage = 0, phase = 0;
-            bool ok = true;
-            for (int32_t w = pair; w < total && ok; w += npairs) {
+            uint32_t stage = 0, phase = 0, qi = 0, qphase = 0;
+            // dynamic schedule: work items in increasing order (row tiles of one weight tile side by side).
+            // The even CTA publishes the item after the current one before the current one's loads, so
+            // the counter's round trip and the cross-CTA publication overlap the MMAs.
+            int32_t w = total, w_next = total;
+            bool ok;
+            if (rank == 0) {
+                ok = publish_tile(sh, p, total, qi, qphase, w, abort);
+                if (ok && w < total) ok = publish_tile(sh, p, total, qi, qphase, w_next, abort);
+            } else {
+                ok = next_tile_thread(sh, rank, qi, qphase, w, abort, p.ctl);
+            }
+            while (ok && w < total) {
                 Tile t;
                 decode_tile(sh, E, w, t);
                 const uint64_t pol_w = (sh.off[t.e + 1] - sh.off[t.e] > kBNMax) ? pol_w_reuse : pol_w_once;
@@ -283,6 +350,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     issued_parity[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
+                if (!ok) break;
+                if (rank == 0) {
+                    w = w_next;
+                    if (w < total) ok = publish_tile(sh, p, total, qi, qphase, w_next, abort);
+                } else {
+                    ok = next_tile_thread(sh, rank, qi, qphase, w, abort, p.ctl);
+                }
             }
             if (!ok || *abort) {
                 for (int s = 0; s < kStages; s++)
@@ -300,9 +374,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int tile_row = p.swiglu ? (int)rank * 64 + quad * 16 + (lane & 15) : quad * 32 + lane;
         const uint32_t sfa_off = kOffSFA + ((p.swiglu && lane >= 16) ? kTileSFBytes : 0) + (tile_row & 31) * 16 +
                                  (tile_row >> 5) * 4;
-        uint32_t stage = 0, phase = 0;
+        uint32_t stage = 0, phase = 0, qi = 0, qphase = 0;
         bool ok = true;
-        for (int32_t w = pair; w < total && ok; w += npairs) {
+        while (ok) {
+            int32_t w;
+            if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl) || w >= total) break;
             for (int32_t kt = 0; kt < ksteps_total; kt++) {
                 if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl)) { ok = false; break; }
                 tc_fence_after();
@@ -339,9 +415,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t idesc_base = (1u << 7) | (1u << 10) | ((uint32_t)((2 * kBM) >> 4) << 24);
             const uint32_t peer_empty0 = cluster_smem_addr(&sh.empty[0], 1);
             const uint32_t own_empty0 = cluster_smem_addr(&sh.empty[0], 0);
-            uint32_t stage = 0, phase = 0, aphase = 0;
+            uint32_t stage = 0, phase = 0, aphase = 0, qi = 0, qphase = 0;
             bool ok = true;
-            for (int32_t w = pair; w < total && ok; w += npairs) {
+            while (ok) {
+                int32_t w;
+                if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl)) { ok = false; break; }
+                if (w >= total) break;
                 Tile t;
                 decode_tile(sh, E, w, t);
                 const uint32_t idesc = idesc_base | ((uint32_t)(t.bn >> 3) << 17);
@@ -396,8 +475,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const bool up_lane = lane >= 16;
         const float a_g = __ldg(p.a_gscale);
         uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
-        uint32_t aphase = 0;
-        for (int32_t w = pair; w < total; w += npairs) {
+        uint32_t aphase = 0, qi = 0, qphase = 0;
+        while (true) {
+            int32_t w;
+            if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl) || w >= total) break;
             Tile t;
             decode_tile(sh, E, w, t);
             if (!warp_wait(&sh.acc_full, aphase, abort, p.ctl)) break;
@@ -481,6 +562,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     cluster_sync();
     tc_fence_after();
     if (warp == 2) tmem_dealloc_pair(tmem, kTmemCols);
+    // The last CTA to finish leaves the work counters at zero for the next launch that draws this slot.
+    if (tid == 0 && atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+        atomicExch(p.sched, 0u);
+        atomicExch(p.sched + 1, 0u);
+    }
 }
 
 }  // namespace gp
@@ -541,6 +627,8 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     prm.K = K;
     prm.swiglu = swiglu;
     prm.amax_out = out_amax;
+    prm.sched = sched_counter_slot();
+    if (!prm.sched) return NVFP4_ERR_CUDA;
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
