@@ -11,7 +11,7 @@
 // Design (chosen for B200, not the SM120 tiles the pages analyse):
 //  * Swap-AB orientation. Experts see 16-256 rows, so the 128-row MMA M side
 //    holds weight rows and the activation rows ride on the MMA N side
-//    (16..64, in steps of 16, picked per tile on the device). Every weight byte
+//    (16..64 or 16..128, in steps of 16, picked per tile on the device). Every weight byte
 //    is read once per (expert, row tile); decode is a pure weight stream.
 //  * Tile = 2 x 128 weight rows x up to 64 activation rows, K stage = 256.
 //    SWIGLU pairs gate rows [n0, n0+128) with up rows [N/2+n0, ...) so both
@@ -41,10 +41,12 @@
 //    tables, checked against the
 //    device's opt-in limit before launch (the same predicate
 //    nvfp4_can_implement() reports, so a passing check never fails to launch).
-//  * Persistent CTAs (one per SM) walk (expert, column tile, row tile) work
-//    items read from device-resident expert offsets; no host synchronisation.
-//    Two TMEM accumulator buffers let the epilogue of one tile overlap the
-//    main loop of the next.
+//  * Persistent CTAs (one per SM) take (expert, column tile, row tile) work
+//    items from a grid-wide counter (dynamic schedule: CTAs that run ahead take
+//    the tail) and read expert offsets from device memory; no host
+//    synchronisation. The producer passes each item to the other warp roles
+//    through a small ring in shared memory. Two TMEM accumulator buffers let the
+//    epilogue of one tile overlap the main loop of the next (narrow shape).
 //  * Every wait is bounded (%globaltimer); on expiry the kernel latches
 //    NVFP4_ERR_DEVICE_TIMEOUT, drains its in-flight copies and MMAs, frees
 //    tensor memory and returns.

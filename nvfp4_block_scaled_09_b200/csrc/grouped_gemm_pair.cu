@@ -18,8 +18,10 @@
 // Synchronisation uses no multicast: the peer's scale-writer and epilogue warps
 // arrive on the even CTA's barriers through cluster addresses (mapa), and the
 // even CTA's MMA completions are committed to each CTA's barrier separately.
-// Every wait is bounded as in the one-SM kernel; a cluster barrier guards the
-// release of tensor memory.
+// Work items come from a grid-wide counter (dynamic schedule); the even CTA
+// takes each one and writes it into both CTAs' work-item rings. Every wait is
+// bounded as in the one-SM kernel; a cluster barrier guards the release of
+// tensor memory.
 #include "common.cuh"
 
 namespace nvfp4 {
