@@ -292,7 +292,7 @@ class MoEBench:
                               P(b + lay["g_x"]), 0, scratch, sbytes, s)
         rec(1)
         st |= L.moe_permute(P(self.ids.data_ptr()), T, k, E, P(b + lay["q_x"]), P(b + lay["sf_x"]), H,
-                            P(b + lay["q_perm"]), P(b + lay["sf_perm"]), P(b + lay["offsets"]),
+                            P(b + lay["q_perm"]), P(b + lay["sf_perm"]), nv.SF_KSTAGE, P(b + lay["offsets"]),
                             P(b + lay["perm_src"]), P(b + lay["inv_perm"]), scratch, sbytes, s)
         rec(2)
         if gemm_ev is not None:
@@ -305,7 +305,7 @@ class MoEBench:
             gemm_ev[1].record()
         rec(3)
         st |= L.nvfp4_quantize_from_amax(P(b + lay["h"]), R, I, P(b + lay["amax_h"]), P(b + lay["q_h"]),
-                                         P(b + lay["sf_h"]), P(b + lay["g_h"]), 0, s)
+                                         P(b + lay["sf_h"]), P(b + lay["g_h"]), nv.SF_KSTAGE, s)
         rec(4)
         st |= L.moe_grouped_gemm_nvfp4(P(b + lay["q_h"]), P(b + lay["sf_h"]), P(b + lay["g_h"]),
                                        P(W.w2.packed.data_ptr()), P(W.w2.gscale.data_ptr()),
@@ -530,7 +530,7 @@ def main_dense(args, cfg, metric, world, rank, local_rank):
     pw = nv.prepare_expert_weights(b)
     del b
     a_q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
-    a_sf = torch.empty((M, K // 16), dtype=torch.uint8, device=dev)
+    a_sf = torch.empty((K // 256, M, 16), dtype=torch.uint8, device=dev)   # K-stage slabs (the GEMM's layout)
     a_g = torch.empty(1, dtype=torch.float32, device=dev)
     qws = torch.empty(nv.quantize_workspace_size(M, K), dtype=torch.uint8, device=dev)
     c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -540,7 +540,7 @@ def main_dense(args, cfg, metric, world, rank, local_rank):
     def step(e0=None, e1=None, e2=None):
         if e0 is not None:
             e0.record()
-        nv.quantize(a, q=a_q, sf=a_sf, g=a_g, ws=qws)
+        nv.quantize(a, q=a_q, sf=a_sf, g=a_g, ws=qws, layout=nv.SF_KSTAGE)
         if e1 is not None:
             e1.record()
         nv.grouped_gemm(a_q, a_sf, a_g, pw, off, False, out=c)

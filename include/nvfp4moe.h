@@ -74,8 +74,14 @@ typedef enum { NVFP4_EPI_NONE = 0, NVFP4_EPI_SWIGLU = 1 } nvfp4_epilogue;
  *   (row block rb, step kc) pair is a 512-byte atom at ((rb * (K/64)) + kc) * 512,
  *   and inside it the scale of row r, block b sits at
  *   (r % 32) * 16 + ((r % 128) / 32) * 4 + (b % 4).
- *   Requires rows % 128 == 0 and K % 64 == 0. */
-typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1 } nvfp4_sf_layout;
+ *   Requires rows % 128 == 0 and K % 64 == 0.
+ * NVFP4_SF_KSTAGE: one [rows x 16 bytes] slab per 256-element K step: the scale
+ *   of row r, block b sits at ((b / 16) * rows + r) * 16 + (b % 16). The 16
+ *   scales of a K step are one 16-byte piece per row, and the pieces of
+ *   consecutive rows are adjacent, so any run of rows of one K step is one
+ *   contiguous copy. Requires K % 256 == 0. The grouped GEMM reads its
+ *   activation scales in this layout. */
+typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1, NVFP4_SF_KSTAGE = 2 } nvfp4_sf_layout;
 
 /* ------------------------------------------------------------------------ */
 /* nvfp4_quantize: BF16 -> packed E2M1 codes + E4M3 block scales + FP32      */
@@ -91,7 +97,7 @@ typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1 } nvfp4_sf_layout;
 /* Arguments:                                                                */
 /*   x                [rows, K] BF16 bits, device, 16-byte aligned           */
 /*   rows, K          rows >= 1, K % 16 == 0 (MMA_TILED: rows % 128 == 0,    */
-/*                    K % 64 == 0)                                           */
+/*                    K % 64 == 0; KSTAGE: K % 256 == 0)                     */
 /*   global_scale_in  device FP32 scalar or NULL (dynamic amax)             */
 /*   q                [rows, K/2] bytes, device, 8-byte aligned              */
 /*   sf               rows*K/16 bytes, device, in `layout`                   */
@@ -134,20 +140,24 @@ NVFP4_API nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows,
 /*   Inside expert e, pairs are ordered by token t ascending, then slot j.   */
 /*   perm_src[p] = source token of permuted row p;                           */
 /*   inv_perm[t*k + j] = permuted row of pair (t, j);                        */
-/*   q_perm[p] = q[perm_src[p]] (K/2 bytes), sf_perm[p] = sf[perm_src[p]]    */
-/*   (K/16 bytes, row-major scales).                                         */
+/*   q_perm[p] = q[perm_src[p]] (K/2 bytes); the K/16 scale bytes of row p   */
+/*   are those of row perm_src[p] of sf, written in sf_perm_layout:          */
+/*   NVFP4_SF_KSTAGE (what the grouped GEMM reads; T*k rows per slab) or     */
+/*   NVFP4_SF_ROWMAJOR (sf_perm[p] = sf[perm_src[p]], e.g. for sending rows  */
+/*   to other ranks).                                                        */
 /* Arguments: topk_ids [T, k] int32 (device) with ids in [0, E), distinct   */
 /*   within a token (violations latch NVFP4_ERR_DEVICE_INPUT); 1 <= T,       */
 /*   1 <= k <= 32, 1 <= E <= 1024, T*k < 2^31; K % 256 == 0; q [T, K/2],    */
-/*   sf [T, K/16] row-major; outputs q_perm [T*k, K/2], sf_perm [T*k, K/16], */
-/*   expert_offsets [E+1], perm_src [T*k], inv_perm [T*k]; all device,       */
-/*   16-byte aligned. ws of moe_permute_workspace_size() bytes.              */
+/*   sf [T, K/16] row-major; outputs q_perm [T*k, K/2], sf_perm (T*k*K/16    */
+/*   bytes), expert_offsets [E+1], perm_src [T*k], inv_perm [T*k]; all       */
+/*   device, 16-byte aligned. ws of moe_permute_workspace_size() bytes.      */
+/*   Any other sf_perm_layout returns NVFP4_ERR_INVALID_ARG.                 */
 /* ------------------------------------------------------------------------ */
 NVFP4_API size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E);
 NVFP4_API nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
                          const uint8_t* q, const uint8_t* sf, int64_t K,
-                         uint8_t* q_perm, uint8_t* sf_perm, int32_t* expert_offsets,
-                         int32_t* perm_src, int32_t* inv_perm,
+                         uint8_t* q_perm, uint8_t* sf_perm, nvfp4_sf_layout sf_perm_layout,
+                         int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
                          void* ws, size_t ws_bytes, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
@@ -173,8 +183,9 @@ NVFP4_API nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k
 #define NVFP4_PERMUTE_NOALLOC_SCRATCH_ENTRIES 65536
 NVFP4_API nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
                                  const uint8_t* q, const uint8_t* sf, int64_t K,
-                                 uint8_t* q_perm, uint8_t* sf_perm, int32_t* expert_offsets,
-                                 int32_t* perm_src, int32_t* inv_perm, nvfp4_stream_t stream);
+                                 uint8_t* q_perm, uint8_t* sf_perm, nvfp4_sf_layout sf_perm_layout,
+                                 int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
+                                 nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* moe_grouped_gemm_nvfp4: one launch for every expert's FP4 block-scaled    */
@@ -189,7 +200,9 @@ NVFP4_API nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, i
 /*           (rows [0, N/2) of each W_e are the gate, [N/2, N) the up        */
 /*           projection),                                     out [rows, N/2]*/
 /* Arguments:                                                                */
-/*   a_q [max_rows, K/2], a_sf [max_rows, K/16] row-major, a_gscale scalar   */
+/*   a_q [max_rows, K/2]; a_sf: max_rows*K/16 bytes in NVFP4_SF_KSTAGE with  */
+/*     max_rows rows per slab (as moe_permute writes it for T*k rows);       */
+/*     a_gscale scalar                                                       */
 /*   w_packed: the weights [E, N, K] packed by nvfp4_pack_weights() as one   */
 /*     [E*N, K] matrix (nvfp4_packed_weight_bytes(E*N, K) bytes);           */
 /*     w_gscale [E]                                                          */
@@ -271,10 +284,10 @@ NVFP4_API nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* i
 /* ------------------------------------------------------------------------ */
 typedef struct {
     size_t q_x, sf_x, g_x;                 /* quantised x [T, H/2], [T, H/16], scalar */
-    size_t q_perm, sf_perm;                /* [T*k, H/2], [T*k, H/16] */
+    size_t q_perm, sf_perm;                /* [T*k, H/2]; T*k*H/16 bytes, NVFP4_SF_KSTAGE */
     size_t offsets, perm_src, inv_perm;    /* [E+1], [T*k], [T*k] int32 */
     size_t h;                              /* [T*k, I] BF16 */
-    size_t q_h, sf_h, g_h;                 /* [T*k, I/2], [T*k, I/16], scalar */
+    size_t q_h, sf_h, g_h;                 /* [T*k, I/2]; T*k*I/16 bytes, NVFP4_SF_KSTAGE; scalar */
     size_t amax_h;                         /* uint32: max |h| (BF16 bits), from the gate/up GEMM */
     size_t y;                              /* [T*k, H] BF16 */
     size_t scratch;                        /* quantize / permute scratch */
@@ -330,7 +343,9 @@ typedef struct {                 /* fields up to `threads` describe the narrow (
 
 NVFP4_API nvfp4_status nvfp4_gemm_get_plan(nvfp4_gemm_plan* plan);
 /* Expect-tx bytes one stage's TMA and bulk copies deliver for a tile of `tokens` rows
- * (wide != 0: the wide tile shape). -1 when tokens is outside [1, tile maximum]. */
+ * (wide != 0: the wide tile shape): both packed weight tiles, the activation rows
+ * rounded up to 16 and the `tokens` rows' 16 scale bytes of the K step. -1 when
+ * tokens is outside [1, tile maximum]. */
 NVFP4_API int64_t nvfp4_gemm_stage_tx_bytes(int32_t tokens, int32_t wide);
 /* Pure host check against a given opt-in shared-memory budget (bytes per block). */
 NVFP4_API nvfp4_status nvfp4_can_implement_with_budget(int64_t N, int64_t K, int32_t E, nvfp4_epilogue epi,

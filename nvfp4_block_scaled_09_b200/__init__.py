@@ -35,7 +35,7 @@ STATUS = {
 }
 OK = 0
 EPI_NONE, EPI_SWIGLU = 0, 1
-SF_ROWMAJOR, SF_MMA_TILED = 0, 1
+SF_ROWMAJOR, SF_MMA_TILED, SF_KSTAGE = 0, 1, 2
 
 
 class NVFP4Error(RuntimeError):
@@ -77,9 +77,9 @@ def lib():
         L.nvfp4_quantize.restype = st
         L.moe_permute_workspace_size.argtypes = [i32, i32, i32]
         L.moe_permute_workspace_size.restype = sz
-        L.moe_permute.argtypes = [P, i32, i32, i32, P, P, i64, P, P, P, P, P, P, sz, P]
+        L.moe_permute.argtypes = [P, i32, i32, i32, P, P, i64, P, P, ctypes.c_int, P, P, P, P, sz, P]
         L.moe_permute.restype = st
-        L.moe_permute_noalloc.argtypes = [P, i32, i32, i32, P, P, i64, P, P, P, P, P, P]
+        L.moe_permute_noalloc.argtypes = [P, i32, i32, i32, P, P, i64, P, P, ctypes.c_int, P, P, P, P]
         L.moe_permute_noalloc.restype = st
         L.moe_grouped_gemm_nvfp4.argtypes = [P, P, P, P, P, P, i32, i64, i64, i64, ctypes.c_int, P, P]
         L.moe_grouped_gemm_nvfp4.restype = st
@@ -151,6 +151,13 @@ def _bits(t: torch.Tensor) -> torch.Tensor:
 
 # ----------------------------------------------------------------------------- quantize
 
+def _sf_empty(rows: int, K: int, layout: int, dev) -> torch.Tensor:
+    """Scale buffer of a [rows, K] tensor: [K/256, rows, 16] in the K-stage layout, else [rows, K/16]."""
+    if layout == SF_KSTAGE:
+        return torch.empty((K // 256, rows, 16), dtype=torch.uint8, device=dev)
+    return torch.empty((rows, K // 16), dtype=torch.uint8, device=dev)
+
+
 def quantize_workspace_size(rows: int, K: int) -> int:
     return int(lib().nvfp4_quantize_workspace_size(rows, K))
 
@@ -158,13 +165,14 @@ def quantize_workspace_size(rows: int, K: int) -> int:
 def quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None, layout: int = SF_ROWMAJOR,
              q: torch.Tensor | None = None, sf: torch.Tensor | None = None, g: torch.Tensor | None = None,
              ws: torch.Tensor | None = None, stream=None):
-    """x [rows, K] bf16 -> (q uint8 [rows, K/2], sf uint8 [rows*K/16], g float32 [1] = g_dec)."""
+    """x [rows, K] bf16 -> (q uint8 [rows, K/2], sf uint8, g float32 [1] = g_dec). sf is [rows, K/16] for
+    SF_ROWMAJOR and SF_MMA_TILED, [K/256, rows, 16] for SF_KSTAGE (the grouped GEMM's activation scales)."""
     _require_cuda(x, global_scale)
     x = _bits(x)
     rows, K = x.shape
     dev = x.device
     q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else q
-    sf = torch.empty((rows, K // 16), dtype=torch.uint8, device=dev) if sf is None else sf
+    sf = _sf_empty(rows, K, layout, dev) if sf is None else sf
     g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else g
     if ws is None and global_scale is None:
         ws = torch.empty(max(quantize_workspace_size(rows, K), 16), dtype=torch.uint8, device=dev)
@@ -194,7 +202,7 @@ def quantize_from_amax(x: torch.Tensor, amax_bits: torch.Tensor, layout: int = S
     rows, K = x.shape
     dev = x.device
     q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else q
-    sf = torch.empty((rows, K // 16), dtype=torch.uint8, device=dev) if sf is None else sf
+    sf = _sf_empty(rows, K, layout, dev) if sf is None else sf
     g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else g
     _check(lib().nvfp4_quantize_from_amax(_ptr(x), rows, K, _ptr(amax_bits), _ptr(q), _ptr(sf), _ptr(g), layout,
                                           _stream(stream)), "nvfp4_quantize_from_amax")
@@ -265,7 +273,9 @@ class Permuted:
 
 
 def permute(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_experts: int, ws=None,
-            stream=None) -> Permuted:
+            stream=None, sf_layout: int = SF_KSTAGE) -> Permuted:
+    """Group the routed rows by expert. sf is row-major [T, K/16]; sf_perm comes out in sf_layout:
+    SF_KSTAGE (what grouped_gemm reads, [K/256, T*k, 16]) or SF_ROWMAJOR ([T*k, K/16])."""
     _require_cuda(topk_ids, q, sf)
     if topk_ids.dtype != torch.int32:
         raise TypeError("topk_ids must be int32")
@@ -276,7 +286,7 @@ def permute(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_exper
     dev = q.device
     out = Permuted(
         q_perm=torch.empty((R, K // 2), dtype=torch.uint8, device=dev),
-        sf_perm=torch.empty((R, K // 16), dtype=torch.uint8, device=dev),
+        sf_perm=_sf_empty(R, K, sf_layout, dev),
         offsets=torch.empty(num_experts + 1, dtype=torch.int32, device=dev),
         perm_src=torch.empty(R, dtype=torch.int32, device=dev),
         inv_perm=torch.empty(R, dtype=torch.int32, device=dev),
@@ -284,13 +294,13 @@ def permute(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_exper
     if ws is None:
         ws = torch.empty(max(permute_workspace_size(T, k, num_experts), 16), dtype=torch.uint8, device=dev)
     _check(lib().moe_permute(_ptr(topk_ids), T, k, num_experts, _ptr(q), _ptr(sf), K, _ptr(out.q_perm),
-                             _ptr(out.sf_perm), _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm), _ptr(ws),
-                             ws.numel(), _stream(stream)), "moe_permute")
+                             _ptr(out.sf_perm), sf_layout, _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm),
+                             _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
     return out
 
 
 def permute_noalloc(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_experts: int,
-                    stream=None) -> Permuted:
+                    stream=None, sf_layout: int = SF_KSTAGE) -> Permuted:
     """moe_permute without a workspace: the library's own fixed device array holds the count table
     (for callers that cannot allocate device memory; see moe_permute_noalloc in the header)."""
     _require_cuda(topk_ids, q, sf)
@@ -303,24 +313,27 @@ def permute_noalloc(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, n
     dev = q.device
     out = Permuted(
         q_perm=torch.empty((R, K // 2), dtype=torch.uint8, device=dev),
-        sf_perm=torch.empty((R, K // 16), dtype=torch.uint8, device=dev),
+        sf_perm=_sf_empty(R, K, sf_layout, dev),
         offsets=torch.empty(num_experts + 1, dtype=torch.int32, device=dev),
         perm_src=torch.empty(R, dtype=torch.int32, device=dev),
         inv_perm=torch.empty(R, dtype=torch.int32, device=dev),
     )
     _check(lib().moe_permute_noalloc(_ptr(topk_ids), T, k, num_experts, _ptr(q), _ptr(sf), K, _ptr(out.q_perm),
-                                     _ptr(out.sf_perm), _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm),
-                                     _stream(stream)), "moe_permute_noalloc")
+                                     _ptr(out.sf_perm), sf_layout, _ptr(out.offsets), _ptr(out.perm_src),
+                                     _ptr(out.inv_perm), _stream(stream)), "moe_permute_noalloc")
     return out
 
 
 # ----------------------------------------------------------------------------- grouped GEMM
 
 def grouped_gemm(a_q, a_sf, a_g, w: PackedWeights, offsets, swiglu: bool, out=None, stream=None, amax_out=None):
-    """Per-expert NVFP4 GEMM. Returns bf16 [rows, N] (or [rows, N/2] with SwiGLU). With amax_out (device int32
-    [1], zeroed by the caller) the kernel also raises it to max |out| as BF16 bits."""
+    """Per-expert NVFP4 GEMM. a_sf holds the activation scales in the K-stage layout ([K/256, rows, 16], as
+    permute() and quantize(layout=SF_KSTAGE) write them). Returns bf16 [rows, N] (or [rows, N/2] with SwiGLU).
+    With amax_out (device int32 [1], zeroed by the caller) the kernel also raises it to max |out| as BF16 bits."""
     _require_cuda(a_q, a_sf, a_g, w.packed, w.gscale, offsets, amax_out)
     rows = a_q.shape[0]
+    if a_sf.dim() != 3 or tuple(a_sf.shape) != (w.K // 256, rows, 16):
+        raise ValueError(f"a_sf must be K-stage scales of shape {(w.K // 256, rows, 16)}, got {tuple(a_sf.shape)}")
     E = offsets.numel() - 1
     N, K = w.N, w.K
     nout = N // 2 if swiglu else N

@@ -189,13 +189,13 @@ extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_i
         return NVFP4_ERR_CUDA;
     if ((st = nvfp4_quantize(x, T, H, nullptr, q_x, sf_x, g_x, NVFP4_SF_ROWMAJOR, scratch, scratch_bytes, stream)))
         return st;
-    if ((st = moe_permute(topk_ids, T, k, E, q_x, sf_x, H, q_perm, sf_perm, off, perm_src, inv_perm, scratch,
-                          scratch_bytes, stream)))
+    if ((st = moe_permute(topk_ids, T, k, E, q_x, sf_x, H, q_perm, sf_perm, NVFP4_SF_KSTAGE, off, perm_src, inv_perm,
+                          scratch, scratch_bytes, stream)))
         return st;
     if ((st = moe_grouped_gemm_nvfp4_amax(q_perm, sf_perm, g_x, w13_packed, w13_gscale, off, E, R, 2 * I, H,
                                           NVFP4_EPI_SWIGLU, h, amax_h, stream)))
         return st;
-    if ((st = nvfp4_quantize_from_amax(h, R, I, amax_h, q_h, sf_h, g_h, NVFP4_SF_ROWMAJOR, stream))) return st;
+    if ((st = nvfp4_quantize_from_amax(h, R, I, amax_h, q_h, sf_h, g_h, NVFP4_SF_KSTAGE, stream))) return st;
     if ((st = moe_grouped_gemm_nvfp4(q_h, sf_h, g_h, w2_packed, w2_gscale, off, E, R, H, I, NVFP4_EPI_NONE, y,
                                      stream)))
         return st;

@@ -42,7 +42,7 @@ nvfp4_status check_launch();          // maps cudaGetLastError to a status
 size_t pair_gemm_smem_bytes();
 int pair_gemm_tokens_max();
 int pair_gemm_store_cols(int swiglu);   // output columns of one epilogue warp's tensor-store box
-nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full, const CUtensorMap& tm_sf,
+nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full,
                                       const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const uint8_t* a_sf,
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,

@@ -24,8 +24,8 @@
 //    ~15% faster from HBM than strided 2-D tiles).
 //  * Warp roles ("Peering into the CUTLASS Kernel Scheduler", The Discovery:
 //    explicit warp-specialised schedules that give A loads, B loads, MMA and
-//    epilogue their own warps): warp 0 issues the weight bulk copies and the
-//    TMA tiles of activations and of their row-major scales; warps 8-11 (one
+//    epilogue their own warps): warp 0 issues the weight bulk copies, the
+//    TMA tiles of activations and one bulk copy of their scales; warps 8-11 (one
 //    per TMEM lane quadrant) store every stage's
 //    scales into a per-stage TMEM ring with tcgen05.st; warp 2 owns tensor
 //    memory and issues only tcgen05.mma (scale copies issued on the MMA pipe
@@ -35,8 +35,14 @@
 //  * Stage accounting: the expected transaction bytes of a stage are the A
 //    tile bytes plus its scale bytes plus the B tile bytes ("Peering into the
 //    CUTLASS SharedStorage", The Message: MK bytes + NK bytes per stage): two
-//    packed weight tiles (codes + scales), the activation tile and one box of
-//    its scales.
+//    packed weight tiles (codes + scales), the activation tile and its rows'
+//    scales.
+//  * Activation scales come in the K-stage layout (one [rows x 16 B] slab per
+//    256-element K step), so a tile's scales for one stage are one contiguous
+//    run, fetched with one bulk copy. A 16-byte-wide TMA box over row-major
+//    scales costs one request per row: measured on B200 (loads alone, all SMs),
+//    such a 256-row box took ~190 ns per stage and brought the CTA-pair
+//    stage's loads from ~280 to ~440 ns.
 //  * Shared memory: 4 stages x 46 KB (narrow) or 54 KB (wide) + scheduler
 //    tables, checked against the
 //    device's opt-in limit before launch (the same predicate
@@ -199,8 +205,7 @@ __device__ __forceinline__ bool next_tile(Shared& sh, uint32_t& qi, uint32_t& qp
 
 template <class C>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_sf,
-                        const Params p) {
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const Params p) {
     constexpr int kBNMax = C::kBNMax;
     constexpr int kOffSFB = C::kOffSFB;
     constexpr int kStageBytes = C::kStageBytes;
@@ -222,7 +227,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         prefetch_tensormap(&tm_a);
-        prefetch_tensormap(&tm_sf);
         sh.abort = 0;
         for (int s = 0; s < kStages; s++) {
             mbar_init(&sh.full_tma[s], 1);
@@ -339,8 +343,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool reuse = (sh.off[t.e + 1] - sh.off[t.e]) > kBNMax;
                 const uint64_t pol_w = reuse ? pol_w_reuse : pol_w_once;
                 // MK part: two packed weight tiles (codes + scales); NK part: the activation
-                // tile and one box of its row-major scales (kBNMax rows x 16 bytes).
-                const uint32_t tx = (uint32_t)(kNumA * kPackedTileBytes + t.bn * kRowBytes + kBNMax * 16);
+                // tile and the tile's rows of the K step's scale slab (16 bytes per row, one
+                // contiguous run in the K-stage layout).
+                const uint32_t tx = (uint32_t)(kNumA * kPackedTileBytes + t.bn * kRowBytes + t.rows * 16);
+                const uint8_t* sfb = p.a_sf + (int64_t)t.row0 * 16;
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
                     if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
                     uint8_t* sb = stages + (size_t)stage * kStageBytes;
@@ -351,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bulk_load(sb + kOffA1, wp1 + (size_t)kt * kPackedTileBytes, kPackedTileBytes, bar, pol_w);
                     for (int32_t i = 0; i < t.bn / kBNStep; i++)
                         tma_load_2d(sb + kOffB + i * kBNStep * kRowBytes, &tm_a, kx, t.row0 + i * kBNStep, bar, pol_a);
-                    tma_load_2d(sb + kOffSFB, &tm_sf, kt * 16, t.row0, bar, pol_a);
+                    bulk_load(sb + kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, bar, pol_a);
                     issued[stage] = true;
                     issued_parity[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -430,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tcgen05.cp on the MMA pipe serialises with the MMAs around it).
         // MMA reads: row m of a weight block at lane m, column base + 4 kc + m/32;
         // activation row n at lane n % 32 of every quadrant, column base + 4 kc + n/32.
-        // Activation scales arrive by TMA as [rows][16 bytes] (row-major, one stage).
+        // Activation scales arrive as [rows][16 bytes] (the tile's rows of one K-stage slab).
         const int quad = warp & 3;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         uint32_t stage = 0, phase = 0, qi = 0, qphase = 0;
@@ -662,8 +668,8 @@ extern "C" int64_t nvfp4_gemm_stage_tx_bytes(int32_t tokens, int32_t wide) {
     if (tokens <= 0 || tokens > bn_max) return -1;
     const int64_t bn = (tokens + gg::kBNStep - 1) / gg::kBNStep * gg::kBNStep;
     // MK part: the two weight tiles with their scales (packed together); NK part: the activation
-    // tile plus one TMA box of its scales (bn_max rows x 16 bytes).
-    return (int64_t)gg::kNumA * gg::kPackedTileBytes + bn * gg::kRowBytes + bn_max * 16;
+    // tile plus its rows' 16 scale bytes of the K step (one bulk copy from the K-stage slab).
+    return (int64_t)gg::kNumA * gg::kPackedTileBytes + bn * gg::kRowBytes + (int64_t)tokens * 16;
 }
 
 extern "C" nvfp4_status nvfp4_can_implement_with_budget(int64_t N, int64_t K, int32_t E, nvfp4_epilogue epi,
@@ -687,8 +693,7 @@ extern "C" nvfp4_status nvfp4_can_implement(int64_t N, int64_t K, int32_t E, nvf
 }
 
 template <class C>
-static nvfp4_status launch_variant(const CUtensorMap& tm_a, const uint8_t* a_sf, const gg::Params& prm,
-                                   cudaStream_t s) {
+static nvfp4_status launch_variant(const CUtensorMap& tm_a, const gg::Params& prm, cudaStream_t s) {
     static bool configured[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
@@ -698,10 +703,7 @@ static nvfp4_status launch_variant(const CUtensorMap& tm_a, const uint8_t* a_sf,
             return NVFP4_ERR_CUDA;
         configured[dev] = true;
     }
-    CUtensorMap tm_sf;  // one stage of activation scales: kBNMax rows x 16 bytes
-    if (!encode_rows_map(&tm_sf, a_sf, prm.max_rows, prm.K / 16, C::kBNMax, 16)) return NVFP4_ERR_CUDA;
-    launch_pdl(gg::grouped_gemm_kernel<C>, dim3(device_sm_count()), dim3(gg::kThreads), C::kSmemBytes, s, tm_a, tm_sf,
-               prm);
+    launch_pdl(gg::grouped_gemm_kernel<C>, dim3(device_sm_count()), dim3(gg::kThreads), C::kSmemBytes, s, tm_a, prm);
     return NVFP4_OK;
 }
 
@@ -757,9 +759,6 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const ui
     prm.ctl.flags = debug_flags();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (max_rows >= kPairMinAvgRows * (int64_t)E) {
-        CUtensorMap tm_sf;  // one stage of activation scales for a whole pair tile: 256 rows x 16 bytes
-        if (!encode_rows_map(&tm_sf, a_sf, max_rows, K / 16, (uint32_t)pair_gemm_tokens_max(), 16))
-            return NVFP4_ERR_CUDA;
         CUtensorMap tm_a_full;  // one CTA's half of a full pair tile: 128 rows x 128 bytes
         if (!encode_rows_map(&tm_a_full, a_q, max_rows, K / 2, (uint32_t)pair_gemm_tokens_max() / 2, 128))
             return NVFP4_ERR_CUDA;
@@ -769,12 +768,12 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const ui
             return NVFP4_ERR_CUDA;
         CUtensorMap tm_wsw = tm_a;  // SWIGLU: interleaved gate/up weight slabs (unused otherwise)
         if (prm.swiglu && !encode_swiglu_weights_map(&tm_wsw, w_packed, E, N, K)) return NVFP4_ERR_CUDA;
-        return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_sf, tm_out, tm_wsw, a_sf, a_gscale, w_packed, w_gscale,
+        return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_out, tm_wsw, a_sf, a_gscale, w_packed, w_gscale,
                                         expert_offsets, E, max_rows, N, K, prm.swiglu, out, out_amax, s, status);
     }
     const bool wide = max_rows >= kWideMinAvgRows * (int64_t)E;
     const nvfp4_status ls =
-        wide ? launch_variant<gg::Wide>(tm_a, a_sf, prm, s) : launch_variant<gg::Narrow>(tm_a, a_sf, prm, s);
+        wide ? launch_variant<gg::Wide>(tm_a, prm, s) : launch_variant<gg::Narrow>(tm_a, prm, s);
     if (ls != NVFP4_OK) return ls;
     count_launch();
     return check_launch();

@@ -15,6 +15,11 @@
 // lanes 32q+16..32q+31: the matching up rows), so one warp reads both halves of
 // its 16 output columns and pairs them with a lane shuffle.
 //
+// One 256-column accumulator per CTA (the scale ring takes the rest of tensor
+// memory), so the epilogue warps first drain it into registers as final BF16
+// values and hand it back to the MMA warp; staging and storing those values
+// then overlaps the next tile's main loop.
+//
 // Synchronisation uses no multicast: the peer's scale-writer and epilogue warps
 // arrive on the even CTA's barriers through cluster addresses (mapa), and the
 // even CTA's MMA completions are committed to each CTA's barrier separately.
@@ -41,10 +46,11 @@ constexpr int kTileSFBytes = 2048;
 constexpr int kOffA = 0;                          // 128 weight rows x 128 B (SwiGLU: gate/up slabs of 16 rows, interleaved)
 constexpr int kOffSFA = kCodeBytes;               // scales of one packed tile (SwiGLU: gate tile's, then up tile's)
 constexpr int kOffB = kOffSFA + 2 * kTileSFBytes;  // this CTA's half of the activation rows
-constexpr int kOffSFB = kOffB + (kBNMax / 2) * kRowBytes;  // row-major scales of all kBNMax rows
+constexpr int kOffSFB = kOffB + (kBNMax / 2) * kRowBytes;  // scales of all the tile's rows, 16 bytes each
 constexpr int kStageBytes = kOffSFB + kBNMax * 16;         // 40960
 constexpr int kThreads = 512;                     // warps: 0 loads, 2 MMA, 4-7 + 12-15 epilogue, 8-11 scales
 constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant, alternating 32-token chunks
+constexpr int kChunksPerWarp = kBNMax / 32 / 2;   // 32-token chunks one epilogue warp drains per tile
 constexpr int kMaxE = 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = kBNMax;             // one 128-lane x 256-column accumulator per CTA
@@ -226,8 +232,8 @@ namespace gp {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_full,
-                             const __grid_constant__ CUtensorMap tm_sf, const __grid_constant__ CUtensorMap tm_out,
-                             const __grid_constant__ CUtensorMap tm_wsw, const Params p) {
+                             const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_wsw,
+                             const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
@@ -242,7 +248,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         prefetch_tensormap(&tm_a);
         prefetch_tensormap(&tm_a_full);
-        prefetch_tensormap(&tm_sf);
         prefetch_tensormap(&tm_out);
         if (p.swiglu) prefetch_tensormap(&tm_wsw);
         sh.abort = 0;
@@ -324,7 +329,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int32_t my_rows = t.bn / 2;
                 const int32_t my_row0 = t.row0 + (int32_t)rank * my_rows;
                 const uint32_t a_bytes = p.swiglu ? 2u * (kCodeBytes / 2 + kTileSFBytes) : (uint32_t)kPackedTileBytes;
-                const uint32_t tx = a_bytes + (uint32_t)my_rows * kRowBytes + kBNMax * 16;
+                // both CTAs stage the scales of all the tile's rows: one contiguous run of the K step's
+                // slab (K-stage layout), 16 bytes per row
+                const uint32_t tx = a_bytes + (uint32_t)my_rows * kRowBytes + (uint32_t)t.rows * 16u;
+                const uint8_t* sfb = p.a_sf + (int64_t)t.row0 * 16;
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
                     if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
                     uint8_t* sb = stages + (size_t)stage * kStageBytes;
@@ -347,7 +355,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             tma_load_2d(sb + kOffB + i * kBoxRows * kRowBytes, &tm_a, kt * kRowBytes,
                                         my_row0 + i * kBoxRows, bar, pol_a);
                     }
-                    tma_load_2d(sb + kOffSFB, &tm_sf, kt * 16, t.row0, bar, pol_a);
+                    bulk_load(sb + kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, bar, pol_a);
                     issued[stage] = true;
                     issued_parity[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -468,8 +476,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 4) {  // warps 4-7 and 12-15
         // ================= epilogue (both CTAs) =================
-        // TMEM lane = A row of this CTA, column = token of the tile. Per 32-token chunk each warp
-        // converts its 32 lanes to BF16 in a private shared block and writes 16-byte row pieces.
+        // TMEM lane = A row of this CTA, column = token of the tile. Each warp drains its 32-token
+        // chunks into registers, releases the accumulator, then per chunk stages a BF16 block in its
+        // private shared buffer and stores it (tensor store, or 16-byte row pieces for a partial chunk).
         const int quad = warp & 3;
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const int half = warp >= 12 ? 1 : 0;  // this warp takes the chunks c with c % 2 == half
@@ -486,68 +495,96 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!warp_wait(&sh.acc_full, aphase, abort, p.ctl)) break;
             tc_fence_after();
             const float alpha = a_g * __ldg(p.w_gscale + t.e);
-            for (int c = half; c * 32 < t.bn; c += 2) {
-                float v[32];
-                tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v);
-                tmem_ld_wait();
-                const int nrows = min(32, t.rows - c * 32);
-                const int32_t r0 = t.row0 + c * 32;
-                // the previous chunk's tensor store has finished reading the staging block
-                if (lane == 0) bulk_wait_group_read0();
-                __syncwarp();
-                int32_t col;      // first output column of this warp's block
-                int lane_cols;    // lanes per 16-byte row piece in the direct-store path: 2 (SwiGLU) or 4
-                if (p.swiglu) {
-                    // lane l < 16 holds gate, lane l + 16 up, of output column 16 quad + l; lane l
-                    // produces the even tokens, lane l + 16 the odd ones
+            // 1. Drain: this warp's chunks (c = half, half + 2, ...) become final BF16 values in registers,
+            //    two per word (SWIGLU: 16 outputs per chunk, NONE: 32), and the accumulator goes back to
+            //    the MMA warp at once: the next tile's main loop runs while 2. stages and stores them.
+            uint32_t pk[kChunksPerWarp][16];
 #pragma unroll
-                    for (int j = 0; j < 16; j++) {
-                        const float send = up_lane ? v[2 * j] : v[2 * j + 1];
-                        const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
-                        const float g = alpha * (up_lane ? recv : v[2 * j]);
-                        const float u = alpha * (up_lane ? v[2 * j + 1] : recv);
-                        const float h = swiglu_f32(g, u);
-                        const uint16_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(h));
-                        if (2 * j + (up_lane ? 1 : 0) < nrows) amax = max(amax, (uint32_t)(hb & 0x7FFFu));
-                        stg[(2 * j + (up_lane ? 1 : 0)) * 16 + (lane & 15)] = hb;
-                    }
-                    col = t.nt * kBM + (int32_t)rank * 64 + quad * 16;
-                    lane_cols = 2;
-                } else {
+            for (int ci = 0; ci < kChunksPerWarp; ci++) {
+                const int c = half + 2 * ci;
+                if (c * 32 < t.bn) {
+                    float v[32];
+                    tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v);
+                    tmem_ld_wait();
+                    const int nrows = min(32, t.rows - c * 32);
+                    if (p.swiglu) {
+                        // lane l < 16 holds gate, lane l + 16 up, of output column 16 quad + l; lane l
+                        // produces the even tokens, lane l + 16 the odd ones
 #pragma unroll
-                    for (int i = 0; i < 32; i++) {
-                        const uint16_t b = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i]));
-                        if (i < nrows) amax = max(amax, (uint32_t)(b & 0x7FFFu));
-                        stg[i * 32 + lane] = b;
+                        for (int j = 0; j < 16; j++) {
+                            const float send = up_lane ? v[2 * j] : v[2 * j + 1];
+                            const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
+                            const float g = alpha * (up_lane ? recv : v[2 * j]);
+                            const float u = alpha * (up_lane ? v[2 * j + 1] : recv);
+                            const uint32_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(swiglu_f32(g, u)));
+                            if (2 * j + (up_lane ? 1 : 0) < nrows) amax = max(amax, hb & 0x7FFFu);
+                            if (j & 1) pk[ci][j >> 1] |= hb << 16;
+                            else pk[ci][j >> 1] = hb;
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            const uint32_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i]));
+                            const uint32_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i + 1]));
+                            if (i < nrows) amax = max(amax, b0 & 0x7FFFu);
+                            if (i + 1 < nrows) amax = max(amax, b1 & 0x7FFFu);
+                            pk[ci][i >> 1] = b0 | (b1 << 16);
+                        }
                     }
-                    col = t.nt * 2 * kBM + (int32_t)rank * kBM + quad * 32;
-                    lane_cols = 4;
-                }
-                if (nrows == 32) {
-                    // a whole chunk of the expert: one asynchronous tensor store of the block
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tm_out, stg, col, r0);
-                        bulk_commit_group();
-                    }
-                } else {
-                    // the expert's last, partial chunk: rows past its end belong to the next expert
-                    __syncwarp();
-                    const int64_t ldo = p.swiglu ? p.N / 2 : p.N;
-                    const int row_elems = 8 * lane_cols;
-                    const int rows_per_pass = 32 / lane_cols;
-                    for (int r = lane / lane_cols; r < nrows; r += rows_per_pass) {
-                        const int piece = 8 * (lane % lane_cols);
-                        *reinterpret_cast<uint4*>(p.out + (int64_t)(r0 + r) * ldo + col + piece) =
-                            *reinterpret_cast<const uint4*>(stg + r * row_elems + piece);
-                    }
-                    __syncwarp();
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) arrive_on_leader(&sh.acc_empty, rank);
+            // 2. Write out: per chunk, stage a 32-token block in shared memory and store it
+#pragma unroll
+            for (int ci = 0; ci < kChunksPerWarp; ci++) {
+                const int c = half + 2 * ci;
+                if (c * 32 < t.bn) {
+                    const int nrows = min(32, t.rows - c * 32);
+                    const int32_t r0 = t.row0 + c * 32;
+                    // the previous chunk's tensor store has finished reading the staging block
+                    if (lane == 0) bulk_wait_group_read0();
+                    __syncwarp();
+                    int32_t col;      // first output column of this warp's block
+                    int lane_cols;    // lanes per 16-byte row piece in the direct-store path: 2 (SwiGLU) or 4
+                    if (p.swiglu) {
+#pragma unroll
+                        for (int j = 0; j < 16; j++)
+                            stg[(2 * j + (up_lane ? 1 : 0)) * 16 + (lane & 15)] =
+                                (uint16_t)((j & 1) ? (pk[ci][j >> 1] >> 16) : (pk[ci][j >> 1] & 0xFFFFu));
+                        col = t.nt * kBM + (int32_t)rank * 64 + quad * 16;
+                        lane_cols = 2;
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; i++)
+                            stg[i * 32 + lane] = (uint16_t)((i & 1) ? (pk[ci][i >> 1] >> 16) : (pk[ci][i >> 1] & 0xFFFFu));
+                        col = t.nt * 2 * kBM + (int32_t)rank * kBM + quad * 32;
+                        lane_cols = 4;
+                    }
+                    if (nrows == 32) {
+                        // a whole chunk of the expert: one asynchronous tensor store of the block
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tm_out, stg, col, r0);
+                            bulk_commit_group();
+                        }
+                    } else {
+                        // the expert's last, partial chunk: rows past its end belong to the next expert
+                        __syncwarp();
+                        const int64_t ldo = p.swiglu ? p.N / 2 : p.N;
+                        const int row_elems = 8 * lane_cols;
+                        const int rows_per_pass = 32 / lane_cols;
+                        for (int r = lane / lane_cols; r < nrows; r += rows_per_pass) {
+                            const int piece = 8 * (lane % lane_cols);
+                            *reinterpret_cast<uint4*>(p.out + (int64_t)(r0 + r) * ldo + col + piece) =
+                                *reinterpret_cast<const uint4*>(stg + r * row_elems + piece);
+                        }
+                        __syncwarp();
+                    }
+                }
+            }
             aphase ^= 1u;
         }
         if (lane == 0) bulk_wait_group0();  // this warp's tensor stores completed
@@ -583,7 +620,7 @@ int pair_gemm_tokens_max() { return gp::kBNMax; }
 int pair_gemm_store_cols(int swiglu) { return swiglu ? 16 : 32; }  // 32 tokens x this many BF16 columns
 
 // Launches the pair kernel; the caller validated every argument (same contract as the one-SM kernel).
-nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full, const CUtensorMap& tm_sf,
+nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full,
                                       const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const uint8_t* a_sf,
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
@@ -635,7 +672,7 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
     launch_pdl(gp::grouped_gemm_pair_kernel, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes, s, tm_a, tm_a_full,
-               tm_sf, tm_out, tm_wsw, prm);
+               tm_out, tm_wsw, prm);
     count_launch();
     return check_launch();
 }

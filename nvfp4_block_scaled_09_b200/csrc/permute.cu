@@ -13,7 +13,11 @@
 //              order. A token lists each expert at most once, so slot order
 //              inside a token never decides a rank.
 //   4. gather: one warp per output row copies K/2 code bytes and K/16 scale
-//              bytes with 16-byte vector loads and stores.
+//              bytes with 16-byte vector loads and stores. The scales go out
+//              row-major or in the K-stage layout (the 16 bytes of each
+//              256-element K step into that step's [R x 16 B] slab; the 8
+//              warps of a CTA write 8 adjacent rows, so each slab receives
+//              128 contiguous bytes per CTA).
 #include <mutex>
 
 #include "common.cuh"
@@ -129,6 +133,7 @@ __global__ void __launch_bounds__(kTok) permute_rank_kernel(const int32_t* __res
 }
 
 // One warp per output row; rows whose source index is invalid become zeros.
+template <bool kKStage>
 __global__ void __launch_bounds__(256) permute_gather_kernel(const uint4* __restrict__ q, const uint4* __restrict__ sf,
                                                              int64_t qvec, int64_t sfvec,
                                                              const int32_t* __restrict__ perm_src, int32_t T,
@@ -146,8 +151,11 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(const uint4* __rest
     uint4* qd = q_perm + p * qvec;
     for (int64_t i = lane; i < qvec; i += 32) qd[i] = ok ? __ldg(qs + i) : zero;
     const uint4* ss = sf + (int64_t)(ok ? src : 0) * sfvec;
-    uint4* sd = sf_perm + p * sfvec;
-    for (int64_t i = lane; i < sfvec; i += 32) sd[i] = ok ? __ldg(ss + i) : zero;
+    for (int64_t i = lane; i < sfvec; i += 32) {
+        const uint4 v = ok ? __ldg(ss + i) : zero;
+        if (kKStage) sf_perm[i * R + p] = v;   // K step i's slab, row p
+        else sf_perm[p * sfvec + i] = v;
+    }
 }
 
 }  // namespace
@@ -157,6 +165,14 @@ using namespace nvfp4;
 
 static inline int32_t permute_chunks(int32_t T) { return (T + kTok - 1) / kTok; }
 
+static void launch_gather(const uint8_t* q, const uint8_t* sf, int64_t K, const int32_t* perm_src, int32_t T,
+                          int64_t R, uint8_t* q_perm, uint8_t* sf_perm, nvfp4_sf_layout layout, cudaStream_t s) {
+    auto kernel = layout == NVFP4_SF_KSTAGE ? permute_gather_kernel<true> : permute_gather_kernel<false>;
+    launch_pdl(kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, s, reinterpret_cast<const uint4*>(q),
+               reinterpret_cast<const uint4*>(sf), K / 32, K / 256, perm_src, T, R, reinterpret_cast<uint4*>(q_perm),
+               reinterpret_cast<uint4*>(sf_perm));
+}
+
 extern "C" size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E) {
     (void)k;
     if (T <= 0 || E <= 0) return 0;
@@ -165,10 +181,11 @@ extern "C" size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E) {
 
 extern "C" nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E, const uint8_t* q,
                                     const uint8_t* sf, int64_t K, uint8_t* q_perm, uint8_t* sf_perm,
-                                    int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm, void* ws,
-                                    size_t ws_bytes, nvfp4_stream_t stream) {
+                                    nvfp4_sf_layout sf_perm_layout, int32_t* expert_offsets, int32_t* perm_src,
+                                    int32_t* inv_perm, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
     if (!topk_ids || !q || !sf || !q_perm || !sf_perm || !expert_offsets || !perm_src || !inv_perm)
         return NVFP4_ERR_INVALID_ARG;
+    if (sf_perm_layout != NVFP4_SF_ROWMAJOR && sf_perm_layout != NVFP4_SF_KSTAGE) return NVFP4_ERR_INVALID_ARG;
     if (T <= 0 || k <= 0 || E <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
     if (k > 32 || E > kMaxE || (int64_t)T * k >= (int64_t)1 << 31 || K % 256 != 0)
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -189,10 +206,7 @@ extern "C" nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t 
     launch_pdl(permute_scan_kernel, dim3(1), dim3(kMaxE), 0, s, counts, nchunks, E, expert_offsets);
     const size_t rank_smem = (size_t)E * kWordsPerExpert * sizeof(uint32_t);
     launch_pdl(permute_rank_kernel, dim3(nchunks), dim3(kTok), rank_smem, s, topk_ids, T, k, E, counts, perm_src, inv_perm, status);
-    const int64_t gblocks = (R + 7) / 8;
-    launch_pdl(permute_gather_kernel, dim3((unsigned)gblocks), dim3(256), 0, s,
-        reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(sf), K / 32, K / 256, perm_src, T, R,
-        reinterpret_cast<uint4*>(q_perm), reinterpret_cast<uint4*>(sf_perm));
+    launch_gather(q, sf, K, perm_src, T, R, q_perm, sf_perm, sf_perm_layout, s);
     count_launch(4);
     return check_launch();
 }
@@ -227,10 +241,12 @@ int32_t* noalloc_scratch_ptr() {
 
 extern "C" nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
                                             const uint8_t* q, const uint8_t* sf, int64_t K, uint8_t* q_perm,
-                                            uint8_t* sf_perm, int32_t* expert_offsets, int32_t* perm_src,
-                                            int32_t* inv_perm, nvfp4_stream_t stream) {
+                                            uint8_t* sf_perm, nvfp4_sf_layout sf_perm_layout,
+                                            int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
+                                            nvfp4_stream_t stream) {
     if (!topk_ids || !q || !sf || !q_perm || !sf_perm || !expert_offsets || !perm_src || !inv_perm)
         return NVFP4_ERR_INVALID_ARG;
+    if (sf_perm_layout != NVFP4_SF_ROWMAJOR && sf_perm_layout != NVFP4_SF_KSTAGE) return NVFP4_ERR_INVALID_ARG;
     if (T <= 0 || k <= 0 || E <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
     if (k > 32 || E > kMaxE || (int64_t)T * k >= (int64_t)1 << 31 || K % 256 != 0)
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -248,9 +264,7 @@ extern "C" nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, 
     launch_pdl(permute_scan_kernel, dim3(1), dim3(kMaxE), 0, s, counts, nchunks, E, expert_offsets);
     const size_t rank_smem = (size_t)E * kWordsPerExpert * sizeof(uint32_t);
     launch_pdl(permute_rank_kernel, dim3(nchunks), dim3(kTok), rank_smem, s, topk_ids, T, k, E, counts, perm_src, inv_perm, status);
-    launch_pdl(permute_gather_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, s,
-        reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(sf), K / 32, K / 256, perm_src, T, R,
-        reinterpret_cast<uint4*>(q_perm), reinterpret_cast<uint4*>(sf_perm));
+    launch_gather(q, sf, K, perm_src, T, R, q_perm, sf_perm, sf_perm_layout, s);
     count_launch(4);
     return check_launch();
 }

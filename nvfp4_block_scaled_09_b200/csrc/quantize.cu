@@ -111,7 +111,8 @@ __device__ __forceinline__ GlobalScale global_scale(float amax, const float* gde
     return g;
 }
 
-template <bool kTiled>
+// kLayout: the nvfp4_sf_layout the block scales are written in.
+template <int kLayout>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, int64_t rows, int64_t K,
                                                             const float* __restrict__ gdec_in,
                                                             const uint32_t* __restrict__ partial, int npartial,
@@ -169,10 +170,14 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
         }
         q[b] = packed;
         int64_t sf_off;
-        if (kTiled) {
+        if (kLayout == NVFP4_SF_MMA_TILED) {
             const int64_t r = b / blocks_per_row, kb = b - r * blocks_per_row;
             const int64_t atom = (r >> 7) * (K >> 6) + (kb >> 2);
             sf_off = atom * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
+        } else if (kLayout == NVFP4_SF_KSTAGE) {
+            // slab of the 256-element K step kb / 16, row r's 16-byte piece, byte kb % 16
+            const int64_t r = b / blocks_per_row, kb = b - r * blocks_per_row;
+            sf_off = ((kb >> 4) * rows + r) * 16 + (kb & 15);
         } else {
             sf_off = b;
         }
@@ -198,12 +203,11 @@ static void launch_quantize(const uint16_t* x, int64_t rows, int64_t K, const fl
     const int64_t cap = (int64_t)device_sm_count() * 16;
     if (grid_q > cap) grid_q = cap;
     if (grid_q < 1) grid_q = 1;
-    if (layout == NVFP4_SF_MMA_TILED)
-        launch_pdl(quantize_kernel<true>, dim3((int)grid_q), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x),
-                   rows, K, global_scale_in, partial, npartial, reinterpret_cast<uint2*>(q), sf, global_scale_out);
-    else
-        launch_pdl(quantize_kernel<false>, dim3((int)grid_q), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x),
-                   rows, K, global_scale_in, partial, npartial, reinterpret_cast<uint2*>(q), sf, global_scale_out);
+    auto kernel = layout == NVFP4_SF_MMA_TILED ? quantize_kernel<NVFP4_SF_MMA_TILED>
+                  : layout == NVFP4_SF_KSTAGE  ? quantize_kernel<NVFP4_SF_KSTAGE>
+                                               : quantize_kernel<NVFP4_SF_ROWMAJOR>;
+    launch_pdl(kernel, dim3((int)grid_q), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x), rows, K,
+               global_scale_in, partial, npartial, reinterpret_cast<uint2*>(q), sf, global_scale_out);
 }
 
 }  // namespace nvfp4
@@ -220,9 +224,11 @@ extern "C" nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t 
                                        void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
     if (!x || !q || !sf || !global_scale_out) return NVFP4_ERR_INVALID_ARG;
     if (rows <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
-    if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_MMA_TILED) return NVFP4_ERR_INVALID_ARG;
+    if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_MMA_TILED && layout != NVFP4_SF_KSTAGE)
+        return NVFP4_ERR_INVALID_ARG;
     if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (layout == NVFP4_SF_MMA_TILED && (rows % 128 != 0 || K % 64 != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (layout == NVFP4_SF_KSTAGE && K % 256 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x) || !aligned8(q)) return NVFP4_ERR_MISALIGNED;
     if (((uintptr_t)global_scale_out & 3u) || (global_scale_in && ((uintptr_t)global_scale_in & 3u)))
         return NVFP4_ERR_MISALIGNED;
@@ -248,9 +254,11 @@ extern "C" nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows
                                                  nvfp4_sf_layout layout, nvfp4_stream_t stream) {
     if (!x || !q || !sf || !global_scale_out || !amax_bits) return NVFP4_ERR_INVALID_ARG;
     if (rows <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
-    if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_MMA_TILED) return NVFP4_ERR_INVALID_ARG;
+    if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_MMA_TILED && layout != NVFP4_SF_KSTAGE)
+        return NVFP4_ERR_INVALID_ARG;
     if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (layout == NVFP4_SF_MMA_TILED && (rows % 128 != 0 || K % 64 != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (layout == NVFP4_SF_KSTAGE && K % 256 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x) || !aligned8(q)) return NVFP4_ERR_MISALIGNED;
     if (((uintptr_t)global_scale_out & 3u) || ((uintptr_t)amax_bits & 3u)) return NVFP4_ERR_MISALIGNED;
     launch_quantize(x, rows, K, nullptr, amax_bits, 1, q, sf, global_scale_out, layout,

@@ -6,8 +6,10 @@ G ranks each hold their own tokens and the weights of E/G consecutive experts. O
      the whole batch, so every rank's FP4 rows are the rows one GPU would produce for all G*T tokens.
   2. moe_permute over all E experts. Each rank's experts are consecutive, so the expert-ordered rows are
      also grouped by the rank that owns them.
-  3. all-to-all of the per-expert row counts, then of the FP4 codes and scales (dispatch).
-  4. The received rows (source-major) are regrouped by local expert with a second moe_permute (k = 1).
+  3. all-to-all of the per-expert row counts, then of the FP4 codes and scales (dispatch; the scales of
+     this permute are row-major, so that each row's bytes are contiguous).
+  4. The received rows (source-major) are regrouped by local expert with a second moe_permute (k = 1),
+     whose scales come out in the K-stage layout the grouped GEMM reads.
   5. The gate/up GEMM reports the amax of h; an all-reduce (max) makes it the amax over all ranks' rows;
      h is quantised from it and the down GEMM runs. A k = 1 combine with weight 1 (an exact copy) puts
      the rows back in arrival order.
@@ -37,11 +39,13 @@ class LibraryOps:
     def amax(self, x):
         return nv.amax(x)
 
-    def quantize_from_amax(self, x, amax_bits):
-        return nv.quantize_from_amax(x, amax_bits)
+    def quantize_from_amax(self, x, amax_bits, gemm_operand=False):
+        # row-major scales for x (they travel to other ranks row by row); K-stage slabs for an operand of
+        # the grouped GEMM
+        return nv.quantize_from_amax(x, amax_bits, layout=nv.SF_KSTAGE if gemm_operand else nv.SF_ROWMAJOR)
 
-    def permute(self, ids, q, sf, num_experts):
-        return nv.permute(ids, q, sf, num_experts)
+    def permute(self, ids, q, sf, num_experts, gemm_operand=False):
+        return nv.permute(ids, q, sf, num_experts, sf_layout=nv.SF_KSTAGE if gemm_operand else nv.SF_ROWMAJOR)
 
     def gemm(self, a_q, a_sf, a_g, w, offsets, swiglu, amax_out=None):
         return nv.grouped_gemm(a_q, a_sf, a_g, w, offsets, swiglu, amax_out=amax_out)
@@ -107,11 +111,12 @@ def ep_moe_layer(x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor, 
     amax_h = torch.zeros(1, dtype=torch.int32, device=dev)
     if Rr > 0:
         local_ids = np.repeat(np.tile(np.arange(El, dtype=np.int32), G), recv_e.reshape(-1))
-        loc = ops.permute(torch.from_numpy(local_ids.reshape(-1, 1)).to(dev), q_recv, sf_recv, El)
+        loc = ops.permute(torch.from_numpy(local_ids.reshape(-1, 1)).to(dev), q_recv, sf_recv, El,
+                          gemm_operand=True)
         h = ops.gemm(loc.q_perm, loc.sf_perm, g_x, local_weights.w13, loc.offsets, True, amax_out=amax_h)
     dist.all_reduce(amax_h, op=dist.ReduceOp.MAX, group=group)
     if Rr > 0:
-        q_h, sf_h, g_h = ops.quantize_from_amax(h, amax_h)
+        q_h, sf_h, g_h = ops.quantize_from_amax(h, amax_h, gemm_operand=True)
         y_loc = ops.gemm(q_h, sf_h, g_h, local_weights.w2, loc.offsets, False)
         y_recv = ops.combine(y_loc, loc.inv_perm, torch.ones((Rr, 1), dtype=torch.float32, device=dev))
     else:

@@ -35,6 +35,21 @@ def untile_sf(sf_tiled, rows, K):
     return flat[off]
 
 
+def kstage_sf_to_rowmajor(sf_kstage, rows, K, sel=None):
+    """NVFP4_SF_KSTAGE bytes -> row-major [rows, K/16] (or only the rows in `sel`). The header's definition:
+    one [rows x 16 bytes] slab per 256-element K step, row r's scale of block b at
+    ((b // 16) * rows + r) * 16 + b % 16 -- i.e. the bytes form an array [K/256, rows, 16]."""
+    slabs = np.ascontiguousarray(sf_kstage).reshape(K // 256, rows, 16)
+    if sel is not None:
+        slabs = slabs[:, np.asarray(sel), :]
+    return np.ascontiguousarray(slabs.transpose(1, 0, 2)).reshape(-1, K // 16)
+
+
+def rowmajor_sf_to_kstage(sf_rowmajor, rows, K):
+    """Row-major [rows, K/16] scales -> the NVFP4_SF_KSTAGE array [K/256, rows, 16]."""
+    return np.ascontiguousarray(np.asarray(sf_rowmajor).reshape(rows, K // 256, 16).transpose(1, 0, 2))
+
+
 def bf16_to_f64(bits):
     bits = np.ascontiguousarray(bits).view(np.uint16)
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

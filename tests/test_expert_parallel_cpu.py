@@ -47,12 +47,12 @@ class OracleOps:
         b = _bits(x)
         return torch.tensor([int((b & 0x7FFF).max()) if b.size else 0], dtype=torch.int32)
 
-    def quantize_from_amax(self, x, amax_bits):
+    def quantize_from_amax(self, x, amax_bits, gemm_operand=False):   # row-major scales throughout
         amax = float(self.o.bf16_bits_to_f64(np.array([int(amax_bits[0])], dtype=np.uint16))[0])
         q, sf, g = self.o.quantize_with_amax(_bits(x), amax)
         return torch.from_numpy(q), torch.from_numpy(sf), torch.tensor([g], dtype=torch.float32)
 
-    def permute(self, ids, q, sf, num_experts):
+    def permute(self, ids, q, sf, num_experts, gemm_operand=False):
         off, src, inv = self.o.permute(ids.numpy(), num_experts)
         return SimpleNamespace(q_perm=torch.from_numpy(self.o.gather_rows(q.numpy(), src)),
                                sf_perm=torch.from_numpy(self.o.gather_rows(sf.numpy(), src)),

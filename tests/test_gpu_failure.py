@@ -10,7 +10,7 @@ import torch
 import nvfp4_block_scaled_09_b200 as nv
 import oracle
 import workloads
-from tests.helpers import compare_bf16, gpu_bf16, host, host_bits, require_gpu
+from tests.helpers import compare_bf16, gpu_bf16, host, host_bits, kstage_sf_to_rowmajor, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 def small_case():
     rows, N, K = [16, 16], 256, 256
     a_bits = workloads.random_bf16_bits((32, K), seed=21)
-    a_q, a_sf, a_g = nv.quantize(gpu_bf16(a_bits))
+    a_q, a_sf, a_g = nv.quantize(gpu_bf16(a_bits), layout=nv.SF_KSTAGE)
     w = workloads.normal_bf16((2, N, K), 0.02, 21, workloads.TAG_W13, device="cuda")
     pw = nv.prepare_expert_weights(w, keep_rowmajor=True)
     off = torch.tensor([0, 16, 32], dtype=torch.int32, device="cuda")
@@ -41,7 +41,8 @@ def test_stalled_producer_times_out_then_context_recovers():
     assert nv.device_status() == 0
     out = nv.grouped_gemm(a_q, a_sf, a_g, pw, off, False)
     assert nv.device_status() == 0
-    ref = oracle.grouped_gemm(host(a_q), host(a_sf), host(a_g)[0], host(pw.q), host(pw.sf), host(pw.gscale),
+    ref = oracle.grouped_gemm(host(a_q), kstage_sf_to_rowmajor(host(a_sf), 32, 256), host(a_g)[0], host(pw.q),
+                              host(pw.sf), host(pw.gscale),
                               np.array([0, 16, 32], np.int32), 256, 256, False)
     compare_bf16(host_bits(out), oracle.bf16_round(ref), "gemm after a timed-out launch", exact=ref)
     # every counter slot of the dynamic schedule (the timed-out launch's among them) is clean when drawn

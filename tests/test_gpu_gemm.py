@@ -13,7 +13,8 @@ import torch
 import nvfp4_block_scaled_09_b200 as nv
 import oracle
 import workloads
-from tests.helpers import compare_bf16, gpu_bf16, host, host_bits, require_gpu, unpack_weights
+from tests.helpers import (compare_bf16, gpu_bf16, host, host_bits, kstage_sf_to_rowmajor, require_gpu,
+                           unpack_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -28,17 +29,19 @@ def make_case(rows, N, K, seed, a_std=1.0, w_std=0.02, pad_rows=0):
     The GEMM's max_rows is the activation row count, so padding rows changes the tile shape it picks."""
     E = len(rows)
     R = int(sum(rows))
-    a_bits = workloads.random_bf16_bits((max(R + pad_rows, 1), K), seed=seed, std=a_std)
-    a_q, a_sf, a_g = nv.quantize(gpu_bf16(a_bits))
+    rows_a = max(R + pad_rows, 1)
+    a_bits = workloads.random_bf16_bits((rows_a, K), seed=seed, std=a_std)
+    a_q, a_sf, a_g = nv.quantize(gpu_bf16(a_bits), layout=nv.SF_KSTAGE)   # the GEMM's activation-scale layout
     w = workloads.normal_bf16((E, N, K), w_std, seed, workloads.TAG_W13, device="cuda")
     pw = nv.prepare_expert_weights(w, keep_rowmajor=True)
     off = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
     torch.cuda.synchronize()
     # the GPU's operands are the oracle's operands: check their quantisation first
     oq, osf, og = oracle.quantize(a_bits)
-    assert np.array_equal(host(a_q), oq) and np.array_equal(host(a_sf), osf) and host(a_g)[0] == og
-    return dict(a_q=a_q, a_sf=a_sf, a_g=a_g, pw=pw, off=torch.from_numpy(off).cuda(), off_np=off, w=w, E=E, R=R,
-                N=N, K=K)
+    a_sf_rm = kstage_sf_to_rowmajor(host(a_sf), rows_a, K)
+    assert np.array_equal(host(a_q), oq) and np.array_equal(a_sf_rm, osf) and host(a_g)[0] == og
+    return dict(a_q=a_q, a_sf=a_sf, a_sf_rm=a_sf_rm, a_g=a_g, pw=pw, off=torch.from_numpy(off).cuda(), off_np=off,
+                w=w, E=E, R=R, N=N, K=K)
 
 
 def oracle_operands(c):
@@ -71,7 +74,7 @@ def run_full(rows, N, K, swiglu, seed, pad_rows=0):
     check_weights_quantised_and_packed(c, range(min(c["E"], 3)))
     w_q, w_sf, w_g = oracle_operands(c)
     R = c["R"]
-    ref = oracle.grouped_gemm(host(c["a_q"])[:R], host(c["a_sf"])[:R], host(c["a_g"])[0], w_q, w_sf, w_g,
+    ref = oracle.grouped_gemm(host(c["a_q"])[:R], c["a_sf_rm"][:R], host(c["a_g"])[0], w_q, w_sf, w_g,
                               c["off_np"], N, K, swiglu)
     got = host_bits(out)[: c["R"]]
     return compare_bf16(got, oracle.bf16_round(ref), f"gemm rows={rows} N={N} K={K} swiglu={swiglu}", exact=ref)
@@ -185,7 +188,7 @@ def sampled_check(a_q, a_sf, a_g, c_w, off_np, N, K, swiglu, out, experts, n_col
     rr, cc = np.meshgrid(np.arange(a_rows.size), cols, indexing="ij")
     rr, cc = rr.ravel(), cc.ravel()
     aq = host(a_q)[a_rows]
-    asf = host(a_sf)[a_rows]
+    asf = kstage_sf_to_rowmajor(host(a_sf), a_q.shape[0], K, sel=a_rows)
     ref = oracle.grouped_gemm_at(aq, asf, float(host(a_g)[0]), w_q, w_sf, w_g, np.array(sub_off, np.int32), N, K,
                                  swiglu, rr, cc)
     got = host_bits(out)[a_rows[rr], cc]
@@ -195,7 +198,7 @@ def sampled_check(a_q, a_sf, a_g, c_w, off_np, N, K, swiglu, out, experts, n_col
 def test_dense_8192_sampled():
     M = N = K = 8192
     a_bits_t = workloads.normal_bf16((M, K), 1.0, 0, workloads.TAG_A, device="cuda")
-    a_q, a_sf, a_g = nv.quantize(a_bits_t)
+    a_q, a_sf, a_g = nv.quantize(a_bits_t, layout=nv.SF_KSTAGE)
     b = workloads.normal_bf16((1, N, K), 0.02, 0, workloads.TAG_B, device="cuda")
     pw = nv.prepare_expert_weights(b, keep_rowmajor=True)
     off = torch.tensor([0, M], dtype=torch.int32, device="cuda")
@@ -203,7 +206,8 @@ def test_dense_8192_sampled():
     assert nv.device_status() == 0
     # quantisation of a sample of A rows against the oracle
     oq, osf, og = oracle.quantize(host_bits(a_bits_t[:256]), float(host(a_g)[0]))
-    assert np.array_equal(host(a_q[:256]), oq) and np.array_equal(host(a_sf[:256]), osf)
+    a_sf_rm = kstage_sf_to_rowmajor(host(a_sf), M, K)
+    assert np.array_equal(host(a_q[:256]), oq) and np.array_equal(a_sf_rm[:256], osf)
     uq, usf = unpack_weights(host(pw.packed[0]), N, K)
     assert np.array_equal(uq, host(pw.q[0])) and np.array_equal(usf, host(pw.sf[0]))
     rng = np.random.default_rng(5)
@@ -211,7 +215,7 @@ def test_dense_8192_sampled():
     cols = rng.choice(N, size=48, replace=False)
     rr, cc = np.meshgrid(rows, cols, indexing="ij")
     rr, cc = rr.ravel(), cc.ravel()
-    ref = oracle.grouped_gemm_at(host(a_q), host(a_sf), float(host(a_g)[0]), host(pw.q), host(pw.sf),
+    ref = oracle.grouped_gemm_at(host(a_q), a_sf_rm, float(host(a_g)[0]), host(pw.q), host(pw.sf),
                                  host(pw.gscale), np.array([0, M], np.int32), N, K, False, rr, cc)
     compare_bf16(host_bits(out)[rr, cc], oracle.bf16_round(ref), "dense 8192", exact=ref)
 
@@ -245,7 +249,7 @@ def test_moe_layer_gemms_full_size_sampled(name):
     experts = sorted(set(e for e in experts if counts[e] > 0))
     # activations already in expert order (permute is tested on its own)
     a = workloads.normal_bf16((R, H), 1.0, 0, workloads.TAG_X, device="cuda")
-    a_q, a_sf, a_g = nv.quantize(a)
+    a_q, a_sf, a_g = nv.quantize(a, layout=nv.SF_KSTAGE)
     w13, kept13 = build_layer_weights(E, 2 * I, H, workloads.TAG_W13, set(experts))
     off = torch.from_numpy(off_np).cuda()
     h = nv.grouped_gemm(a_q, a_sf, a_g, w13, off, True)
@@ -263,7 +267,7 @@ def test_moe_layer_gemms_full_size_sampled(name):
     sampled_check(a_q, a_sf, a_g, host_w(kept13, w13.gscale), off_np, 2 * I, H, True, h, experts, n_cols=32)
 
     # down projection on the GPU's own h
-    hq, hsf, hg = nv.quantize(h)
+    hq, hsf, hg = nv.quantize(h, layout=nv.SF_KSTAGE)
     w2, kept2 = build_layer_weights(E, H, I, workloads.TAG_W2, set(experts))
     y = nv.grouped_gemm(hq, hsf, hg, w2, off, False)
     assert nv.device_status() == 0

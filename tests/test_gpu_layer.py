@@ -36,7 +36,7 @@ def staged_layer(x, ids, w, weights, E):
     perm = nv.permute(ids, q, sf, E)
     amax = torch.zeros(1, dtype=torch.int32, device=x.device)
     h = nv.grouped_gemm(perm.q_perm, perm.sf_perm, g, weights.w13, perm.offsets, True, amax_out=amax)
-    qh, sfh, gh = nv.quantize_from_amax(h, amax)
+    qh, sfh, gh = nv.quantize_from_amax(h, amax, layout=nv.SF_KSTAGE)
     # the amax side output equals the amax pass of the dynamic quantiser on h
     assert torch.equal(gh, nv.quantize(h)[2])
     y = nv.grouped_gemm(qh, sfh, gh, weights.w2, perm.offsets, False)

@@ -1,5 +1,7 @@
 """moe_permute on the GPU against the oracle: offsets, indices and gathered
-bytes bit-exact, for every routing pattern of the workloads."""
+bytes bit-exact, for every routing pattern of the workloads, with the scales
+written in either layout (K-stage slabs, as the grouped GEMM reads them, and
+row-major)."""
 import numpy as np
 import pytest
 import torch
@@ -7,7 +9,7 @@ import torch
 import nvfp4_block_scaled_09_b200 as nv
 import oracle
 import workloads
-from tests.helpers import host, require_gpu
+from tests.helpers import host, kstage_sf_to_rowmajor, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -17,19 +19,24 @@ def _gpu():
     require_gpu()
 
 
-def run(ids, E, K, seed=0):
-    T = ids.shape[0]
+def run(ids, E, K, seed=0, sf_layout=nv.SF_KSTAGE):
+    T, k = ids.shape
     rng = np.random.default_rng(seed)
     q = rng.integers(0, 256, size=(T, K // 2), dtype=np.uint8)
     sf = rng.integers(0, 256, size=(T, K // 16), dtype=np.uint8)
-    out = nv.permute(torch.from_numpy(ids).cuda(), torch.from_numpy(q).cuda(), torch.from_numpy(sf).cuda(), E)
+    out = nv.permute(torch.from_numpy(ids).cuda(), torch.from_numpy(q).cuda(), torch.from_numpy(sf).cuda(), E,
+                     sf_layout=sf_layout)
     assert nv.device_status() == 0
     off, src, inv = oracle.permute(ids, E)
     assert np.array_equal(host(out.offsets), off)
     assert np.array_equal(host(out.perm_src), src)
     assert np.array_equal(host(out.inv_perm), inv)
     assert np.array_equal(host(out.q_perm), oracle.gather_rows(q, src))
-    assert np.array_equal(host(out.sf_perm), oracle.gather_rows(sf, src))
+    sf_perm = host(out.sf_perm)
+    if sf_layout == nv.SF_KSTAGE:
+        assert sf_perm.shape == (K // 256, T * k, 16)
+        sf_perm = kstage_sf_to_rowmajor(sf_perm, T * k, K)
+    assert np.array_equal(sf_perm, oracle.gather_rows(sf, src))
 
 
 @pytest.mark.parametrize("name", ["moe_decode_t512", "moe_zipf_t1024", "moe_prefill_t8192"])
@@ -43,6 +50,14 @@ def test_workload_routing(name):
 def test_ragged_shapes(T, E, k, kind):
     ids, _ = workloads.routing(T, E, k, kind, seed=T)
     run(ids, E, 256, seed=T)
+
+
+@pytest.mark.parametrize("T,E,k,K", [(37, 5, 3, 768), (300, 64, 8, 2048)])
+def test_scale_layouts(T, E, k, K):
+    # several K steps, so the K-stage slabs and the row-major rows differ; both layouts from one routing
+    ids, _ = workloads.routing(T, E, k, "uniform", seed=T)
+    run(ids, E, K, seed=T, sf_layout=nv.SF_KSTAGE)
+    run(ids, E, K, seed=T, sf_layout=nv.SF_ROWMAJOR)
 
 
 def test_invalid_and_duplicate_ids_latch_status():

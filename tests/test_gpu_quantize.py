@@ -8,7 +8,7 @@ import torch
 import nvfp4_block_scaled_09_b200 as nv
 import oracle
 import workloads
-from tests.helpers import gpu_bf16, host, require_gpu, untile_sf
+from tests.helpers import gpu_bf16, host, kstage_sf_to_rowmajor, require_gpu, untile_sf
 
 pytestmark = pytest.mark.gpu
 
@@ -71,6 +71,17 @@ def test_tiled_layout_is_a_permutation_of_rowmajor():
     assert np.array_equal(untile_sf(sf_t, 256, 512), osf)
 
 
+@pytest.mark.parametrize("rows,K", [(1, 256), (37, 768), (300, 6144)])
+def test_kstage_layout_is_a_permutation_of_rowmajor(rows, K):
+    # the grouped GEMM's activation-scale layout: one [rows x 16 B] slab per 256-element K step
+    x = workloads.random_bf16_bits((rows, K), seed=rows, std=1.0)
+    q, sf_k, g = gpu_quantize(x, layout=nv.SF_KSTAGE)
+    oq, osf, og = oracle.quantize(x)
+    assert sf_k.shape == (K // 256, rows, 16)
+    assert g == og and np.array_equal(q, oq)
+    assert np.array_equal(kstage_sf_to_rowmajor(sf_k, rows, K), osf)
+
+
 def test_decode_activation_size():
     # x of the 512-token decode layer, and an h-sized tensor
     check(workloads.random_bf16_bits((512, 6144), seed=12))
@@ -86,6 +97,10 @@ def test_rejects_bad_arguments():
     with pytest.raises(nv.NVFP4Error) as e:
         nv.quantize(x, layout=nv.SF_MMA_TILED)
     assert e.value.status == 3
+    x = torch.zeros((4, 128), dtype=torch.bfloat16, device="cuda")   # K-stage slabs need K % 256 == 0
+    with pytest.raises(nv.NVFP4Error) as e:
+        nv.quantize(x, layout=nv.SF_KSTAGE, sf=torch.empty((4, 8), dtype=torch.uint8, device="cuda"))
+    assert e.value.status == 3
 
 
 @pytest.mark.parametrize("rows,K,std,seed", [(1, 16, 1.0, 10), (96, 2048, 0.5, 11), (300, 512, 3.0, 12)])
@@ -100,3 +115,7 @@ def test_from_amax_equals_dynamic(rows, K, std, seed):
         assert np.float32(host(g)[0]) == og
         assert np.array_equal(host(sf).reshape(osf.shape), osf)
         assert np.array_equal(host(q), oq)
+        if K % 256 == 0:   # the same in the K-stage layout (what the layer feeds the down GEMM)
+            qk, sfk, gk = nv.quantize_from_amax(gpu_bf16(bits), amax, layout=nv.SF_KSTAGE)
+            assert np.float32(host(gk)[0]) == og and np.array_equal(host(qk), oq)
+            assert np.array_equal(kstage_sf_to_rowmajor(host(sfk), rows, K), osf)

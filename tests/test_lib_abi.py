@@ -50,16 +50,17 @@ def test_can_implement_shapes_and_budget(L):
 
 def test_stage_transaction_bytes_are_tile_sums(L):
     # Per stage: (A tile bits + A scale bits) + (B tile bits + B scale bits), in bytes, for
-    # packed E2M1 (4 bits) and one 8-bit scale per 16 elements. The B scales travel as one
-    # box covering the tile shape's maximum row count.
+    # packed E2M1 (4 bits) and one 8-bit scale per 16 elements. The B rows are rounded up to
+    # the 16-row TMA box; the B scales (one contiguous run of the K-stage slab) cover exactly
+    # the tile's rows.
     plan = nv.gemm_plan()
     bk = plan["stage_k"]
     wrows = plan["tile_weight_rows"]
     a_bits = wrows * bk * 4
     sfa_bits = wrows * (bk // 16) * 8
     for wide, bn_max in ((False, plan["tile_tokens_max"]), (True, plan["wide_tile_tokens_max"])):
-        sfb_bits = bn_max * (bk // 16) * 8
         for tokens in (1, 15, 16, 17, 32, 48, 64, 65, 100, 128):
+            sfb_bits = tokens * (bk // 16) * 8
             if tokens > bn_max:
                 assert nv.gemm_stage_tx_bytes(tokens, wide) == -1
                 continue
@@ -93,8 +94,12 @@ def test_invalid_arguments_rejected_before_any_cuda_call(L):
     assert L.moe_unpermute_combine(None, None, None, 1, 1, 8, None, None) == 1
     p = ctypes.c_void_p(16)
     assert L.moe_unpermute_combine(p, p, p, 1, 1, 12, p, None) == 3     # H % 8 != 0
-    assert L.moe_permute(p, 4, 8, 2000, p, p, 256, p, p, p, p, p, p, 1 << 20, None) == 3  # E > 1024
-    assert L.moe_permute(p, 4, 8, 8, p, p, 256, p, p, p, p, p, None, 0, None) == 4       # no workspace
+    assert L.moe_permute(p, 4, 8, 2000, p, p, 256, p, p, 2, p, p, p, p, 1 << 20, None) == 3  # E > 1024
+    assert L.moe_permute(p, 4, 8, 8, p, p, 256, p, p, 2, p, p, p, None, 0, None) == 4       # no workspace
+    assert L.moe_permute(p, 4, 8, 8, p, p, 256, p, p, 1, p, p, p, p, 1 << 20, None) == 1    # tiled sf_perm
+    assert L.moe_permute_noalloc(p, 4, 8, 8, p, p, 256, p, p, 7, p, p, p, None) == 1        # unknown layout
+    assert L.nvfp4_quantize(p, 4, 128, p, p, p, p, 2, None, 0, None) == 3   # K-stage layout: K % 256 != 0
+    assert L.nvfp4_quantize(p, 4, 256, p, p, p, p, 3, None, 0, None) == 1   # unknown layout
     assert L.nvfp4_quantize_from_amax(None, 4, 32, None, None, None, None, 0, None) == 1
     assert L.nvfp4_quantize_from_amax(p, 4, 32, ctypes.c_void_p(18), p, p, p, 0, None) == 2  # amax word misaligned
     assert L.moe_grouped_gemm_nvfp4_amax(p, p, p, p, p, p, 1, 16, 256, 256, 0, p, ctypes.c_void_p(18), None) == 2

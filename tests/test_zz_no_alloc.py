@@ -30,14 +30,14 @@ def call_noalloc(ids, q, sf, E, K):
     R = T * k
     out = {
         "q_perm": torch.empty((R, K // 2), dtype=torch.uint8, device="cuda"),
-        "sf_perm": torch.empty((R, K // 16), dtype=torch.uint8, device="cuda"),
+        "sf_perm": torch.empty((K // 256, R, 16), dtype=torch.uint8, device="cuda"),   # K-stage slabs
         "offsets": torch.empty(E + 1, dtype=torch.int32, device="cuda"),
         "perm_src": torch.empty(R, dtype=torch.int32, device="cuda"),
         "inv_perm": torch.empty(R, dtype=torch.int32, device="cuda"),
     }
     st = nv.lib().moe_permute_noalloc(
         P(ids.data_ptr()), T, k, E, P(q.data_ptr()), P(sf.data_ptr()), K, P(out["q_perm"].data_ptr()),
-        P(out["sf_perm"].data_ptr()), P(out["offsets"].data_ptr()), P(out["perm_src"].data_ptr()),
+        P(out["sf_perm"].data_ptr()), nv.SF_KSTAGE, P(out["offsets"].data_ptr()), P(out["perm_src"].data_ptr()),
         P(out["inv_perm"].data_ptr()), P(torch.cuda.current_stream().cuda_stream))
     assert st == 0, nv.status_string(st)
     return out
@@ -68,5 +68,5 @@ def test_noalloc_rejects_shapes_beyond_its_array():
     # ceil(T / 256) * E must fit the fixed array; 65535 tokens x 1024 experts does not
     T, k, E, K = 65535, 1, 1024, 256
     d = P(256)
-    st = nv.lib().moe_permute_noalloc(d, T, k, E, d, d, K, d, d, d, d, d, None)
+    st = nv.lib().moe_permute_noalloc(d, T, k, E, d, d, K, d, d, nv.SF_KSTAGE, d, d, d, None)
     assert st == 3, nv.status_string(st)
