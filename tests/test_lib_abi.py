@@ -103,3 +103,30 @@ def test_invalid_arguments_rejected_before_any_cuda_call(L):
     assert L.nvfp4_quantize_from_amax(None, 4, 32, None, None, None, None, 0, None) == 1
     assert L.nvfp4_quantize_from_amax(p, 4, 32, ctypes.c_void_p(18), p, p, p, 0, None) == 2  # amax word misaligned
     assert L.moe_grouped_gemm_nvfp4_amax(p, p, p, p, p, p, 1, 16, 256, 256, 0, p, ctypes.c_void_p(18), None) == 2
+
+
+def test_layout_helpers_follow_the_header_definitions():
+    # The host-side layout converters the GPU tests use, checked byte by byte against the index formulas the
+    # header states (K-stage: ((b / 16) * rows + r) * 16 + b % 16; MMA-tiled: 512-byte atoms), on shapes with
+    # several K steps and a row count that is not a multiple of anything.
+    import numpy as np
+    from tests.helpers import kstage_sf_to_rowmajor, rowmajor_sf_to_kstage, untile_sf
+    rng = np.random.default_rng(0)
+    rows, K = 37, 768
+    rm = rng.integers(0, 256, size=(rows, K // 16), dtype=np.uint8)
+    ks = rowmajor_sf_to_kstage(rm, rows, K)
+    assert ks.shape == (K // 256, rows, 16)
+    flat = ks.reshape(-1)
+    for r in range(rows):
+        for b in range(K // 16):
+            assert flat[((b // 16) * rows + r) * 16 + b % 16] == rm[r, b]
+    assert np.array_equal(kstage_sf_to_rowmajor(ks, rows, K), rm)
+    sel = np.array([36, 0, 17])
+    assert np.array_equal(kstage_sf_to_rowmajor(ks, rows, K, sel=sel), rm[sel])
+    rows_t, K_t = 256, 128
+    rm_t = rng.integers(0, 256, size=(rows_t, K_t // 16), dtype=np.uint8)
+    tiled = np.zeros(rows_t * K_t // 16, dtype=np.uint8)
+    for r in range(rows_t):
+        for b in range(K_t // 16):
+            tiled[((r // 128) * (K_t // 64) + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4] = rm_t[r, b]
+    assert np.array_equal(untile_sf(tiled, rows_t, K_t), rm_t)
