@@ -149,6 +149,19 @@ def _bits(t: torch.Tensor) -> torch.Tensor:
     return t.contiguous()
 
 
+def _need(t: torch.Tensor, nbytes: int, what: str, dtype=None) -> torch.Tensor:
+    """A caller-given buffer the library reads or writes `nbytes` of: contiguous, large enough, of `dtype`
+    when given (the library sees only a pointer, so a short buffer would be overrun on the device)."""
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise ValueError(f"{what} holds {have} bytes; the call needs {nbytes}")
+    return t
+
+
 # ----------------------------------------------------------------------------- quantize
 
 def _sf_empty(rows: int, K: int, layout: int, dev) -> torch.Tensor:
@@ -171,9 +184,9 @@ def quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None, layout: 
     x = _bits(x)
     rows, K = x.shape
     dev = x.device
-    q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else q
-    sf = _sf_empty(rows, K, layout, dev) if sf is None else sf
-    g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else g
+    q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else _need(q, rows * K // 2, "q")
+    sf = _sf_empty(rows, K, layout, dev) if sf is None else _need(sf, rows * K // 16, "sf")
+    g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else _need(g, 4, "g", torch.float32)
     if ws is None and global_scale is None:
         ws = torch.empty(max(quantize_workspace_size(rows, K), 16), dtype=torch.uint8, device=dev)
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
@@ -188,6 +201,7 @@ def amax(x: torch.Tensor, amax_bits: torch.Tensor | None = None, stream=None) ->
     x = _bits(x)
     if amax_bits is None:
         amax_bits = torch.zeros(1, dtype=torch.int32, device=x.device)
+    _need(amax_bits, 4, "amax_bits")
     _check(lib().nvfp4_amax(_ptr(x), x.shape[0], x.shape[1], _ptr(amax_bits), _stream(stream)), "nvfp4_amax")
     return amax_bits
 
@@ -201,9 +215,10 @@ def quantize_from_amax(x: torch.Tensor, amax_bits: torch.Tensor, layout: int = S
     x = _bits(x)
     rows, K = x.shape
     dev = x.device
-    q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else q
-    sf = _sf_empty(rows, K, layout, dev) if sf is None else sf
-    g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else g
+    _need(amax_bits, 4, "amax_bits")
+    q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else _need(q, rows * K // 2, "q")
+    sf = _sf_empty(rows, K, layout, dev) if sf is None else _need(sf, rows * K // 16, "sf")
+    g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else _need(g, 4, "g", torch.float32)
     _check(lib().nvfp4_quantize_from_amax(_ptr(x), rows, K, _ptr(amax_bits), _ptr(q), _ptr(sf), _ptr(g), layout,
                                           _stream(stream)), "nvfp4_quantize_from_amax")
     return q, sf, g
@@ -219,8 +234,12 @@ def pack_weights(q: torch.Tensor, sf: torch.Tensor, out: torch.Tensor | None = N
     rows, half = q.shape[-2], q.shape[-1]
     rows = q.numel() // half
     K = half * 2
+    _need(q, rows * K // 2, "q")
+    _need(sf, rows * K // 16, "sf")
     if out is None:
         out = torch.empty(packed_weight_bytes(rows, K), dtype=torch.uint8, device=q.device)
+    else:
+        _need(out, packed_weight_bytes(rows, K), "out")
     _check(lib().nvfp4_pack_weights(_ptr(q), _ptr(sf), rows, K, _ptr(out), _stream(stream)), "nvfp4_pack_weights")
     return out
 
@@ -337,8 +356,14 @@ def grouped_gemm(a_q, a_sf, a_g, w: PackedWeights, offsets, swiglu: bool, out=No
     E = offsets.numel() - 1
     N, K = w.N, w.K
     nout = N // 2 if swiglu else N
+    _need(a_q, rows * K // 2, "a_q")
+    _need(a_sf, rows * K // 16, "a_sf")
+    if amax_out is not None:
+        _need(amax_out, 4, "amax_out")
     if out is None:
         out = torch.empty((rows, nout), dtype=torch.bfloat16, device=a_q.device)
+    else:
+        _need(out, rows * nout * 2, "out", torch.bfloat16)
     _check(lib().moe_grouped_gemm_nvfp4_amax(_ptr(a_q), _ptr(a_sf), _ptr(a_g), _ptr(w.packed), _ptr(w.gscale),
                                              _ptr(offsets), E, rows, N, K, EPI_SWIGLU if swiglu else EPI_NONE,
                                              _ptr(out), _ptr(amax_out), _stream(stream)), "moe_grouped_gemm_nvfp4_amax")
@@ -368,8 +393,12 @@ def unpermute_combine(y: torch.Tensor, inv_perm: torch.Tensor, topk_w: torch.Ten
     _require_cuda(y, inv_perm, topk_w)
     T, k = topk_w.shape
     H = y.shape[1]
+    if y.shape[0] < T * k or inv_perm.numel() < T * k:
+        raise ValueError(f"y and inv_perm need {T * k} rows for T={T}, k={k}")
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
+    else:
+        _need(out, T * H * 2, "out", torch.bfloat16)
     _check(lib().moe_unpermute_combine(_ptr(y.contiguous()), _ptr(inv_perm), _ptr(topk_w.contiguous()), T, k, H,
                                        _ptr(out), _stream(stream)), "moe_unpermute_combine")
     return out
@@ -418,6 +447,8 @@ def moe_layer(x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor, w: 
         ws = layer_workspace(T, k, E, H, I, x.device)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    else:
+        _need(out, T * H * 2, "out", torch.bfloat16)
     _check(lib().moe_layer_nvfp4(_ptr(x), _ptr(topk_ids.contiguous()), _ptr(topk_w.contiguous()), T, k, E, H, I,
                                  _ptr(w.w13.packed), _ptr(w.w13.gscale), _ptr(w.w2.packed), _ptr(w.w2.gscale),
                                  _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "moe_layer_nvfp4")

@@ -130,3 +130,20 @@ def test_layout_helpers_follow_the_header_definitions():
         for b in range(K_t // 16):
             tiled[((r // 128) * (K_t // 64) + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4] = rm_t[r, b]
     assert np.array_equal(untile_sf(tiled, rows_t, K_t), rm_t)
+
+
+def test_binding_rejects_short_or_strided_buffers():
+    # The library sees only pointers; the binding refuses caller buffers it would overrun (checked here on
+    # host tensors: the same helper guards every caller-given output of the binding).
+    import pytest
+    import torch
+    need = nv._need
+    t = torch.empty((4, 8), dtype=torch.uint8)
+    assert need(t, 32, "sf") is t
+    with pytest.raises(ValueError):
+        need(t, 33, "sf")
+    with pytest.raises(ValueError):
+        need(torch.empty((8, 8), dtype=torch.uint8)[:, ::2], 16, "sf")     # not contiguous
+    with pytest.raises(TypeError):
+        need(torch.empty(1, dtype=torch.float64), 4, "g", torch.float32)
+    assert need(torch.empty((3, 5), dtype=torch.bfloat16), 30, "out", torch.bfloat16).numel() == 15
