@@ -15,6 +15,9 @@ arithmetic, with its citations of the pages, lives in that file:
   Required: each expert multiplies the subset of tokens routed to it).
 - ``grouped_gemm`` / ``grouped_gemm_at``: per-expert block-scaled dot products
   in FP64, global scales, optional SwiGLU on gate/up halves.
+- ``route_topk``: the router -- top-k logits per token (lower index first
+  among equal values) and the softmax of the chosen k (the pages describe no
+  router; the reading is stated in the C source).
 - ``combine``: top-k weighted sum of expert outputs in FP64 (the final MoE
   output write of "Peering into the CUTLASS Kernel", Input Knowledge Required
   item 5).
@@ -60,6 +63,9 @@ def lib():
         L.oracle_grouped_gemm.argtypes = [P, P, f32, P, P, P, P, i32, i64, i64, i32, P]
         L.oracle_grouped_gemm_at.argtypes = [P, P, f32, P, P, P, P, i32, i64, i64, i32, P, P, i64, P]
         L.oracle_combine.argtypes = [P, P, P, i32, i32, i64, P]
+        L.oracle_route_topk.argtypes = [P, i32, i32, i32, P, P]
+        L.oracle_grouped_gemm_bound.argtypes = [P, P, f32, P, P, P, P, i32, i64, i64, i32, P]
+        L.oracle_grouped_gemm_bound_at.argtypes = [P, P, f32, P, P, P, P, i32, i64, i64, i32, P, P, i64, P]
         L.oracle_num_threads.restype = ctypes.c_int
         L.oracle_set_num_threads.argtypes = [ctypes.c_int]
         _lib = L
@@ -227,6 +233,42 @@ def grouped_gemm_at(a_q, a_sf, a_g, w_q, w_sf, w_g, offsets, N, K, swiglu: bool,
     return out
 
 
+def route_topk(logits: np.ndarray, k: int):
+    """Router: logits [T, E] FP32 -> (topk_ids [T, k] int32, topk_w [T, k] float32)."""
+    z = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = z.shape
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    ids = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float32)
+    lib().oracle_route_topk(_p(z), T, E, int(k), _p(ids), _p(w))
+    return ids, w
+
+
+def grouped_gemm_bound(a_q, a_sf, a_g, w_q, w_sf, w_g, offsets, N, K, swiglu: bool, rows=None, cols=None):
+    """Per-output bound on |FP32-path result - exact result| (the error model of the tensor-core path: exact
+    16-element block partials, FP32 accumulation over the K/16 blocks, FP32 epilogue; see the C source).
+    Every output like grouped_gemm(), or only the (rows, cols) points like grouped_gemm_at()."""
+    a_q = np.ascontiguousarray(a_q, dtype=np.uint8)
+    a_sf = np.ascontiguousarray(a_sf, dtype=np.uint8)
+    w_q = np.ascontiguousarray(w_q, dtype=np.uint8)
+    w_sf = np.ascontiguousarray(w_sf, dtype=np.uint8)
+    w_g = np.ascontiguousarray(w_g, dtype=np.float32)
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    if rows is None:
+        nout = N // 2 if swiglu else N
+        out = np.empty((int(off[-1]), nout), dtype=np.float64)
+        lib().oracle_grouped_gemm_bound(_p(a_q), _p(a_sf), float(a_g), _p(w_q), _p(w_sf), _p(w_g), _p(off),
+                                        off.size - 1, N, K, 1 if swiglu else 0, _p(out))
+        return out
+    r = np.ascontiguousarray(rows, dtype=np.int64)
+    c = np.ascontiguousarray(cols, dtype=np.int64)
+    out = np.empty(r.size, dtype=np.float64)
+    lib().oracle_grouped_gemm_bound_at(_p(a_q), _p(a_sf), float(a_g), _p(w_q), _p(w_sf), _p(w_g), _p(off),
+                                       off.size - 1, N, K, 1 if swiglu else 0, _p(r), _p(c), r.size, _p(out))
+    return out
+
+
 def combine(y_bf16: np.ndarray, inv_perm: np.ndarray, topk_w: np.ndarray) -> np.ndarray:
     """FP64 result [T, H] of the top-k weighted combine."""
     y = _u16(y_bf16)
@@ -242,5 +284,5 @@ def combine(y_bf16: np.ndarray, inv_perm: np.ndarray, topk_w: np.ndarray) -> np.
 __all__ = [
     "lib", "num_threads", "set_num_threads", "e2m1_decode", "e2m1_encode", "e4m3_decode", "e4m3_encode",
     "bf16_to_float", "bf16_from_double", "bf16_round", "bf16_bits_to_f64", "amax", "quantize", "dequantize",
-    "permute", "gather_rows", "grouped_gemm", "grouped_gemm_at", "combine",
+    "permute", "gather_rows", "grouped_gemm", "grouped_gemm_at", "combine", "route_topk", "grouped_gemm_bound",
 ]

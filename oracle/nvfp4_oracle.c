@@ -278,6 +278,54 @@ int oracle_permute(const int32_t* ids, int32_t T, int32_t k, int32_t E,
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Router: top-k experts of each token by logit, then the softmax of the    */
+/* chosen logits. The pages do not describe the router; the MoE grouped     */
+/* GEMM only needs "the subset of tokens routed to" each expert ("Peering   */
+/* into the CUTLASS Kernel Cache", Knowledge Required). Reading taken: the  */
+/* k largest logits by value, the lower expert index first among equal      */
+/* values (+0 and -0 are equal), listed in that order; weights = softmax    */
+/* over the whole row restricted to the chosen k and renormalised, which is */
+/* the softmax of the k chosen logits alone:                                */
+/*   w[t, j] = exp(z[ids[t, j]] - m) / sum_i exp(z[ids[t, i]] - m),         */
+/*   m = z[ids[t, 0]], the sum over i ascending, all in FP64, rounded once  */
+/*   to FP32. A token whose largest chosen logit is -inf gets 1/k each.     */
+/* Logits are finite or -inf (no NaN, no +inf); 1 <= k <= E.                */
+/* ------------------------------------------------------------------------ */
+
+void oracle_route_topk(const float* z, int32_t T, int32_t E, int32_t k, int32_t* ids, float* w) {
+    unsigned char* taken = (unsigned char*)malloc((size_t)E);
+    double* ex = (double*)malloc(sizeof(double) * (size_t)k);
+    for (int32_t t = 0; t < T; t++) {
+        const float* zt = z + (int64_t)t * E;
+        int32_t* it = ids + (int64_t)t * k;
+        memset(taken, 0, (size_t)E);
+        /* explicit selection: k passes, each picking the largest untaken logit */
+        for (int32_t j = 0; j < k; j++) {
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; e++) {
+                if (taken[e]) continue;
+                if (best < 0 || zt[e] > zt[best]) best = e;   /* strict: an equal later value never wins */
+            }
+            taken[best] = 1;
+            it[j] = best;
+        }
+        const double m = (double)zt[it[0]];
+        if (isinf(m) && m < 0) {
+            for (int32_t j = 0; j < k; j++) w[(int64_t)t * k + j] = (float)(1.0 / (double)k);
+            continue;
+        }
+        double sum = 0.0;
+        for (int32_t j = 0; j < k; j++) {
+            ex[j] = exp((double)zt[it[j]] - m);
+            sum += ex[j];
+        }
+        for (int32_t j = 0; j < k; j++) w[(int64_t)t * k + j] = (float)(ex[j] / sum);
+    }
+    free(ex);
+    free(taken);
+}
+
 /* Row gather: dst row p is a byte copy of src row idx[p]. */
 void oracle_gather_rows(const uint8_t* src, int64_t row_bytes, const int32_t* idx, int64_t n,
                         uint8_t* dst) {
@@ -374,6 +422,133 @@ void oracle_grouped_gemm_at(const uint8_t* a_q, const uint8_t* a_sf, float a_g,
             v = silu(v) * u;
         }
         out[i] = v;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP32 error bound of a GEMM output computed the way a tensor-core path    */
+/* computes it (test infrastructure: it decides which one-ulp BF16          */
+/* disagreements are rounding ties, not what the result is).               */
+/* Model: a 16-element block's partial P_b = sum of its 16 products of      */
+/* decoded values is exact in FP32 (E2M1 x E2M1 products are multiples of  */
+/* 1/4 below 37, so their sum needs at most 11 bits, times an E4M3 x E4M3   */
+/* scale product of at most 8 significant bits); the K/16 partials are      */
+/* accumulated in FP32; alpha = FP32(g_A * g_W) and alpha * acc are FP32    */
+/* products; SwiGLU uses single-precision fast exp and division. First-     */
+/* order bounds, u = 2^-24, gamma_n = n u / (1 - n u):                       */
+/*   NONE:   |y' - y| <= |alpha| gamma_{K/16} sum_b |P_b| (1 + 2u)          */
+/*                       + 2.01 u |alpha acc|                                */
+/*   SWIGLU: with dg, du the NONE bounds of gate and up,                    */
+/*           |h' - h| <= 1.1 dg (|up| + du) + |silu(gate)| du               */
+/*                       + (8 + 2 |gate|) 2^-23 |h|                          */
+/*   (1.1 bounds |silu'|; the last term covers the fast exp and division.)  */
+/* ------------------------------------------------------------------------ */
+
+static double block_dot(const double* a, const double* w, int64_t K, double* sabs) {
+    double acc = 0.0, t = 0.0;
+    for (int64_t b = 0; b < K / 16; b++) {
+        double p = 0.0;
+        for (int i = 0; i < 16; i++) p += a[b * 16 + i] * w[b * 16 + i];
+        acc += p;
+        t += fabs(p);
+    }
+    *sabs = t;
+    return acc;
+}
+
+static double bound_plain(double alpha, double acc, double sabs, int64_t K) {
+    const double u = 5.9604644775390625e-08, nu = (double)(K / 16) * u;
+    return fabs(alpha) * (nu / (1.0 - nu)) * sabs * (1.0 + 2.0 * u) + 2.01 * u * fabs(alpha * acc);
+}
+
+static double bound_swiglu(double alpha, double accg, double sg, double accu, double su, int64_t K) {
+    const double g = alpha * accg, up = alpha * accu;
+    const double dg = bound_plain(alpha, accg, sg, K), du = bound_plain(alpha, accu, su, K);
+    const double h = silu(g) * up;
+    return 1.1 * dg * (fabs(up) + du) + fabs(silu(g)) * du + (8.0 + 2.0 * fabs(g)) * 1.1920928955078125e-07 * fabs(h);
+}
+
+/* Bound of every output of oracle_grouped_gemm (same arguments), bound [off[E], Nout]. */
+void oracle_grouped_gemm_bound(const uint8_t* a_q, const uint8_t* a_sf, float a_g,
+                               const uint8_t* w_q, const uint8_t* w_sf, const float* w_g,
+                               const int32_t* off, int32_t E, int64_t N, int64_t K, int32_t epi,
+                               double* bound) {
+    init_tables();
+    int64_t Nout = epi == 1 ? N / 2 : N;
+    for (int32_t e = 0; e < E; e++) {
+        int64_t m0 = off[e], M = off[e + 1] - off[e];
+        if (M <= 0) continue;
+        double alpha = (double)a_g * (double)w_g[e];
+        double* A = (double*)malloc((size_t)(M * K) * sizeof(double));
+        for (int64_t m = 0; m < M; m++)
+            dq_row(a_q + (m0 + m) * (K / 2), a_sf + (m0 + m) * (K / 16), K, A + m * K);
+        const uint8_t* wq = w_q + (int64_t)e * N * (K / 2);
+        const uint8_t* wsf = w_sf + (int64_t)e * N * (K / 16);
+#pragma omp parallel
+        {
+            double* wg = (double*)malloc((size_t)K * sizeof(double));
+            double* wu = (double*)malloc((size_t)K * sizeof(double));
+#pragma omp for schedule(static)
+            for (int64_t n = 0; n < Nout; n++) {
+                dq_row(wq + n * (K / 2), wsf + n * (K / 16), K, wg);
+                if (epi == 1) dq_row(wq + (N / 2 + n) * (K / 2), wsf + (N / 2 + n) * (K / 16), K, wu);
+                for (int64_t m = 0; m < M; m++) {
+                    double sg, su;
+                    const double ag = block_dot(A + m * K, wg, K, &sg);
+                    double b;
+                    if (epi == 1) {
+                        const double au = block_dot(A + m * K, wu, K, &su);
+                        b = bound_swiglu(alpha, ag, sg, au, su, K);
+                    } else {
+                        b = bound_plain(alpha, ag, sg, K);
+                    }
+                    bound[(m0 + m) * Nout + n] = b;
+                }
+            }
+            free(wg);
+            free(wu);
+        }
+        free(A);
+    }
+}
+
+/* Bound at the selected (row, col) points only (same arguments as oracle_grouped_gemm_at). */
+static double block_dot_row(const uint8_t* aq, const uint8_t* asf, const uint8_t* wq, const uint8_t* wsf,
+                            int64_t K, double* sabs) {
+    double acc = 0.0, t = 0.0;
+    for (int64_t b = 0; b < K / 16; b++) {
+        double p = 0.0;
+        for (int64_t k = b * 16; k < b * 16 + 16; k++) p += dq_elem(aq, asf, k) * dq_elem(wq, wsf, k);
+        acc += p;
+        t += fabs(p);
+    }
+    *sabs = t;
+    return acc;
+}
+
+void oracle_grouped_gemm_bound_at(const uint8_t* a_q, const uint8_t* a_sf, float a_g,
+                                  const uint8_t* w_q, const uint8_t* w_sf, const float* w_g,
+                                  const int32_t* off, int32_t E, int64_t N, int64_t K, int32_t epi,
+                                  const int64_t* rows, const int64_t* cols, int64_t n_pts, double* bound) {
+    init_tables();
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t i = 0; i < n_pts; i++) {
+        int64_t m = rows[i], n = cols[i];
+        int32_t e = expert_of_row(off, E, m);
+        if (e < 0) { bound[i] = NAN; continue; }
+        double alpha = (double)a_g * (double)w_g[e];
+        const uint8_t* aq = a_q + m * (K / 2);
+        const uint8_t* asf = a_sf + m * (K / 16);
+        const uint8_t* wq = w_q + (int64_t)e * N * (K / 2);
+        const uint8_t* wsf = w_sf + (int64_t)e * N * (K / 16);
+        double sg, su;
+        const double ag = block_dot_row(aq, asf, wq + n * (K / 2), wsf + n * (K / 16), K, &sg);
+        if (epi == 1) {
+            const double au = block_dot_row(aq, asf, wq + (N / 2 + n) * (K / 2), wsf + (N / 2 + n) * (K / 16), K, &su);
+            bound[i] = bound_swiglu(alpha, ag, sg, au, su, K);
+        } else {
+            bound[i] = bound_plain(alpha, ag, sg, K);
+        }
     }
 }
 

@@ -6,7 +6,7 @@ import torch
 import nvfp4_block_scaled_09_b200 as nv
 import oracle
 import workloads
-from tests.helpers import compare_bf16, gpu_bf16, host, host_bits, require_gpu
+from tests.helpers import combine_band, compare_bf16, gpu_bf16, host, host_bits, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -25,7 +25,7 @@ def test_combine_parity(T, E, k, H):
     out = nv.unpermute_combine(gpu_bf16(y), torch.from_numpy(inv).cuda(), torch.from_numpy(w).cuda())
     exact = oracle.combine(y, inv, w)
     ref = oracle.bf16_round(exact)
-    compare_bf16(host_bits(out), ref, "combine", exact=exact)
+    compare_bf16(host_bits(out), ref, "combine", exact=exact, band=combine_band(y, inv, w))
     # FP64 accumulation of exact products in the oracle's order: bit-identical
     assert np.array_equal(host_bits(out), ref)
 

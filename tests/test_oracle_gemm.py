@@ -188,3 +188,70 @@ def test_combine_matches_einsum():
     yf = oracle.bf16_bits_to_f64(y)
     want = np.einsum("tj,tjh->th", w.astype(np.float64), yf[inv.reshape(T, k)])
     assert np.allclose(oracle.combine(y, inv, w), want, rtol=1e-14, atol=1e-300)
+
+
+# ---- the FP32-path error bound used to recognise rounding ties -------------------------------------------
+
+def _decoded(q, sf):
+    """Decoded block-scaled values (no global scale) with the oracle's own codecs, in FP64."""
+    e2 = np.array([oracle.e2m1_decode(c) for c in range(16)])
+    e4 = np.array([oracle.e4m3_decode(b) for b in range(256)])
+    codes = np.stack([q & 15, q >> 4], axis=-1).reshape(q.shape[0], -1)
+    return e2[codes] * np.repeat(e4[sf], 16, axis=1)
+
+
+def _fp32_model(a, w, alpha, order_rng):
+    """One FP32 computation of the kind the bound covers: exact 16-element block partials, accumulated in
+    FP32 in a random order, times FP32 alpha, rounded in FP32."""
+    P = (a.reshape(a.shape[0], -1, 16)[:, None, :, :] * w.reshape(w.shape[0], -1, 16)[None, :, :, :]).sum(-1)
+    Pf = P.astype(np.float32)
+    assert np.array_equal(Pf.astype(np.float64), P)        # block partials are exact in FP32
+    acc = np.zeros(P.shape[:2], dtype=np.float32)
+    for b in order_rng.permutation(P.shape[2]):
+        acc = (acc + Pf[:, :, b]).astype(np.float32)
+    return (np.float32(alpha) * acc).astype(np.float32)
+
+
+@pytest.mark.parametrize("K", [256, 2048])
+def test_fp32_bound_covers_fp32_accumulation(K):
+    rng = np.random.default_rng(K)
+    M, N = 6, 8
+    a_bits = workloads.random_bf16_bits((M, K), seed=K)
+    w_bits = workloads.random_bf16_bits((N, K), seed=K + 1, std=0.02)
+    aq, asf, ag = oracle.quantize(a_bits)
+    wq, wsf, wg = oracle.quantize(w_bits)
+    off = np.array([0, M], np.int32)
+    exact = oracle.grouped_gemm(aq, asf, ag, wq[None], wsf[None], np.array([wg]), off, N, K, False)
+    bound = oracle.grouped_gemm_bound(aq, asf, ag, wq[None], wsf[None], np.array([wg]), off, N, K, False)
+    alpha = np.float32(np.float32(ag) * np.float32(wg))
+    A, W = _decoded(aq, asf), _decoded(wq, wsf)
+    worst = 0.0
+    for trial in range(20):
+        got = _fp32_model(A, W, alpha, rng).astype(np.float64)
+        assert np.all(np.abs(got - exact) <= bound)
+        worst = max(worst, float(np.max(np.abs(got - exact) / bound)))
+    assert worst > 1e-4      # the bound is not vacuous: some orders use a visible share of it
+    # the sampled form gives the same bound at the same points
+    rr, cc = np.array([0, 3, 5]), np.array([7, 0, 2])
+    assert np.array_equal(oracle.grouped_gemm_bound(aq, asf, ag, wq[None], wsf[None], np.array([wg]), off, N, K,
+                                                    False, rr, cc), bound[rr, cc])
+
+
+def test_fp32_bound_swiglu_covers_fp32_epilogue():
+    rng = np.random.default_rng(5)
+    M, N, K = 5, 8, 512
+    a_bits = workloads.random_bf16_bits((M, K), seed=50)
+    w_bits = workloads.random_bf16_bits((N, K), seed=51, std=0.05)
+    aq, asf, ag = oracle.quantize(a_bits)
+    wq, wsf, wg = oracle.quantize(w_bits)
+    off = np.array([0, M], np.int32)
+    exact = oracle.grouped_gemm(aq, asf, ag, wq[None], wsf[None], np.array([wg]), off, N, K, True)
+    bound = oracle.grouped_gemm_bound(aq, asf, ag, wq[None], wsf[None], np.array([wg]), off, N, K, True)
+    alpha = np.float32(np.float32(ag) * np.float32(wg))
+    A, W = _decoded(aq, asf), _decoded(wq, wsf)
+    for trial in range(10):
+        y = _fp32_model(A, W, alpha, rng)
+        g, u = y[:, : N // 2], y[:, N // 2:]
+        h = (g / (np.float32(1) + np.exp(-g))).astype(np.float32) * u      # single-precision SiLU and product
+        assert np.all(np.abs(h.astype(np.float64) - exact) <= bound)
+    assert np.all(bound > 0) and np.all(bound < 1e-3 * np.sqrt(np.mean(exact ** 2)))

@@ -53,13 +53,14 @@ def derive_seed(seed: int, tag: int, index: int = 0) -> int:
     return (int(seed) * 1_000_003 + int(tag) * 10_007 + int(index)) & 0x7FFF_FFFF_FFFF
 
 
-def routing(T: int, E: int, k: int, kind: str = "uniform", seed: int = 0, zipf_s: float = 1.1,
-            zero_experts: int = 0):
-    """Return (topk_ids int32 [T, k], topk_w float32 [T, k])."""
+def router_logits(T: int, E: int, kind: str = "uniform", seed: int = 0, zipf_s: float = 1.1,
+                  zero_experts: int = 0) -> np.ndarray:
+    """Router logits [T, E] (float64): N(0, 1) for uniform routing; log p_e + Gumbel(0, 1) for Zipf routing
+    (experts with p_e = 0 get -inf)."""
     rng = np.random.Generator(np.random.PCG64(derive_seed(seed, TAG_ROUTER)))
     if kind == "uniform":
-        z = rng.standard_normal((T, E))
-    elif kind == "zipf":
+        return rng.standard_normal((T, E))
+    if kind == "zipf":
         order = rng.permutation(E)                  # order[r] = expert with popularity rank r
         p = np.zeros(E)
         ranks = np.arange(1, E + 1, dtype=np.float64)
@@ -70,9 +71,14 @@ def routing(T: int, E: int, k: int, kind: str = "uniform", seed: int = 0, zipf_s
         with np.errstate(divide="ignore"):
             logp = np.log(p)
         gumbel = -np.log(-np.log(rng.uniform(np.finfo(np.float64).tiny, 1.0, size=(T, E))))
-        z = logp[None, :] + gumbel
-    else:
-        raise ValueError(kind)
+        return logp[None, :] + gumbel
+    raise ValueError(kind)
+
+
+def routing(T: int, E: int, k: int, kind: str = "uniform", seed: int = 0, zipf_s: float = 1.1,
+            zero_experts: int = 0):
+    """Return (topk_ids int32 [T, k], topk_w float32 [T, k]) drawn on the host from router_logits()."""
+    z = router_logits(T, E, kind, seed, zipf_s, zero_experts)
     ids = np.argsort(-z, axis=1, kind="stable")[:, :k].astype(np.int32)
     zs = np.take_along_axis(z, ids, axis=1)
     zs = zs - zs.max(axis=1, keepdims=True)
