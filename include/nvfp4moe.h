@@ -23,6 +23,15 @@
  *  - Streams: every call is asynchronous on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream). No call synchronises with the host except
  *    nvfp4_get_device_status().
+ *  - Concurrency of the grouped GEMM (and of the layer calls that run it):
+ *    each launch hands out its work items from a counter in the library's
+ *    device memory. Launches draw 64 such counters in turn and the last CTA
+ *    of a launch leaves its counter at zero, so up to 64 grouped GEMMs may be
+ *    in flight on one device at once (any streams). A CUDA graph that
+ *    captured a grouped GEMM keeps the counter its capture drew: replays of
+ *    such a graph must run one after another (one stream, or ordered by
+ *    events) and must not overlap direct launches; two launches that share a
+ *    counter at the same time hand out tiles twice or not at all.
  *  - Errors: argument, alignment, shape and capability problems are reported
  *    synchronously, before anything is launched. Launch failures map to
  *    NVFP4_ERR_CUDA. Problems only visible on the device (expert ids out of
@@ -79,8 +88,10 @@ typedef enum { NVFP4_EPI_NONE = 0, NVFP4_EPI_SWIGLU = 1 } nvfp4_epilogue;
  *   of row r, block b sits at ((b / 16) * rows + r) * 16 + (b % 16). The 16
  *   scales of a K step are one 16-byte piece per row, and the pieces of
  *   consecutive rows are adjacent, so any run of rows of one K step is one
- *   contiguous copy. Requires K % 256 == 0. The grouped GEMM reads its
- *   activation scales in this layout. */
+ *   contiguous copy. Requires K % 128 == 0 and a 16-byte aligned buffer of
+ *   ceil(K/256) * rows * 16 bytes: when K % 256 == 128 the last slab holds
+ *   8 scales per row and 8 zero bytes (zero scales) after them. The grouped
+ *   GEMM reads its activation scales in this layout. */
 typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1, NVFP4_SF_KSTAGE = 2 } nvfp4_sf_layout;
 
 /* ------------------------------------------------------------------------ */
@@ -97,10 +108,11 @@ typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA_TILED = 1, NVFP4_SF_KSTAGE = 
 /* Arguments:                                                                */
 /*   x                [rows, K] BF16 bits, device, 16-byte aligned           */
 /*   rows, K          rows >= 1, K % 16 == 0 (MMA_TILED: rows % 128 == 0,    */
-/*                    K % 64 == 0; KSTAGE: K % 256 == 0)                     */
+/*                    K % 64 == 0; KSTAGE: K % 128 == 0)                     */
 /*   global_scale_in  device FP32 scalar or NULL (dynamic amax)             */
 /*   q                [rows, K/2] bytes, device, 8-byte aligned              */
-/*   sf               rows*K/16 bytes, device, in `layout`                   */
+/*   sf               rows*K/16 bytes (KSTAGE: ceil(K/256)*rows*16, 16-byte  */
+/*                    aligned), device, in `layout`                          */
 /*   global_scale_out device FP32 scalar receiving g_dec (may equal         */
 /*                    global_scale_in)                                       */
 /*   ws, ws_bytes     device scratch of nvfp4_quantize_workspace_size() bytes*/
@@ -147,10 +159,11 @@ NVFP4_API nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows,
 /*   to other ranks).                                                        */
 /* Arguments: topk_ids [T, k] int32 (device) with ids in [0, E), distinct   */
 /*   within a token (violations latch NVFP4_ERR_DEVICE_INPUT); 1 <= T,       */
-/*   1 <= k <= 32, 1 <= E <= 1024, T*k < 2^31; K % 256 == 0; q [T, K/2],    */
+/*   1 <= k <= 32, 1 <= E <= 1024, T*k < 2^31; q [T, K/2],                  */
 /*   sf [T, K/16] row-major; outputs q_perm [T*k, K/2], sf_perm (T*k*K/16    */
-/*   bytes), expert_offsets [E+1], perm_src [T*k], inv_perm [T*k]; all       */
-/*   device, 16-byte aligned. ws of moe_permute_workspace_size() bytes.      */
+/*   bytes; KSTAGE: ceil(K/256)*T*k*16), expert_offsets [E+1], perm_src      */
+/*   [T*k], inv_perm [T*k]; all device, 16-byte aligned. K % 128 == 0.       */
+/*   ws of moe_permute_workspace_size() bytes.                               */
 /*   Any other sf_perm_layout returns NVFP4_ERR_INVALID_ARG.                 */
 /* ------------------------------------------------------------------------ */
 NVFP4_API size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E);
@@ -200,16 +213,21 @@ NVFP4_API nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, i
 /*           (rows [0, N/2) of each W_e are the gate, [N/2, N) the up        */
 /*           projection),                                     out [rows, N/2]*/
 /* Arguments:                                                                */
-/*   a_q [max_rows, K/2]; a_sf: max_rows*K/16 bytes in NVFP4_SF_KSTAGE with  */
-/*     max_rows rows per slab (as moe_permute writes it for T*k rows);       */
-/*     a_gscale scalar                                                       */
+/*   a_q [max_rows, K/2]; a_sf: ceil(K/256)*max_rows*16 bytes in            */
+/*     NVFP4_SF_KSTAGE with max_rows rows per slab (as moe_permute writes   */
+/*     it for T*k rows); a_gscale scalar                                     */
 /*   w_packed: the weights [E, N, K] packed by nvfp4_pack_weights() as one   */
 /*     [E*N, K] matrix (nvfp4_packed_weight_bytes(E*N, K) bytes);           */
 /*     w_gscale [E]                                                          */
 /*   expert_offsets [E+1] (device; non-decreasing, off[0] >= 0,              */
 /*   off[E] <= max_rows, else NVFP4_ERR_DEVICE_INPUT is latched and the      */
 /*   offending experts are skipped)                                          */
-/*   Shapes: 1 <= E <= 1024, N % 256 == 0, K % 256 == 0, max_rows >= 0.      */
+/*   Shapes: 1 <= E <= 1024, K % 128 == 0, max_rows >= 0; NONE: N % 128 == 0;*/
+/*   SWIGLU: N % 256 == 0 (N / 2 % 128 == 0: the gate and the up rows of an  */
+/*   output column sit in the same TMEM lane of two 128-row weight blocks,  */
+/*   so half-blocks of gate rows are not offered; the survey's N / 2 % 64   */
+/*   is narrowed to this). K % 256 == 128 runs a last stage of 128 K-       */
+/*   elements; NONE with N % 256 == 128 a last column tile of 128 rows.     */
 /*   All pointers device, 16-byte aligned. Rows outside every expert's range */
 /*   are not written.                                                        */
 /* ------------------------------------------------------------------------ */
@@ -237,14 +255,17 @@ NVFP4_API nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const uin
 /* nvfp4_pack_weights: one-time packing of a quantised weight matrix         */
 /* [rows, K] (codes q [rows, K/2], row-major scales sf [rows, K/16]) into   */
 /* the tiles the grouped GEMM streams. Tile (rb, kt) = rows [128 rb, +128) x */
-/* K [256 kt, +256) is 18432 contiguous bytes at (rb*(K/256) + kt) * 18432:  */
+/* K [256 kt, +256) is 18432 contiguous bytes at (rb*ceil(K/256) + kt) *     */
+/* 18432 (K % 256 == 128: the last tile of a row block holds 128 K-elements  */
+/* and zero codes and zero scales in place of the other 128):                */
 /*   [0, 16384): code bytes, row r at r*128, its 16-byte piece c (K bytes    */
 /*   16c..16c+15 of the tile row) at (c XOR (r % 8)) * 16 (the 128-byte      */
 /*   swizzle the tensor core reads);                                         */
 /*   [16384, 18432): scales, K step kc (64 elements) at kc*512, row r's 4    */
 /*   scale bytes of that step at (r % 32)*16 + (r / 32)*4.                   */
-/* rows % 128 == 0, K % 256 == 0; all pointers device, 16-byte aligned;      */
-/* packed holds nvfp4_packed_weight_bytes(rows, K) bytes (= rows*(K/2+K/16)).*/
+/* rows % 128 == 0, K % 128 == 0; all pointers device, 16-byte aligned;      */
+/* packed holds nvfp4_packed_weight_bytes(rows, K) bytes                     */
+/* (= rows * ceil(K/256) * 144: rows*(K/2+K/16) when K % 256 == 0).          */
 /* ------------------------------------------------------------------------ */
 NVFP4_API size_t nvfp4_packed_weight_bytes(int64_t rows, int64_t K);
 NVFP4_API nvfp4_status nvfp4_pack_weights(const uint8_t* q, const uint8_t* sf, int64_t rows, int64_t K,
@@ -267,6 +288,26 @@ NVFP4_API nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* i
                                    nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* moe_route_topk: the router -- for each token, the k experts with the     */
+/* largest logits and their weights. The grouped GEMM multiplies each       */
+/* expert's weights by "the subset of tokens routed to it" ("Peering into   */
+/* the CUTLASS Kernel Cache", Knowledge Required); the pages do not describe */
+/* the router, so this is the plainest reading of top-k softmax routing:    */
+/*   topk_ids[t, j] = index of the j-th largest logits[t, :] (equal values: */
+/*     the lower index first; -0 equals +0);                                */
+/*   topk_w[t, j]   = exp(z_j - z_0) / sum_{i<k} exp(z_i - z_0) with        */
+/*     z_j = logits[t, topk_ids[t, j]] -- the softmax over all E restricted */
+/*     to the chosen k and renormalised -- computed in FP64 (the sum over i */
+/*     ascending) and rounded once to FP32; 1/k each when z_0 is -inf.      */
+/* Arguments: logits [T, E] FP32 (device, 4-byte aligned; finite or -inf,   */
+/*   no NaN or +inf); topk_ids [T, k] int32 and topk_w [T, k] FP32 (device, */
+/*   4-byte aligned). 1 <= T, 1 <= E <= 1024, 1 <= k <= min(E, 32). The ids  */
+/*   of a token are distinct, as moe_permute requires.                      */
+/* ------------------------------------------------------------------------ */
+NVFP4_API nvfp4_status moe_route_topk(const float* logits, int32_t T, int32_t E, int32_t k, int32_t* topk_ids,
+                            float* topk_w, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* moe_layer_nvfp4: the whole MoE FFN in one call, every step in this        */
 /* library's kernels, in this order: quantize(x) -> moe_permute ->           */
 /* grouped GEMM gate/up (SWIGLU, N = 2I, K = H, amax of h as a side output)  */
@@ -277,20 +318,21 @@ NVFP4_API nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* i
 /*   w13_packed (W13 [E, 2I, H] packed as an [E*2I, H] matrix), w13_gscale   */
 /*   [E]; w2_packed (W2 [E, H, I] packed as [E*H, I]), w2_gscale [E];        */
 /*   out [T, H] BF16.                                                        */
-/*   H % 256 == 0, I % 128 == 0 (2I % 256 == 0 and I % 256 == 0 for the down */
-/*   GEMM's K), plus the limits of the calls above. ws of                    */
+/*   H % 128 == 0, I % 128 == 0, plus the limits of the calls above. ws of   */
 /*   moe_layer_workspace_size() bytes holds every intermediate; its layout   */
 /*   is reported by moe_layer_workspace_layout().                            */
 /* ------------------------------------------------------------------------ */
 typedef struct {
     size_t q_x, sf_x, g_x;                 /* quantised x [T, H/2], [T, H/16], scalar */
-    size_t q_perm, sf_perm;                /* [T*k, H/2]; T*k*H/16 bytes, NVFP4_SF_KSTAGE */
+    size_t q_perm, sf_perm;                /* [T*k, H/2]; ceil(H/256)*T*k*16 bytes, NVFP4_SF_KSTAGE */
     size_t offsets, perm_src, inv_perm;    /* [E+1], [T*k], [T*k] int32 */
     size_t h;                              /* [T*k, I] BF16 */
-    size_t q_h, sf_h, g_h;                 /* [T*k, I/2]; T*k*I/16 bytes, NVFP4_SF_KSTAGE; scalar */
+    size_t q_h, sf_h, g_h;                 /* [T*k, I/2]; ceil(I/256)*T*k*16 bytes, NVFP4_SF_KSTAGE; scalar */
     size_t amax_h;                         /* uint32: max |h| (BF16 bits), from the gate/up GEMM */
     size_t y;                              /* [T*k, H] BF16 */
     size_t scratch;                        /* quantize / permute scratch */
+    size_t topk_ids, topk_w;               /* [T, k] int32 / FP32: the router's output
+                                              (moe_layer_nvfp4_from_logits only) */
     size_t total;
 } nvfp4_layer_workspace;
 
@@ -302,6 +344,16 @@ NVFP4_API nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_id
                              const uint8_t* w13_packed, const float* w13_gscale,
                              const uint8_t* w2_packed, const float* w2_gscale,
                              uint16_t* out, void* ws, size_t ws_bytes, nvfp4_stream_t stream);
+/* moe_layer_nvfp4_from_logits: moe_route_topk(logits [T, E] FP32, k) into   */
+/* the workspace's topk_ids / topk_w, then moe_layer_nvfp4 on them. Same     */
+/* results as the two calls in sequence; same arguments as moe_layer_nvfp4   */
+/* with the router logits (device, 4-byte aligned) in place of the routing, */
+/* and the router's limits (k <= 32, E <= 1024, finite or -inf logits).      */
+NVFP4_API nvfp4_status moe_layer_nvfp4_from_logits(const uint16_t* x, const float* logits,
+                                         int32_t T, int32_t k, int32_t E, int64_t H, int64_t I,
+                                         const uint8_t* w13_packed, const float* w13_gscale,
+                                         const uint8_t* w2_packed, const float* w2_gscale,
+                                         uint16_t* out, void* ws, size_t ws_bytes, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Capability and pipeline plan of the grouped GEMM.                         */

@@ -15,7 +15,9 @@ Calls (same names as the C ABI):
   amax                -> nvfp4_amax
   pack_weights        -> nvfp4_pack_weights
   unpermute_combine   -> moe_unpermute_combine
+  route_topk          -> moe_route_topk
   moe_layer           -> moe_layer_nvfp4
+  moe_layer_from_logits -> moe_layer_nvfp4_from_logits
 """
 from __future__ import annotations
 
@@ -47,7 +49,7 @@ class NVFP4Error(RuntimeError):
 class LayerWorkspace(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "q_x", "sf_x", "g_x", "q_perm", "sf_perm", "offsets", "perm_src", "inv_perm", "h", "q_h", "sf_h", "g_h",
-        "amax_h", "y", "scratch", "total")]
+        "amax_h", "y", "scratch", "topk_ids", "topk_w", "total")]
 
 
 class GemmPlan(ctypes.Structure):
@@ -96,6 +98,10 @@ def lib():
         L.moe_layer_workspace_size.argtypes = [i32, i32, i32, i64, i64]
         L.moe_layer_workspace_size.restype = sz
         L.moe_layer_nvfp4.argtypes = [P, P, P, i32, i32, i32, i64, i64, P, P, P, P, P, P, sz, P]
+        L.moe_layer_nvfp4_from_logits.argtypes = [P, P, i32, i32, i32, i64, i64, P, P, P, P, P, P, sz, P]
+        L.moe_layer_nvfp4_from_logits.restype = st
+        L.moe_route_topk.argtypes = [P, i32, i32, i32, P, P, P]
+        L.moe_route_topk.restype = st
         L.nvfp4_packed_weight_bytes.argtypes = [i64, i64]
         L.nvfp4_packed_weight_bytes.restype = sz
         L.nvfp4_pack_weights.argtypes = [P, P, i64, i64, P, P]
@@ -164,10 +170,19 @@ def _need(t: torch.Tensor, nbytes: int, what: str, dtype=None) -> torch.Tensor:
 
 # ----------------------------------------------------------------------------- quantize
 
+def kstage_slabs(K: int) -> int:
+    """K-stage scale slabs of a K-element row: one per 256 elements, the last one zero-padded when K % 256."""
+    return (K + 255) // 256
+
+
+def sf_bytes(rows: int, K: int, layout: int) -> int:
+    return kstage_slabs(K) * rows * 16 if layout == SF_KSTAGE else rows * K // 16
+
+
 def _sf_empty(rows: int, K: int, layout: int, dev) -> torch.Tensor:
-    """Scale buffer of a [rows, K] tensor: [K/256, rows, 16] in the K-stage layout, else [rows, K/16]."""
+    """Scale buffer of a [rows, K] tensor: [ceil(K/256), rows, 16] in the K-stage layout, else [rows, K/16]."""
     if layout == SF_KSTAGE:
-        return torch.empty((K // 256, rows, 16), dtype=torch.uint8, device=dev)
+        return torch.empty((kstage_slabs(K), rows, 16), dtype=torch.uint8, device=dev)
     return torch.empty((rows, K // 16), dtype=torch.uint8, device=dev)
 
 
@@ -185,7 +200,7 @@ def quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None, layout: 
     rows, K = x.shape
     dev = x.device
     q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else _need(q, rows * K // 2, "q")
-    sf = _sf_empty(rows, K, layout, dev) if sf is None else _need(sf, rows * K // 16, "sf")
+    sf = _sf_empty(rows, K, layout, dev) if sf is None else _need(sf, sf_bytes(rows, K, layout), "sf")
     g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else _need(g, 4, "g", torch.float32)
     if ws is None and global_scale is None:
         ws = torch.empty(max(quantize_workspace_size(rows, K), 16), dtype=torch.uint8, device=dev)
@@ -217,7 +232,7 @@ def quantize_from_amax(x: torch.Tensor, amax_bits: torch.Tensor, layout: int = S
     dev = x.device
     _need(amax_bits, 4, "amax_bits")
     q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else _need(q, rows * K // 2, "q")
-    sf = _sf_empty(rows, K, layout, dev) if sf is None else _need(sf, rows * K // 16, "sf")
+    sf = _sf_empty(rows, K, layout, dev) if sf is None else _need(sf, sf_bytes(rows, K, layout), "sf")
     g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else _need(g, 4, "g", torch.float32)
     _check(lib().nvfp4_quantize_from_amax(_ptr(x), rows, K, _ptr(amax_bits), _ptr(q), _ptr(sf), _ptr(g), layout,
                                           _stream(stream)), "nvfp4_quantize_from_amax")
@@ -246,7 +261,7 @@ def pack_weights(q: torch.Tensor, sf: torch.Tensor, out: torch.Tensor | None = N
 
 @dataclass
 class PackedWeights:
-    packed: torch.Tensor          # [E, N*(K/2 + K/16)] bytes, packed tiles
+    packed: torch.Tensor          # [E, packed_weight_bytes(N, K)] bytes, packed tiles
     gscale: torch.Tensor          # [E] FP32 global scales (dequantisation multipliers)
     E: int
     N: int
@@ -261,7 +276,7 @@ def prepare_expert_weights(w: torch.Tensor, keep_rowmajor: bool = False, stream=
     _require_cuda(w)
     E, N, K = w.shape
     dev = w.device
-    packed = torch.empty((E, N * (K // 2 + K // 16)), dtype=torch.uint8, device=dev)
+    packed = torch.empty((E, packed_weight_bytes(N, K)), dtype=torch.uint8, device=dev)
     g = torch.empty(E, dtype=torch.float32, device=dev)
     qk = torch.empty((E, N, K // 2), dtype=torch.uint8, device=dev) if keep_rowmajor else None
     sk = torch.empty((E, N, K // 16), dtype=torch.uint8, device=dev) if keep_rowmajor else None
@@ -303,6 +318,8 @@ def permute(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_exper
     K = q.shape[1] * 2
     R = T * k
     dev = q.device
+    _need(q, T * K // 2, "q")
+    _need(sf, T * K // 16, "sf")
     out = Permuted(
         q_perm=torch.empty((R, K // 2), dtype=torch.uint8, device=dev),
         sf_perm=_sf_empty(R, K, sf_layout, dev),
@@ -330,6 +347,8 @@ def permute_noalloc(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, n
     K = q.shape[1] * 2
     R = T * k
     dev = q.device
+    _need(q, T * K // 2, "q")
+    _need(sf, T * K // 16, "sf")
     out = Permuted(
         q_perm=torch.empty((R, K // 2), dtype=torch.uint8, device=dev),
         sf_perm=_sf_empty(R, K, sf_layout, dev),
@@ -351,13 +370,14 @@ def grouped_gemm(a_q, a_sf, a_g, w: PackedWeights, offsets, swiglu: bool, out=No
     With amax_out (device int32 [1], zeroed by the caller) the kernel also raises it to max |out| as BF16 bits."""
     _require_cuda(a_q, a_sf, a_g, w.packed, w.gscale, offsets, amax_out)
     rows = a_q.shape[0]
-    if a_sf.dim() != 3 or tuple(a_sf.shape) != (w.K // 256, rows, 16):
-        raise ValueError(f"a_sf must be K-stage scales of shape {(w.K // 256, rows, 16)}, got {tuple(a_sf.shape)}")
+    if a_sf.dim() != 3 or tuple(a_sf.shape) != (kstage_slabs(w.K), rows, 16):
+        raise ValueError(f"a_sf must be K-stage scales of shape {(kstage_slabs(w.K), rows, 16)}, "
+                         f"got {tuple(a_sf.shape)}")
     E = offsets.numel() - 1
     N, K = w.N, w.K
     nout = N // 2 if swiglu else N
     _need(a_q, rows * K // 2, "a_q")
-    _need(a_sf, rows * K // 16, "a_sf")
+    _need(a_sf, sf_bytes(rows, K, SF_KSTAGE), "a_sf")
     if amax_out is not None:
         _need(amax_out, 4, "amax_out")
     if out is None:
@@ -393,6 +413,8 @@ def unpermute_combine(y: torch.Tensor, inv_perm: torch.Tensor, topk_w: torch.Ten
     _require_cuda(y, inv_perm, topk_w)
     T, k = topk_w.shape
     H = y.shape[1]
+    _need(inv_perm, T * k * 4, "inv_perm", torch.int32)
+    _need(topk_w, T * k * 4, "topk_w", torch.float32)
     if y.shape[0] < T * k or inv_perm.numel() < T * k:
         raise ValueError(f"y and inv_perm need {T * k} rows for T={T}, k={k}")
     if out is None:
@@ -402,6 +424,26 @@ def unpermute_combine(y: torch.Tensor, inv_perm: torch.Tensor, topk_w: torch.Ten
     _check(lib().moe_unpermute_combine(_ptr(y.contiguous()), _ptr(inv_perm), _ptr(topk_w.contiguous()), T, k, H,
                                        _ptr(out), _stream(stream)), "moe_unpermute_combine")
     return out
+
+
+# ----------------------------------------------------------------------------- router
+
+def route_topk(logits: torch.Tensor, k: int, ids: torch.Tensor | None = None, w: torch.Tensor | None = None,
+               stream=None):
+    """Router: logits [T, E] float32 -> (topk_ids int32 [T, k], topk_w float32 [T, k]): the k largest logits
+    per token (lower index first among equal values) and the softmax of the chosen k."""
+    _require_cuda(logits)
+    if logits.dtype != torch.float32:
+        raise TypeError("logits must be float32")
+    _need(logits, logits.numel() * 4, "logits")
+    T, E = logits.shape
+    dev = logits.device
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev) if ids is None else _need(ids, T * k * 4, "ids",
+                                                                                          torch.int32)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev) if w is None else _need(w, T * k * 4, "w",
+                                                                                      torch.float32)
+    _check(lib().moe_route_topk(_ptr(logits), T, E, k, _ptr(ids), _ptr(w), _stream(stream)), "moe_route_topk")
+    return ids, w
 
 
 # ----------------------------------------------------------------------------- layer
@@ -452,6 +494,28 @@ def moe_layer(x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor, w: 
     _check(lib().moe_layer_nvfp4(_ptr(x), _ptr(topk_ids.contiguous()), _ptr(topk_w.contiguous()), T, k, E, H, I,
                                  _ptr(w.w13.packed), _ptr(w.w13.gscale), _ptr(w.w2.packed), _ptr(w.w2.gscale),
                                  _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "moe_layer_nvfp4")
+    return out
+
+
+def moe_layer_from_logits(x: torch.Tensor, logits: torch.Tensor, k: int, w: MoEWeights, ws=None, out=None,
+                          stream=None):
+    """moe_layer() with the routing computed by the router kernel from logits [T, E] float32."""
+    _require_cuda(x, logits)
+    x = _bits(x)
+    T, H = x.shape
+    E, I = w.num_experts, w.intermediate
+    if logits.dtype != torch.float32 or tuple(logits.shape) != (T, E):
+        raise ValueError(f"logits must be float32 [{T}, {E}]")
+    _need(logits, T * E * 4, "logits")
+    if ws is None:
+        ws = layer_workspace(T, k, E, H, I, x.device)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    else:
+        _need(out, T * H * 2, "out", torch.bfloat16)
+    _check(lib().moe_layer_nvfp4_from_logits(_ptr(x), _ptr(logits), T, k, E, H, I, _ptr(w.w13.packed),
+                                             _ptr(w.w13.gscale), _ptr(w.w2.packed), _ptr(w.w2.gscale), _ptr(out),
+                                             _ptr(ws), ws.numel(), _stream(stream)), "moe_layer_nvfp4_from_logits")
     return out
 
 

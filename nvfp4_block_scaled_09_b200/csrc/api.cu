@@ -126,13 +126,13 @@ extern "C" nvfp4_status moe_layer_workspace_layout(int32_t T, int32_t k, int32_t
     L->sf_x = take((size_t)T * H / 16);
     L->g_x = take(sizeof(float));
     L->q_perm = take(R * H / 2);
-    L->sf_perm = take(R * H / 16);
+    L->sf_perm = take(R * ((size_t)H + 255) / 256 * 16);   // K-stage slabs (the last one zero-padded)
     L->offsets = take(sizeof(int32_t) * ((size_t)E + 1));
     L->perm_src = take(sizeof(int32_t) * R);
     L->inv_perm = take(sizeof(int32_t) * R);
     L->h = take(R * I * 2);
     L->q_h = take(R * I / 2);
-    L->sf_h = take(R * I / 16);
+    L->sf_h = take(R * ((size_t)I + 255) / 256 * 16);
     L->g_h = take(sizeof(float));
     L->amax_h = take(sizeof(uint32_t));
     L->y = take(R * H * 2);
@@ -141,6 +141,8 @@ extern "C" nvfp4_status moe_layer_workspace_layout(int32_t T, int32_t k, int32_t
     if (qx > scratch) scratch = qx;
     if (qh > scratch) scratch = qh;
     L->scratch = take(scratch);
+    L->topk_ids = take(sizeof(int32_t) * (size_t)T * (size_t)k);
+    L->topk_w = take(sizeof(float) * (size_t)T * (size_t)k);
     L->total = o;
     return NVFP4_OK;
 }
@@ -151,12 +153,13 @@ extern "C" size_t moe_layer_workspace_size(int32_t T, int32_t k, int32_t E, int6
     return L.total;
 }
 
-extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_ids, const float* topk_w, int32_t T,
-                                        int32_t k, int32_t E, int64_t H, int64_t I, const uint8_t* w13_packed,
-                                        const float* w13_gscale, const uint8_t* w2_packed, const float* w2_gscale,
-                                        uint16_t* out, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
-    if (!x || !topk_ids || !topk_w || !w13_packed || !w13_gscale || !w2_packed || !w2_gscale || !out)
-        return NVFP4_ERR_INVALID_ARG;
+// The layer; with `logits` non-null the router first writes the routing into the workspace.
+static nvfp4_status layer(const uint16_t* x, const float* logits, const int32_t* topk_ids, const float* topk_w,
+                          int32_t T, int32_t k, int32_t E, int64_t H, int64_t I, const uint8_t* w13_packed,
+                          const float* w13_gscale, const uint8_t* w2_packed, const float* w2_gscale, uint16_t* out,
+                          void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!x || !w13_packed || !w13_gscale || !w2_packed || !w2_gscale || !out) return NVFP4_ERR_INVALID_ARG;
+    if (logits == nullptr && (!topk_ids || !topk_w)) return NVFP4_ERR_INVALID_ARG;
     nvfp4_layer_workspace L;
     nvfp4_status st = moe_layer_workspace_layout(T, k, E, H, I, &L);
     if (st != NVFP4_OK) return st;
@@ -164,6 +167,10 @@ extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_i
     if (!aligned16(ws)) return NVFP4_ERR_MISALIGNED;
     if ((st = nvfp4_can_implement(2 * I, H, E, NVFP4_EPI_SWIGLU)) != NVFP4_OK) return st;
     if ((st = nvfp4_can_implement(H, I, E, NVFP4_EPI_NONE)) != NVFP4_OK) return st;
+    if (logits != nullptr) {
+        if (E > 1024 || k > 32 || k > E) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+        if ((uintptr_t)logits & 3u) return NVFP4_ERR_MISALIGNED;
+    }
     uint8_t* b = static_cast<uint8_t*>(ws);
     const int64_t R = (int64_t)T * k;
     uint8_t* q_x = b + L.q_x;
@@ -181,12 +188,19 @@ extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_i
     uint32_t* amax_h = reinterpret_cast<uint32_t*>(b + L.amax_h);
     uint16_t* y = reinterpret_cast<uint16_t*>(b + L.y);
     void* scratch = b + L.scratch;
-    const size_t scratch_bytes = L.total - L.scratch;
+    const size_t scratch_bytes = L.topk_ids - L.scratch;
 
     // the gate/up GEMM raises amax_h; it starts from 0 (before the first kernel, so that every kernel
     // boundary after it keeps its programmatic launch)
     if (cudaMemsetAsync(amax_h, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return NVFP4_ERR_CUDA;
+    if (logits != nullptr) {
+        int32_t* ids_ws = reinterpret_cast<int32_t*>(b + L.topk_ids);
+        float* w_ws = reinterpret_cast<float*>(b + L.topk_w);
+        if ((st = moe_route_topk(logits, T, E, k, ids_ws, w_ws, stream))) return st;
+        topk_ids = ids_ws;
+        topk_w = w_ws;
+    }
     if ((st = nvfp4_quantize(x, T, H, nullptr, q_x, sf_x, g_x, NVFP4_SF_ROWMAJOR, scratch, scratch_bytes, stream)))
         return st;
     if ((st = moe_permute(topk_ids, T, k, E, q_x, sf_x, H, q_perm, sf_perm, NVFP4_SF_KSTAGE, off, perm_src, inv_perm,
@@ -200,4 +214,23 @@ extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_i
                                      stream)))
         return st;
     return moe_unpermute_combine(y, inv_perm, topk_w, T, k, H, out, stream);
+}
+
+extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_ids, const float* topk_w, int32_t T,
+                                        int32_t k, int32_t E, int64_t H, int64_t I, const uint8_t* w13_packed,
+                                        const float* w13_gscale, const uint8_t* w2_packed, const float* w2_gscale,
+                                        uint16_t* out, void* ws, size_t ws_bytes, nvfp4_stream_t stream) {
+    if (!topk_ids || !topk_w) return NVFP4_ERR_INVALID_ARG;
+    return layer(x, nullptr, topk_ids, topk_w, T, k, E, H, I, w13_packed, w13_gscale, w2_packed, w2_gscale, out, ws,
+                 ws_bytes, stream);
+}
+
+extern "C" nvfp4_status moe_layer_nvfp4_from_logits(const uint16_t* x, const float* logits, int32_t T, int32_t k,
+                                                    int32_t E, int64_t H, int64_t I, const uint8_t* w13_packed,
+                                                    const float* w13_gscale, const uint8_t* w2_packed,
+                                                    const float* w2_gscale, uint16_t* out, void* ws, size_t ws_bytes,
+                                                    nvfp4_stream_t stream) {
+    if (!logits) return NVFP4_ERR_INVALID_ARG;
+    return layer(x, logits, nullptr, nullptr, T, k, E, H, I, w13_packed, w13_gscale, w2_packed, w2_gscale, out, ws,
+                 ws_bytes, stream);
 }

@@ -56,6 +56,8 @@
 //  * Every wait is bounded (%globaltimer); on expiry the kernel latches
 //    NVFP4_ERR_DEVICE_TIMEOUT, drains its in-flight copies and MMAs, frees
 //    tensor memory and returns.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace nvfp4 {
@@ -223,7 +225,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int32_t E = p.E;
-    const int32_t n_col_tiles = (int32_t)(p.swiglu ? (p.N / 2) / kBM : p.N / (kNumA * kBM));
+    // NONE with N % 256 == 128: the last column tile holds one 128-row weight block ("half" tile)
+    const int32_t n_col_tiles = (int32_t)(p.swiglu ? (p.N / 2) / kBM : (p.N + kNumA * kBM - 1) / (kNumA * kBM));
+    const bool half_cols = !p.swiglu && (p.N % (kNumA * kBM)) != 0;
 
     if (tid == 0) {
         prefetch_tensormap(&tm_a);
@@ -304,7 +308,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
     const int32_t total = sh.total_tiles;
-    const int32_t ksteps_total = (int32_t)(p.K / kBK);
+    // K % 256 == 128: the last stage holds 128 K-elements (2 MMA K-steps); its weight tiles and activation
+    // scales are zero-padded, and the activation tile's second half is outside the tensor (zero-filled)
+    const int32_t ksteps_total = (int32_t)((p.K + kBK - 1) / kBK);
+    const int last_ksteps = (p.K % kBK) ? (int)((p.K % kBK) / 64) : kKSteps;
 
     if (warp == 0) {
         // ================= TMA producer =================
@@ -342,10 +349,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint8_t* wp1 = p.w_packed + (wr1 / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
                 const bool reuse = (sh.off[t.e + 1] - sh.off[t.e]) > kBNMax;
                 const uint64_t pol_w = reuse ? pol_w_reuse : pol_w_once;
-                // MK part: two packed weight tiles (codes + scales); NK part: the activation
+                const int n_a = (half_cols && t.nt == n_col_tiles - 1) ? 1 : kNumA;   // weight blocks of this tile
+                // MK part: the packed weight tiles (codes + scales); NK part: the activation
                 // tile and the tile's rows of the K step's scale slab (16 bytes per row, one
                 // contiguous run in the K-stage layout).
-                const uint32_t tx = (uint32_t)(kNumA * kPackedTileBytes + t.bn * kRowBytes + t.rows * 16);
+                const uint32_t tx = (uint32_t)(n_a * kPackedTileBytes + t.bn * kRowBytes + t.rows * 16);
                 const uint8_t* sfb = p.a_sf + (int64_t)t.row0 * 16;
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
                     if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
@@ -354,7 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(bar, tx);
                     const int32_t kx = kt * kRowBytes;
                     bulk_load(sb + kOffA0, wp0 + (size_t)kt * kPackedTileBytes, kPackedTileBytes, bar, pol_w);
-                    bulk_load(sb + kOffA1, wp1 + (size_t)kt * kPackedTileBytes, kPackedTileBytes, bar, pol_w);
+                    if (n_a == kNumA)
+                        bulk_load(sb + kOffA1, wp1 + (size_t)kt * kPackedTileBytes, kPackedTileBytes, bar, pol_w);
                     for (int32_t i = 0; i < t.bn / kBNStep; i++)
                         tma_load_2d(sb + kOffB + i * kBNStep * kRowBytes, &tm_a, kx, t.row0 + i * kBNStep, bar, pol_a);
                     bulk_load(sb + kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, bar, pol_a);
@@ -387,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             Tile t;
             decode_tile<kBNMax>(sh, E, n_col_tiles, w, t);
             const uint32_t idesc = idesc_base | ((uint32_t)(t.bn >> 3) << 17);
+            const int n_a = (half_cols && t.nt == n_col_tiles - 1) ? 1 : kNumA;
             if (!warp_wait(&sh.acc_empty[abuf], aphase ^ 1u, abort, p.ctl)) { ok = false; break; }
             tc_fence_after();
             for (int32_t kt = 0; kt < ksteps_total; kt++) {
@@ -399,12 +409,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) {
                     const uint32_t sb = smem_u32(stages + (size_t)stage * kStageBytes);
                     const uint32_t sf = tmem + kTmemSFRing + stage * kTmemSFSlot;
+                    const int n_kc = kt == ksteps_total - 1 ? last_ksteps : kKSteps;
 #pragma unroll
                     for (int kc = 0; kc < kKSteps; kc++) {
+                        if (kc >= n_kc) break;
                         const uint64_t bdesc = make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2);
                         const uint32_t acc = (kt | kc) != 0;
 #pragma unroll
                         for (int a = 0; a < kNumA; a++) {
+                            if (a >= n_a) break;
                             const uint64_t adesc = make_smem_desc(sb + a * kPackedTileBytes + kc * 32, 16, 1024, 2);
                             mma_mxf4nvf4(tmem + abuf * (kNumA * kAccCols) + a * kAccCols, adesc, bdesc, idesc,
                                          sf + a * 4 * kKSteps + 4 * kc, sf + kNumA * 4 * kKSteps + 4 * kc, acc);
@@ -498,6 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t cbase = tmem + lane_base + abuf * (kNumA * kAccCols);
             const float alpha = a_g * __ldg(p.w_gscale + t.e);
+            const bool second = !(half_cols && t.nt == n_col_tiles - 1);   // NONE: the second weight block exists
             for (int c = 0; c * 16 < t.bn; c++) {
                 float v0[16], v1[16];
                 tmem_ld_32x32b_x16(cbase + c * 16, v0);
@@ -524,10 +538,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 16; i++) {
                         if (i < nrows) {
                             const uint16_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v0[i]));
-                            const uint16_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v1[i]));
-                            amax = max(amax, (uint32_t)max(b0 & 0x7FFFu, b1 & 0x7FFFu));
+                            amax = max(amax, (uint32_t)(b0 & 0x7FFFu));
                             o[(int64_t)i * ldo] = b0;
-                            o[(int64_t)i * ldo + kBM] = b1;
+                            if (second) {
+                                const uint16_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v1[i]));
+                                amax = max(amax, (uint32_t)(b1 & 0x7FFFu));
+                                o[(int64_t)i * ldo + kBM] = b1;
+                            }
                         }
                     }
                 }
@@ -619,7 +636,7 @@ static bool encode_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t col
 static bool encode_swiglu_weights_map(CUtensorMap* m, const void* w_packed, int32_t E, int64_t N, int64_t K) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
-    const int64_t ksteps = K / 256;
+    const int64_t ksteps = (K + 255) / 256;
     const int64_t tile_bytes = 18432;
     const int64_t up_stride = (N / 2 / 128) * ksteps * tile_bytes;
     const int64_t tiles = ((int64_t)E * N - N / 2) / 128 * ksteps;
@@ -676,7 +693,9 @@ extern "C" nvfp4_status nvfp4_can_implement_with_budget(int64_t N, int64_t K, in
                                                         int64_t smem_optin_bytes) {
     if (epi != NVFP4_EPI_NONE && epi != NVFP4_EPI_SWIGLU) return NVFP4_ERR_INVALID_ARG;
     if (N <= 0 || K <= 0 || E <= 0) return NVFP4_ERR_INVALID_ARG;
-    if (E > gg::kMaxE || N % (gg::kNumA * gg::kBM) != 0 || K % gg::kBK != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (E > gg::kMaxE || K % (gg::kBK / 2) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    // NONE: 128-row weight blocks; SWIGLU: gate and up halves of 128-row blocks each (N / 2 % 128 == 0)
+    if (N % (epi == NVFP4_EPI_SWIGLU ? gg::kNumA * gg::kBM : gg::kBM) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if ((int64_t)E * N > INT32_MAX || K / 2 > INT32_MAX) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     // both tile shapes must fit: the launcher picks one from the rows per expert
     int64_t need = (int64_t)(gg::Wide::kSmemBytes > gg::Narrow::kSmemBytes ? gg::Wide::kSmemBytes
@@ -693,16 +712,19 @@ extern "C" nvfp4_status nvfp4_can_implement(int64_t N, int64_t K, int32_t E, nvf
 }
 
 template <class C>
-static nvfp4_status launch_variant(const CUtensorMap& tm_a, const gg::Params& prm, cudaStream_t s) {
-    static bool configured[64] = {};
+static nvfp4_status launch_variant(const CUtensorMap& tm_a, gg::Params prm, cudaStream_t s) {
+    // the kernel's shared-memory opt-in, once per device (thread-safe)
+    static std::once_flag once[64];
+    static cudaError_t set_result[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
-    if (!configured[dev]) {
-        if (cudaFuncSetAttribute(gg::grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)C::kSmemBytes) != cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        configured[dev] = true;
-    }
+    std::call_once(once[dev], [&] {
+        set_result[dev] = cudaFuncSetAttribute(gg::grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)C::kSmemBytes);
+    });
+    if (set_result[dev] != cudaSuccess) return NVFP4_ERR_CUDA;
+    prm.sched = sched_counter_slot();
+    if (!prm.sched) return NVFP4_ERR_CUDA;
     launch_pdl(gg::grouped_gemm_kernel<C>, dim3(device_sm_count()), dim3(gg::kThreads), C::kSmemBytes, s, tm_a, prm);
     return NVFP4_OK;
 }
@@ -752,13 +774,13 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const ui
     prm.K = K;
     prm.swiglu = epi == NVFP4_EPI_SWIGLU ? 1 : 0;
     prm.amax_out = out_amax;
-    prm.sched = sched_counter_slot();
-    if (!prm.sched) return NVFP4_ERR_CUDA;
+    prm.sched = nullptr;   // drawn by the launcher that runs (one slot per launch)
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (max_rows >= kPairMinAvgRows * (int64_t)E) {
+    // the CTA-pair tile covers 256 weight rows per column tile: NONE with N % 256 == 128 stays on one SM
+    if (max_rows >= kPairMinAvgRows * (int64_t)E && N % (2 * gg::kBM) == 0) {
         CUtensorMap tm_a_full;  // one CTA's half of a full pair tile: 128 rows x 128 bytes
         if (!encode_rows_map(&tm_a_full, a_q, max_rows, K / 2, (uint32_t)pair_gemm_tokens_max() / 2, 128))
             return NVFP4_ERR_CUDA;

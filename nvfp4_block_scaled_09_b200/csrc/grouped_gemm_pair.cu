@@ -27,10 +27,22 @@
 // takes each one and writes it into both CTAs' work-item rings. Every wait is
 // bounded as in the one-SM kernel; a cluster barrier guards the release of
 // tensor memory.
+#include <mutex>
+
 #include "common.cuh"
+
+#ifndef NVFP4_PAIR_SPLIT_SF
+#define NVFP4_PAIR_SPLIT_SF 0
+#endif
+#ifndef NVFP4_PAIR_PREFETCH
+#define NVFP4_PAIR_PREFETCH 0
+#endif
 
 namespace nvfp4 {
 namespace gp {
+
+constexpr bool kSplitSF = NVFP4_PAIR_SPLIT_SF != 0;     // scales on their own barrier, ahead of the operands
+constexpr int kPrefetchAhead = NVFP4_PAIR_PREFETCH;     // weight stages brought into L2 ahead (0: none)
 
 constexpr int kBM = 128;                          // weight rows per CTA (MMA M = 256 per pair)
 constexpr int kBK = 256;                          // K elements per stage
@@ -62,13 +74,16 @@ static_assert(kStageBytes % 1024 == 0 && kOffB % 1024 == 0, "swizzled tiles need
 constexpr int kTileRing = 4;                      // work items the even CTA may publish ahead
 constexpr int kTileConsumersPerCta = 13;          // even CTA: MMA warp + 4 scale writers + 8 epilogue warps;
                                                   // odd CTA: its producer + 4 scale writers + 8 epilogue warps
+constexpr int kTileConsumers = 2 * kTileConsumersPerCta + (kSplitSF ? 1 : 0);  // + the odd CTA's relay warp
 
 struct Shared {
     alignas(16) uint16_t ostage[kEpiWarps][32 * 32];  // epilogue: one 32-token x 32-column BF16 block per warp
     uint64_t tq_full[kTileRing];  // the even CTA published tq[i] (in this CTA's copy of the ring)
     uint64_t tq_empty[kTileRing]; // even CTA: every consumer warp of both CTAs read entry i
     int32_t tq[kTileRing];        // work item index (>= total: no more work)
-    uint64_t full_tma[kStages];   // this CTA's loads of the stage landed
+    uint64_t full_tma[kStages];   // this CTA's loads of the stage landed (split: its operand codes)
+    uint64_t full_sf[kStages];    // split: this CTA's scale bytes of the stage landed
+    uint64_t op_peer[kStages];    // split, even CTA: the odd CTA's operand codes landed (relay arrival)
     uint64_t sf_ready[kStages];   // even CTA: both CTAs' scales are in TMEM (8 warp arrivals)
     uint64_t empty[kStages];      // the pair's MMAs of the stage completed (commit from the even CTA)
     uint64_t acc_full;            // the pair's MMAs of the tile completed
@@ -180,6 +195,22 @@ __device__ __forceinline__ bool publish_tile(Shared& sh, const Params& p, int32_
     return true;
 }
 
+// Packed weight tiles of work item t at K step 0 for CTA `rank`: NONE: g = this CTA's 128 rows, u = the
+// other CTA's; SWIGLU: g = the gate tile, u = the up tile of the item's 128 output columns (both CTAs).
+__device__ __forceinline__ void weight_tiles(const Params& p, const Tile& t, uint32_t rank, int32_t ksteps,
+                                             const uint8_t*& g, const uint8_t*& u) {
+    const int64_t tile_stride = (int64_t)ksteps * kPackedTileBytes;
+    if (p.swiglu) {
+        const int64_t gate_base = (int64_t)t.e * p.N + (int64_t)t.nt * kBM;
+        g = p.w_packed + (gate_base / kBM) * tile_stride;
+        u = p.w_packed + ((gate_base + p.N / 2) / kBM) * tile_stride;
+    } else {
+        const int64_t base = (int64_t)t.e * p.N + (int64_t)t.nt * 2 * kBM;
+        g = p.w_packed + (base / kBM + rank) * tile_stride;
+        u = p.w_packed + (base / kBM + (rank ^ 1u)) * tile_stride;
+    }
+}
+
 // Expert offsets and the first work item of each expert (every CTA builds its own copy).
 __device__ __forceinline__ void build_schedule(Shared& sh, const Params& p, int32_t n_col_tiles) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -243,7 +274,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t rank = cluster_ctarank();
     const int32_t E = p.E;
     const int32_t n_col_tiles = (int32_t)(p.swiglu ? (p.N / 2) / kBM : p.N / (2 * kBM));
-    const int32_t ksteps_total = (int32_t)(p.K / kBK);
+    // K % 256 == 128: the last stage holds 128 K-elements (2 MMA K-steps); weights and activation scales
+    // are zero-padded there, and the activation tile's second half is outside the tensor (zero-filled)
+    const int32_t ksteps_total = (int32_t)((p.K + kBK - 1) / kBK);
+    const int last_ksteps = (p.K % kBK) ? (int)((p.K % kBK) / 64) : kKSteps;
 
     if (tid == 0) {
         prefetch_tensormap(&tm_a);
@@ -253,6 +287,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         sh.abort = 0;
         for (int s = 0; s < kStages; s++) {
             mbar_init(&sh.full_tma[s], 1);
+            mbar_init(&sh.full_sf[s], 1);
+            mbar_init(&sh.op_peer[s], 1);
             mbar_init(&sh.sf_ready[s], 8);
             mbar_init(&sh.empty[s], 1);
         }
@@ -261,7 +297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_init(&sh.drain, 1);
         for (int i = 0; i < kTileRing; i++) {
             mbar_init(&sh.tq_full[i], 1);
-            mbar_init(&sh.tq_empty[i], 2 * kTileConsumersPerCta);
+            mbar_init(&sh.tq_empty[i], kTileConsumers);
         }
         fence_barrier_init();
     }
@@ -307,46 +343,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             } else {
                 ok = next_tile_thread(sh, rank, qi, qphase, w, abort, p.ctl);
             }
+            const int32_t first_w = w;
             while (ok && w < total) {
                 Tile t;
                 decode_tile(sh, E, w, t);
                 const uint64_t pol_w = (sh.off[t.e + 1] - sh.off[t.e] > kBNMax) ? pol_w_reuse : pol_w_once;
                 // weight rows of this CTA, as (packed tile base, byte offset of the first row's codes)
-                const uint8_t* g_tile;   // NONE: the whole 128-row tile; SWIGLU: the gate tile
-                const uint8_t* u_tile = nullptr;
-                uint32_t half = 0;
-                int32_t sw_tile0 = 0;    // SWIGLU: packed-tile index of the gate tile at K step 0
-                if (p.swiglu) {
-                    const int64_t gate_base = (int64_t)t.e * p.N + (int64_t)t.nt * kBM;
-                    g_tile = p.w_packed + (gate_base / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
-                    u_tile = p.w_packed + ((gate_base + p.N / 2) / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
-                    half = rank * 64;
-                    sw_tile0 = (int32_t)((gate_base / kBM) * ksteps_total);
-                } else {
-                    const int64_t base = (int64_t)t.e * p.N + (int64_t)t.nt * 2 * kBM + rank * kBM;
-                    g_tile = p.w_packed + (base / kBM) * ksteps_total * (int64_t)kPackedTileBytes;
-                }
+                const uint8_t* g_tile;   // NONE: this CTA's 128-row tile; SWIGLU: the gate tile
+                const uint8_t* u_tile;   // NONE: the other CTA's tile; SWIGLU: the up tile
+                weight_tiles(p, t, rank, ksteps_total, g_tile, u_tile);
+                const uint32_t half = p.swiglu ? rank * 64 : 0;
+                const int32_t sw_tile0 = (int32_t)((g_tile - p.w_packed) / kPackedTileBytes);  // SWIGLU: gate tile index at K step 0
                 const int32_t my_rows = t.bn / 2;
                 const int32_t my_row0 = t.row0 + (int32_t)rank * my_rows;
-                const uint32_t a_bytes = p.swiglu ? 2u * (kCodeBytes / 2 + kTileSFBytes) : (uint32_t)kPackedTileBytes;
+                // SWIGLU: 16 KB of interleaved gate/up codes + both tiles' 2 KB of scales; NONE: one packed tile
+                const uint32_t a_sf_bytes = p.swiglu ? 2u * kTileSFBytes : (uint32_t)kTileSFBytes;
                 // both CTAs stage the scales of all the tile's rows: one contiguous run of the K step's
                 // slab (K-stage layout), 16 bytes per row
-                const uint32_t tx = a_bytes + (uint32_t)my_rows * kRowBytes + (uint32_t)t.rows * 16u;
+                const uint32_t sf_tx = a_sf_bytes + (uint32_t)t.rows * 16u;
+                const uint32_t op_tx = (uint32_t)kCodeBytes + (uint32_t)my_rows * kRowBytes;
                 const uint8_t* sfb = p.a_sf + (int64_t)t.row0 * 16;
+                // L2 prefetch of the weight stream kPrefetchAhead stages ahead (even CTA, for both CTAs'
+                // tiles), continuing into the next work item's first stages
+                const uint8_t* pf_g = nullptr;
+                const uint8_t* pf_u = nullptr;
+                uint64_t pf_pol = pol_w_once;
+                if (kPrefetchAhead > 0 && rank == 0 && w_next < total) {
+                    Tile tn;
+                    decode_tile(sh, E, w_next, tn);
+                    weight_tiles(p, tn, 0, ksteps_total, pf_g, pf_u);
+                    pf_pol = (sh.off[tn.e + 1] - sh.off[tn.e] > kBNMax) ? pol_w_reuse : pol_w_once;
+                }
+                if (kPrefetchAhead > 0 && rank == 0 && w == first_w) {
+                    // the first work item: its own first stages were not prefetched by a previous item
+                    for (int32_t kt = 0; kt < min(kPrefetchAhead, ksteps_total); kt++) {
+                        bulk_prefetch_l2(g_tile + (size_t)kt * kPackedTileBytes, kPackedTileBytes, pol_w);
+                        bulk_prefetch_l2(u_tile + (size_t)kt * kPackedTileBytes, kPackedTileBytes, pol_w);
+                    }
+                }
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
                     if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
                     uint8_t* sb = stages + (size_t)stage * kStageBytes;
                     uint64_t* bar = &sh.full_tma[stage];
-                    mbar_arrive_expect_tx(bar, tx);
+                    uint64_t* sbar = kSplitSF ? &sh.full_sf[stage] : bar;
+                    if (kSplitSF) {
+                        mbar_arrive_expect_tx(sbar, sf_tx);
+                        mbar_arrive_expect_tx(bar, op_tx);
+                    } else {
+                        mbar_arrive_expect_tx(bar, sf_tx + op_tx);
+                    }
                     const size_t ko = (size_t)kt * kPackedTileBytes;
+                    // scales first: they are small and their consumers (the scale writers) run ahead of the MMAs
+                    if (p.swiglu) {
+                        bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, sbar, pol_w);
+                        bulk_load(sb + kOffSFA + kTileSFBytes, u_tile + ko + kCodeBytes, kTileSFBytes, sbar, pol_w);
+                    } else if (kSplitSF) {
+                        bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, sbar, pol_w);
+                    }
+                    bulk_load(sb + kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, sbar, pol_a);
                     if (p.swiglu) {
                         // 16-row slabs (2 KB, whole swizzle atoms) of this CTA's half: gate slab q -> A rows
                         // 32q.., up slab q -> 32q+16.. (one box: bytes x rows x gate/up x slab x tile)
                         tma_load_5d(sb + kOffA, &tm_wsw, 0, 0, 0, (int32_t)(half / 16), sw_tile0 + kt, bar, pol_w);
-                        bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
-                        bulk_load(sb + kOffSFA + kTileSFBytes, u_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
+                    } else if (kSplitSF) {
+                        bulk_load(sb + kOffA, g_tile + ko, kCodeBytes, bar, pol_w);
                     } else {
-                        bulk_load(sb + kOffA, g_tile + ko, kPackedTileBytes, bar, pol_w);
+                        bulk_load(sb + kOffA, g_tile + ko, kPackedTileBytes, bar, pol_w);   // codes + scales
                     }
                     if (my_rows == kBNMax / 2) {
                         tma_load_2d(sb + kOffB, &tm_a_full, kt * kRowBytes, my_row0, bar, pol_a);
@@ -355,7 +417,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             tma_load_2d(sb + kOffB + i * kBoxRows * kRowBytes, &tm_a, kt * kRowBytes,
                                         my_row0 + i * kBoxRows, bar, pol_a);
                     }
-                    bulk_load(sb + kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, bar, pol_a);
+                    if (kPrefetchAhead > 0 && rank == 0) {
+                        const int32_t ka = kt + kPrefetchAhead;
+                        if (ka < ksteps_total) {
+                            bulk_prefetch_l2(g_tile + (size_t)ka * kPackedTileBytes, kPackedTileBytes, pol_w);
+                            bulk_prefetch_l2(u_tile + (size_t)ka * kPackedTileBytes, kPackedTileBytes, pol_w);
+                        } else if (pf_g != nullptr && ka - ksteps_total < ksteps_total) {
+                            const size_t kn = (size_t)(ka - ksteps_total) * kPackedTileBytes;
+                            bulk_prefetch_l2(pf_g + kn, kPackedTileBytes, pf_pol);
+                            bulk_prefetch_l2(pf_u + kn, kPackedTileBytes, pf_pol);
+                        }
+                    }
                     issued[stage] = true;
                     issued_parity[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -369,8 +441,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok || *abort) {
-                for (int s = 0; s < kStages; s++)
-                    if (issued[s]) mbar_wait_drain(&sh.full_tma[s], issued_parity[s], 200000000ull);
+                for (int s = 0; s < kStages; s++) {
+                    if (!issued[s]) continue;
+                    mbar_wait_drain(&sh.full_tma[s], issued_parity[s], 200000000ull);
+                    if (kSplitSF) mbar_wait_drain(&sh.full_sf[s], issued_parity[s], 200000000ull);
+                }
             }
         }
         __syncwarp();
@@ -390,7 +465,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int32_t w;
             if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl) || w >= total) break;
             for (int32_t kt = 0; kt < ksteps_total; kt++) {
-                if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl)) { ok = false; break; }
+                if (!warp_wait(kSplitSF ? &sh.full_sf[stage] : &sh.full_tma[stage], phase, abort, p.ctl)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint8_t* sb = stages + (size_t)stage * kStageBytes;
                 const uint32_t slot = tmem + lane_addr + kTmemSFRing + stage * kSFSlot;
@@ -438,6 +516,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
                     if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl) ||
+                        (kSplitSF && !warp_wait(&sh.op_peer[stage], phase, abort, p.ctl)) ||
                         !warp_wait(&sh.sf_ready[stage], phase, abort, p.ctl)) {
                         ok = false;
                         break;
@@ -446,8 +525,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (lane == 0) {
                         const uint32_t sb = smem_u32(stages + (size_t)stage * kStageBytes);
                         const uint32_t sf = tmem + kTmemSFRing + stage * kSFSlot;
+                        const int n_kc = kt == ksteps_total - 1 ? last_ksteps : kKSteps;
 #pragma unroll
                         for (int kc = 0; kc < kKSteps; kc++) {
+                            if (kc >= n_kc) break;
                             mma_mxf4nvf4_pair(tmem, make_smem_desc(sb + kOffA + kc * 32, 16, 1024, 2),
                                               make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2), idesc,
                                               sf + 4 * kc, sf + 16 + 8 * kc, (kt | kc) != 0);
@@ -472,6 +553,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     mbar_wait_drain(&sh.drain, 0, 200000000ull);
                 }
                 __syncwarp();
+            }
+        } else if (kSplitSF) {
+            // ================= relay (odd CTA): this CTA's operand codes of a stage landed =================
+            uint32_t stage = 0, phase = 0, qi = 0, qphase = 0;
+            const uint32_t peer0 = cluster_smem_addr(&sh.op_peer[0], 0);
+            bool ok = true;
+            while (ok) {
+                int32_t w;
+                if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl) || w >= total) break;
+                for (int32_t kt = 0; kt < ksteps_total; kt++) {
+                    if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl)) { ok = false; break; }
+                    if (lane == 0) mbar_arrive_cluster(peer0 + stage * 8);
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
             }
         }
     } else if (warp >= 4) {  // warps 4-7 and 12-15
@@ -626,14 +721,17 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
                                       int swiglu, uint16_t* out, uint32_t* out_amax, cudaStream_t s,
                                       uint32_t* status) {
-    static bool configured[64] = {};
+    // once per device (thread-safe): the shared-memory opt-in and the persistent grid size
+    static std::once_flag once[64];
     static int grid_for[64] = {};
+    static nvfp4_status set_result[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
-    if (!configured[dev]) {
+    std::call_once(once[dev], [&] {
+        set_result[dev] = NVFP4_ERR_CUDA;
         if (cudaFuncSetAttribute(gp::grouped_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gp::kSmemBytes) != cudaSuccess)
-            return NVFP4_ERR_CUDA;
+            return;
         // as many pairs as can be resident at once (persistent grid)
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)device_sm_count() / 2 * 2);
@@ -648,11 +746,14 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
         cfg.numAttrs = 1;
         int clusters = 0;
         if (cudaOccupancyMaxActiveClusters(&clusters, gp::grouped_gemm_pair_kernel, &cfg) != cudaSuccess ||
-            clusters <= 0)
-            return NVFP4_ERR_SMEM_BUDGET;
+            clusters <= 0) {
+            set_result[dev] = NVFP4_ERR_SMEM_BUDGET;
+            return;
+        }
         grid_for[dev] = 2 * clusters < device_sm_count() ? 2 * clusters : device_sm_count() / 2 * 2;
-        configured[dev] = true;
-    }
+        set_result[dev] = NVFP4_OK;
+    });
+    if (set_result[dev] != NVFP4_OK) return set_result[dev];
     gp::Params prm;
     prm.a_sf = a_sf;
     prm.a_gscale = a_gscale;

@@ -133,7 +133,9 @@ __global__ void __launch_bounds__(kTok) permute_rank_kernel(const int32_t* __res
 }
 
 // One warp per output row; rows whose source index is invalid become zeros.
-template <bool kKStage>
+// kHalf: K % 256 == 128. A row-major scale row is then 8 bytes past a multiple of 16, so the scales
+// move in 8-byte units, and the last K-stage slab gets the row's last 8 scales plus 8 zero bytes.
+template <bool kKStage, bool kHalf>
 __global__ void __launch_bounds__(256) permute_gather_kernel(const uint4* __restrict__ q, const uint4* __restrict__ sf,
                                                              int64_t qvec, int64_t sfvec,
                                                              const int32_t* __restrict__ perm_src, int32_t T,
@@ -150,11 +152,27 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(const uint4* __rest
     const uint4* qs = q + (int64_t)(ok ? src : 0) * qvec;
     uint4* qd = q_perm + p * qvec;
     for (int64_t i = lane; i < qvec; i += 32) qd[i] = ok ? __ldg(qs + i) : zero;
-    const uint4* ss = sf + (int64_t)(ok ? src : 0) * sfvec;
-    for (int64_t i = lane; i < sfvec; i += 32) {
-        const uint4 v = ok ? __ldg(ss + i) : zero;
-        if (kKStage) sf_perm[i * R + p] = v;   // K step i's slab, row p
-        else sf_perm[p * sfvec + i] = v;
+    if (!kHalf) {
+        const uint4* ss = sf + (int64_t)(ok ? src : 0) * sfvec;
+        for (int64_t i = lane; i < sfvec; i += 32) {
+            const uint4 v = ok ? __ldg(ss + i) : zero;
+            if (kKStage) sf_perm[i * R + p] = v;   // K step i's slab, row p
+            else sf_perm[p * sfvec + i] = v;
+        }
+    } else {
+        // sfvec counts 8-byte units here (K / 128 per row)
+        const uint2* ss = reinterpret_cast<const uint2*>(sf) + (int64_t)(ok ? src : 0) * sfvec;
+        const uint2 z2 = make_uint2(0u, 0u);
+        if (kKStage) {
+            for (int64_t i = lane; i < (sfvec + 1) / 2; i += 32) {
+                const uint2 lo = ok ? __ldg(ss + 2 * i) : z2;
+                const uint2 hi = (ok && 2 * i + 1 < sfvec) ? __ldg(ss + 2 * i + 1) : z2;
+                sf_perm[i * R + p] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+            }
+        } else {
+            uint2* sd = reinterpret_cast<uint2*>(sf_perm) + p * sfvec;
+            for (int64_t i = lane; i < sfvec; i += 32) sd[i] = ok ? __ldg(ss + i) : z2;
+        }
     }
 }
 
@@ -167,10 +185,12 @@ static inline int32_t permute_chunks(int32_t T) { return (T + kTok - 1) / kTok; 
 
 static void launch_gather(const uint8_t* q, const uint8_t* sf, int64_t K, const int32_t* perm_src, int32_t T,
                           int64_t R, uint8_t* q_perm, uint8_t* sf_perm, nvfp4_sf_layout layout, cudaStream_t s) {
-    auto kernel = layout == NVFP4_SF_KSTAGE ? permute_gather_kernel<true> : permute_gather_kernel<false>;
+    const bool kstage = layout == NVFP4_SF_KSTAGE, half = K % 256 != 0;
+    auto kernel = kstage ? (half ? permute_gather_kernel<true, true> : permute_gather_kernel<true, false>)
+                         : (half ? permute_gather_kernel<false, true> : permute_gather_kernel<false, false>);
     launch_pdl(kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, s, reinterpret_cast<const uint4*>(q),
-               reinterpret_cast<const uint4*>(sf), K / 32, K / 256, perm_src, T, R, reinterpret_cast<uint4*>(q_perm),
-               reinterpret_cast<uint4*>(sf_perm));
+               reinterpret_cast<const uint4*>(sf), K / 32, half ? K / 128 : K / 256, perm_src, T, R,
+               reinterpret_cast<uint4*>(q_perm), reinterpret_cast<uint4*>(sf_perm));
 }
 
 extern "C" size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E) {
@@ -187,7 +207,7 @@ extern "C" nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t 
         return NVFP4_ERR_INVALID_ARG;
     if (sf_perm_layout != NVFP4_SF_ROWMAJOR && sf_perm_layout != NVFP4_SF_KSTAGE) return NVFP4_ERR_INVALID_ARG;
     if (T <= 0 || k <= 0 || E <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
-    if (k > 32 || E > kMaxE || (int64_t)T * k >= (int64_t)1 << 31 || K % 256 != 0)
+    if (k > 32 || E > kMaxE || (int64_t)T * k >= (int64_t)1 << 31 || K % 128 != 0)
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(topk_ids) || !aligned16(q) || !aligned16(sf) || !aligned16(q_perm) || !aligned16(sf_perm) ||
         !aligned16(expert_offsets) || !aligned16(perm_src) || !aligned16(inv_perm))
@@ -248,7 +268,7 @@ extern "C" nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, 
         return NVFP4_ERR_INVALID_ARG;
     if (sf_perm_layout != NVFP4_SF_ROWMAJOR && sf_perm_layout != NVFP4_SF_KSTAGE) return NVFP4_ERR_INVALID_ARG;
     if (T <= 0 || k <= 0 || E <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
-    if (k > 32 || E > kMaxE || (int64_t)T * k >= (int64_t)1 << 31 || K % 256 != 0)
+    if (k > 32 || E > kMaxE || (int64_t)T * k >= (int64_t)1 << 31 || K % 128 != 0)
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int32_t nchunks = permute_chunks(T);
     if ((int64_t)nchunks * E > NVFP4_PERMUTE_NOALLOC_SCRATCH_ENTRIES) return NVFP4_ERR_UNSUPPORTED_SHAPE;

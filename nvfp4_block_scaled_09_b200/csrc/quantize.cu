@@ -178,6 +178,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
             // slab of the 256-element K step kb / 16, row r's 16-byte piece, byte kb % 16
             const int64_t r = b / blocks_per_row, kb = b - r * blocks_per_row;
             sf_off = ((kb >> 4) * rows + r) * 16 + (kb & 15);
+            // K % 256 == 128: the last slab's piece holds 8 scales; its other 8 bytes are zero scales
+            if ((blocks_per_row & 15) == 8 && kb == blocks_per_row - 1)
+                *reinterpret_cast<uint2*>(sf + sf_off + 1) = make_uint2(0u, 0u);
         } else {
             sf_off = b;
         }
@@ -228,8 +231,8 @@ extern "C" nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t 
         return NVFP4_ERR_INVALID_ARG;
     if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (layout == NVFP4_SF_MMA_TILED && (rows % 128 != 0 || K % 64 != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (layout == NVFP4_SF_KSTAGE && K % 256 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(x) || !aligned8(q)) return NVFP4_ERR_MISALIGNED;
+    if (layout == NVFP4_SF_KSTAGE && K % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned8(q) || (layout == NVFP4_SF_KSTAGE && !aligned16(sf))) return NVFP4_ERR_MISALIGNED;
     if (((uintptr_t)global_scale_out & 3u) || (global_scale_in && ((uintptr_t)global_scale_in & 3u)))
         return NVFP4_ERR_MISALIGNED;
     const int64_t nvec = rows * K / 8;
@@ -258,8 +261,8 @@ extern "C" nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows
         return NVFP4_ERR_INVALID_ARG;
     if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (layout == NVFP4_SF_MMA_TILED && (rows % 128 != 0 || K % 64 != 0)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (layout == NVFP4_SF_KSTAGE && K % 256 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(x) || !aligned8(q)) return NVFP4_ERR_MISALIGNED;
+    if (layout == NVFP4_SF_KSTAGE && K % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned8(q) || (layout == NVFP4_SF_KSTAGE && !aligned16(sf))) return NVFP4_ERR_MISALIGNED;
     if (((uintptr_t)global_scale_out & 3u) || ((uintptr_t)amax_bits & 3u)) return NVFP4_ERR_MISALIGNED;
     launch_quantize(x, rows, K, nullptr, amax_bits, 1, q, sf, global_scale_out, layout,
                     reinterpret_cast<cudaStream_t>(stream));

@@ -76,14 +76,17 @@ def run_full(rows, N, K, swiglu, seed, pad_rows=0):
     R = c["R"]
     ref = oracle.grouped_gemm(host(c["a_q"])[:R], c["a_sf_rm"][:R], host(c["a_g"])[0], w_q, w_sf, w_g,
                               c["off_np"], N, K, swiglu)
+    band = oracle.grouped_gemm_bound(host(c["a_q"])[:R], c["a_sf_rm"][:R], host(c["a_g"])[0], w_q, w_sf, w_g,
+                                     c["off_np"], N, K, swiglu)
     got = host_bits(out)[: c["R"]]
-    return compare_bf16(got, oracle.bf16_round(ref), f"gemm rows={rows} N={N} K={K} swiglu={swiglu}", exact=ref)
+    return compare_bf16(got, oracle.bf16_round(ref), f"gemm rows={rows} N={N} K={K} swiglu={swiglu}", exact=ref,
+                        band=band)
 
 
 def test_tiny_config():
     # 4 experts x 16 rows, K = N = 256, plain epilogue
     stats = run_full([16, 16, 16, 16], 256, 256, False, seed=0)
-    assert stats["exact_frac"] > 0.95
+    assert stats["exact_frac"] > 0.97
 
 
 @pytest.mark.parametrize("swiglu", [False, True])
@@ -155,6 +158,24 @@ def test_deeper_k_and_wider_n(swiglu):
     run_full([5, 40, 200], 768, 2048, swiglu, seed=2)
 
 
+@pytest.mark.parametrize("N,K,swiglu", [(128, 128, False), (384, 384, False), (128, 640, False), (256, 128, True),
+                                        (512, 384, True)])
+def test_k_and_n_multiples_of_128(N, K, swiglu):
+    # the boundary's smallest steps: K at its minimum 128, K % 256 == 128 (a last stage of 128 K-elements over
+    # zero-padded weight tiles and scale slabs), and, for the plain epilogue, N % 256 == 128 (a last column
+    # tile of one 128-row weight block); narrow tiles
+    assert nv.can_implement(N, K, 6, swiglu) == 0
+    run_full([0, 5, 16, 33, 64, 1], N, K, swiglu, seed=N + K)
+
+
+@pytest.mark.parametrize("N,K,swiglu,pad", [(384, 384, False, 1200), (512, 384, True, 1200),
+                                            (384, 128, False, 0)])
+def test_k_and_n_multiples_of_128_wide_and_pair(N, K, swiglu, pad):
+    # the same shapes on the wide one-SM tile (NONE with N % 256 == 128 stays on one SM even when the rows
+    # per expert would pick CTA pairs) and on the CTA-pair kernel (SwiGLU, K % 256 == 128)
+    run_full([0, 200, 256, 257, 40], N, K, swiglu, seed=N * K, pad_rows=pad)
+
+
 def test_rows_outside_experts_untouched():
     c = make_case([10, 0, 20], 256, 256, seed=3)
     R = c["R"]
@@ -191,8 +212,10 @@ def sampled_check(a_q, a_sf, a_g, c_w, off_np, N, K, swiglu, out, experts, n_col
     asf = kstage_sf_to_rowmajor(host(a_sf), a_q.shape[0], K, sel=a_rows)
     ref = oracle.grouped_gemm_at(aq, asf, float(host(a_g)[0]), w_q, w_sf, w_g, np.array(sub_off, np.int32), N, K,
                                  swiglu, rr, cc)
+    band = oracle.grouped_gemm_bound(aq, asf, float(host(a_g)[0]), w_q, w_sf, w_g, np.array(sub_off, np.int32), N,
+                                     K, swiglu, rr, cc)
     got = host_bits(out)[a_rows[rr], cc]
-    return compare_bf16(got, oracle.bf16_round(ref), f"sampled N={N} K={K} swiglu={swiglu}", exact=ref)
+    return compare_bf16(got, oracle.bf16_round(ref), f"sampled N={N} K={K} swiglu={swiglu}", exact=ref, band=band)
 
 
 def test_dense_8192_sampled():
@@ -217,7 +240,9 @@ def test_dense_8192_sampled():
     rr, cc = rr.ravel(), cc.ravel()
     ref = oracle.grouped_gemm_at(host(a_q), a_sf_rm, float(host(a_g)[0]), host(pw.q), host(pw.sf),
                                  host(pw.gscale), np.array([0, M], np.int32), N, K, False, rr, cc)
-    compare_bf16(host_bits(out)[rr, cc], oracle.bf16_round(ref), "dense 8192", exact=ref)
+    band = oracle.grouped_gemm_bound(host(a_q), a_sf_rm, float(host(a_g)[0]), host(pw.q), host(pw.sf),
+                                     host(pw.gscale), np.array([0, M], np.int32), N, K, False, rr, cc)
+    compare_bf16(host_bits(out)[rr, cc], oracle.bf16_round(ref), "dense 8192", exact=ref, band=band)
 
 
 def build_layer_weights(E, N, K, tag, keep):

@@ -71,13 +71,14 @@ def test_tiled_layout_is_a_permutation_of_rowmajor():
     assert np.array_equal(untile_sf(sf_t, 256, 512), osf)
 
 
-@pytest.mark.parametrize("rows,K", [(1, 256), (37, 768), (300, 6144)])
+@pytest.mark.parametrize("rows,K", [(1, 256), (37, 768), (300, 6144), (5, 128), (33, 384)])
 def test_kstage_layout_is_a_permutation_of_rowmajor(rows, K):
-    # the grouped GEMM's activation-scale layout: one [rows x 16 B] slab per 256-element K step
+    # the grouped GEMM's activation-scale layout: one [rows x 16 B] slab per 256-element K step (K % 256 == 128:
+    # the last slab zero-padded, which the converter checks)
     x = workloads.random_bf16_bits((rows, K), seed=rows, std=1.0)
     q, sf_k, g = gpu_quantize(x, layout=nv.SF_KSTAGE)
     oq, osf, og = oracle.quantize(x)
-    assert sf_k.shape == (K // 256, rows, 16)
+    assert sf_k.shape == ((K + 255) // 256, rows, 16)
     assert g == og and np.array_equal(q, oq)
     assert np.array_equal(kstage_sf_to_rowmajor(sf_k, rows, K), osf)
 

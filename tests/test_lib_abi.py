@@ -36,8 +36,14 @@ def test_can_implement_shapes_and_budget(L):
     assert nv.can_implement(6144, 2048, 256, False, big) == 0
     assert nv.can_implement(8192, 8192, 1, False, big) == 0
     assert nv.can_implement(256, 256, 4, False, big) == 0
+    # K % 128 and, for the plain epilogue, N % 128; SwiGLU needs N % 256 (gate and up 128-row blocks)
+    assert nv.can_implement(128, 128, 4, False, big) == 0
+    assert nv.can_implement(384, 384, 4, False, big) == 0
+    assert nv.can_implement(4096, 6144 + 128, 256, True, big) == 0
     assert nv.can_implement(4096 + 128, 6144, 256, True, big) == 3
-    assert nv.can_implement(4096, 6144 + 128, 256, True, big) == 3
+    assert nv.can_implement(4096, 6144 + 64, 256, True, big) == 3
+    assert nv.can_implement(128 + 64, 128, 4, False, big) == 3
+    assert nv.can_implement(128, 64, 4, False, big) == 3
     assert nv.can_implement(4096, 6144, 1025, True, big) == 3
     assert nv.can_implement(0, 6144, 8, True, big) == 1
     # a budget below either tile shape's shared memory is refused before any launch
@@ -98,7 +104,9 @@ def test_invalid_arguments_rejected_before_any_cuda_call(L):
     assert L.moe_permute(p, 4, 8, 8, p, p, 256, p, p, 2, p, p, p, None, 0, None) == 4       # no workspace
     assert L.moe_permute(p, 4, 8, 8, p, p, 256, p, p, 1, p, p, p, p, 1 << 20, None) == 1    # tiled sf_perm
     assert L.moe_permute_noalloc(p, 4, 8, 8, p, p, 256, p, p, 7, p, p, p, None) == 1        # unknown layout
-    assert L.nvfp4_quantize(p, 4, 128, p, p, p, p, 2, None, 0, None) == 3   # K-stage layout: K % 256 != 0
+    assert L.nvfp4_quantize(p, 4, 64, p, p, p, p, 2, None, 0, None) == 3    # K-stage layout: K % 128 != 0
+    assert L.nvfp4_quantize(p, 4, 128, p, p, ctypes.c_void_p(24), p, 2, None, 0, None) == 2  # K-stage sf misaligned
+    assert L.moe_permute(p, 4, 8, 8, p, p, 192, p, p, 2, p, p, p, p, 1 << 20, None) == 3    # K % 128 != 0
     assert L.nvfp4_quantize(p, 4, 256, p, p, p, p, 3, None, 0, None) == 1   # unknown layout
     assert L.nvfp4_quantize_from_amax(None, 4, 32, None, None, None, None, 0, None) == 1
     assert L.nvfp4_quantize_from_amax(p, 4, 32, ctypes.c_void_p(18), p, p, p, 0, None) == 2  # amax word misaligned
@@ -123,6 +131,16 @@ def test_layout_helpers_follow_the_header_definitions():
     assert np.array_equal(kstage_sf_to_rowmajor(ks, rows, K), rm)
     sel = np.array([36, 0, 17])
     assert np.array_equal(kstage_sf_to_rowmajor(ks, rows, K, sel=sel), rm[sel])
+    # K % 256 == 128: ceil(K/256) slabs, the last one's second 8 bytes of every row are zero scales
+    K_h = 384
+    rm_h = rng.integers(0, 256, size=(rows, K_h // 16), dtype=np.uint8)
+    ks_h = rowmajor_sf_to_kstage(rm_h, rows, K_h)
+    assert ks_h.shape == (2, rows, 16) and not ks_h[1, :, 8:].any()
+    flat_h = ks_h.reshape(-1)
+    for r in range(rows):
+        for b in range(K_h // 16):
+            assert flat_h[((b // 16) * rows + r) * 16 + b % 16] == rm_h[r, b]
+    assert np.array_equal(kstage_sf_to_rowmajor(ks_h, rows, K_h), rm_h)
     rows_t, K_t = 256, 128
     rm_t = rng.integers(0, 256, size=(rows_t, K_t // 16), dtype=np.uint8)
     tiled = np.zeros(rows_t * K_t // 16, dtype=np.uint8)
