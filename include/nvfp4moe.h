@@ -252,6 +252,34 @@ NVFP4_API nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const uin
                                          uint32_t* out_amax, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* moe_grouped_gemm_nvfp4_finalize: the down GEMM with the top-k combine     */
+/* fused into its epilogue -- the FINALIZE epilogue that performs the final */
+/* MoE output write ("Peering into the CUTLASS Kernel", Input Knowledge     */
+/* Required, item 5).                                                        */
+/*   The GEMM (NONE epilogue) writes y [max_rows, N] as moe_grouped_gemm_    */
+/*   nvfp4 does, and out [T, N] = moe_unpermute_combine(y, inv_perm,        */
+/*   topk_w) -- the same bits: for every (token, 128-column block) the CTA  */
+/*   that writes the token's k-th row of that block sums the k rows in FP64 */
+/*   in slot order with one final rounding, whichever rows came first.      */
+/* Arguments: the GEMM's as in moe_grouped_gemm_nvfp4 (NONE epilogue, y is   */
+/*   its output); perm_src [max_rows] (row -> token), inv_perm [T*k]         */
+/*   ((token, slot) -> row) as moe_permute writes them, topk_w [T, k] FP32,  */
+/*   T * k <= max_rows, k <= 32; counters: moe_finalize_counters_size(T, N)  */
+/*   bytes of device memory, zero before the first call (each call leaves   */
+/*   it zero again; re-zero it after a call that reported an error);        */
+/*   out [T, N] BF16. All device, 4-byte aligned (y and out as for the       */
+/*   GEMM). Calls sharing one counters buffer must not overlap.              */
+/* ------------------------------------------------------------------------ */
+NVFP4_API size_t moe_finalize_counters_size(int32_t T, int64_t N);
+NVFP4_API nvfp4_status moe_grouped_gemm_nvfp4_finalize(const uint8_t* a_q, const uint8_t* a_sf,
+                                             const float* a_gscale, const uint8_t* w_packed,
+                                             const float* w_gscale, const int32_t* expert_offsets,
+                                             int32_t E, int64_t max_rows, int64_t N, int64_t K,
+                                             uint16_t* y, const int32_t* perm_src, const int32_t* inv_perm,
+                                             const float* topk_w, int32_t T, int32_t k, uint32_t* counters,
+                                             uint16_t* out, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* nvfp4_pack_weights: one-time packing of a quantised weight matrix         */
 /* [rows, K] (codes q [rows, K/2], row-major scales sf [rows, K/16]) into   */
 /* the tiles the grouped GEMM streams. Tile (rb, kt) = rows [128 rb, +128) x */
@@ -329,6 +357,8 @@ typedef struct {
     size_t h;                              /* [T*k, I] BF16 */
     size_t q_h, sf_h, g_h;                 /* [T*k, I/2]; ceil(I/256)*T*k*16 bytes, NVFP4_SF_KSTAGE; scalar */
     size_t amax_h;                         /* uint32: max |h| (BF16 bits), from the gate/up GEMM */
+    size_t fin_counters;                   /* the down GEMM's fused-combine counters, right after amax_h
+                                              (both zeroed by one memset at the start of each call) */
     size_t y;                              /* [T*k, H] BF16 */
     size_t scratch;                        /* quantize / permute scratch */
     size_t topk_ids, topk_w;               /* [T, k] int32 / FP32: the router's output

@@ -49,7 +49,7 @@ class NVFP4Error(RuntimeError):
 class LayerWorkspace(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "q_x", "sf_x", "g_x", "q_perm", "sf_perm", "offsets", "perm_src", "inv_perm", "h", "q_h", "sf_h", "g_h",
-        "amax_h", "y", "scratch", "topk_ids", "topk_w", "total")]
+        "amax_h", "fin_counters", "y", "scratch", "topk_ids", "topk_w", "total")]
 
 
 class GemmPlan(ctypes.Structure):
@@ -102,6 +102,11 @@ def lib():
         L.moe_layer_nvfp4_from_logits.restype = st
         L.moe_route_topk.argtypes = [P, i32, i32, i32, P, P, P]
         L.moe_route_topk.restype = st
+        L.moe_finalize_counters_size.argtypes = [i32, i64]
+        L.moe_finalize_counters_size.restype = sz
+        L.moe_grouped_gemm_nvfp4_finalize.argtypes = [P, P, P, P, P, P, i32, i64, i64, i64, P, P, P, P, i32, i32, P,
+                                                      P, P]
+        L.moe_grouped_gemm_nvfp4_finalize.restype = st
         L.nvfp4_packed_weight_bytes.argtypes = [i64, i64]
         L.nvfp4_packed_weight_bytes.restype = sz
         L.nvfp4_pack_weights.argtypes = [P, P, i64, i64, P, P]
@@ -388,6 +393,40 @@ def grouped_gemm(a_q, a_sf, a_g, w: PackedWeights, offsets, swiglu: bool, out=No
                                              _ptr(offsets), E, rows, N, K, EPI_SWIGLU if swiglu else EPI_NONE,
                                              _ptr(out), _ptr(amax_out), _stream(stream)), "moe_grouped_gemm_nvfp4_amax")
     return out
+
+
+def finalize_counters(T: int, N: int, device="cuda") -> torch.Tensor:
+    """Zeroed arrival counters for grouped_gemm_finalize (each call leaves them zero)."""
+    n = int(lib().moe_finalize_counters_size(T, N))
+    return torch.zeros(max(n // 4, 1), dtype=torch.int32, device=device)
+
+
+def grouped_gemm_finalize(a_q, a_sf, a_g, w: PackedWeights, offsets, perm_src, inv_perm, topk_w, counters,
+                          y=None, out=None, stream=None):
+    """Down GEMM (plain epilogue) with the top-k combine fused into its epilogue: returns (out [T, N] bf16,
+    y [rows, N] bf16). perm_src / inv_perm as permute() returns them, topk_w [T, k] float32."""
+    _require_cuda(a_q, a_sf, a_g, w.packed, w.gscale, offsets, perm_src, inv_perm, topk_w, counters)
+    rows = a_q.shape[0]
+    T, k = topk_w.shape
+    N, K = w.N, w.K
+    E = offsets.numel() - 1
+    if a_sf.dim() != 3 or tuple(a_sf.shape) != (kstage_slabs(K), rows, 16):
+        raise ValueError(f"a_sf must be K-stage scales of shape {(kstage_slabs(K), rows, 16)}")
+    _need(a_q, rows * K // 2, "a_q")
+    _need(a_sf, sf_bytes(rows, K, SF_KSTAGE), "a_sf")
+    _need(perm_src, rows * 4, "perm_src", torch.int32)
+    _need(inv_perm, T * k * 4, "inv_perm", torch.int32)
+    _need(topk_w, T * k * 4, "topk_w", torch.float32)
+    _need(counters, int(lib().moe_finalize_counters_size(T, N)), "counters")
+    y = torch.empty((rows, N), dtype=torch.bfloat16, device=a_q.device) if y is None else \
+        _need(y, rows * N * 2, "y", torch.bfloat16)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device=a_q.device) if out is None else \
+        _need(out, T * N * 2, "out", torch.bfloat16)
+    _check(lib().moe_grouped_gemm_nvfp4_finalize(_ptr(a_q), _ptr(a_sf), _ptr(a_g), _ptr(w.packed), _ptr(w.gscale),
+                                                 _ptr(offsets), E, rows, N, K, _ptr(y), _ptr(perm_src),
+                                                 _ptr(inv_perm), _ptr(topk_w), T, k, _ptr(counters), _ptr(out),
+                                                 _stream(stream)), "moe_grouped_gemm_nvfp4_finalize")
+    return out, y
 
 
 def can_implement(N: int, K: int, E: int, swiglu: bool, smem_budget: int | None = None) -> int:

@@ -135,6 +135,7 @@ extern "C" nvfp4_status moe_layer_workspace_layout(int32_t T, int32_t k, int32_t
     L->sf_h = take(R * ((size_t)I + 255) / 256 * 16);
     L->g_h = take(sizeof(float));
     L->amax_h = take(sizeof(uint32_t));
+    L->fin_counters = take(moe_finalize_counters_size(T, H));
     L->y = take(R * H * 2);
     size_t scratch = moe_permute_workspace_size(T, k, E);
     const size_t qx = nvfp4_quantize_workspace_size(T, H), qh = nvfp4_quantize_workspace_size((int64_t)R, I);
@@ -190,9 +191,12 @@ static nvfp4_status layer(const uint16_t* x, const float* logits, const int32_t*
     void* scratch = b + L.scratch;
     const size_t scratch_bytes = L.topk_ids - L.scratch;
 
-    // the gate/up GEMM raises amax_h; it starts from 0 (before the first kernel, so that every kernel
-    // boundary after it keeps its programmatic launch)
-    if (cudaMemsetAsync(amax_h, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    uint32_t* fin_counters = reinterpret_cast<uint32_t*>(b + L.fin_counters);
+    // the gate/up GEMM raises amax_h and the down GEMM counts rows into fin_counters; both start from 0
+    // (one memset before the first kernel, so that every kernel boundary after it keeps its
+    // programmatic launch)
+    if (cudaMemsetAsync(amax_h, 0, L.fin_counters + moe_finalize_counters_size(T, H) - L.amax_h,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     if (logits != nullptr) {
         int32_t* ids_ws = reinterpret_cast<int32_t*>(b + L.topk_ids);
@@ -210,10 +214,10 @@ static nvfp4_status layer(const uint16_t* x, const float* logits, const int32_t*
                                           NVFP4_EPI_SWIGLU, h, amax_h, stream)))
         return st;
     if ((st = nvfp4_quantize_from_amax(h, R, I, amax_h, q_h, sf_h, g_h, NVFP4_SF_KSTAGE, stream))) return st;
-    if ((st = moe_grouped_gemm_nvfp4(q_h, sf_h, g_h, w2_packed, w2_gscale, off, E, R, H, I, NVFP4_EPI_NONE, y,
-                                     stream)))
-        return st;
-    return moe_unpermute_combine(y, inv_perm, topk_w, T, k, H, out, stream);
+    // the down GEMM with the top-k combine fused into its epilogue (same bits as the GEMM followed by
+    // moe_unpermute_combine)
+    return moe_grouped_gemm_nvfp4_finalize(q_h, sf_h, g_h, w2_packed, w2_gscale, off, E, R, H, I, y, perm_src,
+                                           inv_perm, topk_w, T, k, fin_counters, out, stream);
 }
 
 extern "C" nvfp4_status moe_layer_nvfp4(const uint16_t* x, const int32_t* topk_ids, const float* topk_w, int32_t T,

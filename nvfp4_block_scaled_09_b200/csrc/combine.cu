@@ -24,14 +24,6 @@ __device__ __forceinline__ void acc_bf16x2(double& a0, double& a1, uint32_t w, d
     a1 = fma(s, (double)__uint_as_float(w & 0xFFFF0000u), a1);
 }
 
-// FP64 -> BF16, round to nearest even, in effect a single rounding: truncate to
-// FP32, mark inexactness in the last bit (round-to-odd), then round to BF16.
-__device__ __forceinline__ uint32_t f64_to_bf16_bits(double d) {
-    float f = __double2float_rz(d);
-    if ((double)f != d) f = __uint_as_float(__float_as_uint(f) | 1u);
-    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(double lo, double hi) {
     return f64_to_bf16_bits(lo) | (f64_to_bf16_bits(hi) << 16);
 }

@@ -29,6 +29,16 @@ struct DeviceCtl {
     uint32_t flags;        // kCtl* test flags
 };
 
+// The grouped GEMM's fused top-k combine (moe_grouped_gemm_nvfp4_finalize); off when out == nullptr.
+struct Finalize {
+    const int32_t* src;    // [rows] token of each activation row (moe_permute's perm_src)
+    const int32_t* inv;    // [T * k] row of each (token, slot) (moe_permute's inv_perm)
+    const float* w;        // [T, k] combine weights
+    uint32_t* counters;    // [T, col_blocks] arrivals per (token, 128-column block); zero on entry, left zero
+    uint16_t* out;         // [T, N] combined BF16 output
+    int32_t T, k, col_blocks;
+};
+
 // Host-side registry (api.cu).
 uint32_t* status_word_ptr();          // nullptr on failure
 uint32_t* sched_counter_slot();       // two zeroed words for one GEMM launch's dynamic schedule (nullptr on failure)
@@ -46,8 +56,8 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
                                       const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const uint8_t* a_sf,
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
-                                      int swiglu, uint16_t* out, uint32_t* out_amax, cudaStream_t s,
-                                      uint32_t* status);
+                                      int swiglu, uint16_t* out, uint32_t* out_amax, const Finalize& fin,
+                                      cudaStream_t s, uint32_t* status);
 
 #ifdef __CUDACC__
 // Launch `kernel` on `s` with programmatic stream serialization (see pdl_wait()).
@@ -342,6 +352,31 @@ __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_
 // without branches (fast exponential and division, a few fp32 ulp: far below the BF16 output's
 // resolution). For g below about -88 the exponential overflows and the result is -0 * u.
 __device__ __forceinline__ float swiglu_f32(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
+// FP64 -> BF16, round to nearest even, in effect a single rounding: truncate to FP32, mark inexactness
+// in the last bit (round-to-odd), then round to BF16. (The combine's final rounding, shared by the
+// separate combine kernel and the GEMM's fused combine so the two agree bit for bit.)
+__device__ __forceinline__ uint32_t f64_to_bf16_bits(double d) {
+    float f = __double2float_rz(d);
+    if ((double)f != d) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// One output element of the top-k weighted combine: sum over the token's slots j ascending of
+// w[t, j] * y[inv_perm[t*k + j], col] in FP64 (each product of an FP32 weight and a BF16 value is exact),
+// negative rows skipped; y is read past L1 (other SMs wrote it). Returns the BF16 bits.
+__device__ __forceinline__ uint32_t combine_element(const uint16_t* y, int64_t ldy, const int32_t* inv_perm,
+                                                    const float* w, int32_t t, int32_t k, int64_t col) {
+    double acc = 0.0;
+    for (int32_t j = 0; j < k; j++) {
+        const int32_t p = __ldg(inv_perm + (int64_t)t * k + j);
+        if (p < 0) continue;
+        const double s = (double)__ldg(w + (int64_t)t * k + j);
+        const uint32_t b = __ldcg(reinterpret_cast<const unsigned short*>(y + (int64_t)p * ldy + col));
+        acc = fma(s, (double)__uint_as_float(b << 16), acc);
+    }
+    return f64_to_bf16_bits(acc);
+}
 
 // ---- thread-block clusters and CTA pairs (cta_group::2) ---------------------
 

@@ -103,6 +103,8 @@ struct Shared {
     int32_t total_tiles;
     int32_t off[kMaxE + 1];
     int32_t tile_start[kMaxE + 1];
+    int32_t fin_tok[128];                        // fused combine: tokens of this tile whose last row it wrote
+    uint64_t fin_bar;                            // fused combine: the 4 epilogue warps meet (bounded waits)
 };
 
 // Two tile shapes share one kernel body:
@@ -152,6 +154,7 @@ struct Params {
     uint32_t* amax_out;   // nullable: raised to max |out| (BF16 bits)
     uint32_t* sched;      // this launch's work counter [0] and finished-CTA counter [1]; zero at launch
     DeviceCtl ctl;
+    Finalize fin;         // fused top-k combine (NONE epilogue), off when fin.out == nullptr
 };
 
 struct Tile {
@@ -242,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sh.acc_empty[b], 4);
         }
         mbar_init(&sh.drain, 1);
+        mbar_init(&sh.fin_bar, 4);
         for (int i = 0; i < kTileRing; i++) {
             mbar_init(&sh.tq_full[i], 1);
             mbar_init(&sh.tq_empty[i], kTileConsumers);
@@ -500,7 +504,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const float a_g = __ldg(p.a_gscale);
         uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
-        uint32_t abuf = 0, aphase = 0, qi = 0, qphase = 0;
+        uint32_t abuf = 0, aphase = 0, qi = 0, qphase = 0, fphase = 0;
+        // the 4 epilogue warps meet here (fused combine only); false when a wait ran out
+        auto epi_sync = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.fin_bar);
+            const bool ok = warp_wait(&sh.fin_bar, fphase, abort, p.ctl);
+            fphase ^= 1u;
+            return ok;
+        };
         while (true) {
             int32_t w;
             if (!next_tile(sh, qi, qphase, w, lane, abort, p.ctl)) break;
@@ -553,6 +565,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.acc_empty[abuf]);
             if (++abuf == (uint32_t)C::kAccBufs) { abuf = 0; aphase ^= 1u; }
+            if (p.fin.out != nullptr) {
+                // Fused combine. Every row of this tile holds one (token, slot) product for the tile's output
+                // columns; count the rows in per (token, column tile). The CTA that brings a token's count
+                // to k writes that token's combined output for these columns, whichever CTA wrote the other
+                // k - 1 rows, with the combine's arithmetic, so the result does not depend on the order.
+                __threadfence();                            // this thread's y stores, device-wide, first
+                if (!epi_sync()) break;
+                const int i = (warp - 4) * 32 + lane;
+                int32_t tok = -1;
+                if (i < t.rows) {
+                    const int32_t tk = __ldg(p.fin.src + t.row0 + i);
+                    if (tk >= 0 && tk < p.fin.T) {
+                        uint32_t* cnt = p.fin.counters + (int64_t)tk * p.fin.col_blocks + 2 * t.nt;
+                        if (atomicAdd(cnt, 1u) == (uint32_t)(p.fin.k - 1)) {
+                            atomicExch(cnt, 0u);            // left at zero for the next launch
+                            tok = tk;
+                        }
+                    }
+                }
+                sh.fin_tok[i] = tok;
+                __threadfence();                            // the other rows' stores are visible before the reads
+                if (!epi_sync()) break;
+                const int64_t col = (int64_t)t.nt * (kNumA * kBM) + r;
+                for (int j = 0; j < t.rows; j++) {
+                    const int32_t tk = sh.fin_tok[j];
+                    if (tk < 0) continue;
+                    p.fin.out[(int64_t)tk * p.N + col] =
+                        (uint16_t)combine_element(p.out, p.N, p.fin.inv, p.fin.w, tk, p.fin.k, col);
+                    if (second)
+                        p.fin.out[(int64_t)tk * p.N + col + kBM] =
+                            (uint16_t)combine_element(p.out, p.N, p.fin.inv, p.fin.w, tk, p.fin.k, col + kBM);
+                }
+                if (!epi_sync()) break;                     // fin_tok is rewritten by the next tile
+            }
         }
         if (p.amax_out != nullptr) {
             amax = __reduce_max_sync(0xFFFFFFFFu, amax);
@@ -738,11 +784,11 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
                                        epi, out, nullptr, stream);
 }
 
-extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
-                                                    const uint8_t* w_packed, const float* w_gscale,
-                                                    const int32_t* expert_offsets, int32_t E, int64_t max_rows,
-                                                    int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
-                                                    uint32_t* out_amax, nvfp4_stream_t stream) {
+// Validates, encodes the tensor maps and launches one of the three kernels.
+static nvfp4_status grouped_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
+                                 const uint8_t* w_packed, const float* w_gscale, const int32_t* expert_offsets,
+                                 int32_t E, int64_t max_rows, int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
+                                 uint32_t* out_amax, const Finalize& fin, nvfp4_stream_t stream) {
     if (!a_q || !a_sf || !a_gscale || !w_packed || !w_gscale || !expert_offsets || !out)
         return NVFP4_ERR_INVALID_ARG;
     if ((uintptr_t)out_amax & 3u) return NVFP4_ERR_MISALIGNED;
@@ -774,6 +820,7 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const ui
     prm.K = K;
     prm.swiglu = epi == NVFP4_EPI_SWIGLU ? 1 : 0;
     prm.amax_out = out_amax;
+    prm.fin = fin;
     prm.sched = nullptr;   // drawn by the launcher that runs (one slot per launch)
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
@@ -791,7 +838,7 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const ui
         CUtensorMap tm_wsw = tm_a;  // SWIGLU: interleaved gate/up weight slabs (unused otherwise)
         if (prm.swiglu && !encode_swiglu_weights_map(&tm_wsw, w_packed, E, N, K)) return NVFP4_ERR_CUDA;
         return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_out, tm_wsw, a_sf, a_gscale, w_packed, w_gscale,
-                                        expert_offsets, E, max_rows, N, K, prm.swiglu, out, out_amax, s, status);
+                                        expert_offsets, E, max_rows, N, K, prm.swiglu, out, out_amax, fin, s, status);
     }
     const bool wide = max_rows >= kWideMinAvgRows * (int64_t)E;
     const nvfp4_status ls =
@@ -799,4 +846,46 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const ui
     if (ls != NVFP4_OK) return ls;
     count_launch();
     return check_launch();
+}
+
+extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
+                                                    const uint8_t* w_packed, const float* w_gscale,
+                                                    const int32_t* expert_offsets, int32_t E, int64_t max_rows,
+                                                    int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
+                                                    uint32_t* out_amax, nvfp4_stream_t stream) {
+    const Finalize none = {};
+    return grouped_gemm(a_q, a_sf, a_gscale, w_packed, w_gscale, expert_offsets, E, max_rows, N, K, epi, out, out_amax,
+                        none, stream);
+}
+
+extern "C" size_t moe_finalize_counters_size(int32_t T, int64_t N) {
+    if (T <= 0 || N <= 0) return 0;
+    return (size_t)T * (size_t)((N + 127) / 128) * sizeof(uint32_t);
+}
+
+extern "C" nvfp4_status moe_grouped_gemm_nvfp4_finalize(const uint8_t* a_q, const uint8_t* a_sf,
+                                                        const float* a_gscale, const uint8_t* w_packed,
+                                                        const float* w_gscale, const int32_t* expert_offsets,
+                                                        int32_t E, int64_t max_rows, int64_t N, int64_t K,
+                                                        uint16_t* y, const int32_t* perm_src,
+                                                        const int32_t* inv_perm, const float* topk_w, int32_t T,
+                                                        int32_t k, uint32_t* counters, uint16_t* out,
+                                                        nvfp4_stream_t stream) {
+    if (!perm_src || !inv_perm || !topk_w || !counters || !out || !y) return NVFP4_ERR_INVALID_ARG;
+    if (T <= 0 || k <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (k > 32 || (int64_t)T * k > max_rows) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (((uintptr_t)perm_src & 3u) || ((uintptr_t)inv_perm & 3u) || ((uintptr_t)topk_w & 3u) ||
+        ((uintptr_t)counters & 3u) || ((uintptr_t)out & 1u))
+        return NVFP4_ERR_MISALIGNED;
+    Finalize fin;
+    fin.src = perm_src;
+    fin.inv = inv_perm;
+    fin.w = topk_w;
+    fin.counters = counters;
+    fin.out = out;
+    fin.T = T;
+    fin.k = k;
+    fin.col_blocks = (int32_t)((N + 127) / 128);
+    return grouped_gemm(a_q, a_sf, a_gscale, w_packed, w_gscale, expert_offsets, E, max_rows, N, K, NVFP4_EPI_NONE, y,
+                        nullptr, fin, stream);
 }

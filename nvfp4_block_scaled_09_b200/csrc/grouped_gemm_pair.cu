@@ -94,6 +94,8 @@ struct Shared {
     int32_t total_tiles;
     int32_t off[kMaxE + 1];
     int32_t tile_start[kMaxE + 1];
+    int32_t fin_tok[kBNMax];      // fused combine: tokens of this tile whose last row this CTA wrote
+    uint64_t fin_bar;             // fused combine: this CTA's 8 epilogue warps meet (bounded waits)
 };
 
 constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Shared);
@@ -114,6 +116,7 @@ struct Params {
     uint32_t* amax_out;   // nullable: raised to max |out| (BF16 bits)
     uint32_t* sched;      // this launch's work counter [0] and finished-CTA counter [1]; zero at launch
     DeviceCtl ctl;
+    Finalize fin;         // fused top-k combine (NONE epilogue), off when fin.out == nullptr
 };
 
 struct Tile {
@@ -295,6 +298,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_init(&sh.acc_full, 1);
         mbar_init(&sh.acc_empty, 2 * kEpiWarps);
         mbar_init(&sh.drain, 1);
+        mbar_init(&sh.fin_bar, kEpiWarps);
         for (int i = 0; i < kTileRing; i++) {
             mbar_init(&sh.tq_full[i], 1);
             mbar_init(&sh.tq_empty[i], kTileConsumers);
@@ -581,7 +585,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const bool up_lane = lane >= 16;
         const float a_g = __ldg(p.a_gscale);
         uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
-        uint32_t aphase = 0, qi = 0, qphase = 0;
+        uint32_t aphase = 0, qi = 0, qphase = 0, fphase = 0;
+        // this CTA's 8 epilogue warps meet here (fused combine only); false when a wait ran out
+        auto epi_sync = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.fin_bar);
+            const bool ok = warp_wait(&sh.fin_bar, fphase, abort, p.ctl);
+            fphase ^= 1u;
+            return ok;
+        };
         while (true) {
             int32_t w;
             if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl) || w >= total) break;
@@ -657,8 +669,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         col = t.nt * 2 * kBM + (int32_t)rank * kBM + quad * 32;
                         lane_cols = 4;
                     }
-                    if (nrows == 32) {
+                    if (nrows == 32 && p.fin.out == nullptr) {
                         // a whole chunk of the expert: one asynchronous tensor store of the block
+                        // (the fused combine stores directly: its last arrivers read these rows back)
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
@@ -681,6 +694,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             aphase ^= 1u;
+            if (p.fin.out != nullptr) {
+                // Fused combine over this CTA's 128 output columns: count the tile's rows in per (token,
+                // 128-column block); the CTA that brings a count to k writes that token's combined output
+                // for these columns (see the one-SM kernel: the result does not depend on the order).
+                __threadfence();                            // this thread's y stores, device-wide, first
+                if (!epi_sync()) break;
+                const int i = (half * 4 + quad) * 32 + lane;
+                int32_t tok = -1;
+                if (i < t.rows) {
+                    const int32_t tk = __ldg(p.fin.src + t.row0 + i);
+                    if (tk >= 0 && tk < p.fin.T) {
+                        uint32_t* cnt = p.fin.counters + (int64_t)tk * p.fin.col_blocks + 2 * t.nt + rank;
+                        if (atomicAdd(cnt, 1u) == (uint32_t)(p.fin.k - 1)) {
+                            atomicExch(cnt, 0u);            // left at zero for the next launch
+                            tok = tk;
+                        }
+                    }
+                }
+                sh.fin_tok[i] = tok;
+                __threadfence();                            // the other rows' stores are visible before the reads
+                if (!epi_sync()) break;
+                const int64_t col = (int64_t)t.nt * 2 * kBM + (int64_t)rank * kBM + (i & (kBM - 1));
+                for (int j = i >> 7; j < t.rows; j += 2) {
+                    const int32_t tk = sh.fin_tok[j];
+                    if (tk >= 0)
+                        p.fin.out[(int64_t)tk * p.N + col] =
+                            (uint16_t)combine_element(p.out, p.N, p.fin.inv, p.fin.w, tk, p.fin.k, col);
+                }
+                if (!epi_sync()) break;                     // fin_tok is rewritten by the next tile
+            }
         }
         if (lane == 0) bulk_wait_group0();  // this warp's tensor stores completed
         __syncwarp();
@@ -719,8 +762,8 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
                                       const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const uint8_t* a_sf,
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
-                                      int swiglu, uint16_t* out, uint32_t* out_amax, cudaStream_t s,
-                                      uint32_t* status) {
+                                      int swiglu, uint16_t* out, uint32_t* out_amax, const Finalize& fin,
+                                      cudaStream_t s, uint32_t* status) {
     // once per device (thread-safe): the shared-memory opt-in and the persistent grid size
     static std::once_flag once[64];
     static int grid_for[64] = {};
@@ -767,6 +810,7 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     prm.K = K;
     prm.swiglu = swiglu;
     prm.amax_out = out_amax;
+    prm.fin = fin;
     prm.sched = sched_counter_slot();
     if (!prm.sched) return NVFP4_ERR_CUDA;
     prm.ctl.status = status;
