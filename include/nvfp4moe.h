@@ -252,6 +252,32 @@ NVFP4_API nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const uin
                                          uint32_t* out_amax, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* moe_grouped_gemm_nvfp4_quant: the gate/up GEMM (SWIGLU) with its output  */
+/* h quantised to NVFP4 in the epilogue, by a static (calibrated) global    */
+/* scale, in place of BF16 h -- the producer-side fusion that leaves no h   */
+/* in memory for the down GEMM's activations ("Peering into the CUTLASS     */
+/* Kernel Cache", Knowledge Required: the grouped GEMM of a                 */
+/* Mixture-of-Experts layer; the format of "Peering into the CUTLASS        */
+/* SharedStorage", Input Knowledge Required, item 3).                        */
+/*   q_h, sf_h = nvfp4_quantize(h, global_scale_in = h_gscale,              */
+/*               layout = NVFP4_SF_KSTAGE) bit for bit, where h [max_rows,  */
+/*               N/2] is what moe_grouped_gemm_nvfp4(..., SWIGLU) writes;   */
+/*   h_amax (nullable, zeroed by the caller) is raised to max |h| as BF16   */
+/*   bits -- the amax a dynamic scale would use, to calibrate the next call */
+/*   (g_dec = amax / 2688).                                                 */
+/* Arguments: as moe_grouped_gemm_nvfp4 with the SWIGLU epilogue, plus      */
+/*   h_gscale (device FP32 scalar, g_dec of h), q_h [max_rows, N/4] and     */
+/*   sf_h (ceil((N/2)/256) * max_rows * 16 bytes, K-stage slabs of max_rows */
+/*   rows), both device, 16-byte aligned. Rows outside every expert are not */
+/*   written.                                                                */
+/* ------------------------------------------------------------------------ */
+NVFP4_API nvfp4_status moe_grouped_gemm_nvfp4_quant(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
+                                          const uint8_t* w_packed, const float* w_gscale,
+                                          const int32_t* expert_offsets, int32_t E, int64_t max_rows,
+                                          int64_t N, int64_t K, const float* h_gscale, uint8_t* q_h,
+                                          uint8_t* sf_h, uint32_t* h_amax, nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* moe_grouped_gemm_nvfp4_finalize: the down GEMM with the top-k combine     */
 /* fused into its epilogue -- the FINALIZE epilogue that performs the final */
 /* MoE output write ("Peering into the CUTLASS Kernel", Input Knowledge     */

@@ -102,6 +102,8 @@ def lib():
         L.moe_layer_nvfp4_from_logits.restype = st
         L.moe_route_topk.argtypes = [P, i32, i32, i32, P, P, P]
         L.moe_route_topk.restype = st
+        L.moe_grouped_gemm_nvfp4_quant.argtypes = [P, P, P, P, P, P, i32, i64, i64, i64, P, P, P, P, P]
+        L.moe_grouped_gemm_nvfp4_quant.restype = st
         L.moe_finalize_counters_size.argtypes = [i32, i64]
         L.moe_finalize_counters_size.restype = sz
         L.moe_grouped_gemm_nvfp4_finalize.argtypes = [P, P, P, P, P, P, i32, i64, i64, i64, P, P, P, P, i32, i32, P,
@@ -393,6 +395,34 @@ def grouped_gemm(a_q, a_sf, a_g, w: PackedWeights, offsets, swiglu: bool, out=No
                                              _ptr(offsets), E, rows, N, K, EPI_SWIGLU if swiglu else EPI_NONE,
                                              _ptr(out), _ptr(amax_out), _stream(stream)), "moe_grouped_gemm_nvfp4_amax")
     return out
+
+
+def grouped_gemm_quant(a_q, a_sf, a_g, w: PackedWeights, offsets, h_gscale, q_h=None, sf_h=None, amax_out=None,
+                       stream=None):
+    """Gate/up GEMM (SwiGLU) whose epilogue writes h as NVFP4 with the static global scale h_gscale (device
+    float32 [1], g_dec): returns (q_h uint8 [rows, N/4], sf_h uint8 K-stage [ceil((N/2)/256), rows, 16]), the
+    bytes nvfp4_quantize(h, global_scale=h_gscale, layout=SF_KSTAGE) gives for the BF16 h grouped_gemm writes.
+    amax_out (device int32 [1], zeroed by the caller) is raised to max |h| as BF16 bits."""
+    _require_cuda(a_q, a_sf, a_g, w.packed, w.gscale, offsets, h_gscale, amax_out)
+    rows = a_q.shape[0]
+    N, K = w.N, w.K
+    E = offsets.numel() - 1
+    hc = N // 2
+    if a_sf.dim() != 3 or tuple(a_sf.shape) != (kstage_slabs(K), rows, 16):
+        raise ValueError(f"a_sf must be K-stage scales of shape {(kstage_slabs(K), rows, 16)}")
+    _need(a_q, rows * K // 2, "a_q")
+    _need(a_sf, sf_bytes(rows, K, SF_KSTAGE), "a_sf")
+    _need(h_gscale, 4, "h_gscale", torch.float32)
+    if amax_out is not None:
+        _need(amax_out, 4, "amax_out")
+    q_h = torch.empty((rows, hc // 2), dtype=torch.uint8, device=a_q.device) if q_h is None else \
+        _need(q_h, rows * hc // 2, "q_h")
+    sf_h = _sf_empty(rows, hc, SF_KSTAGE, a_q.device) if sf_h is None else _need(sf_h, sf_bytes(rows, hc, SF_KSTAGE),
+                                                                                  "sf_h")
+    _check(lib().moe_grouped_gemm_nvfp4_quant(_ptr(a_q), _ptr(a_sf), _ptr(a_g), _ptr(w.packed), _ptr(w.gscale),
+                                              _ptr(offsets), E, rows, N, K, _ptr(h_gscale), _ptr(q_h), _ptr(sf_h),
+                                              _ptr(amax_out), _stream(stream)), "moe_grouped_gemm_nvfp4_quant")
+    return q_h, sf_h
 
 
 def finalize_counters(T: int, N: int, device="cuda") -> torch.Tensor:

@@ -29,6 +29,15 @@ struct DeviceCtl {
     uint32_t flags;        // kCtl* test flags
 };
 
+// The gate/up GEMM's quantised h (moe_grouped_gemm_nvfp4_quant): the SwiGLU epilogue writes h as NVFP4
+// with a static global scale instead of BF16 h; off when q == nullptr.
+struct QuantOut {
+    const float* gdec;     // device scalar: the static global scale of h (dequantisation multiplier g_dec)
+    uint8_t* q;            // [rows, N/4] E2M1 codes of h [rows, N/2]
+    uint8_t* sf;           // h's block scales in the K-stage layout, rows_per_slab rows per slab
+    int64_t rows_per_slab;
+};
+
 // The grouped GEMM's fused top-k combine (moe_grouped_gemm_nvfp4_finalize); off when out == nullptr.
 struct Finalize {
     const int32_t* src;    // [rows] token of each activation row (moe_permute's perm_src)
@@ -57,7 +66,7 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
                                       int swiglu, uint16_t* out, uint32_t* out_amax, const Finalize& fin,
-                                      cudaStream_t s, uint32_t* status);
+                                      const QuantOut& qo, cudaStream_t s, uint32_t* status);
 
 #ifdef __CUDACC__
 // Launch `kernel` on `s` with programmatic stream serialization (see pdl_wait()).
@@ -352,6 +361,52 @@ __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_
 // without branches (fast exponential and division, a few fp32 ulp: far below the BF16 output's
 // resolution). For g below about -88 the exponential overflows and the result is -0 * u.
 __device__ __forceinline__ float swiglu_f32(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
+// FP32 -> E4M3, round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint32_t f32_to_e4m3_satfinite(float s) {
+    uint16_t pair;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(0.0f), "f"(s));
+    return pair & 0xFFu;
+}
+
+// Non-negative finite E4M3 byte -> FP32 (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+    if (e == 0) return (float)m * 0.001953125f;  // m * 2^-9, exact
+    return __uint_as_float(((e + 120u) << 23) | (m << 20));  // (1 + m/8) * 2^(e-7)
+}
+
+// FP32 -> E2M1 code (low 4 bits), round to nearest even, saturating to +-6, the sign kept on zero.
+__device__ __forceinline__ uint32_t f32_to_e2m1(float y) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tmov.b32 %0, {t, t, t, t};\n\t}"
+        : "=r"(w) : "f"(0.0f), "f"(y));
+    return w & 15u;
+}
+
+// Block quantisation step shared by every quantiser (nvfp4_quantize and the GEMM epilogue that writes
+// quantised h): the E4M3 scale of a 16-element block from its amax, and the FP32 factor that takes the
+// block's values onto the E2M1 grid (0 when the scale is 0: the block's codes are +0).
+__device__ __forceinline__ uint32_t block_scale(float amax_b, float g_enc, float& f) {
+    const float s = __fmul_rn(__fdiv_rn(amax_b, 6.0f), g_enc);
+    const uint32_t S = f32_to_e4m3_satfinite(s);
+    const float sfv = e4m3_to_f32(S);
+    f = sfv != 0.0f ? __fdiv_rn(g_enc, sfv) : 0.0f;
+    return S;
+}
+
+// One E2M1 code per lane of a half-warp whose 16 lanes hold one 16-element block of a row (BF16 bits
+// hb; valid = the lane's element exists): the block's scale byte (returned) and the lane's code, by the
+// quantiser's steps with the given g_enc. Every lane of the warp must call it.
+__device__ __forceinline__ uint32_t quantize_half_warp_block(uint32_t hb, bool valid, float g_enc, uint32_t& code) {
+    uint32_t a = valid ? (hb & 0x7FFFu) : 0u;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+    float f;
+    const uint32_t S = block_scale(__uint_as_float(a << 16), g_enc, f);
+    code = (S != 0u && valid) ? f32_to_e2m1(__fmul_rn(__uint_as_float(hb << 16), f)) : 0u;
+    return S;
+}
 
 // FP64 -> BF16, round to nearest even, in effect a single rounding: truncate to FP32, mark inexactness
 // in the last bit (round-to-odd), then round to BF16. (The combine's final rounding, shared by the

@@ -155,6 +155,7 @@ struct Params {
     uint32_t* sched;      // this launch's work counter [0] and finished-CTA counter [1]; zero at launch
     DeviceCtl ctl;
     Finalize fin;         // fused top-k combine (NONE epilogue), off when fin.out == nullptr
+    QuantOut qo;          // quantised h (SWIGLU epilogue), off when qo.q == nullptr
 };
 
 struct Tile {
@@ -503,6 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = quad * 32 + lane;         // accumulator row = weight row within a block
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const float a_g = __ldg(p.a_gscale);
+        const float h_genc = p.qo.q != nullptr ? __fdiv_rn(1.0f, __ldg(p.qo.gdec)) : 0.0f;   // static scale of h
         uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
         uint32_t abuf = 0, aphase = 0, qi = 0, qphase = 0, fphase = 0;
         // the 4 epilogue warps meet here (fused combine only); false when a wait ran out
@@ -530,7 +532,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_32x32b_x16(cbase + kAccCols + c * 16, v1);
                 tmem_ld_wait();
                 const int nrows = min(16, t.rows - c * 16);
-                if (p.swiglu) {
+                if (p.swiglu && p.qo.q != nullptr) {
+                    // h as NVFP4: lanes 16h..16h+15 of this warp hold one 16-column block of each token row
+                    const int64_t hcols = p.N / 2;
+                    const int64_t n = (int64_t)t.nt * kBM + r;               // this lane's column of h
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        const bool valid = i < nrows;
+                        const float g = alpha * v0[i], u = alpha * v1[i];
+                        const uint32_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(swiglu_f32(g, u)));
+                        if (valid) amax = max(amax, (uint32_t)(hb & 0x7FFFu));
+                        uint32_t code;
+                        const uint32_t S = quantize_half_warp_block(hb, valid, h_genc, code);
+                        const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, code, 1);
+                        const int64_t row = (int64_t)t.row0 + c * 16 + i;
+                        if (valid && (lane & 1) == 0) p.qo.q[row * (hcols / 2) + n / 2] = (uint8_t)(code | (hi << 4));
+                        if (valid && (lane & 15) == 0) {
+                            const int64_t b = n >> 4;
+                            uint8_t* piece = p.qo.sf + ((b >> 4) * p.qo.rows_per_slab + row) * 16;
+                            piece[b & 15] = (uint8_t)S;
+                            if ((hcols & 255) == 128 && b == (hcols >> 4) - 1)   // the last slab's padding
+                                *reinterpret_cast<uint2*>(piece + 8) = make_uint2(0u, 0u);
+                        }
+                    }
+                } else if (p.swiglu) {
                     const int64_t ldo = p.N / 2;
                     uint16_t* o = p.out + ((int64_t)t.row0 + c * 16) * ldo + (int64_t)t.nt * kBM + r;
 #pragma unroll
@@ -788,7 +813,9 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4(const uint8_t* a_q, const uint8_t
 static nvfp4_status grouped_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
                                  const uint8_t* w_packed, const float* w_gscale, const int32_t* expert_offsets,
                                  int32_t E, int64_t max_rows, int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
-                                 uint32_t* out_amax, const Finalize& fin, nvfp4_stream_t stream) {
+                                 uint32_t* out_amax, const Finalize& fin, const QuantOut& qo, nvfp4_stream_t stream) {
+    // quantised h replaces the BF16 output: `out` then only anchors the (unused) output tensor map
+    if (qo.q != nullptr) out = reinterpret_cast<uint16_t*>(qo.q);
     if (!a_q || !a_sf || !a_gscale || !w_packed || !w_gscale || !expert_offsets || !out)
         return NVFP4_ERR_INVALID_ARG;
     if ((uintptr_t)out_amax & 3u) return NVFP4_ERR_MISALIGNED;
@@ -821,6 +848,7 @@ static nvfp4_status grouped_gemm(const uint8_t* a_q, const uint8_t* a_sf, const 
     prm.swiglu = epi == NVFP4_EPI_SWIGLU ? 1 : 0;
     prm.amax_out = out_amax;
     prm.fin = fin;
+    prm.qo = qo;
     prm.sched = nullptr;   // drawn by the launcher that runs (one slot per launch)
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
@@ -832,13 +860,15 @@ static nvfp4_status grouped_gemm(const uint8_t* a_q, const uint8_t* a_sf, const 
         if (!encode_rows_map(&tm_a_full, a_q, max_rows, K / 2, (uint32_t)pair_gemm_tokens_max() / 2, 128))
             return NVFP4_ERR_CUDA;
         CUtensorMap tm_out;  // one epilogue warp's 32-token block of the output
-        const int64_t out_cols = prm.swiglu ? N / 2 : N;
+        // (with quantised h the map spans the codes buffer, [max_rows, N/4] bytes, and is never used)
+        const int64_t out_cols = qo.q != nullptr ? N / 8 : prm.swiglu ? N / 2 : N;
         if (!encode_out_map(&tm_out, out, max_rows, out_cols, (uint32_t)pair_gemm_store_cols(prm.swiglu)))
             return NVFP4_ERR_CUDA;
         CUtensorMap tm_wsw = tm_a;  // SWIGLU: interleaved gate/up weight slabs (unused otherwise)
         if (prm.swiglu && !encode_swiglu_weights_map(&tm_wsw, w_packed, E, N, K)) return NVFP4_ERR_CUDA;
         return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_out, tm_wsw, a_sf, a_gscale, w_packed, w_gscale,
-                                        expert_offsets, E, max_rows, N, K, prm.swiglu, out, out_amax, fin, s, status);
+                                        expert_offsets, E, max_rows, N, K, prm.swiglu, out, out_amax, fin, qo, s,
+                                        status);
     }
     const bool wide = max_rows >= kWideMinAvgRows * (int64_t)E;
     const nvfp4_status ls =
@@ -854,8 +884,26 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4_amax(const uint8_t* a_q, const ui
                                                     int64_t N, int64_t K, nvfp4_epilogue epi, uint16_t* out,
                                                     uint32_t* out_amax, nvfp4_stream_t stream) {
     const Finalize none = {};
+    const QuantOut bf16_out = {};
     return grouped_gemm(a_q, a_sf, a_gscale, w_packed, w_gscale, expert_offsets, E, max_rows, N, K, epi, out, out_amax,
-                        none, stream);
+                        none, bf16_out, stream);
+}
+
+extern "C" nvfp4_status moe_grouped_gemm_nvfp4_quant(const uint8_t* a_q, const uint8_t* a_sf, const float* a_gscale,
+                                                     const uint8_t* w_packed, const float* w_gscale,
+                                                     const int32_t* expert_offsets, int32_t E, int64_t max_rows,
+                                                     int64_t N, int64_t K, const float* h_gscale, uint8_t* q_h,
+                                                     uint8_t* sf_h, uint32_t* h_amax, nvfp4_stream_t stream) {
+    if (!h_gscale || !q_h || !sf_h) return NVFP4_ERR_INVALID_ARG;
+    if (((uintptr_t)h_gscale & 3u) || !aligned16(q_h) || !aligned16(sf_h)) return NVFP4_ERR_MISALIGNED;
+    QuantOut qo;
+    qo.gdec = h_gscale;
+    qo.q = q_h;
+    qo.sf = sf_h;
+    qo.rows_per_slab = max_rows;
+    const Finalize none = {};
+    return grouped_gemm(a_q, a_sf, a_gscale, w_packed, w_gscale, expert_offsets, E, max_rows, N, K, NVFP4_EPI_SWIGLU,
+                        nullptr, h_amax, none, qo, stream);
 }
 
 extern "C" size_t moe_finalize_counters_size(int32_t T, int64_t N) {
@@ -886,6 +934,7 @@ extern "C" nvfp4_status moe_grouped_gemm_nvfp4_finalize(const uint8_t* a_q, cons
     fin.T = T;
     fin.k = k;
     fin.col_blocks = (int32_t)((N + 127) / 128);
+    const QuantOut bf16_out = {};
     return grouped_gemm(a_q, a_sf, a_gscale, w_packed, w_gscale, expert_offsets, E, max_rows, N, K, NVFP4_EPI_NONE, y,
-                        nullptr, fin, stream);
+                        nullptr, fin, bf16_out, stream);
 }

@@ -117,6 +117,7 @@ struct Params {
     uint32_t* sched;      // this launch's work counter [0] and finished-CTA counter [1]; zero at launch
     DeviceCtl ctl;
     Finalize fin;         // fused top-k combine (NONE epilogue), off when fin.out == nullptr
+    QuantOut qo;          // quantised h (SWIGLU epilogue), off when qo.q == nullptr
 };
 
 struct Tile {
@@ -584,6 +585,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint16_t* stg = sh.ostage[half * 4 + quad];
         const bool up_lane = lane >= 16;
         const float a_g = __ldg(p.a_gscale);
+        const float h_genc = p.qo.q != nullptr ? __fdiv_rn(1.0f, __ldg(p.qo.gdec)) : 0.0f;   // static scale of h
         uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
         uint32_t aphase = 0, qi = 0, qphase = 0, fphase = 0;
         // this CTA's 8 epilogue warps meet here (fused combine only); false when a wait ran out
@@ -624,7 +626,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             const float g = alpha * (up_lane ? recv : v[2 * j]);
                             const float u = alpha * (up_lane ? v[2 * j + 1] : recv);
                             const uint32_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(swiglu_f32(g, u)));
-                            if (2 * j + (up_lane ? 1 : 0) < nrows) amax = max(amax, hb & 0x7FFFu);
+                            const bool valid = 2 * j + (up_lane ? 1 : 0) < nrows;
+                            if (valid) amax = max(amax, hb & 0x7FFFu);
+                            if (p.qo.q != nullptr) {
+                                // h as NVFP4: lanes 0-15 hold one 16-column block of token 2j, lanes 16-31
+                                // the same block of token 2j + 1
+                                uint32_t code;
+                                const uint32_t S = quantize_half_warp_block(hb, valid, h_genc, code);
+                                const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, code, 1);
+                                const int64_t hcols = p.N / 2;
+                                const int64_t n = (int64_t)t.nt * kBM + (int64_t)rank * 64 + quad * 16 + (lane & 15);
+                                const int64_t row = (int64_t)t.row0 + c * 32 + 2 * j + (up_lane ? 1 : 0);
+                                if (valid && (lane & 1) == 0)
+                                    p.qo.q[row * (hcols / 2) + n / 2] = (uint8_t)(code | (hi << 4));
+                                if (valid && (lane & 15) == 0) {
+                                    const int64_t b = n >> 4;
+                                    uint8_t* piece = p.qo.sf + ((b >> 4) * p.qo.rows_per_slab + row) * 16;
+                                    piece[b & 15] = (uint8_t)S;
+                                    if ((hcols & 255) == 128 && b == (hcols >> 4) - 1)   // the last slab's padding
+                                        *reinterpret_cast<uint2*>(piece + 8) = make_uint2(0u, 0u);
+                                }
+                            }
                             if (j & 1) pk[ci][j >> 1] |= hb << 16;
                             else pk[ci][j >> 1] = hb;
                         }
@@ -643,9 +665,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) arrive_on_leader(&sh.acc_empty, rank);
-            // 2. Write out: per chunk, stage a 32-token block in shared memory and store it
+            // 2. Write out: per chunk, stage a 32-token block in shared memory and store it (quantised h was
+            //    written in 1.)
 #pragma unroll
             for (int ci = 0; ci < kChunksPerWarp; ci++) {
+                if (p.qo.q != nullptr) break;
                 const int c = half + 2 * ci;
                 if (c * 32 < t.bn) {
                     const int nrows = min(32, t.rows - c * 32);
@@ -763,7 +787,7 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
                                       int swiglu, uint16_t* out, uint32_t* out_amax, const Finalize& fin,
-                                      cudaStream_t s, uint32_t* status) {
+                                      const QuantOut& qo, cudaStream_t s, uint32_t* status) {
     // once per device (thread-safe): the shared-memory opt-in and the persistent grid size
     static std::once_flag once[64];
     static int grid_for[64] = {};
@@ -811,6 +835,7 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     prm.swiglu = swiglu;
     prm.amax_out = out_amax;
     prm.fin = fin;
+    prm.qo = qo;
     prm.sched = sched_counter_slot();
     if (!prm.sched) return NVFP4_ERR_CUDA;
     prm.ctl.status = status;

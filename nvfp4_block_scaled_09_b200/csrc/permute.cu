@@ -132,6 +132,85 @@ __global__ void __launch_bounds__(kTok) permute_rank_kernel(const int32_t* __res
     }
 }
 
+// Small batches in one CTA (1024 threads) and one launch: count, scan and stable rank. Shared memory holds
+// one bit per (expert, token) and, per 32-token word, the number of the expert's pairs before that word
+// (the expert's offset included), so a pair's position is that prefix plus the popcount of the earlier
+// tokens in its word: token order inside each expert, as the multi-kernel path produces.
+__global__ void __launch_bounds__(kMaxE) permute_small_kernel(const int32_t* __restrict__ ids, int32_t T, int32_t k,
+                                                                int32_t E, int32_t* __restrict__ offsets,
+                                                                int32_t* __restrict__ perm_src,
+                                                                int32_t* __restrict__ inv_perm, uint32_t* status) {
+    pdl_launch_dependents();
+    pdl_wait();
+    extern __shared__ uint32_t small_sm[];
+    __shared__ int32_t warp_sums[kMaxE / 32];
+    const int W = (T + 31) / 32;                  // 32-token words per expert
+    uint32_t* bits = small_sm;                    // [E][W]
+    int32_t* pre = reinterpret_cast<int32_t*>(small_sm + (size_t)E * W);   // [E][W]
+    const int tid = threadIdx.x;
+    for (int i = tid; i < E * W; i += kMaxE) bits[i] = 0u;
+    __syncthreads();
+    const int64_t R = (int64_t)T * k;
+    bool bad = false;
+    for (int64_t i = tid; i < R; i += kMaxE) {
+        const int32_t t = (int32_t)(i / k);
+        const int32_t e = ids[i];
+        if (e >= 0 && e < E) {
+            const uint32_t bit = 1u << (t & 31);
+            if (atomicOr(&bits[e * W + (t >> 5)], bit) & bit) bad = true;   // expert listed twice by one token
+        } else {
+            bad = true;
+        }
+    }
+    if (bad) atomicOr(status, kStatusBadInput);
+    __syncthreads();
+    int32_t total = 0;
+    if (tid < E)
+        for (int w = 0; w < W; w++) total += __popc(bits[tid * W + w]);
+    // exclusive scan of the experts' totals
+    const int lane = tid & 31, warp = tid >> 5;
+    int32_t incl = total;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int32_t sacc = warp_sums[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t v = __shfl_up_sync(0xFFFFFFFFu, sacc, o);
+            if (lane >= o) sacc += v;
+        }
+        warp_sums[lane] = sacc;
+    }
+    __syncthreads();
+    if (tid < E) {
+        const int32_t excl = incl - total + (warp > 0 ? warp_sums[warp - 1] : 0);
+        offsets[tid] = excl;
+        if (tid == E - 1) offsets[E] = excl + total;
+        int32_t run = excl;
+        for (int w = 0; w < W; w++) {
+            pre[tid * W + w] = run;
+            run += __popc(bits[tid * W + w]);
+        }
+    }
+    __syncthreads();
+    for (int64_t i = tid; i < R; i += kMaxE) {
+        const int32_t t = (int32_t)(i / k);
+        const int32_t e = ids[i];
+        int32_t pos = -1;
+        if (e >= 0 && e < E) {
+            const int w = t >> 5;
+            pos = pre[e * W + w] + __popc(bits[e * W + w] & ((1u << (t & 31)) - 1u));
+            perm_src[pos] = t;
+        }
+        inv_perm[i] = pos;
+    }
+}
+
 // One warp per output row; rows whose source index is invalid become zeros.
 // kHalf: K % 256 == 128. A row-major scale row is then 8 bytes past a multiple of 16, so the scales
 // move in 8-byte units, and the last K-stage slab gets the row's last 8 scales plus 8 zero bytes.
@@ -183,6 +262,23 @@ using namespace nvfp4;
 
 static inline int32_t permute_chunks(int32_t T) { return (T + kTok - 1) / kTok; }
 
+// The one-CTA path takes up to this many pairs and this much shared memory (2 * E * ceil(T/32) words).
+constexpr int64_t kSmallMaxPairs = 32768;
+constexpr size_t kSmallMaxSmem = 160 * 1024;
+
+// Opt the one-CTA kernel into the shared memory it may need, once per device.
+static bool small_kernel_ready() {
+    static std::once_flag once[64];
+    static bool ok[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::call_once(once[dev], [&] {
+        ok[dev] = cudaFuncSetAttribute(permute_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmallMaxSmem) == cudaSuccess;
+    });
+    return ok[dev];
+}
+
 static void launch_gather(const uint8_t* q, const uint8_t* sf, int64_t K, const int32_t* perm_src, int32_t T,
                           int64_t R, uint8_t* q_perm, uint8_t* sf_perm, nvfp4_sf_layout layout, cudaStream_t s) {
     const bool kstage = layout == NVFP4_SF_KSTAGE, half = K % 256 != 0;
@@ -222,6 +318,15 @@ extern "C" nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t 
     int32_t* counts = static_cast<int32_t*>(ws);
     const int64_t R = (int64_t)T * k;
 
+    // small batches (decode): one CTA ranks every pair, then the gather -- two launches
+    const size_t small_smem = 2 * (size_t)E * (size_t)((T + 31) / 32) * sizeof(uint32_t);
+    if (R <= kSmallMaxPairs && small_smem <= kSmallMaxSmem && small_kernel_ready()) {
+        launch_pdl(permute_small_kernel, dim3(1), dim3(kMaxE), small_smem, s, topk_ids, T, k, E, expert_offsets,
+                   perm_src, inv_perm, status);
+        launch_gather(q, sf, K, perm_src, T, R, q_perm, sf_perm, sf_perm_layout, s);
+        count_launch(2);
+        return check_launch();
+    }
     launch_pdl(permute_count_kernel, dim3(nchunks), dim3(kTok), 0, s, topk_ids, T, k, E, counts, status);
     launch_pdl(permute_scan_kernel, dim3(1), dim3(kMaxE), 0, s, counts, nchunks, E, expert_offsets);
     const size_t rank_smem = (size_t)E * kWordsPerExpert * sizeof(uint32_t);

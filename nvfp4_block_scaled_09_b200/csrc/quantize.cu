@@ -64,20 +64,6 @@ __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const uint4* __r
     }
 }
 
-// FP32 -> E4M3, round to nearest even, saturating to +-448.
-__device__ __forceinline__ uint32_t f32_to_e4m3_satfinite(float s) {
-    uint16_t pair;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(0.0f), "f"(s));
-    return pair & 0xFFu;
-}
-
-// Non-negative finite E4M3 byte -> FP32 (exact).
-__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
-    const uint32_t e = (b >> 3) & 15u, m = b & 7u;
-    if (e == 0) return (float)m * 0.001953125f;  // m * 2^-9, exact
-    return __uint_as_float(((e + 120u) << 23) | (m << 20));  // (1 + m/8) * 2^(e-7)
-}
-
 // Four FP32 values -> four E2M1 pairs packed little-endian: value 2i in the low nibble of byte i.
 __device__ __forceinline__ uint32_t f32x8_to_e2m1x8(const float (&y)[8]) {
     uint32_t out;
@@ -148,12 +134,10 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
 #pragma unroll
         for (int i = 0; i < 8; i++) m = absmax_pair(m, w[i]);
         const float amax_b = bf16_bits_to_f32(fold_pair(m));
-        const float s = __fmul_rn(__fdiv_rn(amax_b, 6.0f), g_enc);
-        const uint32_t S = f32_to_e4m3_satfinite(s);
-        const float sfv = e4m3_to_f32(S);
+        float f;
+        const uint32_t S = block_scale(amax_b, g_enc, f);
         uint2 packed = make_uint2(0u, 0u);
-        if (sfv != 0.0f) {
-            const float f = __fdiv_rn(g_enc, sfv);
+        if (S != 0u) {
             float y[8];
 #pragma unroll
             for (int i = 0; i < 4; i++) {

@@ -46,8 +46,10 @@ def test_workload_routing(name):
 
 
 @pytest.mark.parametrize("T,E,k,kind", [(1, 4, 1, "uniform"), (37, 5, 3, "uniform"), (300, 1024, 8, "zipf"),
-                                        (257, 64, 16, "uniform"), (513, 3, 2, "zipf")])
+                                        (257, 64, 16, "uniform"), (513, 3, 2, "zipf"),
+                                        (5000, 1024, 8, "zipf")])   # > 32768 pairs: the multi-kernel path
 def test_ragged_shapes(T, E, k, kind):
+    # up to 32768 pairs (and 160 KB of rank tables) one CTA ranks every pair; beyond, four kernels do
     ids, _ = workloads.routing(T, E, k, kind, seed=T)
     run(ids, E, 256, seed=T)
 
