@@ -73,3 +73,11 @@ def test_reference_arm_under_torchrun_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    # the reference arm describes the workload with the GPU arm's config object (same keys and values)
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    want = bench.moe_config_dict("moe_decode_t512", workloads.CONFIGS["moe_decode_t512"],
+                                 bench.moe_counts(workloads.CONFIGS["moe_decode_t512"],
+                                                  workloads.config_routing("moe_decode_t512")[0]), 2)
+    assert d["config"] == json.loads(json.dumps(want))
