@@ -29,6 +29,12 @@ struct DeviceCtl {
     uint32_t flags;        // kCtl* test flags
 };
 
+// Epilogue modes of the grouped GEMM kernels (template argument): each instantiation carries only its own
+// epilogue code.
+constexpr int kEpiPlain = 0;      // BF16 output (NONE or SWIGLU)
+constexpr int kEpiFinalize = 1;   // NONE + the fused top-k combine
+constexpr int kEpiQuant = 2;      // SWIGLU with h written as NVFP4
+
 // The gate/up GEMM's quantised h (moe_grouped_gemm_nvfp4_quant): the SwiGLU epilogue writes h as NVFP4
 // with a static global scale instead of BF16 h; off when q == nullptr.
 struct QuantOut {
@@ -417,20 +423,45 @@ __device__ __forceinline__ uint32_t f64_to_bf16_bits(double d) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
-// One output element of the top-k weighted combine: sum over the token's slots j ascending of
-// w[t, j] * y[inv_perm[t*k + j], col] in FP64 (each product of an FP32 weight and a BF16 value is exact),
-// negative rows skipped; y is read past L1 (other SMs wrote it). Returns the BF16 bits.
-__device__ __forceinline__ uint32_t combine_element(const uint16_t* y, int64_t ldy, const int32_t* inv_perm,
-                                                    const float* w, int32_t t, int32_t k, int64_t col) {
-    double acc = 0.0;
-    for (int32_t j = 0; j < k; j++) {
-        const int32_t p = __ldg(inv_perm + (int64_t)t * k + j);
-        if (p < 0) continue;
-        const double s = (double)__ldg(w + (int64_t)t * k + j);
-        const uint32_t b = __ldcg(reinterpret_cast<const unsigned short*>(y + (int64_t)p * ldy + col));
-        acc = fma(s, (double)__uint_as_float(b << 16), acc);
+// Eight adjacent output columns [col, col + 8) of the top-k weighted combine for token t: the sum over the
+// token's slots j ascending of w[t, j] * y[inv_perm[t*k + j], col..] in FP64 (each product of an FP32 weight and
+// a BF16 value is exact), negative rows skipped, rounded once to BF16 and stored as one 16-byte piece. The
+// slots are read in groups of four so their loads overlap; y is read past L1 (other SMs wrote it).
+__device__ __forceinline__ void combine_vec8(const uint16_t* y, int64_t ldy, const int32_t* inv_perm, const float* w,
+                                             int32_t t, int32_t k, int64_t col, uint16_t* out, int64_t ldo) {
+    double a[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) a[i] = 0.0;
+    for (int32_t j0 = 0; j0 < k; j0 += 4) {
+        int32_t p[4];
+        float s[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            p[u] = j0 + u < k ? __ldg(inv_perm + (int64_t)t * k + j0 + u) : -1;
+            s[u] = j0 + u < k ? __ldg(w + (int64_t)t * k + j0 + u) : 0.0f;
+        }
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++)
+            v[u] = p[u] >= 0 ? __ldcg(reinterpret_cast<const uint4*>(y + (int64_t)p[u] * ldy + col)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            if (p[u] < 0) continue;
+            const double sd = (double)s[u];
+            const uint32_t x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                a[2 * i] = fma(sd, (double)__uint_as_float(x[i] << 16), a[2 * i]);
+                a[2 * i + 1] = fma(sd, (double)__uint_as_float(x[i] & 0xFFFF0000u), a[2 * i + 1]);
+            }
+        }
     }
-    return f64_to_bf16_bits(acc);
+    uint4 o;
+    o.x = f64_to_bf16_bits(a[0]) | (f64_to_bf16_bits(a[1]) << 16);
+    o.y = f64_to_bf16_bits(a[2]) | (f64_to_bf16_bits(a[3]) << 16);
+    o.z = f64_to_bf16_bits(a[4]) | (f64_to_bf16_bits(a[5]) << 16);
+    o.w = f64_to_bf16_bits(a[6]) | (f64_to_bf16_bits(a[7]) << 16);
+    *reinterpret_cast<uint4*>(out + (int64_t)t * ldo + col) = o;
 }
 
 // ---- thread-block clusters and CTA pairs (cta_group::2) ---------------------

@@ -209,7 +209,7 @@ __device__ __forceinline__ bool next_tile(Shared& sh, uint32_t& qi, uint32_t& qp
     return true;
 }
 
-template <class C>
+template <class C, int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const Params p) {
     constexpr int kBNMax = C::kBNMax;
@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = quad * 32 + lane;         // accumulator row = weight row within a block
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const float a_g = __ldg(p.a_gscale);
-        const float h_genc = p.qo.q != nullptr ? __fdiv_rn(1.0f, __ldg(p.qo.gdec)) : 0.0f;   // static scale of h
+        const float h_genc = kEpi == kEpiQuant ? __fdiv_rn(1.0f, __ldg(p.qo.gdec)) : 0.0f;   // static scale of h
         uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
         uint32_t abuf = 0, aphase = 0, qi = 0, qphase = 0, fphase = 0;
         // the 4 epilogue warps meet here (fused combine only); false when a wait ran out
@@ -532,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_32x32b_x16(cbase + kAccCols + c * 16, v1);
                 tmem_ld_wait();
                 const int nrows = min(16, t.rows - c * 16);
-                if (p.swiglu && p.qo.q != nullptr) {
+                if (p.swiglu && kEpi == kEpiQuant) {
                     // h as NVFP4: lanes 16h..16h+15 of this warp hold one 16-column block of each token row
                     const int64_t hcols = p.N / 2;
                     const int64_t n = (int64_t)t.nt * kBM + r;               // this lane's column of h
@@ -590,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.acc_empty[abuf]);
             if (++abuf == (uint32_t)C::kAccBufs) { abuf = 0; aphase ^= 1u; }
-            if (p.fin.out != nullptr) {
+            if (kEpi == kEpiFinalize) {
                 // Fused combine. Every row of this tile holds one (token, slot) product for the tile's output
                 // columns; count the rows in per (token, column tile). The CTA that brings a token's count
                 // to k writes that token's combined output for these columns, whichever CTA wrote the other
@@ -612,15 +612,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 sh.fin_tok[i] = tok;
                 __threadfence();                            // the other rows' stores are visible before the reads
                 if (!epi_sync()) break;
-                const int64_t col = (int64_t)t.nt * (kNumA * kBM) + r;
-                for (int j = 0; j < t.rows; j++) {
+                // one warp per token: lane l combines columns [8l, 8l + 8) of the tile's 256 (128 for a half tile)
+                const int64_t col = (int64_t)t.nt * (kNumA * kBM) + lane * 8;
+                const bool lane_on = second || lane * 8 < kBM;
+                for (int j = warp - 4; j < t.rows; j += 4) {
                     const int32_t tk = sh.fin_tok[j];
-                    if (tk < 0) continue;
-                    p.fin.out[(int64_t)tk * p.N + col] =
-                        (uint16_t)combine_element(p.out, p.N, p.fin.inv, p.fin.w, tk, p.fin.k, col);
-                    if (second)
-                        p.fin.out[(int64_t)tk * p.N + col + kBM] =
-                            (uint16_t)combine_element(p.out, p.N, p.fin.inv, p.fin.w, tk, p.fin.k, col + kBM);
+                    if (tk >= 0 && lane_on) combine_vec8(p.out, p.N, p.fin.inv, p.fin.w, tk, p.fin.k, col, p.fin.out, p.N);
                 }
                 if (!epi_sync()) break;                     // fin_tok is rewritten by the next tile
             }
@@ -782,7 +779,7 @@ extern "C" nvfp4_status nvfp4_can_implement(int64_t N, int64_t K, int32_t E, nvf
     return nvfp4_can_implement_with_budget(N, K, E, epi, optin);
 }
 
-template <class C>
+template <class C, int kEpi>
 static nvfp4_status launch_variant(const CUtensorMap& tm_a, gg::Params prm, cudaStream_t s) {
     // the kernel's shared-memory opt-in, once per device (thread-safe)
     static std::once_flag once[64];
@@ -790,13 +787,14 @@ static nvfp4_status launch_variant(const CUtensorMap& tm_a, gg::Params prm, cuda
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
     std::call_once(once[dev], [&] {
-        set_result[dev] = cudaFuncSetAttribute(gg::grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        set_result[dev] = cudaFuncSetAttribute(gg::grouped_gemm_kernel<C, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)C::kSmemBytes);
     });
     if (set_result[dev] != cudaSuccess) return NVFP4_ERR_CUDA;
     prm.sched = sched_counter_slot();
     if (!prm.sched) return NVFP4_ERR_CUDA;
-    launch_pdl(gg::grouped_gemm_kernel<C>, dim3(device_sm_count()), dim3(gg::kThreads), C::kSmemBytes, s, tm_a, prm);
+    launch_pdl(gg::grouped_gemm_kernel<C, kEpi>, dim3(device_sm_count()), dim3(gg::kThreads), C::kSmemBytes, s, tm_a,
+               prm);
     return NVFP4_OK;
 }
 
@@ -871,8 +869,14 @@ static nvfp4_status grouped_gemm(const uint8_t* a_q, const uint8_t* a_sf, const 
                                         status);
     }
     const bool wide = max_rows >= kWideMinAvgRows * (int64_t)E;
-    const nvfp4_status ls =
-        wide ? launch_variant<gg::Wide>(tm_a, prm, s) : launch_variant<gg::Narrow>(tm_a, prm, s);
+    nvfp4_status ls;
+    if (qo.q != nullptr)
+        ls = wide ? launch_variant<gg::Wide, kEpiQuant>(tm_a, prm, s) : launch_variant<gg::Narrow, kEpiQuant>(tm_a, prm, s);
+    else if (fin.out != nullptr)
+        ls = wide ? launch_variant<gg::Wide, kEpiFinalize>(tm_a, prm, s)
+                  : launch_variant<gg::Narrow, kEpiFinalize>(tm_a, prm, s);
+    else
+        ls = wide ? launch_variant<gg::Wide, kEpiPlain>(tm_a, prm, s) : launch_variant<gg::Narrow, kEpiPlain>(tm_a, prm, s);
     if (ls != NVFP4_OK) return ls;
     count_launch();
     return check_launch();

@@ -37,6 +37,9 @@
 #ifndef NVFP4_PAIR_PREFETCH
 #define NVFP4_PAIR_PREFETCH 0
 #endif
+#ifndef NVFP4_PAIR_OLD_ORDER
+#define NVFP4_PAIR_OLD_ORDER 0
+#endif
 
 namespace nvfp4 {
 namespace gp {
@@ -265,6 +268,7 @@ __device__ __forceinline__ void build_schedule(Shared& sh, const Params& p, int3
 namespace nvfp4 {
 namespace gp {
 
+template <int kEpi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_full,
                              const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_wsw,
@@ -398,6 +402,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         mbar_arrive_expect_tx(bar, sf_tx + op_tx);
                     }
                     const size_t ko = (size_t)kt * kPackedTileBytes;
+#if NVFP4_PAIR_OLD_ORDER
+                    if (!kSplitSF) {
+                        // codes, then scales (issue order of the first CTA-pair kernel)
+                        if (p.swiglu) {
+                            tma_load_5d(sb + kOffA, &tm_wsw, 0, 0, 0, (int32_t)(half / 16), sw_tile0 + kt, bar, pol_w);
+                            bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
+                            bulk_load(sb + kOffSFA + kTileSFBytes, u_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
+                        } else {
+                            bulk_load(sb + kOffA, g_tile + ko, kPackedTileBytes, bar, pol_w);
+                        }
+                        if (my_rows == kBNMax / 2) {
+                            tma_load_2d(sb + kOffB, &tm_a_full, kt * kRowBytes, my_row0, bar, pol_a);
+                        } else {
+                            for (int32_t i = 0; i < my_rows / kBoxRows; i++)
+                                tma_load_2d(sb + kOffB + i * kBoxRows * kRowBytes, &tm_a, kt * kRowBytes,
+                                            my_row0 + i * kBoxRows, bar, pol_a);
+                        }
+                        bulk_load(sb + kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, bar, pol_a);
+                        issued[stage] = true;
+                        issued_parity[stage] = phase;
+                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                        continue;
+                    }
+#endif
                     // scales first: they are small and their consumers (the scale writers) run ahead of the MMAs
                     if (p.swiglu) {
                         bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, sbar, pol_w);
@@ -585,7 +613,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint16_t* stg = sh.ostage[half * 4 + quad];
         const bool up_lane = lane >= 16;
         const float a_g = __ldg(p.a_gscale);
-        const float h_genc = p.qo.q != nullptr ? __fdiv_rn(1.0f, __ldg(p.qo.gdec)) : 0.0f;   // static scale of h
+        const float h_genc = kEpi == kEpiQuant ? __fdiv_rn(1.0f, __ldg(p.qo.gdec)) : 0.0f;   // static scale of h
         uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
         uint32_t aphase = 0, qi = 0, qphase = 0, fphase = 0;
         // this CTA's 8 epilogue warps meet here (fused combine only); false when a wait ran out
@@ -628,7 +656,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             const uint32_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(swiglu_f32(g, u)));
                             const bool valid = 2 * j + (up_lane ? 1 : 0) < nrows;
                             if (valid) amax = max(amax, hb & 0x7FFFu);
-                            if (p.qo.q != nullptr) {
+                            if (kEpi == kEpiQuant) {
                                 // h as NVFP4: lanes 0-15 hold one 16-column block of token 2j, lanes 16-31
                                 // the same block of token 2j + 1
                                 uint32_t code;
@@ -669,7 +697,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             //    written in 1.)
 #pragma unroll
             for (int ci = 0; ci < kChunksPerWarp; ci++) {
-                if (p.qo.q != nullptr) break;
+                if (kEpi == kEpiQuant) break;
                 const int c = half + 2 * ci;
                 if (c * 32 < t.bn) {
                     const int nrows = min(32, t.rows - c * 32);
@@ -693,7 +721,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         col = t.nt * 2 * kBM + (int32_t)rank * kBM + quad * 32;
                         lane_cols = 4;
                     }
-                    if (nrows == 32 && p.fin.out == nullptr) {
+                    if (nrows == 32 && kEpi != kEpiFinalize) {
                         // a whole chunk of the expert: one asynchronous tensor store of the block
                         // (the fused combine stores directly: its last arrivers read these rows back)
                         fence_proxy_async_smem();
@@ -718,7 +746,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             aphase ^= 1u;
-            if (p.fin.out != nullptr) {
+            if (kEpi == kEpiFinalize) {
                 // Fused combine over this CTA's 128 output columns: count the tile's rows in per (token,
                 // 128-column block); the CTA that brings a count to k writes that token's combined output
                 // for these columns (see the one-SM kernel: the result does not depend on the order).
@@ -739,12 +767,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 sh.fin_tok[i] = tok;
                 __threadfence();                            // the other rows' stores are visible before the reads
                 if (!epi_sync()) break;
-                const int64_t col = (int64_t)t.nt * 2 * kBM + (int64_t)rank * kBM + (i & (kBM - 1));
-                for (int j = i >> 7; j < t.rows; j += 2) {
+                // one half-warp per token: lane l combines columns [8 (l % 16), +8) of this CTA's 128
+                const int64_t col = (int64_t)t.nt * 2 * kBM + (int64_t)rank * kBM + (lane & 15) * 8;
+                for (int j = 2 * (half * 4 + quad) + (lane >> 4); j < t.rows; j += 2 * kEpiWarps) {
                     const int32_t tk = sh.fin_tok[j];
-                    if (tk >= 0)
-                        p.fin.out[(int64_t)tk * p.N + col] =
-                            (uint16_t)combine_element(p.out, p.N, p.fin.inv, p.fin.w, tk, p.fin.k, col);
+                    if (tk >= 0) combine_vec8(p.out, p.N, p.fin.inv, p.fin.w, tk, p.fin.k, col, p.fin.out, p.N);
                 }
                 if (!epi_sync()) break;                     // fin_tok is rewritten by the next tile
             }
@@ -781,6 +808,18 @@ size_t pair_gemm_smem_bytes() { return gp::kSmemBytes; }
 int pair_gemm_tokens_max() { return gp::kBNMax; }
 int pair_gemm_store_cols(int swiglu) { return swiglu ? 16 : 32; }  // 32 tokens x this many BF16 columns
 
+// The shared-memory opt-in of one instantiation, once per device (thread-safe).
+template <int kEpi>
+static bool pair_kernel_configured(int dev) {
+    static std::once_flag once[64];
+    static bool ok[64] = {};
+    std::call_once(once[dev], [&] {
+        ok[dev] = cudaFuncSetAttribute(gp::grouped_gemm_pair_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)gp::kSmemBytes) == cudaSuccess;
+    });
+    return ok[dev];
+}
+
 // Launches the pair kernel; the caller validated every argument (same contract as the one-SM kernel).
 nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full,
                                       const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const uint8_t* a_sf,
@@ -796,9 +835,7 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
     std::call_once(once[dev], [&] {
         set_result[dev] = NVFP4_ERR_CUDA;
-        if (cudaFuncSetAttribute(gp::grouped_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gp::kSmemBytes) != cudaSuccess)
-            return;
+        if (!pair_kernel_configured<kEpiPlain>(dev)) return;
         // as many pairs as can be resident at once (persistent grid)
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)device_sm_count() / 2 * 2);
@@ -812,7 +849,7 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, gp::grouped_gemm_pair_kernel, &cfg) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveClusters(&clusters, gp::grouped_gemm_pair_kernel<kEpiPlain>, &cfg) != cudaSuccess ||
             clusters <= 0) {
             set_result[dev] = NVFP4_ERR_SMEM_BUDGET;
             return;
@@ -841,8 +878,19 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
-    launch_pdl(gp::grouped_gemm_pair_kernel, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes, s, tm_a, tm_a_full,
-               tm_out, tm_wsw, prm);
+    // every instantiation has the plain one's resources (same shared memory, threads and cluster shape)
+    if (qo.q != nullptr) {
+        if (!pair_kernel_configured<kEpiQuant>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiQuant>, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes, s,
+                   tm_a, tm_a_full, tm_out, tm_wsw, prm);
+    } else if (fin.out != nullptr) {
+        if (!pair_kernel_configured<kEpiFinalize>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiFinalize>, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes,
+                   s, tm_a, tm_a_full, tm_out, tm_wsw, prm);
+    } else {
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain>, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes, s,
+                   tm_a, tm_a_full, tm_out, tm_wsw, prm);
+    }
     count_launch();
     return check_launch();
 }

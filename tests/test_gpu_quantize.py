@@ -98,10 +98,13 @@ def test_rejects_bad_arguments():
     with pytest.raises(nv.NVFP4Error) as e:
         nv.quantize(x, layout=nv.SF_MMA_TILED)
     assert e.value.status == 3
-    x = torch.zeros((4, 128), dtype=torch.bfloat16, device="cuda")   # K-stage slabs need K % 256 == 0
+    x = torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda")    # K-stage slabs need K % 128 == 0
     with pytest.raises(nv.NVFP4Error) as e:
-        nv.quantize(x, layout=nv.SF_KSTAGE, sf=torch.empty((4, 8), dtype=torch.uint8, device="cuda"))
+        nv.quantize(x, layout=nv.SF_KSTAGE)
     assert e.value.status == 3
+    x = torch.zeros((4, 128), dtype=torch.bfloat16, device="cuda")   # one padded slab: 4 rows x 16 bytes
+    with pytest.raises(ValueError):
+        nv.quantize(x, layout=nv.SF_KSTAGE, sf=torch.empty((4, 8), dtype=torch.uint8, device="cuda"))
 
 
 @pytest.mark.parametrize("rows,K,std,seed", [(1, 16, 1.0, 10), (96, 2048, 0.5, 11), (300, 512, 3.0, 12)])
