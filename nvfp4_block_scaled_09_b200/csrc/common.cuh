@@ -68,7 +68,8 @@ size_t pair_gemm_smem_bytes();
 int pair_gemm_tokens_max();
 int pair_gemm_store_cols(int swiglu);   // output columns of one epilogue warp's tensor-store box
 nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full,
-                                      const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const uint8_t* a_sf,
+                                      const CUtensorMap& tm_out, const CUtensorMap& tm_wsw,
+                                      const CUtensorMap& tm_wsf, const uint8_t* a_sf,
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
                                       int swiglu, uint16_t* out, uint32_t* out_amax, const Finalize& fin,
@@ -211,13 +212,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
             smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
-}
-
-// Hint: bring `bytes` (16-byte aligned start, size % 16 == 0) of global memory into L2 ahead of a
-// later copy; nothing waits for it.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes, uint64_t policy) {
-    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(src), "r"(bytes), "l"(policy)
-                 : "memory");
 }
 
 // TMA: 2-D tiled tensor store shared -> global (box at coordinates {c0, c1}, both >= 0), tracked

@@ -414,19 +414,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) {
                     const uint32_t sb = smem_u32(stages + (size_t)stage * kStageBytes);
                     const uint32_t sf = tmem + kTmemSFRing + stage * kTmemSFSlot;
-                    const int n_kc = kt == ksteps_total - 1 ? last_ksteps : kKSteps;
-#pragma unroll
-                    for (int kc = 0; kc < kKSteps; kc++) {
-                        if (kc >= n_kc) break;
+                    auto mma_step = [&](int kc, int a) {
                         const uint64_t bdesc = make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2);
-                        const uint32_t acc = (kt | kc) != 0;
+                        const uint64_t adesc = make_smem_desc(sb + a * kPackedTileBytes + kc * 32, 16, 1024, 2);
+                        mma_mxf4nvf4(tmem + abuf * (kNumA * kAccCols) + a * kAccCols, adesc, bdesc, idesc,
+                                     sf + a * 4 * kKSteps + 4 * kc, sf + kNumA * 4 * kKSteps + 4 * kc, (kt | kc) != 0);
+                    };
+                    if (n_a == kNumA && (kt != ksteps_total - 1 || last_ksteps == kKSteps)) {
 #pragma unroll
-                        for (int a = 0; a < kNumA; a++) {
-                            if (a >= n_a) break;
-                            const uint64_t adesc = make_smem_desc(sb + a * kPackedTileBytes + kc * 32, 16, 1024, 2);
-                            mma_mxf4nvf4(tmem + abuf * (kNumA * kAccCols) + a * kAccCols, adesc, bdesc, idesc,
-                                         sf + a * 4 * kKSteps + 4 * kc, sf + kNumA * 4 * kKSteps + 4 * kc, acc);
-                        }
+                        for (int kc = 0; kc < kKSteps; kc++)
+#pragma unroll
+                            for (int a = 0; a < kNumA; a++) mma_step(kc, a);
+                    } else {
+                        // a half column tile (one weight block) and/or a last stage of 128 K-elements
+                        const int n_kc = kt == ksteps_total - 1 ? last_ksteps : kKSteps;
+                        for (int kc = 0; kc < n_kc; kc++)
+                            for (int a = 0; a < n_a; a++) mma_step(kc, a);
                     }
                     tc_commit(&sh.empty[stage]);
                 }
@@ -701,16 +704,19 @@ static bool encode_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t col
 // packed tile, packed tile index}. A box {128, 16, 2, 4, 1} gathers one CTA's 64 gate rows and the
 // matching 64 up rows, interleaved 16 at a time. Tiles run only over gate tiles plus the ones whose
 // up tile still lies inside the tensor, so no box can leave the allocation.
-static bool encode_swiglu_weights_map(CUtensorMap* m, const void* w_packed, int32_t E, int64_t N, int64_t K) {
+// The same view with a ninth slab (the tile's 2 KB of scales, right after its 16 KB of codes) and a
+// box of one slab: {128, 16, 2, 1, 1} at slab 8 brings the gate and the up tile's scales in one load.
+static bool encode_swiglu_weights_map(CUtensorMap* m, const void* w_packed, int32_t E, int64_t N, int64_t K,
+                                      uint32_t box_slabs) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
     const int64_t ksteps = (K + 255) / 256;
     const int64_t tile_bytes = 18432;
     const int64_t up_stride = (N / 2 / 128) * ksteps * tile_bytes;
     const int64_t tiles = ((int64_t)E * N - N / 2) / 128 * ksteps;
-    cuuint64_t dims[5] = {128u, 16u, 2u, 8u, (cuuint64_t)tiles};
+    cuuint64_t dims[5] = {128u, 16u, 2u, 9u, (cuuint64_t)tiles};
     cuuint64_t strides[4] = {128u, (cuuint64_t)up_stride, 2048u, (cuuint64_t)tile_bytes};
-    cuuint32_t box[5] = {128u, 16u, 2u, 4u, 1u};
+    cuuint32_t box[5] = {128u, 16u, 2u, box_slabs, 1u};
     cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(w_packed), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -863,8 +869,11 @@ static nvfp4_status grouped_gemm(const uint8_t* a_q, const uint8_t* a_sf, const 
         if (!encode_out_map(&tm_out, out, max_rows, out_cols, (uint32_t)pair_gemm_store_cols(prm.swiglu)))
             return NVFP4_ERR_CUDA;
         CUtensorMap tm_wsw = tm_a;  // SWIGLU: interleaved gate/up weight slabs (unused otherwise)
-        if (prm.swiglu && !encode_swiglu_weights_map(&tm_wsw, w_packed, E, N, K)) return NVFP4_ERR_CUDA;
-        return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_out, tm_wsw, a_sf, a_gscale, w_packed, w_gscale,
+        CUtensorMap tm_wsf = tm_a;  // SWIGLU: the gate and up tiles' scales (unused otherwise)
+        if (prm.swiglu && (!encode_swiglu_weights_map(&tm_wsw, w_packed, E, N, K, 4) ||
+                           !encode_swiglu_weights_map(&tm_wsf, w_packed, E, N, K, 1)))
+            return NVFP4_ERR_CUDA;
+        return launch_grouped_gemm_pair(tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, a_sf, a_gscale, w_packed, w_gscale,
                                         expert_offsets, E, max_rows, N, K, prm.swiglu, out, out_amax, fin, qo, s,
                                         status);
     }

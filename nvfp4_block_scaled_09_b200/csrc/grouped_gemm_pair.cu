@@ -31,21 +31,17 @@
 
 #include "common.cuh"
 
-#ifndef NVFP4_PAIR_SPLIT_SF
-#define NVFP4_PAIR_SPLIT_SF 0
+#ifndef NVFP4_PAIR_SKIP_FULL_WAIT
+#define NVFP4_PAIR_SKIP_FULL_WAIT 0
 #endif
-#ifndef NVFP4_PAIR_PREFETCH
-#define NVFP4_PAIR_PREFETCH 0
-#endif
-#ifndef NVFP4_PAIR_OLD_ORDER
-#define NVFP4_PAIR_OLD_ORDER 0
+#ifndef NVFP4_PAIR_SFA_BOX
+#define NVFP4_PAIR_SFA_BOX 0
 #endif
 
 namespace nvfp4 {
 namespace gp {
 
-constexpr bool kSplitSF = NVFP4_PAIR_SPLIT_SF != 0;     // scales on their own barrier, ahead of the operands
-constexpr int kPrefetchAhead = NVFP4_PAIR_PREFETCH;     // weight stages brought into L2 ahead (0: none)
+constexpr bool kSkipFullWait = NVFP4_PAIR_SKIP_FULL_WAIT != 0;   // the MMA warp waits on sf_ready alone
 
 constexpr int kBM = 128;                          // weight rows per CTA (MMA M = 256 per pair)
 constexpr int kBK = 256;                          // K elements per stage
@@ -77,16 +73,14 @@ static_assert(kStageBytes % 1024 == 0 && kOffB % 1024 == 0, "swizzled tiles need
 constexpr int kTileRing = 4;                      // work items the even CTA may publish ahead
 constexpr int kTileConsumersPerCta = 13;          // even CTA: MMA warp + 4 scale writers + 8 epilogue warps;
                                                   // odd CTA: its producer + 4 scale writers + 8 epilogue warps
-constexpr int kTileConsumers = 2 * kTileConsumersPerCta + (kSplitSF ? 1 : 0);  // + the odd CTA's relay warp
+constexpr int kTileConsumers = 2 * kTileConsumersPerCta;
 
 struct Shared {
     alignas(16) uint16_t ostage[kEpiWarps][32 * 32];  // epilogue: one 32-token x 32-column BF16 block per warp
     uint64_t tq_full[kTileRing];  // the even CTA published tq[i] (in this CTA's copy of the ring)
     uint64_t tq_empty[kTileRing]; // even CTA: every consumer warp of both CTAs read entry i
     int32_t tq[kTileRing];        // work item index (>= total: no more work)
-    uint64_t full_tma[kStages];   // this CTA's loads of the stage landed (split: its operand codes)
-    uint64_t full_sf[kStages];    // split: this CTA's scale bytes of the stage landed
-    uint64_t op_peer[kStages];    // split, even CTA: the odd CTA's operand codes landed (relay arrival)
+    uint64_t full_tma[kStages];   // this CTA's loads of the stage landed
     uint64_t sf_ready[kStages];   // even CTA: both CTAs' scales are in TMEM (8 warp arrivals)
     uint64_t empty[kStages];      // the pair's MMAs of the stage completed (commit from the even CTA)
     uint64_t acc_full;            // the pair's MMAs of the tile completed
@@ -272,7 +266,7 @@ template <int kEpi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_full,
                              const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_wsw,
-                             const Params p) {
+                             const __grid_constant__ CUtensorMap tm_wsf, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
@@ -291,12 +285,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tm_a);
         prefetch_tensormap(&tm_a_full);
         prefetch_tensormap(&tm_out);
-        if (p.swiglu) prefetch_tensormap(&tm_wsw);
+        if (p.swiglu) {
+            prefetch_tensormap(&tm_wsw);
+            prefetch_tensormap(&tm_wsf);
+        }
         sh.abort = 0;
         for (int s = 0; s < kStages; s++) {
             mbar_init(&sh.full_tma[s], 1);
-            mbar_init(&sh.full_sf[s], 1);
-            mbar_init(&sh.op_peer[s], 1);
             mbar_init(&sh.sf_ready[s], 8);
             mbar_init(&sh.empty[s], 1);
         }
@@ -352,7 +347,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             } else {
                 ok = next_tile_thread(sh, rank, qi, qphase, w, abort, p.ctl);
             }
-            const int32_t first_w = w;
             while (ok && w < total) {
                 Tile t;
                 decode_tile(sh, E, w, t);
@@ -366,80 +360,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int32_t my_rows = t.bn / 2;
                 const int32_t my_row0 = t.row0 + (int32_t)rank * my_rows;
                 // SWIGLU: 16 KB of interleaved gate/up codes + both tiles' 2 KB of scales; NONE: one packed tile
-                const uint32_t a_sf_bytes = p.swiglu ? 2u * kTileSFBytes : (uint32_t)kTileSFBytes;
+                const uint32_t a_bytes = p.swiglu ? (uint32_t)kCodeBytes + 2u * kTileSFBytes : (uint32_t)kPackedTileBytes;
                 // both CTAs stage the scales of all the tile's rows: one contiguous run of the K step's
                 // slab (K-stage layout), 16 bytes per row
-                const uint32_t sf_tx = a_sf_bytes + (uint32_t)t.rows * 16u;
-                const uint32_t op_tx = (uint32_t)kCodeBytes + (uint32_t)my_rows * kRowBytes;
+                const uint32_t tx = a_bytes + (uint32_t)my_rows * kRowBytes + (uint32_t)t.rows * 16u;
                 const uint8_t* sfb = p.a_sf + (int64_t)t.row0 * 16;
-                // L2 prefetch of the weight stream kPrefetchAhead stages ahead (even CTA, for both CTAs'
-                // tiles), continuing into the next work item's first stages
-                const uint8_t* pf_g = nullptr;
-                const uint8_t* pf_u = nullptr;
-                uint64_t pf_pol = pol_w_once;
-                if (kPrefetchAhead > 0 && rank == 0 && w_next < total) {
-                    Tile tn;
-                    decode_tile(sh, E, w_next, tn);
-                    weight_tiles(p, tn, 0, ksteps_total, pf_g, pf_u);
-                    pf_pol = (sh.off[tn.e + 1] - sh.off[tn.e] > kBNMax) ? pol_w_reuse : pol_w_once;
-                }
-                if (kPrefetchAhead > 0 && rank == 0 && w == first_w) {
-                    // the first work item: its own first stages were not prefetched by a previous item
-                    for (int32_t kt = 0; kt < min(kPrefetchAhead, ksteps_total); kt++) {
-                        bulk_prefetch_l2(g_tile + (size_t)kt * kPackedTileBytes, kPackedTileBytes, pol_w);
-                        bulk_prefetch_l2(u_tile + (size_t)kt * kPackedTileBytes, kPackedTileBytes, pol_w);
-                    }
-                }
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
                     if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
                     uint8_t* sb = stages + (size_t)stage * kStageBytes;
                     uint64_t* bar = &sh.full_tma[stage];
-                    uint64_t* sbar = kSplitSF ? &sh.full_sf[stage] : bar;
-                    if (kSplitSF) {
-                        mbar_arrive_expect_tx(sbar, sf_tx);
-                        mbar_arrive_expect_tx(bar, op_tx);
-                    } else {
-                        mbar_arrive_expect_tx(bar, sf_tx + op_tx);
-                    }
+                    mbar_arrive_expect_tx(bar, tx);
                     const size_t ko = (size_t)kt * kPackedTileBytes;
-#if NVFP4_PAIR_OLD_ORDER
-                    if (!kSplitSF) {
-                        // codes, then scales (issue order of the first CTA-pair kernel)
-                        if (p.swiglu) {
-                            tma_load_5d(sb + kOffA, &tm_wsw, 0, 0, 0, (int32_t)(half / 16), sw_tile0 + kt, bar, pol_w);
-                            bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
-                            bulk_load(sb + kOffSFA + kTileSFBytes, u_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
-                        } else {
-                            bulk_load(sb + kOffA, g_tile + ko, kPackedTileBytes, bar, pol_w);
-                        }
-                        if (my_rows == kBNMax / 2) {
-                            tma_load_2d(sb + kOffB, &tm_a_full, kt * kRowBytes, my_row0, bar, pol_a);
-                        } else {
-                            for (int32_t i = 0; i < my_rows / kBoxRows; i++)
-                                tma_load_2d(sb + kOffB + i * kBoxRows * kRowBytes, &tm_a, kt * kRowBytes,
-                                            my_row0 + i * kBoxRows, bar, pol_a);
-                        }
-                        bulk_load(sb + kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, bar, pol_a);
-                        issued[stage] = true;
-                        issued_parity[stage] = phase;
-                        if (++stage == kStages) { stage = 0; phase ^= 1u; }
-                        continue;
-                    }
-#endif
-                    // scales first: they are small and their consumers (the scale writers) run ahead of the MMAs
-                    if (p.swiglu) {
-                        bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, sbar, pol_w);
-                        bulk_load(sb + kOffSFA + kTileSFBytes, u_tile + ko + kCodeBytes, kTileSFBytes, sbar, pol_w);
-                    } else if (kSplitSF) {
-                        bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, sbar, pol_w);
-                    }
-                    bulk_load(sb + kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, sbar, pol_a);
                     if (p.swiglu) {
                         // 16-row slabs (2 KB, whole swizzle atoms) of this CTA's half: gate slab q -> A rows
                         // 32q.., up slab q -> 32q+16.. (one box: bytes x rows x gate/up x slab x tile)
                         tma_load_5d(sb + kOffA, &tm_wsw, 0, 0, 0, (int32_t)(half / 16), sw_tile0 + kt, bar, pol_w);
-                    } else if (kSplitSF) {
-                        bulk_load(sb + kOffA, g_tile + ko, kCodeBytes, bar, pol_w);
+#if NVFP4_PAIR_SFA_BOX
+                        // both tiles' 2 KB of scales (slab 8 of each tile's view): one load
+                        tma_load_5d(sb + kOffSFA, &tm_wsf, 0, 0, 0, 8, sw_tile0 + kt, bar, pol_w);
+#else
+                        bulk_load(sb + kOffSFA, g_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
+                        bulk_load(sb + kOffSFA + kTileSFBytes, u_tile + ko + kCodeBytes, kTileSFBytes, bar, pol_w);
+#endif
                     } else {
                         bulk_load(sb + kOffA, g_tile + ko, kPackedTileBytes, bar, pol_w);   // codes + scales
                     }
@@ -450,17 +392,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             tma_load_2d(sb + kOffB + i * kBoxRows * kRowBytes, &tm_a, kt * kRowBytes,
                                         my_row0 + i * kBoxRows, bar, pol_a);
                     }
-                    if (kPrefetchAhead > 0 && rank == 0) {
-                        const int32_t ka = kt + kPrefetchAhead;
-                        if (ka < ksteps_total) {
-                            bulk_prefetch_l2(g_tile + (size_t)ka * kPackedTileBytes, kPackedTileBytes, pol_w);
-                            bulk_prefetch_l2(u_tile + (size_t)ka * kPackedTileBytes, kPackedTileBytes, pol_w);
-                        } else if (pf_g != nullptr && ka - ksteps_total < ksteps_total) {
-                            const size_t kn = (size_t)(ka - ksteps_total) * kPackedTileBytes;
-                            bulk_prefetch_l2(pf_g + kn, kPackedTileBytes, pf_pol);
-                            bulk_prefetch_l2(pf_u + kn, kPackedTileBytes, pf_pol);
-                        }
-                    }
+                    bulk_load(sb + kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, bar, pol_a);
                     issued[stage] = true;
                     issued_parity[stage] = phase;
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -474,11 +406,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok || *abort) {
-                for (int s = 0; s < kStages; s++) {
-                    if (!issued[s]) continue;
-                    mbar_wait_drain(&sh.full_tma[s], issued_parity[s], 200000000ull);
-                    if (kSplitSF) mbar_wait_drain(&sh.full_sf[s], issued_parity[s], 200000000ull);
-                }
+                for (int s = 0; s < kStages; s++)
+                    if (issued[s]) mbar_wait_drain(&sh.full_tma[s], issued_parity[s], 200000000ull);
             }
         }
         __syncwarp();
@@ -498,10 +427,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int32_t w;
             if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl) || w >= total) break;
             for (int32_t kt = 0; kt < ksteps_total; kt++) {
-                if (!warp_wait(kSplitSF ? &sh.full_sf[stage] : &sh.full_tma[stage], phase, abort, p.ctl)) {
-                    ok = false;
-                    break;
-                }
+                if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl)) { ok = false; break; }
                 tc_fence_after();
                 const uint8_t* sb = stages + (size_t)stage * kStageBytes;
                 const uint32_t slot = tmem + lane_addr + kTmemSFRing + stage * kSFSlot;
@@ -548,8 +474,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (!warp_wait(&sh.acc_empty, aphase ^ 1u, abort, p.ctl)) { ok = false; break; }
                 tc_fence_after();
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
-                    if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl) ||
-                        (kSplitSF && !warp_wait(&sh.op_peer[stage], phase, abort, p.ctl)) ||
+                    // sf_ready implies both CTAs' loads of the stage landed: every scale writer waits for its
+                    // CTA's loads before arriving
+                    if ((!kSkipFullWait && !warp_wait(&sh.full_tma[stage], phase, abort, p.ctl)) ||
                         !warp_wait(&sh.sf_ready[stage], phase, abort, p.ctl)) {
                         ok = false;
                         break;
@@ -558,13 +485,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (lane == 0) {
                         const uint32_t sb = smem_u32(stages + (size_t)stage * kStageBytes);
                         const uint32_t sf = tmem + kTmemSFRing + stage * kSFSlot;
-                        const int n_kc = kt == ksteps_total - 1 ? last_ksteps : kKSteps;
+                        if (kt != ksteps_total - 1 || last_ksteps == kKSteps) {
 #pragma unroll
-                        for (int kc = 0; kc < kKSteps; kc++) {
-                            if (kc >= n_kc) break;
-                            mma_mxf4nvf4_pair(tmem, make_smem_desc(sb + kOffA + kc * 32, 16, 1024, 2),
-                                              make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2), idesc,
-                                              sf + 4 * kc, sf + 16 + 8 * kc, (kt | kc) != 0);
+                            for (int kc = 0; kc < kKSteps; kc++)
+                                mma_mxf4nvf4_pair(tmem, make_smem_desc(sb + kOffA + kc * 32, 16, 1024, 2),
+                                                  make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2), idesc,
+                                                  sf + 4 * kc, sf + 16 + 8 * kc, (kt | kc) != 0);
+                        } else {
+                            // a last stage of 128 K-elements: its first two K-steps
+                            for (int kc = 0; kc < last_ksteps; kc++)
+                                mma_mxf4nvf4_pair(tmem, make_smem_desc(sb + kOffA + kc * 32, 16, 1024, 2),
+                                                  make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2), idesc,
+                                                  sf + 4 * kc, sf + 16 + 8 * kc, (kt | kc) != 0);
                         }
                         tc_commit_pair(own_empty0 + stage * 8);
                         tc_commit_pair(peer_empty0 + stage * 8);
@@ -586,20 +518,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     mbar_wait_drain(&sh.drain, 0, 200000000ull);
                 }
                 __syncwarp();
-            }
-        } else if (kSplitSF) {
-            // ================= relay (odd CTA): this CTA's operand codes of a stage landed =================
-            uint32_t stage = 0, phase = 0, qi = 0, qphase = 0;
-            const uint32_t peer0 = cluster_smem_addr(&sh.op_peer[0], 0);
-            bool ok = true;
-            while (ok) {
-                int32_t w;
-                if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl) || w >= total) break;
-                for (int32_t kt = 0; kt < ksteps_total; kt++) {
-                    if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl)) { ok = false; break; }
-                    if (lane == 0) mbar_arrive_cluster(peer0 + stage * 8);
-                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
-                }
             }
         }
     } else if (warp >= 4) {  // warps 4-7 and 12-15
@@ -822,7 +740,8 @@ static bool pair_kernel_configured(int dev) {
 
 // Launches the pair kernel; the caller validated every argument (same contract as the one-SM kernel).
 nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full,
-                                      const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const uint8_t* a_sf,
+                                      const CUtensorMap& tm_out, const CUtensorMap& tm_wsw,
+                                      const CUtensorMap& tm_wsf, const uint8_t* a_sf,
                                       const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
                                       const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
                                       int swiglu, uint16_t* out, uint32_t* out_amax, const Finalize& fin,
@@ -882,14 +801,14 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     if (qo.q != nullptr) {
         if (!pair_kernel_configured<kEpiQuant>(dev)) return NVFP4_ERR_CUDA;
         launch_pdl(gp::grouped_gemm_pair_kernel<kEpiQuant>, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes, s,
-                   tm_a, tm_a_full, tm_out, tm_wsw, prm);
+                   tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
     } else if (fin.out != nullptr) {
         if (!pair_kernel_configured<kEpiFinalize>(dev)) return NVFP4_ERR_CUDA;
         launch_pdl(gp::grouped_gemm_pair_kernel<kEpiFinalize>, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes,
-                   s, tm_a, tm_a_full, tm_out, tm_wsw, prm);
+                   s, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
     } else {
         launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain>, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes, s,
-                   tm_a, tm_a_full, tm_out, tm_wsw, prm);
+                   tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
     }
     count_launch();
     return check_launch();
