@@ -191,10 +191,9 @@ static nvfp4_status layer(const uint16_t* x, const float* logits, const int32_t*
     void* scratch = b + L.scratch;
     const size_t scratch_bytes = L.topk_ids - L.scratch;
 
-    uint32_t* fin_counters = reinterpret_cast<uint32_t*>(b + L.fin_counters);
-    // the gate/up GEMM raises amax_h and the down GEMM counts rows into fin_counters; both start from 0
-    // (one memset before the first kernel, so that every kernel boundary after it keeps its
-    // programmatic launch)
+    // the gate/up GEMM raises amax_h; it starts from 0, and so do the fused combine's counters right after it
+    // (one memset before the first kernel, so that every kernel boundary after it keeps its programmatic
+    // launch)
     if (cudaMemsetAsync(amax_h, 0, L.fin_counters + moe_finalize_counters_size(T, H) - L.amax_h,
                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return NVFP4_ERR_CUDA;
@@ -217,7 +216,6 @@ static nvfp4_status layer(const uint16_t* x, const float* logits, const int32_t*
     // the down GEMM, then the combine as its own kernel: measured on B200 faster than the down GEMM with
     // the combine fused into its epilogue (moe_grouped_gemm_nvfp4_finalize gives the same bits) on the
     // decode, Zipf and prefill layers
-    (void)fin_counters;
     if ((st = moe_grouped_gemm_nvfp4(q_h, sf_h, g_h, w2_packed, w2_gscale, off, E, R, H, I, NVFP4_EPI_NONE, y,
                                      stream)))
         return st;
