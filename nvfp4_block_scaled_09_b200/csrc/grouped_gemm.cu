@@ -86,7 +86,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemLimit = 232448;               // B200 opt-in shared memory per block
 
 constexpr int kTileRing = 4;                     // work items the producer may publish ahead of the slowest role
-constexpr int kFinSlots = 4;                     // stored tiles the epilogue may hand ahead to the finalisers
 constexpr int kTileConsumers = 9;                // MMA warp + 4 scale writers + 4 epilogue warps
 
 struct Shared {
@@ -104,10 +103,8 @@ struct Shared {
     int32_t total_tiles;
     int32_t off[kMaxE + 1];
     int32_t tile_start[kMaxE + 1];
-    // fused combine: the epilogue hands each stored tile to the finaliser warps through this ring
-    int4 fin_q[kFinSlots];                       // {first row, rows (< 0: no more tiles), column tile, full width}
-    uint64_t fin_full[kFinSlots];                // the 4 epilogue warps stored and fenced the tile's rows
-    uint64_t fin_empty[kFinSlots];               // both finaliser warps are done with the entry
+    int32_t fin_tok[128];                        // fused combine: tokens of this tile whose last row it wrote
+    uint64_t fin_bar;                            // fused combine: the 4 epilogue warps meet (bounded waits)
 };
 
 // Two tile shapes share one kernel body:
@@ -249,10 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sh.acc_empty[b], 4);
         }
         mbar_init(&sh.drain, 1);
-        for (int i = 0; i < kFinSlots; i++) {
-            mbar_init(&sh.fin_full[i], 4);
-            mbar_init(&sh.fin_empty[i], 2);
-        }
+        mbar_init(&sh.fin_bar, 4);
         for (int i = 0; i < kTileRing; i++) {
             mbar_init(&sh.tq_full[i], 1);
             mbar_init(&sh.tq_empty[i], kTileConsumers);
@@ -507,48 +501,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (++stage == kStages) { stage = 0; phase ^= 1u; }
             }
         }
-    } else if (kEpi == kEpiFinalize && (warp == 1 || warp == 3)) {
-        // ================= finalisers (fused combine) =================
-        // Every row of a stored tile holds one (token, slot) product for the tile's output columns. Each
-        // finaliser warp counts half of the tile's rows in per (token, column tile); the warp that brings a
-        // token's count to k writes the token's combined output for these columns (lane l: columns
-        // [8l, 8l + 8)), whichever CTA wrote the other k - 1 rows, with the combine kernel's arithmetic, so
-        // the result does not depend on the order. The last arriver leaves the counter at zero.
-        const int f = warp == 1 ? 0 : 1;
-        uint32_t fslot = 0, fphase = 0;
-        while (true) {
-            if (!warp_wait(&sh.fin_full[fslot], fphase, abort, p.ctl)) break;
-            const volatile int* qv = reinterpret_cast<volatile int*>(&sh.fin_q[fslot]);
-            const int4 en = make_int4(qv[0], qv[1], qv[2], qv[3]);
-            if (en.y < 0) break;
-            const int64_t col = (int64_t)en.z * (kNumA * kBM) + lane * 8;
-            const bool lane_on = en.w != 0 || lane * 8 < kBM;
-            for (int h = 0; h < 2; h++) {
-                const int i = f * 64 + h * 32 + lane;
-                int32_t tok = -1;
-                if (i < en.y) {
-                    const int32_t tk = __ldg(p.fin.src + en.x + i);
-                    if (tk >= 0 && tk < p.fin.T) {
-                        uint32_t* cnt = p.fin.counters + (int64_t)tk * p.fin.col_blocks + 2 * en.z;
-                        if (atomicAdd(cnt, 1u) == (uint32_t)(p.fin.k - 1)) {
-                            atomicExch(cnt, 0u);
-                            tok = tk;
-                        }
-                    }
-                }
-                uint32_t m = __ballot_sync(0xFFFFFFFFu, tok >= 0);
-                if (m) __threadfence();   // the other rows' stores are visible before the reads
-                while (m) {
-                    const int src_lane = __ffs(m) - 1;
-                    m &= m - 1u;
-                    const int32_t tk = __shfl_sync(0xFFFFFFFFu, tok, src_lane);
-                    if (lane_on) combine_vec8(p.out, p.N, p.fin.inv, p.fin.w, tk, p.fin.k, col, p.fin.out, p.N);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.fin_empty[fslot]);
-            if (++fslot == kFinSlots) { fslot = 0; fphase ^= 1u; }
-        }
     } else if (warp >= 4) {
         // ================= epilogue =================
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
@@ -557,19 +509,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float a_g = __ldg(p.a_gscale);
         const float h_genc = kEpi == kEpiQuant ? __fdiv_rn(1.0f, __ldg(p.qo.gdec)) : 0.0f;   // static scale of h
         uint32_t amax = 0;  // max |stored BF16| of this thread, as BF16 bits
-        uint32_t abuf = 0, aphase = 0, qi = 0, qphase = 0, fslot = 0, fphase = 0;
-        // fused combine: hand a stored tile (or the end, rows < 0) to the finaliser warps; false when a wait
-        // ran out. Warp 4 writes the entry once the finalisers released the slot; the ring entry is complete
-        // when all 4 epilogue warps arrived, so warps 5-7 need not wait for the slot themselves.
-        auto fin_push = [&](int4 entry) -> bool {
-            if (warp == 4) {
-                if (!warp_wait(&sh.fin_empty[fslot], fphase ^ 1u, abort, p.ctl)) return false;
-                if (lane == 0) sh.fin_q[fslot] = entry;
-            }
+        uint32_t abuf = 0, aphase = 0, qi = 0, qphase = 0, fphase = 0;
+        // the 4 epilogue warps meet here (fused combine only); false when a wait ran out
+        auto epi_sync = [&]() -> bool {
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.fin_full[fslot]);
-            if (++fslot == kFinSlots) { fslot = 0; fphase ^= 1u; }
-            return true;
+            if (lane == 0) mbar_arrive(&sh.fin_bar);
+            const bool ok = warp_wait(&sh.fin_bar, fphase, abort, p.ctl);
+            fphase ^= 1u;
+            return ok;
         };
         while (true) {
             int32_t w;
@@ -647,11 +594,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&sh.acc_empty[abuf]);
             if (++abuf == (uint32_t)C::kAccBufs) { abuf = 0; aphase ^= 1u; }
             if (kEpi == kEpiFinalize) {
-                __threadfence();   // this thread's y stores, device-wide, before the finalisers count the rows in
-                if (!fin_push(make_int4(t.row0, t.rows, t.nt, second ? 1 : 0))) break;
+                // Fused combine. Every row of this tile holds one (token, slot) product for the tile's output
+                // columns; count the rows in per (token, column tile). The CTA that brings a token's count
+                // to k writes that token's combined output for these columns, whichever CTA wrote the other
+                // k - 1 rows, with the combine's arithmetic, so the result does not depend on the order.
+                __threadfence();                            // this thread's y stores, device-wide, first
+                if (!epi_sync()) break;
+                const int i = (warp - 4) * 32 + lane;
+                int32_t tok = -1;
+                if (i < t.rows) {
+                    const int32_t tk = __ldg(p.fin.src + t.row0 + i);
+                    if (tk >= 0 && tk < p.fin.T) {
+                        uint32_t* cnt = p.fin.counters + (int64_t)tk * p.fin.col_blocks + 2 * t.nt;
+                        if (atomicAdd(cnt, 1u) == (uint32_t)(p.fin.k - 1)) {
+                            atomicExch(cnt, 0u);            // left at zero for the next launch
+                            tok = tk;
+                        }
+                    }
+                }
+                sh.fin_tok[i] = tok;
+                __threadfence();                            // the other rows' stores are visible before the reads
+                if (!epi_sync()) break;
+                // one warp per token: lane l combines columns [8l, 8l + 8) of the tile's 256 (128 for a half tile)
+                const int64_t col = (int64_t)t.nt * (kNumA * kBM) + lane * 8;
+                const bool lane_on = second || lane * 8 < kBM;
+                for (int j = warp - 4; j < t.rows; j += 4) {
+                    const int32_t tk = sh.fin_tok[j];
+                    if (tk >= 0 && lane_on) combine_vec8(p.out, p.N, p.fin.inv, p.fin.w, tk, p.fin.k, col, p.fin.out, p.N);
+                }
+                if (!epi_sync()) break;                     // fin_tok is rewritten by the next tile
             }
         }
-        if (kEpi == kEpiFinalize) fin_push(make_int4(0, -1, 0, 0));   // no more tiles
         if (p.amax_out != nullptr) {
             amax = __reduce_max_sync(0xFFFFFFFFu, amax);
             if (lane == 0 && amax != 0u) atomicMax(p.amax_out, amax);
