@@ -481,9 +481,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kc = 0; kc < kKSteps; kc++)
                         word[kc] = *reinterpret_cast<const uint32_t*>(src + kc * kSFAtomBytes);
+                    // one column per K-step: the one this quadrant's rows are read from
 #pragma unroll
-                    for (int j = 0; j < 16; j++) v[j] = ((j & 3) == quad) ? word[j >> 2] : 0u;
-                    tmem_st_32x32b_x16(slot + a * 4 * kKSteps, v);
+                    for (int kc = 0; kc < kKSteps; kc++) tmem_st_32x32b_x1(slot + a * 4 * kKSteps + 4 * kc + quad, word[kc]);
                 }
 #pragma unroll
                 for (int kc = 0; kc < kKSteps; kc++) {

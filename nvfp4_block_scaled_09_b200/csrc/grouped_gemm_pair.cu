@@ -20,9 +20,10 @@
 // values and hand it back to the MMA warp; staging and storing those values
 // then overlaps the next tile's main loop.
 //
-// Synchronisation uses no multicast: the peer's scale-writer and epilogue warps
-// arrive on the even CTA's barriers through cluster addresses (mapa), and the
-// even CTA's MMA completions are committed to each CTA's barrier separately.
+// The peer's scale-writer and epilogue warps arrive on the even CTA's barriers
+// through cluster addresses (mapa); the even CTA's MMA completions reach both
+// CTAs' barriers through one commit with a CTA mask (no data moves by multicast;
+// measured 1-3% faster than a commit per CTA).
 // Work items come from a grid-wide counter (dynamic schedule); the even CTA
 // takes each one and writes it into both CTAs' work-item rings. Every wait is
 // bounded as in the one-SM kernel; a cluster barrier guards the release of
@@ -30,6 +31,7 @@
 #include <mutex>
 
 #include "common.cuh"
+
 
 
 namespace nvfp4 {
@@ -420,14 +422,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint8_t* sb = stages + (size_t)stage * kStageBytes;
                 const uint32_t slot = tmem + lane_addr + kTmemSFRing + stage * kSFSlot;
-                uint32_t v16[16];
+                // SFA: one column per K-step, the one this quadrant's rows are read from (the other three
+                // columns of the step belong to the other quadrants; measured: 1% faster than writing all four)
 #pragma unroll
-                for (int kc = 0; kc < kKSteps; kc++) {
-                    const uint32_t word = *reinterpret_cast<const uint32_t*>(sb + sfa_off + kc * 512);
-#pragma unroll
-                    for (int q = 0; q < 4; q++) v16[4 * kc + q] = (q == quad) ? word : 0u;
-                }
-                tmem_st_32x32b_x16(slot, v16);
+                for (int kc = 0; kc < kKSteps; kc++)
+                    tmem_st_32x32b_x1(slot + 4 * kc + quad, *reinterpret_cast<const uint32_t*>(sb + sfa_off + kc * 512));
                 uint32_t v32[32];
 #pragma unroll
                 for (int g = 0; g < 8; g++) {
@@ -449,8 +448,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ================= MMA issuer (even CTA) =================
         if (rank == 0) {
             const uint32_t idesc_base = (1u << 7) | (1u << 10) | ((uint32_t)((2 * kBM) >> 4) << 24);
-            const uint32_t peer_empty0 = cluster_smem_addr(&sh.empty[0], 1);
-            const uint32_t own_empty0 = cluster_smem_addr(&sh.empty[0], 0);
             uint32_t stage = 0, phase = 0, aphase = 0, qi = 0, qphase = 0;
             bool ok = true;
             while (ok) {
@@ -486,16 +483,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                   make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2), idesc,
                                                   sf + 4 * kc, sf + 16 + 8 * kc, (kt | kc) != 0);
                         }
-                        tc_commit_pair(own_empty0 + stage * 8);
-                        tc_commit_pair(peer_empty0 + stage * 8);
+                        tc_commit_pair_both(&sh.empty[stage]);
                     }
                     __syncwarp();
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 if (lane == 0) {
-                    tc_commit_pair(cluster_smem_addr(&sh.acc_full, 0));
-                    tc_commit_pair(cluster_smem_addr(&sh.acc_full, 1));
+                    tc_commit_pair_both(&sh.acc_full);
                 }
                 __syncwarp();
                 aphase ^= 1u;
