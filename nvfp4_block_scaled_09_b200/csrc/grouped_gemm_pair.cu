@@ -45,39 +45,33 @@ constexpr int kKSteps = kBK / 64;
 constexpr int kBNMax = 256;                       // activation rows per pair tile (MMA N)
 constexpr int kBNStep = 32;                       // N granularity: each CTA holds a multiple of 16 rows
 constexpr int kBoxRows = 16;                      // activation TMA box rows
-constexpr int kStages = 5;
 constexpr int kPackedTileBytes = 18432;           // packed weight tile: 16 KB codes + 2 KB scales
 constexpr int kCodeBytes = 16384;
 constexpr int kTileSFBytes = 2048;
 constexpr int kOffA = 0;                          // 128 weight rows x 128 B (SwiGLU: gate/up slabs of 16 rows, interleaved)
 constexpr int kOffSFA = kCodeBytes;               // scales of one packed tile (SwiGLU: gate tile's, then up tile's)
 constexpr int kOffB = kOffSFA + 2 * kTileSFBytes;  // this CTA's half of the activation rows
-constexpr int kOffSFB = kOffB + (kBNMax / 2) * kRowBytes;  // scales of all the tile's rows, 16 bytes each
-constexpr int kStageBytes = kOffSFB + kBNMax * 16;         // 40960
 constexpr int kThreads = 512;                     // warps: 0 loads, 2 MMA, 4-7 + 12-15 epilogue, 8-11 scales
 constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant, alternating 32-token chunks
 constexpr int kChunksPerWarp = kBNMax / 32 / 2;   // 32-token chunks one epilogue warp drains per tile
+                                                  // (plus the tail chunk, columns 256-287, on warps 4-7)
 constexpr int kMaxE = 1024;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCols = kBNMax;             // one 128-lane x 256-column accumulator per CTA
-constexpr uint32_t kSFSlot = 4 * kKSteps + 8 * kKSteps;  // SFA: 4 columns per K step, SFB: 8 (256 rows)
-constexpr uint32_t kTmemSFRing = kAccCols;
-static_assert(kTmemSFRing + kStages * kSFSlot <= kTmemCols, "TMEM budget");
-static_assert(kStageBytes % 1024 == 0 && kOffB % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 
 constexpr int kTileRing = 4;                      // work items the even CTA may publish ahead
 constexpr int kTileConsumersPerCta = 13;          // even CTA: MMA warp + 4 scale writers + 8 epilogue warps;
                                                   // odd CTA: its producer + 4 scale writers + 8 epilogue warps
 constexpr int kTileConsumers = 2 * kTileConsumersPerCta;
 
-struct Shared {
+template <int kStagesT, int kTailT>
+struct SharedT {
     alignas(16) uint16_t ostage[kEpiWarps][32 * 32];  // epilogue: one 32-token x 32-column BF16 block per warp
     uint64_t tq_full[kTileRing];  // the even CTA published tq[i] (in this CTA's copy of the ring)
     uint64_t tq_empty[kTileRing]; // even CTA: every consumer warp of both CTAs read entry i
     int32_t tq[kTileRing];        // work item index (>= total: no more work)
-    uint64_t full_tma[kStages];   // this CTA's loads of the stage landed
-    uint64_t sf_ready[kStages];   // even CTA: both CTAs' scales are in TMEM (8 warp arrivals)
-    uint64_t empty[kStages];      // the pair's MMAs of the stage completed (commit from the even CTA)
+    uint64_t full_tma[kStagesT];  // this CTA's loads of the stage landed
+    uint64_t sf_ready[kStagesT];  // even CTA: both CTAs' scales are in TMEM (8 warp arrivals)
+    uint64_t empty[kStagesT];     // the pair's MMAs of the stage completed (commit from the even CTA)
     uint64_t acc_full;            // the pair's MMAs of the tile completed
     uint64_t acc_empty;           // even CTA: both CTAs' epilogues drained TMEM (2 x kEpiWarps arrivals)
     uint64_t drain;
@@ -86,12 +80,37 @@ struct Shared {
     int32_t total_tiles;
     int32_t off[kMaxE + 1];
     int32_t tile_start[kMaxE + 1];
-    int32_t fin_tok[kBNMax];      // fused combine: tokens of this tile whose last row this CTA wrote
+    int32_t fin_tok[kBNMax + kTailT];   // fused combine: tokens of this tile whose last row this CTA wrote
     uint64_t fin_bar;             // fused combine: this CTA's 8 epilogue warps meet (bounded waits)
 };
 
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Shared);
-static_assert(kSmemBytes + 256 <= 232448, "shared memory budget");
+// Two configurations of the kernel, chosen per launch:
+// - kTails (grouped GEMMs): an expert's rows past its last full 256-row tile ride on that tile when there
+//   are at most kTailMax = 32 of them (a second MMA of N = 32 into accumulator columns 256-287) instead
+//   of taking a tile of their own, which would stream the whole weight tile again for a few rows. Their
+//   buffers cost a shared-memory stage (4 of 43 KB) and the scales' TMEM ring is 3 slots deep (a slot is
+//   written just before its MMAs, so it needs fewer slots than there are stages).
+// - no tails (one expert, dense): 5 stages of 40 KB, one scale slot per stage.
+template <bool kTails>
+struct Cfg {
+    static constexpr int kTailMax = kTails ? 32 : 0;
+    static constexpr int kStages = kTails ? 4 : 5;
+    static constexpr int kOffBT = kOffB + (kBNMax / 2) * kRowBytes;       // this CTA's half of the tail rows
+    static constexpr int kOffSFB = kOffBT + (kTailMax / 2) * kRowBytes;   // scales of all the tile's rows, 16 B each
+    static constexpr int kStageBytes = (kOffSFB + (kBNMax + kTailMax) * 16 + 1023) / 1024 * 1024;
+    static constexpr uint32_t kAccCols = kBNMax + kTailMax;    // one accumulator per CTA (+ the tail's columns)
+    // TMEM scale slot: SFA 4 columns per K step, SFB 8 (256 rows), tail SFB 4 (one used)
+    static constexpr int kSFSlots = kTails ? 3 : kStages;
+    static constexpr uint32_t kSFSlot = (kTails ? 16 : 12) * kKSteps;
+    static constexpr uint32_t kSFTail = 12 * kKSteps;          // tail SFB of K step kc at slot + kSFTail + 4 kc
+    static constexpr uint32_t kTmemSFRing = kAccCols;
+    using Shared = SharedT<kStages, kTailMax>;
+    static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Shared);
+    static_assert(kTmemSFRing + kSFSlots * kSFSlot <= kTmemCols, "TMEM budget");
+    static_assert(kStageBytes % 1024 == 0 && kOffB % 1024 == 0 && kOffBT % 1024 == 0,
+                  "swizzled tiles need 1024-byte alignment");
+    static_assert(kSmemBytes + 256 <= 232448, "shared memory budget");
+};
 
 struct Params {
     const uint8_t* a_sf;
@@ -113,10 +132,20 @@ struct Params {
 };
 
 struct Tile {
-    int32_t e, nt, mt, row0, rows, bn;
+    int32_t e, nt, mt, row0, rows, bn, tail;   // rows = bn-covered rows + tail rows (columns 256..287)
 };
 
-__device__ __forceinline__ void decode_tile(const Shared& sh, int32_t E, int32_t w, Tile& t) {
+// Row tiles of an expert with M rows: 256 rows each, except that a remainder of at most kTailMax rows
+// rides on the last full tile (a second MMA of N = 32 into accumulator columns 256-287) instead of
+// taking a tile of its own, which would stream the whole weight tile again for a few rows.
+template <int kTail>
+__device__ __forceinline__ int32_t row_tiles(int32_t M) {
+    const int32_t full = M / kBNMax, rem = M - full * kBNMax;
+    return full + ((rem > kTail || (full == 0 && rem > 0)) ? 1 : 0);
+}
+
+template <int kTail, class S>
+__device__ __forceinline__ void decode_tile(const S& sh, int32_t E, int32_t w, Tile& t) {
     int32_t lo = 0, hi = E;  // tile_start[lo] <= w < tile_start[hi]
     while (hi - lo > 1) {
         const int32_t mid = (lo + hi) >> 1;
@@ -124,14 +153,16 @@ __device__ __forceinline__ void decode_tile(const Shared& sh, int32_t E, int32_t
         else hi = mid;
     }
     const int32_t M = sh.off[lo + 1] - sh.off[lo];
-    const int32_t mtiles = (M + kBNMax - 1) / kBNMax;
+    const int32_t mtiles = row_tiles<kTail>(M);
     const int32_t local = w - sh.tile_start[lo];
     t.e = lo;
     t.nt = local / mtiles;
     t.mt = local - t.nt * mtiles;
     t.row0 = sh.off[lo] + t.mt * kBNMax;
-    t.rows = min(kBNMax, M - t.mt * kBNMax);
-    t.bn = (t.rows + kBNStep - 1) / kBNStep * kBNStep;
+    t.rows = t.mt == mtiles - 1 ? M - t.mt * kBNMax : kBNMax;
+    const int32_t main_rows = min(t.rows, kBNMax);
+    t.bn = (main_rows + kBNStep - 1) / kBNStep * kBNStep;
+    t.tail = t.rows - main_rows;
 }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, const DeviceCtl& ctl) {
@@ -149,17 +180,20 @@ __device__ __forceinline__ void arrive_on_leader(uint64_t* bar, uint32_t rank) {
 // The even CTA's producer takes each work item from the launch's counter and writes it into both CTAs'
 // copies of the ring (the odd CTA's through distributed shared memory, released at cluster scope); every
 // consumer warp of both CTAs reports on the even CTA's tq_empty once it has read an entry.
-__device__ __forceinline__ bool tq_wait(Shared& sh, uint32_t qi, uint32_t qphase, uint32_t rank, volatile int* abort,
+template <class S>
+__device__ __forceinline__ bool tq_wait(S& sh, uint32_t qi, uint32_t qphase, uint32_t rank, volatile int* abort,
                                         const DeviceCtl& ctl) {
     return rank == 0 ? mbar_wait_bounded(&sh.tq_full[qi], qphase, abort, ctl)
                      : mbar_wait_bounded_acq_cluster(&sh.tq_full[qi], qphase, abort, ctl);
 }
-__device__ __forceinline__ void tq_release(Shared& sh, uint32_t qi, uint32_t rank) {
+template <class S>
+__device__ __forceinline__ void tq_release(S& sh, uint32_t qi, uint32_t rank) {
     if (rank == 0) mbar_arrive(&sh.tq_empty[qi]);
     else mbar_arrive_release_cluster(cluster_smem_addr(&sh.tq_empty[qi], 0));
 }
 // Next work item for a whole consumer warp. False when a wait ran out.
-__device__ __forceinline__ bool next_tile_warp(Shared& sh, uint32_t rank, uint32_t& qi, uint32_t& qphase, int32_t& w,
+template <class S>
+__device__ __forceinline__ bool next_tile_warp(S& sh, uint32_t rank, uint32_t& qi, uint32_t& qphase, int32_t& w,
                                                int lane, volatile int* abort, const DeviceCtl& ctl) {
     const bool ok = __all_sync(0xFFFFFFFFu, tq_wait(sh, qi, qphase, rank, abort, ctl));
     if (!ok) return false;
@@ -170,7 +204,8 @@ __device__ __forceinline__ bool next_tile_warp(Shared& sh, uint32_t rank, uint32
     return true;
 }
 // Next work item for one thread (the odd CTA's producer).
-__device__ __forceinline__ bool next_tile_thread(Shared& sh, uint32_t rank, uint32_t& qi, uint32_t& qphase,
+template <class S>
+__device__ __forceinline__ bool next_tile_thread(S& sh, uint32_t rank, uint32_t& qi, uint32_t& qphase,
                                                  int32_t& w, volatile int* abort, const DeviceCtl& ctl) {
     if (!tq_wait(sh, qi, qphase, rank, abort, ctl)) return false;
     w = *reinterpret_cast<volatile int32_t*>(&sh.tq[qi]);
@@ -179,7 +214,8 @@ __device__ __forceinline__ bool next_tile_thread(Shared& sh, uint32_t rank, uint
     return true;
 }
 // The even CTA's producer: take the next work item of the grid and publish it to both CTAs.
-__device__ __forceinline__ bool publish_tile(Shared& sh, const Params& p, int32_t total, uint32_t& qi,
+template <class S>
+__device__ __forceinline__ bool publish_tile(S& sh, const Params& p, int32_t total, uint32_t& qi,
                                              uint32_t& qphase, int32_t& w, volatile int* abort) {
     w = (int32_t)min(atomicAdd(p.sched, 1u), (uint32_t)total);
     if (!mbar_wait_bounded_acq_cluster(&sh.tq_empty[qi], qphase ^ 1u, abort, p.ctl)) return false;
@@ -208,7 +244,8 @@ __device__ __forceinline__ void weight_tiles(const Params& p, const Tile& t, uin
 }
 
 // Expert offsets and the first work item of each expert (every CTA builds its own copy).
-__device__ __forceinline__ void build_schedule(Shared& sh, const Params& p, int32_t n_col_tiles) {
+template <int kTail, class S>
+__device__ __forceinline__ void build_schedule(S& sh, const Params& p, int32_t n_col_tiles) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int32_t E = p.E;
     const int e0 = tid * 4;
@@ -222,7 +259,7 @@ __device__ __forceinline__ void build_schedule(Shared& sh, const Params& p, int3
         if (e < E) {
             const int32_t a = sh.off[e], b = sh.off[e + 1];
             if (a < 0 || b < a || (int64_t)b > p.max_rows) bad = true;  // inconsistent offsets: skip the expert
-            else cnt[i] = ((b - a + kBNMax - 1) / kBNMax) * n_col_tiles;
+            else cnt[i] = row_tiles<kTail>(b - a) * n_col_tiles;
         }
         local += cnt[i];
     }
@@ -257,15 +294,16 @@ __device__ __forceinline__ void build_schedule(Shared& sh, const Params& p, int3
 namespace nvfp4 {
 namespace gp {
 
-template <int kEpi>
+template <int kEpi, bool kTails>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_full,
                              const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_wsw,
                              const __grid_constant__ CUtensorMap tm_wsf, const Params p) {
+    using C = Cfg<kTails>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
-    Shared& sh = *reinterpret_cast<Shared*>(smem + (size_t)kStages * kStageBytes);
+    typename C::Shared& sh = *reinterpret_cast<typename C::Shared*>(smem + (size_t)C::kStages * C::kStageBytes);
     volatile int* abort = &sh.abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
@@ -285,7 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&tm_wsf);
         }
         sh.abort = 0;
-        for (int s = 0; s < kStages; s++) {
+        for (int s = 0; s < C::kStages; s++) {
             mbar_init(&sh.full_tma[s], 1);
             mbar_init(&sh.sf_ready[s], 8);
             mbar_init(&sh.empty[s], 1);
@@ -305,7 +343,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pdl_wait();
     for (int i = tid; i <= E; i += kThreads) sh.off[i] = __ldg(p.offsets + i);
     __syncthreads();
-    build_schedule(sh, p, n_col_tiles);
+    build_schedule<C::kTailMax>(sh, p, n_col_tiles);
     if (warp == 2) {
         tmem_alloc_pair(&sh.tmem_base, kTmemCols);
         tmem_relinquish_pair();
@@ -319,10 +357,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ================= loads of this CTA's halves =================
-        uint32_t issued_parity[kStages];
-        bool issued[kStages];
+        uint32_t issued_parity[C::kStages];
+        bool issued[C::kStages];
 #pragma unroll
-        for (int s = 0; s < kStages; s++) issued[s] = false, issued_parity[s] = 0;
+        for (int s = 0; s < C::kStages; s++) issued[s] = false, issued_parity[s] = 0;
         if (lane == 0 && !(p.ctl.flags & kCtlStallProducer)) {
             // L2: an expert's activation rows are re-read by each of its column tiles and stay hot on
             // their own; a weight tile is re-read only by the expert's other row tiles, which run
@@ -344,8 +382,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             while (ok && w < total) {
                 Tile t;
-                decode_tile(sh, E, w, t);
-                const uint64_t pol_w = (sh.off[t.e + 1] - sh.off[t.e] > kBNMax) ? pol_w_reuse : pol_w_once;
+                decode_tile<C::kTailMax>(sh, E, w, t);
+                const uint64_t pol_w = row_tiles<C::kTailMax>(sh.off[t.e + 1] - sh.off[t.e]) > 1 ? pol_w_reuse : pol_w_once;
                 // weight rows of this CTA, as (packed tile base, byte offset of the first row's codes)
                 const uint8_t* g_tile;   // NONE: this CTA's 128-row tile; SWIGLU: the gate tile
                 const uint8_t* u_tile;   // NONE: the other CTA's tile; SWIGLU: the up tile
@@ -358,11 +396,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint32_t a_bytes = p.swiglu ? (uint32_t)kCodeBytes + 2u * kTileSFBytes : (uint32_t)kPackedTileBytes;
                 // both CTAs stage the scales of all the tile's rows: one contiguous run of the K step's
                 // slab (K-stage layout), 16 bytes per row
-                const uint32_t tx = a_bytes + (uint32_t)my_rows * kRowBytes + (uint32_t)t.rows * 16u;
+                // (+ this CTA's 16 tail rows when the tile has a tail)
+                const uint32_t tx = a_bytes + (uint32_t)my_rows * kRowBytes +
+                                    (C::kTailMax > 0 && t.tail > 0 ? (C::kTailMax / 2) * kRowBytes : 0u) +
+                                    (uint32_t)t.rows * 16u;
                 const uint8_t* sfb = p.a_sf + (int64_t)t.row0 * 16;
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
                     if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort, p.ctl)) { ok = false; break; }
-                    uint8_t* sb = stages + (size_t)stage * kStageBytes;
+                    uint8_t* sb = stages + (size_t)stage * C::kStageBytes;
                     uint64_t* bar = &sh.full_tma[stage];
                     mbar_arrive_expect_tx(bar, tx);
                     const size_t ko = (size_t)kt * kPackedTileBytes;
@@ -383,10 +424,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             tma_load_2d(sb + kOffB + i * kBoxRows * kRowBytes, &tm_a, kt * kRowBytes,
                                         my_row0 + i * kBoxRows, bar, pol_a);
                     }
-                    bulk_load(sb + kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, bar, pol_a);
+                    if (C::kTailMax > 0 && t.tail > 0)
+                        tma_load_2d(sb + C::kOffBT, &tm_a, kt * kRowBytes, t.row0 + kBNMax + (int32_t)rank * (C::kTailMax / 2),
+                                    bar, pol_a);
+                    bulk_load(sb + C::kOffSFB, sfb + (int64_t)kt * p.max_rows * 16, (uint32_t)t.rows * 16u, bar, pol_a);
                     issued[stage] = true;
                     issued_parity[stage] = phase;
-                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 if (rank == 0) {
@@ -397,7 +441,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok || *abort) {
-                for (int s = 0; s < kStages; s++)
+                for (int s = 0; s < C::kStages; s++)
                     if (issued[s]) mbar_wait_drain(&sh.full_tma[s], issued_parity[s], 200000000ull);
             }
         }
@@ -412,16 +456,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int tile_row = p.swiglu ? (int)rank * 64 + quad * 16 + (lane & 15) : quad * 32 + lane;
         const uint32_t sfa_off = kOffSFA + ((p.swiglu && lane >= 16) ? kTileSFBytes : 0) + (tile_row & 31) * 16 +
                                  (tile_row >> 5) * 4;
-        uint32_t stage = 0, phase = 0, qi = 0, qphase = 0;
+        uint32_t stage = 0, phase = 0, qi = 0, qphase = 0, sfs = 0;
+        uint32_t count = 0;   // stages handled so far
         bool ok = true;
         while (ok) {
             int32_t w;
             if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl) || w >= total) break;
+            Tile t;
+            decode_tile<C::kTailMax>(sh, E, w, t);
             for (int32_t kt = 0; kt < ksteps_total; kt++) {
                 if (!warp_wait(&sh.full_tma[stage], phase, abort, p.ctl)) { ok = false; break; }
+                // the TMEM slot's previous stage (C::kSFSlots back) has had its MMAs completed
+                if (C::kSFSlots < C::kStages && count >= (uint32_t)C::kSFSlots) {
+                    const uint32_t c0 = count - C::kSFSlots;
+                    if (!warp_wait(&sh.empty[c0 % C::kStages], (c0 / C::kStages) & 1u, abort, p.ctl)) { ok = false; break; }
+                }
                 tc_fence_after();
-                const uint8_t* sb = stages + (size_t)stage * kStageBytes;
-                const uint32_t slot = tmem + lane_addr + kTmemSFRing + stage * kSFSlot;
+                const uint8_t* sb = stages + (size_t)stage * C::kStageBytes;
+                const uint32_t slot = tmem + lane_addr + C::kTmemSFRing + sfs * C::kSFSlot;
                 // SFA: one column per K-step, the one this quadrant's rows are read from (the other three
                 // columns of the step belong to the other quadrants; measured: 1% faster than writing all four)
 #pragma unroll
@@ -430,33 +482,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 uint32_t v32[32];
 #pragma unroll
                 for (int g = 0; g < 8; g++) {
-                    const uint4 x = *reinterpret_cast<const uint4*>(sb + kOffSFB + (32 * g + lane) * 16);
+                    const uint4 x = *reinterpret_cast<const uint4*>(sb + C::kOffSFB + (32 * g + lane) * 16);
                     v32[g] = x.x;
                     v32[8 + g] = x.y;
                     v32[16 + g] = x.z;
                     v32[24 + g] = x.w;
                 }
                 tmem_st_32x32b_x32(slot + 16, v32);
+                if (C::kTailMax > 0 && t.tail > 0) {
+                    // tail SFB: tail row 256 + r at lane r of every quadrant, one column per K step
+                    const uint4 x = *reinterpret_cast<const uint4*>(sb + C::kOffSFB + (kBNMax + lane) * 16);
+                    tmem_st_32x32b_x1(slot + C::kSFTail, x.x);
+                    tmem_st_32x32b_x1(slot + C::kSFTail + 4, x.y);
+                    tmem_st_32x32b_x1(slot + C::kSFTail + 8, x.z);
+                    tmem_st_32x32b_x1(slot + C::kSFTail + 12, x.w);
+                }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) arrive_on_leader(&sh.sf_ready[stage], rank);
-                if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                if (++sfs == (uint32_t)C::kSFSlots) sfs = 0;
+                count++;
             }
         }
     } else if (warp == 2) {
         // ================= MMA issuer (even CTA) =================
         if (rank == 0) {
             const uint32_t idesc_base = (1u << 7) | (1u << 10) | ((uint32_t)((2 * kBM) >> 4) << 24);
-            uint32_t stage = 0, phase = 0, aphase = 0, qi = 0, qphase = 0;
+            const uint32_t idesc_tail = idesc_base | ((uint32_t)(C::kTailMax >> 3) << 17);
+            uint32_t stage = 0, phase = 0, aphase = 0, qi = 0, qphase = 0, sfs = 0;
             bool ok = true;
             while (ok) {
                 int32_t w;
                 if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl)) { ok = false; break; }
                 if (w >= total) break;
                 Tile t;
-                decode_tile(sh, E, w, t);
+                decode_tile<C::kTailMax>(sh, E, w, t);
                 const uint32_t idesc = idesc_base | ((uint32_t)(t.bn >> 3) << 17);
+                const bool tail = C::kTailMax > 0 && t.tail > 0;
                 if (!warp_wait(&sh.acc_empty, aphase ^ 1u, abort, p.ctl)) { ok = false; break; }
                 tc_fence_after();
                 for (int32_t kt = 0; kt < ksteps_total; kt++) {
@@ -468,25 +532,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t sb = smem_u32(stages + (size_t)stage * kStageBytes);
-                        const uint32_t sf = tmem + kTmemSFRing + stage * kSFSlot;
+                        const uint32_t sb = smem_u32(stages + (size_t)stage * C::kStageBytes);
+                        const uint32_t sf = tmem + C::kTmemSFRing + sfs * C::kSFSlot;
+                        // the tile's 256 columns, and the tail rows into columns 256-287
+                        auto mma_step = [&](int kc) {
+                            const uint64_t adesc = make_smem_desc(sb + kOffA + kc * 32, 16, 1024, 2);
+                            mma_mxf4nvf4_pair(tmem, adesc, make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2), idesc,
+                                              sf + 4 * kc, sf + 16 + 8 * kc, (kt | kc) != 0);
+                            if (tail)
+                                mma_mxf4nvf4_pair(tmem + kBNMax, adesc, make_smem_desc(sb + C::kOffBT + kc * 32, 16, 1024, 2),
+                                                  idesc_tail, sf + 4 * kc, sf + C::kSFTail + 4 * kc, (kt | kc) != 0);
+                        };
                         if (kt != ksteps_total - 1 || last_ksteps == kKSteps) {
 #pragma unroll
-                            for (int kc = 0; kc < kKSteps; kc++)
-                                mma_mxf4nvf4_pair(tmem, make_smem_desc(sb + kOffA + kc * 32, 16, 1024, 2),
-                                                  make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2), idesc,
-                                                  sf + 4 * kc, sf + 16 + 8 * kc, (kt | kc) != 0);
+                            for (int kc = 0; kc < kKSteps; kc++) mma_step(kc);
                         } else {
                             // a last stage of 128 K-elements: its first two K-steps
-                            for (int kc = 0; kc < last_ksteps; kc++)
-                                mma_mxf4nvf4_pair(tmem, make_smem_desc(sb + kOffA + kc * 32, 16, 1024, 2),
-                                                  make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2), idesc,
-                                                  sf + 4 * kc, sf + 16 + 8 * kc, (kt | kc) != 0);
+                            for (int kc = 0; kc < last_ksteps; kc++) mma_step(kc);
                         }
                         tc_commit_pair_both(&sh.empty[stage]);
                     }
                     __syncwarp();
-                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+                    if (++sfs == (uint32_t)C::kSFSlots) sfs = 0;
                 }
                 if (!ok) break;
                 if (lane == 0) {
@@ -529,13 +597,118 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int32_t w;
             if (!next_tile_warp(sh, rank, qi, qphase, w, lane, abort, p.ctl) || w >= total) break;
             Tile t;
-            decode_tile(sh, E, w, t);
+            decode_tile<C::kTailMax>(sh, E, w, t);
             if (!warp_wait(&sh.acc_full, aphase, abort, p.ctl)) break;
             tc_fence_after();
             const float alpha = a_g * __ldg(p.w_gscale + t.e);
-            // 1. Drain: this warp's chunks (c = half, half + 2, ...) become final BF16 values in registers,
-            //    two per word (SWIGLU: 16 outputs per chunk, NONE: 32), and the accumulator goes back to
-            //    the MMA warp at once: the next tile's main loop runs while 2. stages and stores them.
+            // Chunk c (columns [32 c, +32), tokens row0 + 32 c ...) as final BF16 values, two per word
+            // (SWIGLU: 16 outputs per lane, NONE: 32); quantised h is written here directly
+            auto finish = [&](int c, const float (&v)[32], uint32_t (&pk)[16]) {
+                const int nrows = min(32, t.rows - c * 32);
+                if (p.swiglu) {
+                    // lane l < 16 holds gate, lane l + 16 up, of output column 16 quad + l; lane l
+                    // produces the even tokens, lane l + 16 the odd ones
+#pragma unroll
+                    for (int j = 0; j < 16; j++) {
+                        const float send = up_lane ? v[2 * j] : v[2 * j + 1];
+                        const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
+                        const float g = alpha * (up_lane ? recv : v[2 * j]);
+                        const float u = alpha * (up_lane ? v[2 * j + 1] : recv);
+                        const uint32_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(swiglu_f32(g, u)));
+                        const bool valid = 2 * j + (up_lane ? 1 : 0) < nrows;
+                        if (valid) amax = max(amax, hb & 0x7FFFu);
+                        if (kEpi == kEpiQuant) {
+                            // h as NVFP4: lanes 0-15 hold one 16-column block of token 2j, lanes 16-31
+                            // the same block of token 2j + 1
+                            uint32_t code;
+                            const uint32_t S = quantize_half_warp_block(hb, valid, h_genc, code);
+                            const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, code, 1);
+                            const int64_t hcols = p.N / 2;
+                            const int64_t n = (int64_t)t.nt * kBM + (int64_t)rank * 64 + quad * 16 + (lane & 15);
+                            const int64_t row = (int64_t)t.row0 + c * 32 + 2 * j + (up_lane ? 1 : 0);
+                            if (valid && (lane & 1) == 0)
+                                p.qo.q[row * (hcols / 2) + n / 2] = (uint8_t)(code | (hi << 4));
+                            if (valid && (lane & 15) == 0) {
+                                const int64_t b = n >> 4;
+                                uint8_t* piece = p.qo.sf + ((b >> 4) * p.qo.rows_per_slab + row) * 16;
+                                piece[b & 15] = (uint8_t)S;
+                                if ((hcols & 255) == 128 && b == (hcols >> 4) - 1)   // the last slab's padding
+                                    *reinterpret_cast<uint2*>(piece + 8) = make_uint2(0u, 0u);
+                            }
+                        }
+                        if (j & 1) pk[j >> 1] |= hb << 16;
+                        else pk[j >> 1] = hb;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const uint32_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i]));
+                        const uint32_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i + 1]));
+                        if (i < nrows) amax = max(amax, b0 & 0x7FFFu);
+                        if (i + 1 < nrows) amax = max(amax, b1 & 0x7FFFu);
+                        pk[i >> 1] = b0 | (b1 << 16);
+                    }
+                }
+            };
+            // Chunk c staged as a 32-token block in shared memory and stored
+            auto store = [&](int c, const uint32_t (&pk)[16]) {
+                const int nrows = min(32, t.rows - c * 32);
+                const int32_t r0 = t.row0 + c * 32;
+                // the previous chunk's tensor store has finished reading the staging block
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+                int32_t col;      // first output column of this warp's block
+                int lane_cols;    // lanes per 16-byte row piece in the direct-store path: 2 (SwiGLU) or 4
+                if (p.swiglu) {
+#pragma unroll
+                    for (int j = 0; j < 16; j++)
+                        stg[(2 * j + (up_lane ? 1 : 0)) * 16 + (lane & 15)] =
+                            (uint16_t)((j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu));
+                    col = t.nt * kBM + (int32_t)rank * 64 + quad * 16;
+                    lane_cols = 2;
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; i++)
+                        stg[i * 32 + lane] = (uint16_t)((i & 1) ? (pk[i >> 1] >> 16) : (pk[i >> 1] & 0xFFFFu));
+                    col = t.nt * 2 * kBM + (int32_t)rank * kBM + quad * 32;
+                    lane_cols = 4;
+                }
+                if (nrows == 32 && kEpi != kEpiFinalize) {
+                    // a whole chunk of the expert: one asynchronous tensor store of the block
+                    // (the fused combine stores directly: its last arrivers read these rows back)
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tm_out, stg, col, r0);
+                        bulk_commit_group();
+                    }
+                } else {
+                    // the expert's last, partial chunk: rows past its end belong to the next expert
+                    __syncwarp();
+                    const int64_t ldo = p.swiglu ? p.N / 2 : p.N;
+                    const int row_elems = 8 * lane_cols;
+                    const int rows_per_pass = 32 / lane_cols;
+                    for (int r = lane / lane_cols; r < nrows; r += rows_per_pass) {
+                        const int piece = 8 * (lane % lane_cols);
+                        *reinterpret_cast<uint4*>(p.out + (int64_t)(r0 + r) * ldo + col + piece) =
+                            *reinterpret_cast<const uint4*>(stg + r * row_elems + piece);
+                    }
+                    __syncwarp();
+                }
+            };
+            // 0. The tail rows (columns 256-287), on tiles that have them: warps 4-7 finish and store them
+            //    while the accumulator is still held
+            if (C::kTailMax > 0 && half == 0 && t.tail > 0) {
+                float v[32];
+                tmem_ld_32x32b_x32(tmem + lane_base + kBNMax, v);
+                tmem_ld_wait();
+                uint32_t pkt[16];
+                finish(kBNMax / 32, v, pkt);
+                if (kEpi != kEpiQuant) store(kBNMax / 32, pkt);
+            }
+            // 1. Drain: this warp's chunks (c = half, half + 2, ...) become final values in registers, and
+            //    the accumulator goes back to the MMA warp at once: the next tile's main loop runs while 2.
+            //    stages and stores them.
             uint32_t pk[kChunksPerWarp][16];
 #pragma unroll
             for (int ci = 0; ci < kChunksPerWarp; ci++) {
@@ -544,107 +717,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     float v[32];
                     tmem_ld_32x32b_x32(tmem + lane_base + c * 32, v);
                     tmem_ld_wait();
-                    const int nrows = min(32, t.rows - c * 32);
-                    if (p.swiglu) {
-                        // lane l < 16 holds gate, lane l + 16 up, of output column 16 quad + l; lane l
-                        // produces the even tokens, lane l + 16 the odd ones
-#pragma unroll
-                        for (int j = 0; j < 16; j++) {
-                            const float send = up_lane ? v[2 * j] : v[2 * j + 1];
-                            const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
-                            const float g = alpha * (up_lane ? recv : v[2 * j]);
-                            const float u = alpha * (up_lane ? v[2 * j + 1] : recv);
-                            const uint32_t hb = __bfloat16_as_ushort(__float2bfloat16_rn(swiglu_f32(g, u)));
-                            const bool valid = 2 * j + (up_lane ? 1 : 0) < nrows;
-                            if (valid) amax = max(amax, hb & 0x7FFFu);
-                            if (kEpi == kEpiQuant) {
-                                // h as NVFP4: lanes 0-15 hold one 16-column block of token 2j, lanes 16-31
-                                // the same block of token 2j + 1
-                                uint32_t code;
-                                const uint32_t S = quantize_half_warp_block(hb, valid, h_genc, code);
-                                const uint32_t hi = __shfl_xor_sync(0xFFFFFFFFu, code, 1);
-                                const int64_t hcols = p.N / 2;
-                                const int64_t n = (int64_t)t.nt * kBM + (int64_t)rank * 64 + quad * 16 + (lane & 15);
-                                const int64_t row = (int64_t)t.row0 + c * 32 + 2 * j + (up_lane ? 1 : 0);
-                                if (valid && (lane & 1) == 0)
-                                    p.qo.q[row * (hcols / 2) + n / 2] = (uint8_t)(code | (hi << 4));
-                                if (valid && (lane & 15) == 0) {
-                                    const int64_t b = n >> 4;
-                                    uint8_t* piece = p.qo.sf + ((b >> 4) * p.qo.rows_per_slab + row) * 16;
-                                    piece[b & 15] = (uint8_t)S;
-                                    if ((hcols & 255) == 128 && b == (hcols >> 4) - 1)   // the last slab's padding
-                                        *reinterpret_cast<uint2*>(piece + 8) = make_uint2(0u, 0u);
-                                }
-                            }
-                            if (j & 1) pk[ci][j >> 1] |= hb << 16;
-                            else pk[ci][j >> 1] = hb;
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            const uint32_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i]));
-                            const uint32_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i + 1]));
-                            if (i < nrows) amax = max(amax, b0 & 0x7FFFu);
-                            if (i + 1 < nrows) amax = max(amax, b1 & 0x7FFFu);
-                            pk[ci][i >> 1] = b0 | (b1 << 16);
-                        }
-                    }
+                    finish(c, v, pk[ci]);
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) arrive_on_leader(&sh.acc_empty, rank);
-            // 2. Write out: per chunk, stage a 32-token block in shared memory and store it (quantised h was
-            //    written in 1.)
+            // 2. Write out
 #pragma unroll
             for (int ci = 0; ci < kChunksPerWarp; ci++) {
                 if (kEpi == kEpiQuant) break;
                 const int c = half + 2 * ci;
-                if (c * 32 < t.bn) {
-                    const int nrows = min(32, t.rows - c * 32);
-                    const int32_t r0 = t.row0 + c * 32;
-                    // the previous chunk's tensor store has finished reading the staging block
-                    if (lane == 0) bulk_wait_group_read0();
-                    __syncwarp();
-                    int32_t col;      // first output column of this warp's block
-                    int lane_cols;    // lanes per 16-byte row piece in the direct-store path: 2 (SwiGLU) or 4
-                    if (p.swiglu) {
-#pragma unroll
-                        for (int j = 0; j < 16; j++)
-                            stg[(2 * j + (up_lane ? 1 : 0)) * 16 + (lane & 15)] =
-                                (uint16_t)((j & 1) ? (pk[ci][j >> 1] >> 16) : (pk[ci][j >> 1] & 0xFFFFu));
-                        col = t.nt * kBM + (int32_t)rank * 64 + quad * 16;
-                        lane_cols = 2;
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; i++)
-                            stg[i * 32 + lane] = (uint16_t)((i & 1) ? (pk[ci][i >> 1] >> 16) : (pk[ci][i >> 1] & 0xFFFFu));
-                        col = t.nt * 2 * kBM + (int32_t)rank * kBM + quad * 32;
-                        lane_cols = 4;
-                    }
-                    if (nrows == 32 && kEpi != kEpiFinalize) {
-                        // a whole chunk of the expert: one asynchronous tensor store of the block
-                        // (the fused combine stores directly: its last arrivers read these rows back)
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&tm_out, stg, col, r0);
-                            bulk_commit_group();
-                        }
-                    } else {
-                        // the expert's last, partial chunk: rows past its end belong to the next expert
-                        __syncwarp();
-                        const int64_t ldo = p.swiglu ? p.N / 2 : p.N;
-                        const int row_elems = 8 * lane_cols;
-                        const int rows_per_pass = 32 / lane_cols;
-                        for (int r = lane / lane_cols; r < nrows; r += rows_per_pass) {
-                            const int piece = 8 * (lane % lane_cols);
-                            *reinterpret_cast<uint4*>(p.out + (int64_t)(r0 + r) * ldo + col + piece) =
-                                *reinterpret_cast<const uint4*>(stg + r * row_elems + piece);
-                        }
-                        __syncwarp();
-                    }
-                }
+                if (c * 32 < t.bn) store(c, pk[ci]);
             }
             aphase ^= 1u;
             if (kEpi == kEpiFinalize) {
@@ -653,19 +737,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // for these columns (see the one-SM kernel: the result does not depend on the order).
                 __threadfence();                            // this thread's y stores, device-wide, first
                 if (!epi_sync()) break;
-                const int i = (half * 4 + quad) * 32 + lane;
-                int32_t tok = -1;
-                if (i < t.rows) {
-                    const int32_t tk = __ldg(p.fin.src + t.row0 + i);
-                    if (tk >= 0 && tk < p.fin.T) {
-                        uint32_t* cnt = p.fin.counters + (int64_t)tk * p.fin.col_blocks + 2 * t.nt + rank;
-                        if (atomicAdd(cnt, 1u) == (uint32_t)(p.fin.k - 1)) {
-                            atomicExch(cnt, 0u);            // left at zero for the next launch
-                            tok = tk;
+                for (int i = (half * 4 + quad) * 32 + lane; i < kBNMax + C::kTailMax; i += 32 * kEpiWarps) {
+                    int32_t tok = -1;
+                    if (i < t.rows) {
+                        const int32_t tk = __ldg(p.fin.src + t.row0 + i);
+                        if (tk >= 0 && tk < p.fin.T) {
+                            uint32_t* cnt = p.fin.counters + (int64_t)tk * p.fin.col_blocks + 2 * t.nt + rank;
+                            if (atomicAdd(cnt, 1u) == (uint32_t)(p.fin.k - 1)) {
+                                atomicExch(cnt, 0u);            // left at zero for the next launch
+                                tok = tk;
+                            }
                         }
                     }
+                    sh.fin_tok[i] = tok;
                 }
-                sh.fin_tok[i] = tok;
                 __threadfence();                            // the other rows' stores are visible before the reads
                 if (!epi_sync()) break;
                 // one half-warp per token: lane l combines columns [8 (l % 16), +8) of this CTA's 128
@@ -705,44 +790,39 @@ using namespace nvfp4;
 
 namespace nvfp4 {
 
-size_t pair_gemm_smem_bytes() { return gp::kSmemBytes; }
+size_t pair_gemm_smem_bytes() {
+    return gp::Cfg<true>::kSmemBytes > gp::Cfg<false>::kSmemBytes ? gp::Cfg<true>::kSmemBytes
+                                                                  : gp::Cfg<false>::kSmemBytes;
+}
 int pair_gemm_tokens_max() { return gp::kBNMax; }
 int pair_gemm_store_cols(int swiglu) { return swiglu ? 16 : 32; }  // 32 tokens x this many BF16 columns
 
 // The shared-memory opt-in of one instantiation, once per device (thread-safe).
-template <int kEpi>
+template <int kEpi, bool kTails>
 static bool pair_kernel_configured(int dev) {
     static std::once_flag once[64];
     static bool ok[64] = {};
     std::call_once(once[dev], [&] {
-        ok[dev] = cudaFuncSetAttribute(gp::grouped_gemm_pair_kernel<kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)gp::kSmemBytes) == cudaSuccess;
+        ok[dev] = cudaFuncSetAttribute(gp::grouped_gemm_pair_kernel<kEpi, kTails>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)gp::Cfg<kTails>::kSmemBytes) == cudaSuccess;
     });
     return ok[dev];
 }
 
-// Launches the pair kernel; the caller validated every argument (same contract as the one-SM kernel).
-nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full,
-                                      const CUtensorMap& tm_out, const CUtensorMap& tm_wsw,
-                                      const CUtensorMap& tm_wsf, const uint8_t* a_sf,
-                                      const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
-                                      const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
-                                      int swiglu, uint16_t* out, uint32_t* out_amax, const Finalize& fin,
-                                      const QuantOut& qo, cudaStream_t s, uint32_t* status) {
-    // once per device (thread-safe): the shared-memory opt-in and the persistent grid size
+// As many pairs as can be resident at once (the persistent grid), once per device and configuration.
+template <bool kTails>
+static nvfp4_status pair_grid(int dev, int& grid) {
     static std::once_flag once[64];
     static int grid_for[64] = {};
     static nvfp4_status set_result[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
     std::call_once(once[dev], [&] {
         set_result[dev] = NVFP4_ERR_CUDA;
-        if (!pair_kernel_configured<kEpiPlain>(dev)) return;
-        // as many pairs as can be resident at once (persistent grid)
+        if (!pair_kernel_configured<kEpiPlain, kTails>(dev)) return;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)device_sm_count() / 2 * 2);
         cfg.blockDim = dim3(gp::kThreads);
-        cfg.dynamicSmemBytes = gp::kSmemBytes;
+        cfg.dynamicSmemBytes = gp::Cfg<kTails>::kSmemBytes;
         cudaLaunchAttribute attr;
         attr.id = cudaLaunchAttributeClusterDimension;
         attr.val.clusterDim.x = 2;
@@ -751,7 +831,8 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, gp::grouped_gemm_pair_kernel<kEpiPlain>, &cfg) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveClusters(&clusters, gp::grouped_gemm_pair_kernel<kEpiPlain, kTails>, &cfg) !=
+                cudaSuccess ||
             clusters <= 0) {
             set_result[dev] = NVFP4_ERR_SMEM_BUDGET;
             return;
@@ -759,7 +840,46 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
         grid_for[dev] = 2 * clusters < device_sm_count() ? 2 * clusters : device_sm_count() / 2 * 2;
         set_result[dev] = NVFP4_OK;
     });
-    if (set_result[dev] != NVFP4_OK) return set_result[dev];
+    grid = grid_for[dev];
+    return set_result[dev];
+}
+
+template <bool kTails>
+static nvfp4_status launch_pair_config(int dev, const CUtensorMap& tm_a, const CUtensorMap& tm_a_full,
+                                       const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const CUtensorMap& tm_wsf,
+                                       const gp::Params& prm, cudaStream_t s) {
+    int grid = 0;
+    const nvfp4_status st = pair_grid<kTails>(dev, grid);
+    if (st != NVFP4_OK) return st;
+    const size_t smem = gp::Cfg<kTails>::kSmemBytes;
+    // every instantiation has the plain one's resources (same shared memory, threads and cluster shape)
+    if (prm.qo.q != nullptr) {
+        if (!pair_kernel_configured<kEpiQuant, kTails>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiQuant, kTails>, dim3(grid), dim3(gp::kThreads), smem, s, tm_a,
+                   tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+    } else if (prm.fin.out != nullptr) {
+        if (!pair_kernel_configured<kEpiFinalize, kTails>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiFinalize, kTails>, dim3(grid), dim3(gp::kThreads), smem, s, tm_a,
+                   tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+    } else {
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain, kTails>, dim3(grid), dim3(gp::kThreads), smem, s, tm_a,
+                   tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+    }
+    return NVFP4_OK;
+}
+
+// Launches the pair kernel; the caller validated every argument (same contract as the one-SM kernel).
+// Several experts: the configuration that lets up to 32 rows past a full tile ride on it; one expert
+// (a dense GEMM): the deeper pipeline without that.
+nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full,
+                                      const CUtensorMap& tm_out, const CUtensorMap& tm_wsw,
+                                      const CUtensorMap& tm_wsf, const uint8_t* a_sf,
+                                      const float* a_gscale, const uint8_t* w_packed, const float* w_gscale,
+                                      const int32_t* offsets, int32_t E, int64_t max_rows, int64_t N, int64_t K,
+                                      int swiglu, uint16_t* out, uint32_t* out_amax, const Finalize& fin,
+                                      const QuantOut& qo, cudaStream_t s, uint32_t* status) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
     gp::Params prm;
     prm.a_sf = a_sf;
     prm.a_gscale = a_gscale;
@@ -780,19 +900,9 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
-    // every instantiation has the plain one's resources (same shared memory, threads and cluster shape)
-    if (qo.q != nullptr) {
-        if (!pair_kernel_configured<kEpiQuant>(dev)) return NVFP4_ERR_CUDA;
-        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiQuant>, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes, s,
-                   tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
-    } else if (fin.out != nullptr) {
-        if (!pair_kernel_configured<kEpiFinalize>(dev)) return NVFP4_ERR_CUDA;
-        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiFinalize>, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes,
-                   s, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
-    } else {
-        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain>, dim3(grid_for[dev]), dim3(gp::kThreads), gp::kSmemBytes, s,
-                   tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
-    }
+    const nvfp4_status st = E > 1 ? launch_pair_config<true>(dev, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm, s)
+                                  : launch_pair_config<false>(dev, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm, s);
+    if (st != NVFP4_OK) return st;
     count_launch();
     return check_launch();
 }

@@ -118,6 +118,17 @@ def test_pair_tiles_ragged(swiglu):
 
 
 @pytest.mark.parametrize("swiglu", [False, True])
+@pytest.mark.parametrize("K", [512, 384])
+def test_pair_tiles_tail_rows(swiglu, K):
+    # an expert's rows past its last full 256-row tile ride on that tile when there are at most 32 of them
+    # (a second MMA into accumulator columns 256-287): 256 (no tail), 257 / 272 / 288 (tails of 1, 16, 32),
+    # 289 (a tile of its own), 512 + 1 and 512 + 32 (tail on the second tile), 545 (third tile), with
+    # K % 256 == 128 (a last stage of two K-steps) as well
+    rows = [256, 257, 272, 288, 289, 513, 544, 545]
+    run_full(rows, 512, K, swiglu, seed=13)
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
 def test_pair_tiles_small_ragged_experts(swiglu):
     # padding the activations to 192 rows per expert selects the CTA-pair kernel for experts of 1-33 rows:
     # one-row tiles, a 32-row tile (one full N step), 33 rows (two N steps), an empty expert
