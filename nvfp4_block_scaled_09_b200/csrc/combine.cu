@@ -5,7 +5,7 @@
 //   out[t, :] = BF16( sum_{j ascending} w[t, j] * y[inv_perm[t*k + j], :] )
 //
 // Memory bound (reads k rows of y per token, writes one row): each thread owns
-// 8 consecutive columns (16-byte loads and stores). The sum is accumulated in
+// 8 consecutive columns (16-byte loads and stores; combine_vec8). The sum is accumulated in
 // FP64: a product of an FP32 weight and a BF16 value has at most 32
 // significant bits, so every product is exact and the only roundings are the
 // FP64 additions and one final rounding to BF16 (through round-to-odd FP32,
@@ -19,44 +19,18 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kColsPerThread = 8;
 
-__device__ __forceinline__ void acc_bf16x2(double& a0, double& a1, uint32_t w, double s) {
-    a0 = fma(s, (double)__uint_as_float(w << 16), a0);
-    a1 = fma(s, (double)__uint_as_float(w & 0xFFFF0000u), a1);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(double lo, double hi) {
-    return f64_to_bf16_bits(lo) | (f64_to_bf16_bits(hi) << 16);
-}
-
-__global__ void __launch_bounds__(kThreads) combine_kernel(const uint4* __restrict__ y,
+// One thread per (token, 16-byte column group): all of a token's k <= 8 slots are loaded before any is
+// accumulated, so the k row reads are in flight together (the combine is latency-bound at decode sizes).
+__global__ void __launch_bounds__(kThreads) combine_kernel(const uint16_t* __restrict__ y,
                                                            const int32_t* __restrict__ inv_perm,
                                                            const float* __restrict__ w, int64_t T, int32_t k,
-                                                           int64_t hvec, uint4* __restrict__ out) {
+                                                           int64_t H, uint16_t* __restrict__ out) {
     pdl_launch_dependents();
     pdl_wait();
     const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;  // 16-byte column group
-    if (c >= hvec) return;
-    for (int64_t t = blockIdx.y; t < T; t += gridDim.y) {
-        double a[kColsPerThread];
-#pragma unroll
-        for (int i = 0; i < kColsPerThread; i++) a[i] = 0.0;
-        for (int j = 0; j < k; j++) {
-            const int32_t p = __ldg(inv_perm + t * k + j);
-            if (p < 0) continue;
-            const double s = (double)__ldg(w + t * k + j);
-            const uint4 v = __ldcs(y + (int64_t)p * hvec + c);
-            acc_bf16x2(a[0], a[1], v.x, s);
-            acc_bf16x2(a[2], a[3], v.y, s);
-            acc_bf16x2(a[4], a[5], v.z, s);
-            acc_bf16x2(a[6], a[7], v.w, s);
-        }
-        uint4 o;
-        o.x = pack_bf16x2(a[0], a[1]);
-        o.y = pack_bf16x2(a[2], a[3]);
-        o.z = pack_bf16x2(a[4], a[5]);
-        o.w = pack_bf16x2(a[6], a[7]);
-        out[t * hvec + c] = o;
-    }
+    if (c * kColsPerThread >= H) return;
+    for (int64_t t = blockIdx.y; t < T; t += gridDim.y)
+        combine_vec8<8>(y, H, inv_perm, w, (int32_t)t, k, c * kColsPerThread, out, H);
 }
 
 }  // namespace
@@ -74,8 +48,8 @@ extern "C" nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* 
         return NVFP4_ERR_MISALIGNED;
     const int64_t hvec = H / kColsPerThread;
     dim3 grid((unsigned)((hvec + kThreads - 1) / kThreads), (unsigned)(T < 65535 ? T : 65535));  // tokens loop
-    launch_pdl(combine_kernel, dim3(grid), dim3(kThreads), 0, reinterpret_cast<cudaStream_t>(stream),
-        reinterpret_cast<const uint4*>(y), inv_perm, topk_w, (int64_t)T, k, hvec, reinterpret_cast<uint4*>(out));
+    launch_pdl(combine_kernel, dim3(grid), dim3(kThreads), 0, reinterpret_cast<cudaStream_t>(stream), y, inv_perm,
+               topk_w, (int64_t)T, k, H, out);
     count_launch();
     return check_launch();
 }

@@ -162,6 +162,23 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// mbar_wait_bounded for a wait known to be long: a pause of `pause_ns` between polls.
+__device__ __forceinline__ bool mbar_wait_bounded_pause(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                        const DeviceCtl& ctl, uint32_t pause_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(pause_ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > ctl.timeout_ns) {
+            *abort = 1;
+            atomicOr(ctl.status, kStatusTimeout);
+            return false;
+        }
+    }
+}
+
 // Drain wait used only on the abort path: bounded, never raises flags.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t budget_ns) {
     const uint64_t t0 = global_timer_ns();
@@ -424,26 +441,27 @@ __device__ __forceinline__ uint32_t f64_to_bf16_bits(double d) {
 // Eight adjacent output columns [col, col + 8) of the top-k weighted combine for token t: the sum over the
 // token's slots j ascending of w[t, j] * y[inv_perm[t*k + j], col..] in FP64 (each product of an FP32 weight and
 // a BF16 value is exact), negative rows skipped, rounded once to BF16 and stored as one 16-byte piece. The
-// slots are read in groups of four so their loads overlap; y is read past L1 (other SMs wrote it).
+// slots are read in groups of kGroup so their loads overlap; y is read past L1 (other SMs wrote it).
+template <int kGroup = 4>
 __device__ __forceinline__ void combine_vec8(const uint16_t* y, int64_t ldy, const int32_t* inv_perm, const float* w,
                                              int32_t t, int32_t k, int64_t col, uint16_t* out, int64_t ldo) {
     double a[8];
 #pragma unroll
     for (int i = 0; i < 8; i++) a[i] = 0.0;
-    for (int32_t j0 = 0; j0 < k; j0 += 4) {
-        int32_t p[4];
-        float s[4];
+    for (int32_t j0 = 0; j0 < k; j0 += kGroup) {
+        int32_t p[kGroup];
+        float s[kGroup];
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
+        for (int u = 0; u < kGroup; u++) {
             p[u] = j0 + u < k ? __ldg(inv_perm + (int64_t)t * k + j0 + u) : -1;
             s[u] = j0 + u < k ? __ldg(w + (int64_t)t * k + j0 + u) : 0.0f;
         }
-        uint4 v[4];
+        uint4 v[kGroup];
 #pragma unroll
-        for (int u = 0; u < 4; u++)
+        for (int u = 0; u < kGroup; u++)
             v[u] = p[u] >= 0 ? __ldcg(reinterpret_cast<const uint4*>(y + (int64_t)p[u] * ldy + col)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
+        for (int u = 0; u < kGroup; u++) {
             if (p[u] < 0) continue;
             const double sd = (double)s[u];
             const uint32_t x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
