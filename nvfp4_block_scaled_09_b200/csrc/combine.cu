@@ -19,8 +19,10 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kColsPerThread = 8;
 
-// One thread per (token, 16-byte column group): all of a token's k <= 8 slots are loaded before any is
-// accumulated, so the k row reads are in flight together (the combine is latency-bound at decode sizes).
+// Each thread owns one 16-byte column group and walks tokens blockIdx.y, + gridDim.y, ... (a grid of about
+// three CTAs per SM: no CTA churn). For k <= 8 the next token's slot indices and weights are loaded while
+// the current token's k rows are in flight, so a thread waits for one round of row reads per token (the
+// combine is bound by that latency when each thread handles one token per CTA). Larger k: combine_vec8.
 __global__ void __launch_bounds__(kThreads) combine_kernel(const uint16_t* __restrict__ y,
                                                            const int32_t* __restrict__ inv_perm,
                                                            const float* __restrict__ w, int64_t T, int32_t k,
@@ -29,8 +31,57 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const uint16_t* __res
     pdl_wait();
     const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;  // 16-byte column group
     if (c * kColsPerThread >= H) return;
-    for (int64_t t = blockIdx.y; t < T; t += gridDim.y)
-        combine_vec8<8>(y, H, inv_perm, w, (int32_t)t, k, c * kColsPerThread, out, H);
+    const int64_t col = c * kColsPerThread;
+    if (k > 8) {
+        for (int64_t t = blockIdx.y; t < T; t += gridDim.y)
+            combine_vec8<8>(y, H, inv_perm, w, (int32_t)t, k, col, out, H);
+        return;
+    }
+    int32_t p[8];
+    float s[8];
+    auto load_slots = [&](int64_t t) {
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            p[j] = j < k ? __ldg(inv_perm + t * k + j) : -1;
+            s[j] = j < k ? __ldg(w + t * k + j) : 0.0f;
+        }
+    };
+    int64_t t = blockIdx.y;
+    if (t < T) load_slots(t);
+    while (t < T) {
+        uint4 v[8];
+        float sc[8];
+        int32_t pc[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            pc[j] = p[j];
+            sc[j] = s[j];
+            v[j] = pc[j] >= 0 ? __ldcg(reinterpret_cast<const uint4*>(y + (int64_t)pc[j] * H + col)) : make_uint4(0, 0, 0, 0);
+        }
+        const int64_t tn = t + gridDim.y;
+        if (tn < T) load_slots(tn);   // the next token's slots, while this token's rows are in flight
+        double a[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) a[i] = 0.0;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {   // slots ascending (the oracle's order)
+            if (pc[j] < 0) continue;
+            const double sd = (double)sc[j];
+            const uint32_t x[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                a[2 * i] = fma(sd, (double)__uint_as_float(x[i] << 16), a[2 * i]);
+                a[2 * i + 1] = fma(sd, (double)__uint_as_float(x[i] & 0xFFFF0000u), a[2 * i + 1]);
+            }
+        }
+        uint4 o;
+        o.x = f64_to_bf16_bits(a[0]) | (f64_to_bf16_bits(a[1]) << 16);
+        o.y = f64_to_bf16_bits(a[2]) | (f64_to_bf16_bits(a[3]) << 16);
+        o.z = f64_to_bf16_bits(a[4]) | (f64_to_bf16_bits(a[5]) << 16);
+        o.w = f64_to_bf16_bits(a[6]) | (f64_to_bf16_bits(a[7]) << 16);
+        *reinterpret_cast<uint4*>(out + t * H + col) = o;
+        t = tn;
+    }
 }
 
 }  // namespace
@@ -47,7 +98,12 @@ extern "C" nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* 
     if (!aligned16(y) || !aligned16(out) || ((uintptr_t)inv_perm & 3u) || ((uintptr_t)topk_w & 3u))
         return NVFP4_ERR_MISALIGNED;
     const int64_t hvec = H / kColsPerThread;
-    dim3 grid((unsigned)((hvec + kThreads - 1) / kThreads), (unsigned)(T < 65535 ? T : 65535));  // tokens loop
+    // about three CTAs per SM in all (each thread walks tokens)
+    const int64_t gx = (hvec + kThreads - 1) / kThreads;
+    int64_t gy = ((int64_t)device_sm_count() * 3 + gx - 1) / gx;
+    if (gy > T) gy = T;
+    if (gy > 65535) gy = 65535;
+    dim3 grid((unsigned)gx, (unsigned)gy);
     launch_pdl(combine_kernel, dim3(grid), dim3(kThreads), 0, reinterpret_cast<cudaStream_t>(stream), y, inv_perm,
                topk_w, (int64_t)T, k, H, out);
     count_launch();
