@@ -135,7 +135,10 @@ __global__ void __launch_bounds__(kTok) permute_rank_kernel(const int32_t* __res
 // Small batches in one CTA (1024 threads) and one launch: count, scan and stable rank. Shared memory holds
 // one bit per (expert, token) and, per 32-token word, the number of the expert's pairs before that word
 // (the expert's offset included), so a pair's position is that prefix plus the popcount of the earlier
-// tokens in its word: token order inside each expert, as the multi-kernel path produces.
+// tokens in its word: token order inside each expert, as the multi-kernel path produces. Both tables are
+// word-major ([W][E]), so the per-expert passes read consecutive words across a warp; a thread keeps the
+// expert ids of its first kIdsCached pairs in registers for the second pass.
+constexpr int kIdsCached = 8;
 __global__ void __launch_bounds__(kMaxE) permute_small_kernel(const int32_t* __restrict__ ids, int32_t T, int32_t k,
                                                                 int32_t E, int32_t* __restrict__ offsets,
                                                                 int32_t* __restrict__ perm_src,
@@ -145,28 +148,37 @@ __global__ void __launch_bounds__(kMaxE) permute_small_kernel(const int32_t* __r
     extern __shared__ uint32_t small_sm[];
     __shared__ int32_t warp_sums[kMaxE / 32];
     const int W = (T + 31) / 32;                  // 32-token words per expert
-    uint32_t* bits = small_sm;                    // [E][W]
-    int32_t* pre = reinterpret_cast<int32_t*>(small_sm + (size_t)E * W);   // [E][W]
+    uint32_t* bits = small_sm;                    // [W][E]
+    int32_t* pre = reinterpret_cast<int32_t*>(small_sm + (size_t)E * W);   // [W][E]
     const int tid = threadIdx.x;
     for (int i = tid; i < E * W; i += kMaxE) bits[i] = 0u;
     __syncthreads();
     const int64_t R = (int64_t)T * k;
+    int32_t my_e[kIdsCached];
+#pragma unroll
+    for (int c = 0; c < kIdsCached; c++) {
+        const int64_t i = tid + (int64_t)c * kMaxE;
+        my_e[c] = i < R ? __ldg(ids + i) : -1;
+    }
     bool bad = false;
-    for (int64_t i = tid; i < R; i += kMaxE) {
+    auto mark = [&](int64_t i, int32_t e) {
         const int32_t t = (int32_t)(i / k);
-        const int32_t e = ids[i];
         if (e >= 0 && e < E) {
             const uint32_t bit = 1u << (t & 31);
-            if (atomicOr(&bits[e * W + (t >> 5)], bit) & bit) bad = true;   // expert listed twice by one token
+            if (atomicOr(&bits[(t >> 5) * E + e], bit) & bit) bad = true;   // expert listed twice by one token
         } else {
             bad = true;
         }
-    }
+    };
+#pragma unroll
+    for (int c = 0; c < kIdsCached; c++)
+        if (tid + (int64_t)c * kMaxE < R) mark(tid + (int64_t)c * kMaxE, my_e[c]);
+    for (int64_t i = tid + (int64_t)kIdsCached * kMaxE; i < R; i += kMaxE) mark(i, __ldg(ids + i));
     if (bad) atomicOr(status, kStatusBadInput);
     __syncthreads();
     int32_t total = 0;
     if (tid < E)
-        for (int w = 0; w < W; w++) total += __popc(bits[tid * W + w]);
+        for (int w = 0; w < W; w++) total += __popc(bits[w * E + tid]);
     // exclusive scan of the experts' totals
     const int lane = tid & 31, warp = tid >> 5;
     int32_t incl = total;
@@ -193,22 +205,25 @@ __global__ void __launch_bounds__(kMaxE) permute_small_kernel(const int32_t* __r
         if (tid == E - 1) offsets[E] = excl + total;
         int32_t run = excl;
         for (int w = 0; w < W; w++) {
-            pre[tid * W + w] = run;
-            run += __popc(bits[tid * W + w]);
+            pre[w * E + tid] = run;
+            run += __popc(bits[w * E + tid]);
         }
     }
     __syncthreads();
-    for (int64_t i = tid; i < R; i += kMaxE) {
+    auto place = [&](int64_t i, int32_t e) {
         const int32_t t = (int32_t)(i / k);
-        const int32_t e = ids[i];
         int32_t pos = -1;
         if (e >= 0 && e < E) {
             const int w = t >> 5;
-            pos = pre[e * W + w] + __popc(bits[e * W + w] & ((1u << (t & 31)) - 1u));
+            pos = pre[w * E + e] + __popc(bits[w * E + e] & ((1u << (t & 31)) - 1u));
             perm_src[pos] = t;
         }
         inv_perm[i] = pos;
-    }
+    };
+#pragma unroll
+    for (int c = 0; c < kIdsCached; c++)
+        if (tid + (int64_t)c * kMaxE < R) place(tid + (int64_t)c * kMaxE, my_e[c]);
+    for (int64_t i = tid + (int64_t)kIdsCached * kMaxE; i < R; i += kMaxE) place(i, __ldg(ids + i));
 }
 
 // One warp per output row; rows whose source index is invalid become zeros.
