@@ -565,6 +565,7 @@ void oracle_combine(const uint16_t* y, const int32_t* inv_perm, const float* w,
             double acc = 0.0;
             for (int32_t j = 0; j < k; j++) {
                 int64_t p = inv_perm[(int64_t)t * k + j];
+                if (p < 0) continue;   /* a pair without an expert row (the permute's -1) adds nothing */
                 acc += (double)w[(int64_t)t * k + j] * (double)oracle_bf16_to_float(y[p * H + h]);
             }
             out[(int64_t)t * H + h] = acc;

@@ -190,6 +190,25 @@ def test_combine_matches_einsum():
     assert np.allclose(oracle.combine(y, inv, w), want, rtol=1e-14, atol=1e-300)
 
 
+
+def test_combine_skips_pairs_without_a_row():
+    # a -1 slot (the permute's marker for a pair with an invalid expert) adds nothing: the combine equals the
+    # einsum over the remaining slots, and a token whose slots are all -1 gets zeros
+    T, k, H, E = 6, 3, 32, 6
+    ids, w = workloads.routing(T, E, k, "uniform", seed=6)
+    _, _, inv = oracle.permute(ids, E)
+    inv = inv.copy()
+    inv[1] = -1
+    inv[3 * k: 4 * k] = -1
+    y = workloads.random_bf16_bits((T * k, H), seed=7)
+    yf = oracle.bf16_bits_to_f64(y)
+    inv2 = inv.reshape(T, k)
+    keep = (inv2 >= 0).astype(np.float64)
+    want = np.einsum("tj,tjh->th", w.astype(np.float64) * keep, yf[np.maximum(inv2, 0)])
+    got = oracle.combine(y, inv, w)
+    assert np.allclose(got, want, rtol=1e-14, atol=1e-300)
+    assert np.all(got[3] == 0.0)
+
 # ---- the FP32-path error bound used to recognise rounding ties -------------------------------------------
 
 def _decoded(q, sf):
