@@ -71,7 +71,8 @@ typedef enum {
     NVFP4_ERR_CUDA = 6,              /* a CUDA runtime call or launch failed */
     NVFP4_ERR_DEVICE_TIMEOUT = 7,    /* (device) a bounded pipeline wait ran out */
     NVFP4_ERR_DEVICE_INPUT = 8       /* (device) expert id out of range, duplicate id in a
-                                        token's top-k, or inconsistent expert offsets */
+                                        token's top-k, inconsistent expert offsets, or a
+                                        combine row index past y */
 } nvfp4_status;
 
 typedef enum { NVFP4_EPI_NONE = 0, NVFP4_EPI_SWIGLU = 1 } nvfp4_epilogue;
@@ -332,7 +333,8 @@ NVFP4_API nvfp4_status nvfp4_pack_weights(const uint8_t* q, const uint8_t* sf, i
 /*   out[t, h] = BF16( sum_{j=0..k-1} topk_w[t, j] * y[inv_perm[t*k+j], h] ) */
 /*   accumulated in FP64 over j ascending (each FP32 x BF16 product is exact */
 /*   in FP64) and rounded once to BF16 (nearest even); a negative inv_perm   */
-/*   entry is skipped.                                                       */
+/*   entry is skipped, and so is an entry >= T*k (past the last row of y),  */
+/*   which also latches NVFP4_ERR_DEVICE_INPUT.                              */
 /* Arguments: y [T*k, H] BF16, inv_perm [T*k], topk_w [T, k] FP32, out [T, H]*/
 /*   BF16; y and out 16-byte aligned, inv_perm and topk_w 4-byte aligned;   */
 /*   all device; H % 8 == 0, 1 <= k <= 32, T >= 1.                           */

@@ -20,49 +20,38 @@ constexpr int kThreads = 256;
 constexpr int kColsPerThread = 8;
 
 // Each thread owns one 16-byte column group and walks tokens blockIdx.y, + gridDim.y, ... (a grid of about
-// three CTAs per SM: no CTA churn). For k <= 8 the next token's slot indices and weights are loaded while
-// the current token's k rows are in flight, so a thread waits for one round of row reads per token (the
-// combine is bound by that latency when each thread handles one token per CTA). Larger k: combine_vec8.
+// three CTAs per SM: no CTA churn). Slots go in groups of 8: a group's row indices and weights, then its
+// rows (all in flight together), then its FP64 sums in slot order. For k <= 8 (one group) the next token's
+// slot indices and weights are loaded while the current token's rows are in flight, so a thread waits for
+// one round of row reads per token (the combine is bound by that latency at decode sizes). A row index past
+// the last row of y is skipped and latched as bad input.
+template <bool kOneGroup>   // k <= 8
 __global__ void __launch_bounds__(kThreads) combine_kernel(const uint16_t* __restrict__ y,
                                                            const int32_t* __restrict__ inv_perm,
                                                            const float* __restrict__ w, int64_t T, int32_t k,
-                                                           int64_t H, uint16_t* __restrict__ out) {
+                                                           int64_t H, uint16_t* __restrict__ out, uint32_t* status) {
     pdl_launch_dependents();
     pdl_wait();
     const int64_t c = (int64_t)blockIdx.x * kThreads + threadIdx.x;  // 16-byte column group
     if (c * kColsPerThread >= H) return;
     const int64_t col = c * kColsPerThread;
-    if (k > 8) {
-        for (int64_t t = blockIdx.y; t < T; t += gridDim.y)
-            combine_vec8<8>(y, H, inv_perm, w, (int32_t)t, k, col, out, H);
-        return;
-    }
+    const int64_t R = T * k;
+    bool bad = false;
     int32_t p[8];
     float s[8];
-    auto load_slots = [&](int64_t t) {
+    auto load_slots = [&](int64_t t, int j0) {
 #pragma unroll
         for (int j = 0; j < 8; j++) {
-            p[j] = j < k ? __ldg(inv_perm + t * k + j) : -1;
-            s[j] = j < k ? __ldg(w + t * k + j) : 0.0f;
+            int32_t pj = j0 + j < k ? __ldg(inv_perm + t * k + j0 + j) : -1;
+            if (pj >= R) {
+                bad = true;
+                pj = -1;
+            }
+            p[j] = pj;
+            s[j] = j0 + j < k ? __ldg(w + t * k + j0 + j) : 0.0f;
         }
     };
-    int64_t t = blockIdx.y;
-    if (t < T) load_slots(t);
-    while (t < T) {
-        uint4 v[8];
-        float sc[8];
-        int32_t pc[8];
-#pragma unroll
-        for (int j = 0; j < 8; j++) {
-            pc[j] = p[j];
-            sc[j] = s[j];
-            v[j] = pc[j] >= 0 ? __ldcg(reinterpret_cast<const uint4*>(y + (int64_t)pc[j] * H + col)) : make_uint4(0, 0, 0, 0);
-        }
-        const int64_t tn = t + gridDim.y;
-        if (tn < T) load_slots(tn);   // the next token's slots, while this token's rows are in flight
-        double a[8];
-#pragma unroll
-        for (int i = 0; i < 8; i++) a[i] = 0.0;
+    auto accumulate = [&](const uint4 (&v)[8], const int32_t (&pc)[8], const float (&sc)[8], double (&a)[8]) {
 #pragma unroll
         for (int j = 0; j < 8; j++) {   // slots ascending (the oracle's order)
             if (pc[j] < 0) continue;
@@ -74,14 +63,41 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const uint16_t* __res
                 a[2 * i + 1] = fma(sd, (double)__uint_as_float(x[i] & 0xFFFF0000u), a[2 * i + 1]);
             }
         }
+    };
+    auto store = [&](int64_t t, const double (&a)[8]) {
         uint4 o;
         o.x = f64_to_bf16_bits(a[0]) | (f64_to_bf16_bits(a[1]) << 16);
         o.y = f64_to_bf16_bits(a[2]) | (f64_to_bf16_bits(a[3]) << 16);
         o.z = f64_to_bf16_bits(a[4]) | (f64_to_bf16_bits(a[5]) << 16);
         o.w = f64_to_bf16_bits(a[6]) | (f64_to_bf16_bits(a[7]) << 16);
         *reinterpret_cast<uint4*>(out + t * H + col) = o;
+    };
+    int64_t t = blockIdx.y;
+    if (kOneGroup && t < T) load_slots(t, 0);
+    while (t < T) {
+        const int64_t tn = t + gridDim.y;
+        double a[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) a[i] = 0.0;
+        for (int j0 = 0; j0 < (kOneGroup ? 1 : k); j0 += 8) {
+            if (!kOneGroup) load_slots(t, j0);
+            uint4 v[8];
+            float sc[8];
+            int32_t pc[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                pc[j] = p[j];
+                sc[j] = s[j];
+                v[j] = pc[j] >= 0 ? __ldcg(reinterpret_cast<const uint4*>(y + (int64_t)pc[j] * H + col))
+                                  : make_uint4(0, 0, 0, 0);
+            }
+            if (kOneGroup && tn < T) load_slots(tn, 0);   // the next token's slots, while these rows are in flight
+            accumulate(v, pc, sc, a);
+        }
+        store(t, a);
         t = tn;
     }
+    if (bad) atomicOr(status, kStatusBadInput);
 }
 
 }  // namespace
@@ -104,8 +120,10 @@ extern "C" nvfp4_status moe_unpermute_combine(const uint16_t* y, const int32_t* 
     if (gy > T) gy = T;
     if (gy > 65535) gy = 65535;
     dim3 grid((unsigned)gx, (unsigned)gy);
-    launch_pdl(combine_kernel, dim3(grid), dim3(kThreads), 0, reinterpret_cast<cudaStream_t>(stream), y, inv_perm,
-               topk_w, (int64_t)T, k, H, out);
+    uint32_t* status = status_word_ptr();
+    if (!status) return NVFP4_ERR_CUDA;
+    launch_pdl(k <= 8 ? combine_kernel<true> : combine_kernel<false>, dim3(grid), dim3(kThreads), 0,
+               reinterpret_cast<cudaStream_t>(stream), y, inv_perm, topk_w, (int64_t)T, k, H, out, status);
     count_launch();
     return check_launch();
 }

@@ -39,3 +39,31 @@ def test_one_hot_weights_select_rows_exactly():
     w[:, 1] = 1.0
     out = nv.unpermute_combine(gpu_bf16(y), torch.from_numpy(inv).cuda(), torch.from_numpy(w).cuda())
     assert np.array_equal(host_bits(out), y[inv.reshape(T, k)[:, 1]])
+
+
+def test_combine_chunked_rows_and_skipped_slots():
+    # k = 32 rows of 4000 columns do not fit one shared-memory stage: 1536-column chunks with a ragged last
+    # chunk (928 columns); slots marked -1 are skipped
+    T, E, k, H = 40, 64, 32, 4000
+    ids, w = workloads.routing(T, E, k, "uniform", seed=9)
+    _, _, inv = oracle.permute(ids, E)
+    inv = inv.copy()
+    inv[::7] = -1
+    y = workloads.random_bf16_bits((T * k, H), seed=10)
+    out = nv.unpermute_combine(gpu_bf16(y), torch.from_numpy(inv).cuda(), torch.from_numpy(w).cuda())
+    assert nv.device_status() == 0
+    assert np.array_equal(host_bits(out), oracle.bf16_round(oracle.combine(y, inv, w)))
+
+
+def test_combine_row_index_past_y_is_skipped_and_latched():
+    T, E, k, H = 16, 8, 4, 256
+    ids, w = workloads.routing(T, E, k, "uniform", seed=11)
+    _, _, inv = oracle.permute(ids, E)
+    y = workloads.random_bf16_bits((T * k, H), seed=12)
+    bad = inv.copy()
+    bad[5] = T * k + 3                                     # past the last row of y
+    out = nv.unpermute_combine(gpu_bf16(y), torch.from_numpy(bad).cuda(), torch.from_numpy(w).cuda())
+    assert nv.device_status() == 8                         # NVFP4_ERR_DEVICE_INPUT
+    skipped = inv.copy()
+    skipped[5] = -1
+    assert np.array_equal(host_bits(out), oracle.bf16_round(oracle.combine(y, skipped, w)))
