@@ -175,6 +175,27 @@ NVFP4_API nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k
                          void* ws, size_t ws_bytes, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* moe_quantize_permute: nvfp4_quantize(x) followed by moe_permute of the    */
+/* result, in one call: the same outputs, byte for byte (q_perm, sf_perm,    */
+/* g_x = the global scale nvfp4_quantize would return, expert_offsets,       */
+/* perm_src, inv_perm). Up to 32,768 pairs (and E * ceil(T/32) <= 20,480)   */
+/* it runs as two kernels -- the ranking beside the amax of x, then one that */
+/* quantises each token's row once and writes it to the token's k permuted */
+/* rows -- and never writes x's codes in token order; larger batches       */
+/* quantise into the workspace first. With an invalid expert id the rows   */
+/* past expert_offsets[E] are left unspecified (no pair maps to them).     */
+/* Arguments: x [T, H] BF16 (device, 16-byte aligned), H % 128 == 0; the     */
+/*   rest as moe_permute with K = H; g_x one FP32 (4-byte aligned); ws of    */
+/*   moe_quantize_permute_workspace_size() bytes (16-byte aligned).         */
+/* ------------------------------------------------------------------------ */
+NVFP4_API size_t moe_quantize_permute_workspace_size(int32_t T, int32_t k, int32_t E, int64_t H);
+NVFP4_API nvfp4_status moe_quantize_permute(const uint16_t* x, int32_t T, int64_t H, const int32_t* topk_ids,
+                                  int32_t k, int32_t E, uint8_t* q_perm, uint8_t* sf_perm,
+                                  nvfp4_sf_layout sf_perm_layout, float* g_x, int32_t* expert_offsets,
+                                  int32_t* perm_src, int32_t* inv_perm, void* ws, size_t ws_bytes,
+                                  nvfp4_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* moe_permute_noalloc: moe_permute without a caller workspace. No passage   */
 /* of the pages corresponds to it; it exists for callers that cannot hand    */
 /* the library any device memory of their own -- code running where         */

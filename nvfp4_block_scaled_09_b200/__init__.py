@@ -10,6 +10,7 @@ without a CUDA device the calls raise.
 Calls (same names as the C ABI):
   quantize            -> nvfp4_quantize
   permute             -> moe_permute
+  quantize_permute    -> moe_quantize_permute
   grouped_gemm        -> moe_grouped_gemm_nvfp4 (moe_grouped_gemm_nvfp4_amax with amax_out)
   quantize_from_amax  -> nvfp4_quantize_from_amax
   amax                -> nvfp4_amax
@@ -80,6 +81,10 @@ def lib():
         L.moe_permute_workspace_size.argtypes = [i32, i32, i32]
         L.moe_permute_workspace_size.restype = sz
         L.moe_permute.argtypes = [P, i32, i32, i32, P, P, i64, P, P, ctypes.c_int, P, P, P, P, sz, P]
+        L.moe_quantize_permute_workspace_size.argtypes = [i32, i32, i32, i64]
+        L.moe_quantize_permute_workspace_size.restype = sz
+        L.moe_quantize_permute.argtypes = [P, i32, i64, P, i32, i32, P, P, ctypes.c_int, P, P, P, P, P, sz, P]
+        L.moe_quantize_permute.restype = st
         L.moe_permute.restype = st
         L.moe_permute_noalloc.argtypes = [P, i32, i32, i32, P, P, i64, P, P, ctypes.c_int, P, P, P, P]
         L.moe_permute_noalloc.restype = st
@@ -340,6 +345,41 @@ def permute(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_exper
                              _ptr(out.sf_perm), sf_layout, _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm),
                              _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
     return out
+
+
+def quantize_permute(x: torch.Tensor, topk_ids: torch.Tensor, num_experts: int, ws=None, stream=None,
+                     sf_layout: int = SF_KSTAGE):
+    """quantize(x) then permute of the result in one call (moe_quantize_permute): the same bytes.
+    Returns (Permuted, g) with g the float32 [1] global scale of x."""
+    _require_cuda(x, topk_ids)
+    if topk_ids.dtype != torch.int32:
+        raise TypeError("topk_ids must be int32")
+    topk_ids = topk_ids.contiguous()
+    T, k = topk_ids.shape
+    if x.dim() != 2 or x.shape[0] != T:
+        raise ValueError(f"x must be [T={T}, H]")
+    H = x.shape[1]
+    _need(x, T * H * 2, "x", torch.bfloat16)
+    R = T * k
+    dev = x.device
+    out = Permuted(
+        q_perm=torch.empty((R, H // 2), dtype=torch.uint8, device=dev),
+        sf_perm=_sf_empty(R, H, sf_layout, dev),
+        offsets=torch.empty(num_experts + 1, dtype=torch.int32, device=dev),
+        perm_src=torch.empty(R, dtype=torch.int32, device=dev),
+        inv_perm=torch.empty(R, dtype=torch.int32, device=dev),
+    )
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    need = int(lib().moe_quantize_permute_workspace_size(T, k, num_experts, H))
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    else:
+        _need(ws, need, "ws")
+    _check(lib().moe_quantize_permute(_ptr(x), T, H, _ptr(topk_ids), k, num_experts, _ptr(out.q_perm),
+                                      _ptr(out.sf_perm), sf_layout, _ptr(g), _ptr(out.offsets), _ptr(out.perm_src),
+                                      _ptr(out.inv_perm), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_quantize_permute")
+    return out, g
 
 
 def permute_noalloc(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_experts: int,

@@ -141,6 +141,7 @@ extern "C" nvfp4_status moe_layer_workspace_layout(int32_t T, int32_t k, int32_t
     const size_t qx = nvfp4_quantize_workspace_size(T, H), qh = nvfp4_quantize_workspace_size((int64_t)R, I);
     if (qx > scratch) scratch = qx;
     if (qh > scratch) scratch = qh;
+    if (scratch < 1024) scratch = 1024;   // the fused quantize-permute's amax partials (up to 148 words)
     L->scratch = take(scratch);
     L->topk_ids = take(sizeof(int32_t) * (size_t)T * (size_t)k);
     L->topk_w = take(sizeof(float) * (size_t)T * (size_t)k);
@@ -155,6 +156,14 @@ extern "C" size_t moe_layer_workspace_size(int32_t T, int32_t k, int32_t E, int6
 }
 
 // The layer; with `logits` non-null the router first writes the routing into the workspace.
+// permute.cu: nvfp4_quantize + moe_permute with caller-given token-order buffers and scratch
+namespace nvfp4 {
+nvfp4_status quantize_permute(const uint16_t* x, int32_t T, int64_t H, const int32_t* topk_ids, int32_t k, int32_t E,
+                              uint8_t* q_perm, uint8_t* sf_perm, nvfp4_sf_layout layout, float* g_x,
+                              int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm, uint8_t* q_x,
+                              uint8_t* sf_x, void* scratch, size_t scratch_bytes, cudaStream_t s);
+}  // namespace nvfp4
+
 static nvfp4_status layer(const uint16_t* x, const float* logits, const int32_t* topk_ids, const float* topk_w,
                           int32_t T, int32_t k, int32_t E, int64_t H, int64_t I, const uint8_t* w13_packed,
                           const float* w13_gscale, const uint8_t* w2_packed, const float* w2_gscale, uint16_t* out,
@@ -204,10 +213,9 @@ static nvfp4_status layer(const uint16_t* x, const float* logits, const int32_t*
         topk_ids = ids_ws;
         topk_w = w_ws;
     }
-    if ((st = nvfp4_quantize(x, T, H, nullptr, q_x, sf_x, g_x, NVFP4_SF_ROWMAJOR, scratch, scratch_bytes, stream)))
-        return st;
-    if ((st = moe_permute(topk_ids, T, k, E, q_x, sf_x, H, q_perm, sf_perm, NVFP4_SF_KSTAGE, off, perm_src, inv_perm,
-                          scratch, scratch_bytes, stream)))
+    // x quantised straight into expert order (small batches never write its codes in token order)
+    if ((st = quantize_permute(x, T, H, topk_ids, k, E, q_perm, sf_perm, NVFP4_SF_KSTAGE, g_x, off, perm_src,
+                               inv_perm, q_x, sf_x, scratch, scratch_bytes, reinterpret_cast<cudaStream_t>(stream))))
         return st;
     if ((st = moe_grouped_gemm_nvfp4_amax(q_perm, sf_perm, g_x, w13_packed, w13_gscale, off, E, R, 2 * I, H,
                                           NVFP4_EPI_SWIGLU, h, amax_h, stream)))

@@ -21,6 +21,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "quant_math.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -139,13 +140,10 @@ __global__ void __launch_bounds__(kTok) permute_rank_kernel(const int32_t* __res
 // word-major ([W][E]), so the per-expert passes read consecutive words across a warp; a thread keeps the
 // expert ids of its first kIdsCached pairs in registers for the second pass.
 constexpr int kIdsCached = 8;
-__global__ void __launch_bounds__(kMaxE) permute_small_kernel(const int32_t* __restrict__ ids, int32_t T, int32_t k,
-                                                                int32_t E, int32_t* __restrict__ offsets,
-                                                                int32_t* __restrict__ perm_src,
-                                                                int32_t* __restrict__ inv_perm, uint32_t* status) {
-    pdl_launch_dependents();
-    pdl_wait();
-    extern __shared__ uint32_t small_sm[];
+// The ranking of one CTA of kMaxE threads; small_sm: 2 * E * ceil(T/32) words of shared memory.
+__device__ __forceinline__ void rank_small(const int32_t* __restrict__ ids, int32_t T, int32_t k, int32_t E,
+                                           int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src,
+                                           int32_t* __restrict__ inv_perm, uint32_t* status, uint32_t* small_sm) {
     __shared__ int32_t warp_sums[kMaxE / 32];
     const int W = (T + 31) / 32;                  // 32-token words per expert
     uint32_t* bits = small_sm;                    // [W][E]
@@ -224,6 +222,106 @@ __global__ void __launch_bounds__(kMaxE) permute_small_kernel(const int32_t* __r
     for (int c = 0; c < kIdsCached; c++)
         if (tid + (int64_t)c * kMaxE < R) place(tid + (int64_t)c * kMaxE, my_e[c]);
     for (int64_t i = tid + (int64_t)kIdsCached * kMaxE; i < R; i += kMaxE) place(i, __ldg(ids + i));
+}
+
+__global__ void __launch_bounds__(kMaxE) permute_small_kernel(const int32_t* __restrict__ ids, int32_t T, int32_t k,
+                                                                int32_t E, int32_t* __restrict__ offsets,
+                                                                int32_t* __restrict__ perm_src,
+                                                                int32_t* __restrict__ inv_perm, uint32_t* status) {
+    pdl_launch_dependents();
+    pdl_wait();
+    extern __shared__ uint32_t small_sm[];
+    rank_small(ids, T, k, E, offsets, perm_src, inv_perm, status, small_sm);
+}
+
+// ---- quantise while permuting (small batches): moe_quantize_permute ----------------------------------
+// Front: CTA 0 ranks every pair (rank_small); CTAs 1..G take the packed |x| maximum of a slice of x into
+// partial[blockIdx.x - 1]. The two steps need nothing from each other, so they run side by side.
+__global__ void __launch_bounds__(kMaxE) quantize_permute_front_kernel(
+    const int32_t* __restrict__ ids, int32_t T, int32_t k, int32_t E, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm, uint32_t* status, const uint4* __restrict__ x,
+    int64_t nvec, uint32_t* __restrict__ partial) {
+    pdl_launch_dependents();
+    pdl_wait();
+    extern __shared__ uint32_t small_sm[];
+    if (blockIdx.x == 0) {
+        rank_small(ids, T, k, E, offsets, perm_src, inv_perm, status, small_sm);
+        return;
+    }
+    uint32_t m = 0;
+    const int64_t stride = (int64_t)(gridDim.x - 1) * blockDim.x;
+    for (int64_t i = (int64_t)(blockIdx.x - 1) * blockDim.x + threadIdx.x; i < nvec; i += stride) {
+        const uint4 v = __ldg(x + i);
+        m = absmax_pair(m, v.x);
+        m = absmax_pair(m, v.y);
+        m = absmax_pair(m, v.z);
+        m = absmax_pair(m, v.w);
+    }
+    m = warp_max_u32(fold_pair(m));
+    __shared__ uint32_t s_warp[kMaxE / 32];
+    if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const uint32_t v = warp_max_u32(s_warp[threadIdx.x]);
+        if (threadIdx.x == 0) partial[blockIdx.x - 1] = v;
+    }
+}
+
+// Quantise and scatter: one warp per 32-block piece of token t's BF16 row quantises it once (quantize_block: the quantiser's
+// own steps, with the global scale folded from the front's partials) and writes the codes and scales of
+// every 16-element block to the permuted rows of its k pairs (inv_perm, from the front's ranking). A pair
+// without a row (an invalid expert id, inv_perm -1) is skipped. kKStage: scales in the K-stage layout,
+// else row-major.
+template <bool kKStage>
+__global__ void __launch_bounds__(256) quantize_scatter_kernel(const uint4* __restrict__ x, int32_t T, int64_t K,
+                                                               int32_t k, const uint32_t* __restrict__ partial,
+                                                               int npartial, const int32_t* __restrict__ inv_perm,
+                                                               int64_t R, uint2* __restrict__ q_perm,
+                                                               uint8_t* __restrict__ sf_perm, float* __restrict__ gdec_out) {
+    pdl_launch_dependents();
+    pdl_wait();
+    __shared__ float s_genc;
+    if (threadIdx.x < 32) {
+        uint32_t m = 0;
+        for (int i = threadIdx.x; i < npartial; i += 32) m = max(m, partial[i]);
+        m = warp_max_u32(m);
+        const GlobalScale g = global_scale(bf16_bits_to_f32(m), nullptr);
+        if (threadIdx.x == 0) {
+            s_genc = g.enc;
+            if (blockIdx.x == 0) *gdec_out = g.dec;
+        }
+    }
+    __syncthreads();
+    const float g_enc = s_genc;
+    const int64_t nb = K >> 4;                         // 16-element blocks per row
+    const int64_t nchunk = (nb + 31) / 32;             // 32-block pieces of a row, one warp each
+    const int64_t wi = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int64_t t = wi / nchunk;
+    if (t >= T) return;
+    const int lane = threadIdx.x & 31;
+    const int32_t my_dst = lane < k ? __ldg(inv_perm + t * k + lane) : -1;   // lane j: the row of pair (t, j)
+    const uint4* xs = x + t * (K >> 3);
+    {   // every lane takes part in the shuffles below, active or not
+        const int64_t b = (wi - t * nchunk) * 32 + lane;
+        const bool active = b < nb;
+        uint2 packed = make_uint2(0u, 0u);
+        uint32_t S = 0u;
+        if (active) S = quantize_block(__ldg(xs + 2 * b), __ldg(xs + 2 * b + 1), g_enc, packed);
+        for (int j = 0; j < k; j++) {
+            const int32_t d = __shfl_sync(0xFFFFFFFFu, my_dst, j);
+            if (d < 0 || !active) continue;
+            q_perm[(int64_t)d * nb + b] = packed;
+            if (kKStage) {
+                // slab of the 256-element K step b / 16, row d's 16-byte piece, byte b % 16
+                const int64_t off = ((b >> 4) * R + d) * 16 + (b & 15);
+                sf_perm[off] = (uint8_t)S;
+                // K % 256 == 128: the last slab's piece holds 8 scales; its other 8 bytes are zero scales
+                if ((nb & 15) == 8 && b == nb - 1) *reinterpret_cast<uint2*>(sf_perm + off + 1) = make_uint2(0u, 0u);
+            } else {
+                sf_perm[(int64_t)d * nb + b] = (uint8_t)S;
+            }
+        }
+    }
 }
 
 // One warp per output row; rows whose source index is invalid become zeros.
@@ -349,6 +447,96 @@ extern "C" nvfp4_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t 
     launch_gather(q, sf, K, perm_src, T, R, q_perm, sf_perm, sf_perm_layout, s);
     count_launch(4);
     return check_launch();
+}
+
+// ---------------------------------------------------------------------------
+// moe_quantize_permute: x quantised straight into expert order.
+//
+// Small batches (the one-CTA ranking applies): two launches -- the front (ranking beside the amax
+// partials of x) and the quantise-scatter (each token's row quantised once and written to its k permuted
+// rows) -- and no token-order copy of the codes. Larger batches: nvfp4_quantize into the workspace, then
+// moe_permute (the same bytes either way).
+
+static constexpr int kFrontMaxPartials = 148;
+
+static bool front_kernel_ready() {
+    static std::once_flag once[64];
+    static bool ok[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::call_once(once[dev], [&] {
+        ok[dev] = cudaFuncSetAttribute(quantize_permute_front_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmallMaxSmem) == cudaSuccess;
+    });
+    return ok[dev];
+}
+
+static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+extern "C" size_t moe_quantize_permute_workspace_size(int32_t T, int32_t k, int32_t E, int64_t H) {
+    if (T <= 0 || k <= 0 || E <= 0 || H <= 0 || H % 16 != 0) return 0;
+    size_t scratch = moe_permute_workspace_size(T, k, E);
+    const size_t qws = nvfp4_quantize_workspace_size(T, H);
+    if (qws > scratch) scratch = qws;
+    if ((size_t)kFrontMaxPartials * 4 > scratch) scratch = (size_t)kFrontMaxPartials * 4;
+    return align256((size_t)T * (size_t)H / 2) + align256((size_t)T * (size_t)H / 16) + align256(scratch);
+}
+
+namespace nvfp4 {
+nvfp4_status quantize_permute(const uint16_t* x, int32_t T, int64_t H, const int32_t* topk_ids, int32_t k, int32_t E,
+                              uint8_t* q_perm, uint8_t* sf_perm, nvfp4_sf_layout layout, float* g_x,
+                              int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm, uint8_t* q_x,
+                              uint8_t* sf_x, void* scratch, size_t scratch_bytes, cudaStream_t s) {
+    const int64_t R = (int64_t)T * k;
+    const size_t small_smem = 2 * (size_t)E * (size_t)((T + 31) / 32) * sizeof(uint32_t);
+    const int64_t nvec = (int64_t)T * H / 8;
+    if (R <= kSmallMaxPairs && small_smem <= kSmallMaxSmem && front_kernel_ready()) {
+        uint32_t* status = status_word_ptr();
+        if (!status) return NVFP4_ERR_CUDA;
+        if (scratch_bytes < (size_t)kFrontMaxPartials * 4) return NVFP4_ERR_WORKSPACE;
+        int64_t parts = (nvec + (int64_t)kMaxE * 4 - 1) / ((int64_t)kMaxE * 4);   // ~4 vectors per thread
+        if (parts > kFrontMaxPartials) parts = kFrontMaxPartials;
+        if (parts < 1) parts = 1;
+        uint32_t* partial = static_cast<uint32_t*>(scratch);
+        launch_pdl(quantize_permute_front_kernel, dim3((unsigned)(1 + parts)), dim3(kMaxE), small_smem, s, topk_ids, T,
+                   k, E, expert_offsets, perm_src, inv_perm, status, reinterpret_cast<const uint4*>(x), nvec, partial);
+        auto kernel = layout == NVFP4_SF_KSTAGE ? quantize_scatter_kernel<true> : quantize_scatter_kernel<false>;
+        const int64_t warps = (int64_t)T * ((H / 16 + 31) / 32);
+        launch_pdl(kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, reinterpret_cast<const uint4*>(x), T, H, k,
+                   partial, (int)parts, inv_perm, R, reinterpret_cast<uint2*>(q_perm), sf_perm, g_x);
+        count_launch(2);
+        return check_launch();
+    }
+    nvfp4_status st = nvfp4_quantize(x, T, H, nullptr, q_x, sf_x, g_x, NVFP4_SF_ROWMAJOR, scratch, scratch_bytes, s);
+    if (st != NVFP4_OK) return st;
+    return moe_permute(topk_ids, T, k, E, q_x, sf_x, H, q_perm, sf_perm, layout, expert_offsets, perm_src, inv_perm,
+                       scratch, scratch_bytes, s);
+}
+}  // namespace nvfp4
+
+extern "C" nvfp4_status moe_quantize_permute(const uint16_t* x, int32_t T, int64_t H, const int32_t* topk_ids,
+                                             int32_t k, int32_t E, uint8_t* q_perm, uint8_t* sf_perm,
+                                             nvfp4_sf_layout sf_perm_layout, float* g_x, int32_t* expert_offsets,
+                                             int32_t* perm_src, int32_t* inv_perm, void* ws, size_t ws_bytes,
+                                             nvfp4_stream_t stream) {
+    if (!x || !topk_ids || !q_perm || !sf_perm || !g_x || !expert_offsets || !perm_src || !inv_perm)
+        return NVFP4_ERR_INVALID_ARG;
+    if (sf_perm_layout != NVFP4_SF_ROWMAJOR && sf_perm_layout != NVFP4_SF_KSTAGE) return NVFP4_ERR_INVALID_ARG;
+    if (T <= 0 || k <= 0 || E <= 0 || H <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (k > 32 || E > kMaxE || (int64_t)T * k >= (int64_t)1 << 31 || H % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(topk_ids) || !aligned16(q_perm) || !aligned16(sf_perm) ||
+        !aligned16(expert_offsets) || !aligned16(perm_src) || !aligned16(inv_perm) || ((uintptr_t)g_x & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    const size_t need = moe_quantize_permute_workspace_size(T, k, E, H);
+    if (!ws || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_MISALIGNED;
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    uint8_t* q_x = b;
+    uint8_t* sf_x = q_x + align256((size_t)T * (size_t)H / 2);
+    uint8_t* scratch = sf_x + align256((size_t)T * (size_t)H / 16);
+    const size_t scratch_bytes = need - (size_t)(scratch - b);
+    return quantize_permute(x, T, H, topk_ids, k, E, q_perm, sf_perm, sf_perm_layout, g_x, expert_offsets, perm_src,
+                            inv_perm, q_x, sf_x, scratch, scratch_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
