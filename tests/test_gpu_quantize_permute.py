@@ -37,6 +37,7 @@ def both(T, E, k, H, kind, seed, layout=nv.SF_KSTAGE):
                                           (37, 5, 2, 256, "uniform"),         # ragged, few experts
                                           (1, 1, 1, 128, "uniform"),          # one row, K = 128
                                           (64, 16, 4, 384, "uniform"),        # K % 256 == 128 (half slab)
+                                          (64, 1024, 32, 256, "uniform"),     # E = 1024, k = 32 (every lane a slot)
                                           (5000, 64, 8, 256, "uniform")])     # 40,000 pairs: quantise, then permute
 def test_same_bytes_as_quantize_then_permute(T, E, k, H, kind):
     both(T, E, k, H, kind, seed=T + H)
