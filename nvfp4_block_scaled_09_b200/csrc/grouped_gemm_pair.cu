@@ -15,10 +15,13 @@
 // lanes 32q+16..32q+31: the matching up rows), so one warp reads both halves of
 // its 16 output columns and pairs them with a lane shuffle.
 //
-// One 256-column accumulator per CTA (the scale ring takes the rest of tensor
-// memory), so the epilogue warps first drain it into registers as final BF16
-// values and hand it back to the MMA warp; staging and storing those values
-// then overlaps the next tile's main loop.
+// One accumulator per CTA (256 columns, plus 32 for the rows past an expert's
+// last full tile that ride on it in the configuration with row tails; the scale
+// ring takes the rest of tensor memory), so the epilogue warps first drain it
+// into registers as final BF16 values and hand it back to the MMA warp; staging
+// and storing those values then overlaps the next tile's main loop. Two
+// configurations (Cfg below): row tails, 4 stages and a 3-slot scale ring for
+// several experts; 5 stages and a scale slot per stage for one expert.
 //
 // The peer's scale-writer and epilogue warps arrive on the even CTA's barriers
 // through cluster addresses (mapa); the even CTA's MMA completions reach both
