@@ -23,6 +23,10 @@
 // configurations (Cfg below): row tails, 4 stages and a 3-slot scale ring for
 // several experts; 5 stages and a scale slot per stage for one expert.
 //
+// The kernel is a template on the epilogue mode, the configuration and SwiGLU or plain output, so each
+// instantiation carries only its own epilogue (measured on B200: a runtime SwiGLU switch cost 1-4% on
+// the prefill GEMMs).
+//
 // The peer's scale-writer and epilogue warps arrive on the even CTA's barriers
 // through cluster addresses (mapa); the even CTA's MMA completions reach both
 // CTAs' barriers through one commit with a CTA mask (no data moves by multicast;
@@ -59,11 +63,16 @@ __device__ __forceinline__ uint32_t f32x2_to_bf16x2(uint64_t v) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
-// max |x| over the 16 BF16 pairs of a chunk, as BF16 bits
-__device__ __forceinline__ uint32_t absmax_bf16x2(const uint32_t* pk, int n) {
+// max |x| over the n BF16 pairs of a chunk, as BF16 bits, counting only the halves whose token is below
+// nrows: word i holds tokens stride * i + off (low half) and stride * i + off + stride / 2 (high half)
+__device__ __forceinline__ uint32_t absmax_bf16x2(const uint32_t* pk, int n, int nrows, int stride, int off) {
     uint32_t m = 0;
 #pragma unroll
-    for (int i = 0; i < n; i++) m = __vmaxu2(m, pk[i] & 0x7FFF7FFFu);
+    for (int i = 0; i < n; i++) {
+        const int lo = stride * i + off;
+        const uint32_t mask = (lo < nrows ? 0x7FFFu : 0u) | (lo + stride / 2 < nrows ? 0x7FFF0000u : 0u);
+        m = __vmaxu2(m, pk[i] & mask);
+    }
     return max(m & 0xFFFFu, m >> 16);
 }
 
@@ -324,7 +333,7 @@ __device__ __forceinline__ void build_schedule(S& sh, const Params& p, int32_t n
 namespace nvfp4 {
 namespace gp {
 
-template <int kEpi, bool kTails>
+template <int kEpi, bool kTails, bool kSw>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_full,
                              const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_wsw,
@@ -338,7 +347,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
     const int32_t E = p.E;
-    const int32_t n_col_tiles = (int32_t)(p.swiglu ? (p.N / 2) / kBM : p.N / (2 * kBM));
+    const int32_t n_col_tiles = (int32_t)(kSw ? (p.N / 2) / kBM : p.N / (2 * kBM));
     // K % 256 == 128: the last stage holds 128 K-elements (2 MMA K-steps); weights and activation scales
     // are zero-padded there, and the activation tile's second half is outside the tensor (zero-filled)
     const int32_t ksteps_total = (int32_t)((p.K + kBK - 1) / kBK);
@@ -348,7 +357,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tm_a);
         prefetch_tensormap(&tm_a_full);
         prefetch_tensormap(&tm_out);
-        if (p.swiglu) {
+        if (kSw) {
             prefetch_tensormap(&tm_wsw);
             prefetch_tensormap(&tm_wsf);
         }
@@ -418,12 +427,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint8_t* g_tile;   // NONE: this CTA's 128-row tile; SWIGLU: the gate tile
                 const uint8_t* u_tile;   // NONE: the other CTA's tile; SWIGLU: the up tile
                 weight_tiles(p, t, rank, ksteps_total, g_tile, u_tile);
-                const uint32_t half = p.swiglu ? rank * 64 : 0;
+                const uint32_t half = kSw ? rank * 64 : 0;
                 const int32_t sw_tile0 = (int32_t)((g_tile - p.w_packed) / kPackedTileBytes);  // SWIGLU: gate tile index at K step 0
                 const int32_t my_rows = t.bn / 2;
                 const int32_t my_row0 = t.row0 + (int32_t)rank * my_rows;
                 // SWIGLU: 16 KB of interleaved gate/up codes + both tiles' 2 KB of scales; NONE: one packed tile
-                const uint32_t a_bytes = p.swiglu ? (uint32_t)kCodeBytes + 2u * kTileSFBytes : (uint32_t)kPackedTileBytes;
+                const uint32_t a_bytes = kSw ? (uint32_t)kCodeBytes + 2u * kTileSFBytes : (uint32_t)kPackedTileBytes;
                 // both CTAs stage the scales of all the tile's rows: one contiguous run of the K step's
                 // slab (K-stage layout), 16 bytes per row
                 // (+ this CTA's 16 tail rows when the tile has a tail)
@@ -437,7 +446,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     uint64_t* bar = &sh.full_tma[stage];
                     mbar_arrive_expect_tx(bar, tx);
                     const size_t ko = (size_t)kt * kPackedTileBytes;
-                    if (p.swiglu) {
+                    if (kSw) {
                         // 16-row slabs (2 KB, whole swizzle atoms) of this CTA's half: gate slab q -> A rows
                         // 32q.., up slab q -> 32q+16.. (one box: bytes x rows x gate/up x slab x tile)
                         tma_load_5d(sb + kOffA, &tm_wsw, 0, 0, 0, (int32_t)(half / 16), sw_tile0 + kt, bar, pol_w);
@@ -483,8 +492,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int quad = warp & 3;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         // row of this lane inside its packed tile, and that tile's scale atom in the stage
-        const int tile_row = p.swiglu ? (int)rank * 64 + quad * 16 + (lane & 15) : quad * 32 + lane;
-        const uint32_t sfa_off = kOffSFA + ((p.swiglu && lane >= 16) ? kTileSFBytes : 0) + (tile_row & 31) * 16 +
+        const int tile_row = kSw ? (int)rank * 64 + quad * 16 + (lane & 15) : quad * 32 + lane;
+        const uint32_t sfa_off = kOffSFA + ((kSw && lane >= 16) ? kTileSFBytes : 0) + (tile_row & 31) * 16 +
                                  (tile_row >> 5) * 4;
         uint32_t stage = 0, phase = 0, qi = 0, qphase = 0, sfs = 0;
         uint32_t count = 0;   // stages handled so far
@@ -642,13 +651,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // (SWIGLU: 16 outputs per lane, NONE: 32); quantised h is written here directly
             auto finish = [&](int c, const float (&v)[32], uint32_t (&pk)[16]) {
                 const int nrows = min(32, t.rows - c * 32);
-                if (p.swiglu) {
+                if (kSw) {
                     // lane l < 16 holds gate, lane l + 16 up, of output column 16 quad + l; lane l
                     // produces the even tokens, lane l + 16 the odd ones
                     if (kEpi == kEpiPlain && nrows == 32) {
                         // a whole chunk (the accumulator hold is the epilogue's critical path): two outputs
-                        // per step rounded together to a BF16 pair, amax over the packed pairs at the end
-                        // (measured on the prefill gate/up GEMM: 1.3% faster than the per-output path)
+                        // per step rounded together to a BF16 pair, amax over the pairs at the end (measured
+                        // on the prefill gate/up GEMM: 1.3% faster than one output at a time)
 #pragma unroll
                         for (int j = 0; j < 16; j += 2) {
                             float hv[2];
@@ -663,7 +672,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             const __nv_bfloat162 b2 = __floats2bfloat162_rn(hv[0], hv[1]);
                             pk[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
                         }
-                        if (p.amax_out != nullptr) amax = max(amax, absmax_bf16x2(pk, 8));
+                        // word i: tokens 4 i + (up lane) and 4 i + 2 + (up lane)
+                        if (p.amax_out != nullptr) amax = max(amax, absmax_bf16x2(pk, 8, nrows, 4, up_lane ? 1 : 0));
                         return;
                     }
 #pragma unroll
@@ -698,25 +708,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         else pk[j >> 1] = hb;
                     }
                 } else {
-                    if (nrows == 32) {
-                        // a whole chunk: alpha applied with packed FP32 multiplies, two outputs rounded per
-                        // conversion, amax only when it is asked for (measured on the prefill down GEMM: 5%
-                        // faster than the per-output path; the same bits)
-                        const uint64_t a2 = f32x2_pack(alpha, alpha);
+                    // alpha applied with packed FP32 multiplies, two outputs rounded per conversion, amax
+                    // only when it is asked for (measured on the prefill down GEMM: 5% faster than one
+                    // output at a time; the same bits). Word i: tokens 2 i and 2 i + 1.
+                    const uint64_t a2 = f32x2_pack(alpha, alpha);
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2)
-                            pk[i >> 1] = f32x2_to_bf16x2(f32x2_mul(f32x2_pack(v[i], v[i + 1]), a2));
-                        if (p.amax_out != nullptr) amax = max(amax, absmax_bf16x2(pk, 16));
-                        return;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const uint32_t b0 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i]));
-                        const uint32_t b1 = __bfloat16_as_ushort(__float2bfloat16_rn(alpha * v[i + 1]));
-                        if (i < nrows) amax = max(amax, b0 & 0x7FFFu);
-                        if (i + 1 < nrows) amax = max(amax, b1 & 0x7FFFu);
-                        pk[i >> 1] = b0 | (b1 << 16);
-                    }
+                    for (int i = 0; i < 32; i += 2)
+                        pk[i >> 1] = f32x2_to_bf16x2(f32x2_mul(f32x2_pack(v[i], v[i + 1]), a2));
+                    if (p.amax_out != nullptr) amax = max(amax, absmax_bf16x2(pk, 16, nrows, 2, 0));
                 }
             };
             // Chunk c staged as a 32-token block in shared memory and stored
@@ -728,7 +727,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 int32_t col;      // first output column of this warp's block
                 int lane_cols;    // lanes per 16-byte row piece in the direct-store path: 2 (SwiGLU) or 4
-                if (p.swiglu) {
+                if (kSw) {
 #pragma unroll
                     for (int j = 0; j < 16; j++)
                         stg[(2 * j + (up_lane ? 1 : 0)) * 16 + (lane & 15)] =
@@ -754,7 +753,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 } else {
                     // the expert's last, partial chunk: rows past its end belong to the next expert
                     __syncwarp();
-                    const int64_t ldo = p.swiglu ? p.N / 2 : p.N;
+                    const int64_t ldo = kSw ? p.N / 2 : p.N;
                     const int row_elems = 8 * lane_cols;
                     const int rows_per_pass = 32 / lane_cols;
                     for (int r = lane / lane_cols; r < nrows; r += rows_per_pass) {
@@ -867,12 +866,12 @@ int pair_gemm_tokens_max() { return gp::kBNMax; }
 int pair_gemm_store_cols(int swiglu) { return swiglu ? 16 : 32; }  // 32 tokens x this many BF16 columns
 
 // The shared-memory opt-in of one instantiation, once per device (thread-safe).
-template <int kEpi, bool kTails>
+template <int kEpi, bool kTails, bool kSw>
 static bool pair_kernel_configured(int dev) {
     static std::once_flag once[64];
     static bool ok[64] = {};
     std::call_once(once[dev], [&] {
-        ok[dev] = cudaFuncSetAttribute(gp::grouped_gemm_pair_kernel<kEpi, kTails>,
+        ok[dev] = cudaFuncSetAttribute(gp::grouped_gemm_pair_kernel<kEpi, kTails, kSw>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)gp::Cfg<kTails>::kSmemBytes) == cudaSuccess;
     });
@@ -887,7 +886,7 @@ static nvfp4_status pair_grid(int dev, int& grid) {
     static nvfp4_status set_result[64] = {};
     std::call_once(once[dev], [&] {
         set_result[dev] = NVFP4_ERR_CUDA;
-        if (!pair_kernel_configured<kEpiPlain, kTails>(dev)) return;
+        if (!pair_kernel_configured<kEpiPlain, kTails, false>(dev)) return;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)device_sm_count() / 2 * 2);
         cfg.blockDim = dim3(gp::kThreads);
@@ -900,7 +899,7 @@ static nvfp4_status pair_grid(int dev, int& grid) {
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, gp::grouped_gemm_pair_kernel<kEpiPlain, kTails>, &cfg) !=
+        if (cudaOccupancyMaxActiveClusters(&clusters, gp::grouped_gemm_pair_kernel<kEpiPlain, kTails, false>, &cfg) !=
                 cudaSuccess ||
             clusters <= 0) {
             set_result[dev] = NVFP4_ERR_SMEM_BUDGET;
@@ -922,17 +921,22 @@ static nvfp4_status launch_pair_config(int dev, const CUtensorMap& tm_a, const C
     if (st != NVFP4_OK) return st;
     const size_t smem = gp::Cfg<kTails>::kSmemBytes;
     // every instantiation has the plain one's resources (same shared memory, threads and cluster shape)
+    // quantised h is SWIGLU only, the fused combine NONE only (the caller checked)
     if (prm.qo.q != nullptr) {
-        if (!pair_kernel_configured<kEpiQuant, kTails>(dev)) return NVFP4_ERR_CUDA;
-        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiQuant, kTails>, dim3(grid), dim3(gp::kThreads), smem, s, tm_a,
-                   tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+        if (!pair_kernel_configured<kEpiQuant, kTails, true>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiQuant, kTails, true>, dim3(grid), dim3(gp::kThreads), smem, s,
+                   tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
     } else if (prm.fin.out != nullptr) {
-        if (!pair_kernel_configured<kEpiFinalize, kTails>(dev)) return NVFP4_ERR_CUDA;
-        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiFinalize, kTails>, dim3(grid), dim3(gp::kThreads), smem, s, tm_a,
-                   tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+        if (!pair_kernel_configured<kEpiFinalize, kTails, false>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiFinalize, kTails, false>, dim3(grid), dim3(gp::kThreads), smem,
+                   s, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+    } else if (prm.swiglu) {
+        if (!pair_kernel_configured<kEpiPlain, kTails, true>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain, kTails, true>, dim3(grid), dim3(gp::kThreads), smem, s,
+                   tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
     } else {
-        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain, kTails>, dim3(grid), dim3(gp::kThreads), smem, s, tm_a,
-                   tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain, kTails, false>, dim3(grid), dim3(gp::kThreads), smem, s,
+                   tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
     }
     return NVFP4_OK;
 }
