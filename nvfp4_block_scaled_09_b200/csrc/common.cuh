@@ -378,6 +378,26 @@ __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_
     return d;
 }
 
+// Two FP32 values in one 64-bit register, for the packed FP32 multiply of sm_100 (mul.rn.f32x2: both
+// halves rounded as two scalar multiplies would be)
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// Both halves rounded to BF16 (nearest even), the low half into the low 16 bits
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
 // SwiGLU of one output element: silu(g) * u with silu(g) = g / (1 + e^-g), in single precision
 // without branches: e^-g as 2^(-g log2 e) on the ISA's base-2 exponential (ex2.approx), and the
 // quotient as g times the ISA's approximate reciprocal (rcp.approx) of 1 + e^-g. Both are within a few

@@ -43,26 +43,6 @@
 
 namespace nvfp4 {
 namespace gp {
-// Two FP32 values in one 64-bit register, for the packed FP32 multiply of sm_100 (mul.rn.f32x2: both
-// halves rounded as two scalar multiplies would be)
-__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-// Both halves rounded to BF16 (nearest even), the low half into the low 16 bits
-__device__ __forceinline__ uint32_t f32x2_to_bf16x2(uint64_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
 // max |x| over the n BF16 pairs of a chunk, as BF16 bits, counting only the halves whose token is below
 // nrows: word i holds tokens stride * i + off (low half) and stride * i + off + stride / 2 (high half)
 __device__ __forceinline__ uint32_t absmax_bf16x2(const uint32_t* pk, int n, int nrows, int stride, int off) {
