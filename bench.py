@@ -354,6 +354,7 @@ class MoEBench:
         self.weights = weights
         self.ws = nv.layer_workspace(T, k, E, H, I, device)
         self.lay = nv.layer_workspace_layout(T, k, E, H, I)
+        self.l2_hints = nv.layer_l2_prefetch_bytes(T, k, E, H, I)
         # amax_h and the fused combine's counters: zeroed together at the start of every layer
         self.zeroed = self.ws[self.lay["amax_h"]: self.lay["fin_counters"] + nv.lib().moe_finalize_counters_size(T, H)]
         self.out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
@@ -385,10 +386,12 @@ class MoEBench:
         self.zeroed.zero_()    # as moe_layer_nvfp4's one memset
         rec(0)
         # x quantised into expert order (moe_layer_nvfp4 runs the same kernels on its own workspace)
-        st = L.moe_quantize_permute(P(self.x.data_ptr()), T, H, P(self.ids.data_ptr()), k, E,
-                                    P(b + lay["q_perm"]), P(b + lay["sf_perm"]), nv.SF_KSTAGE, P(b + lay["g_x"]),
-                                    P(b + lay["offsets"]), P(b + lay["perm_src"]), P(b + lay["inv_perm"]),
-                                    P(self.qp_ws.data_ptr()), self.qp_ws.numel(), s)
+        pf13, pf2 = self.l2_hints   # the L2 prefetch hints moe_layer_nvfp4 gives (decode-sized batches)
+        st = L.moe_quantize_permute_prefetch(P(self.x.data_ptr()), T, H, P(self.ids.data_ptr()), k, E,
+                                             P(b + lay["q_perm"]), P(b + lay["sf_perm"]), nv.SF_KSTAGE,
+                                             P(b + lay["g_x"]), P(b + lay["offsets"]), P(b + lay["perm_src"]),
+                                             P(b + lay["inv_perm"]), P(self.qp_ws.data_ptr()), self.qp_ws.numel(),
+                                             P(W.w13.packed.data_ptr()), pf13, s)
         rec(1)
         if gemm_ev is not None:
             gemm_ev[0].record()
@@ -399,8 +402,9 @@ class MoEBench:
         if gemm_ev is not None:
             gemm_ev[1].record()
         rec(2)
-        st |= L.nvfp4_quantize_from_amax(P(b + lay["h"]), R, I, P(b + lay["amax_h"]), P(b + lay["q_h"]),
-                                         P(b + lay["sf_h"]), P(b + lay["g_h"]), nv.SF_KSTAGE, s)
+        st |= L.nvfp4_quantize_from_amax_prefetch(P(b + lay["h"]), R, I, P(b + lay["amax_h"]), P(b + lay["q_h"]),
+                                                  P(b + lay["sf_h"]), P(b + lay["g_h"]), nv.SF_KSTAGE,
+                                                  P(W.w2.packed.data_ptr()), pf2, s)
         rec(3)
         if fused:
             st |= L.moe_grouped_gemm_nvfp4_finalize(P(b + lay["q_h"]), P(b + lay["sf_h"]), P(b + lay["g_h"]),
@@ -511,10 +515,17 @@ def run_moe(args, name, cfg, weights, rank, world, local_rank, dev, peaks, resiz
     shape = ("CTA-pair" if rows_mean >= plan["pair_min_avg_rows"] else
              "wide" if rows_mean >= plan["wide_min_avg_rows"] else "narrow")
     tflops1 = f1 / gemm1_s / 1e12
+    # bytes of each GEMM's weights the kernel before it pulled into L2 (the layer's prefetch hints): the GEMM's
+    # own HBM stream is the algorithmic bytes less those
+    pf1, pf2 = bench.l2_hints
     roof = ({"bound": "tensor", "achieved": tflops1, "peak": fp4_peak, "unit": "TFLOP/s", "frac": tflops1 / fp4_peak,
              "algorithmic_flops": f1} if tensor_bound else
-            {"bound": "hbm", "achieved": g1b / gemm1_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-             "frac": g1b / gemm1_s / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": g1b})
+            {"bound": "hbm", "achieved": (g1b - pf1) / gemm1_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": (g1b - pf1) / gemm1_s / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": g1b})
+    roof["l2_prefetch_bytes"] = pf1
+    if pf1:
+        roof["bytes_note"] = ("achieved counts algorithmic_bytes less l2_prefetch_bytes: the first weight tiles "
+                              "were pulled into L2 by the kernel before this one")
     roof |= {"traffic": measured_traffic(name if not resized else "", "gate_up_dram_bytes_per_launch"),
              "kernel": f"grouped GEMM gate/up + SwiGLU ({shape} tiles)",
              "peak_source": f"{peaks['source']} ({'HBM copy' if not tensor_bound else 'sustained bf16 x 4'})",
@@ -535,9 +546,9 @@ def run_moe(args, name, cfg, weights, rank, world, local_rank, dev, peaks, resiz
                        "note": "same box, same inputs: the down GEMM followed by moe_unpermute_combine (the "
                                "layer's path) against the down GEMM with the combine fused into its epilogue"},
         "roofline": roof,
-        "roofline_down": {"bound": "hbm", "achieved": g2b / gemm2_s / 1e9, "peak": peaks["hbm_gbs"],
-                          "unit": "GB/s", "frac": g2b / gemm2_s / 1e9 / peaks["hbm_gbs"],
-                          "algorithmic_bytes": g2b, "kernel": "grouped GEMM down",
+        "roofline_down": {"bound": "hbm", "achieved": (g2b - pf2) / gemm2_s / 1e9, "peak": peaks["hbm_gbs"],
+                          "unit": "GB/s", "frac": (g2b - pf2) / gemm2_s / 1e9 / peaks["hbm_gbs"],
+                          "algorithmic_bytes": g2b, "l2_prefetch_bytes": pf2, "kernel": "grouped GEMM down",
                           "avg_launch_ms": stage_ms[3], "tensor_frac": f2 / gemm2_s / 1e12 / fp4_peak,
                           "traffic": measured_traffic(name if not resized else "", "down_dram_bytes_per_launch")},
         "clocks": clk, "gpu_launches": int(launches), "e2e": e2e,

@@ -143,6 +143,16 @@ NVFP4_API nvfp4_status nvfp4_amax(const uint16_t* x, int64_t rows, int64_t K, ui
 NVFP4_API nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows, int64_t K, const uint32_t* amax_bits,
                                       uint8_t* q, uint8_t* sf, float* global_scale_out, nvfp4_sf_layout layout,
                                       nvfp4_stream_t stream);
+/* nvfp4_quantize_from_amax_prefetch: the same, and while it runs it pulls  */
+/* the first l2_next_bytes bytes at l2_next (device memory that no kernel   */
+/* in flight writes, e.g. the next GEMM's packed expert weights, taken by   */
+/* its schedule in address order) into L2 with plain prefetches. A hint: the */
+/* outputs do not depend on it; l2_next NULL or 0 bytes prefetches nothing. */
+NVFP4_API nvfp4_status nvfp4_quantize_from_amax_prefetch(const uint16_t* x, int64_t rows, int64_t K,
+                                               const uint32_t* amax_bits, uint8_t* q, uint8_t* sf,
+                                               float* global_scale_out, nvfp4_sf_layout layout,
+                                               const void* l2_next, size_t l2_next_bytes,
+                                               nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* moe_permute: group routed (token, slot) pairs by expert and gather the    */
@@ -194,6 +204,20 @@ NVFP4_API nvfp4_status moe_quantize_permute(const uint16_t* x, int32_t T, int64_
                                   nvfp4_sf_layout sf_perm_layout, float* g_x, int32_t* expert_offsets,
                                   int32_t* perm_src, int32_t* inv_perm, void* ws, size_t ws_bytes,
                                   nvfp4_stream_t stream);
+/* moe_quantize_permute_prefetch: the same, with the L2 prefetch hint of     */
+/* nvfp4_quantize_from_amax_prefetch (issued by the two-kernel path only).  */
+NVFP4_API nvfp4_status moe_quantize_permute_prefetch(const uint16_t* x, int32_t T, int64_t H,
+                                           const int32_t* topk_ids, int32_t k, int32_t E, uint8_t* q_perm,
+                                           uint8_t* sf_perm, nvfp4_sf_layout sf_perm_layout, float* g_x,
+                                           int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
+                                           void* ws, size_t ws_bytes, const void* l2_next,
+                                           size_t l2_next_bytes, nvfp4_stream_t stream);
+/* moe_layer_l2_prefetch_bytes: the prefetch hints moe_layer_nvfp4 gives    */
+/* (bytes of the gate/up and of the down weights: 96 MB and 48 MB, or the   */
+/* whole tensor when smaller; 0 when the experts average 32 rows or more,   */
+/* where the GEMMs do not stream their weights at HBM rate). Host only.     */
+NVFP4_API void moe_layer_l2_prefetch_bytes(int32_t T, int32_t k, int32_t E, int64_t H, int64_t I, size_t* gate_up,
+                                 size_t* down);
 
 /* ------------------------------------------------------------------------ */
 /* moe_permute_noalloc: moe_permute without a caller workspace. No passage   */
@@ -390,7 +414,9 @@ NVFP4_API nvfp4_status moe_route_topk(const float* logits, int32_t T, int32_t E,
 /* grouped GEMM gate/up (SWIGLU, N = 2I, K = H, amax of h as a side output)  */
 /* -> quantize(h) from that amax -> grouped GEMM down (NONE, N = H, K = I)   */
 /* -> moe_unpermute_combine. Results equal the four calls above run one by   */
-/* one (nvfp4_quantize of h with a dynamic scale).                           */
+/* one (nvfp4_quantize of h with a dynamic scale). With fewer than 32 rows   */
+/* per expert, the kernels before each GEMM carry the L2 prefetch hints of   */
+/* moe_layer_l2_prefetch_bytes (the *_prefetch calls): same results.         */
 /* Arguments: x [T, H] BF16, topk_ids [T, k], topk_w [T, k];                 */
 /*   w13_packed (W13 [E, 2I, H] packed as an [E*2I, H] matrix), w13_gscale   */
 /*   [E]; w2_packed (W2 [E, H, I] packed as [E*H, I]), w2_gscale [E];        */

@@ -10,9 +10,10 @@ without a CUDA device the calls raise.
 Calls (same names as the C ABI):
   quantize            -> nvfp4_quantize
   permute             -> moe_permute
-  quantize_permute    -> moe_quantize_permute
+  quantize_permute    -> moe_quantize_permute_prefetch (no hint: moe_quantize_permute's bytes)
   grouped_gemm        -> moe_grouped_gemm_nvfp4 (moe_grouped_gemm_nvfp4_amax with amax_out)
-  quantize_from_amax  -> nvfp4_quantize_from_amax
+  quantize_from_amax  -> nvfp4_quantize_from_amax_prefetch (no hint: nvfp4_quantize_from_amax)
+  layer_l2_prefetch_bytes -> moe_layer_l2_prefetch_bytes
   amax                -> nvfp4_amax
   pack_weights        -> nvfp4_pack_weights
   unpermute_combine   -> moe_unpermute_combine
@@ -85,6 +86,11 @@ def lib():
         L.moe_quantize_permute_workspace_size.restype = sz
         L.moe_quantize_permute.argtypes = [P, i32, i64, P, i32, i32, P, P, ctypes.c_int, P, P, P, P, P, sz, P]
         L.moe_quantize_permute.restype = st
+        L.moe_quantize_permute_prefetch.argtypes = [P, i32, i64, P, i32, i32, P, P, ctypes.c_int, P, P, P, P, P, sz,
+                                                    P, sz, P]
+        L.moe_quantize_permute_prefetch.restype = st
+        L.moe_layer_l2_prefetch_bytes.argtypes = [i32, i32, i32, i64, i64, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.moe_layer_l2_prefetch_bytes.restype = None
         L.moe_permute.restype = st
         L.moe_permute_noalloc.argtypes = [P, i32, i32, i32, P, P, i64, P, P, ctypes.c_int, P, P, P, P]
         L.moe_permute_noalloc.restype = st
@@ -94,6 +100,8 @@ def lib():
         L.moe_grouped_gemm_nvfp4_amax.restype = st
         L.nvfp4_quantize_from_amax.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int, P]
         L.nvfp4_quantize_from_amax.restype = st
+        L.nvfp4_quantize_from_amax_prefetch.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int, P, sz, P]
+        L.nvfp4_quantize_from_amax_prefetch.restype = st
         L.nvfp4_amax.argtypes = [P, i64, i64, P, P]
         L.nvfp4_amax.restype = st
         L.moe_unpermute_combine.argtypes = [P, P, P, i32, i32, i64, P, P]
@@ -233,11 +241,30 @@ def amax(x: torch.Tensor, amax_bits: torch.Tensor | None = None, stream=None) ->
     return amax_bits
 
 
+def _l2_hint(l2_next, l2_next_bytes):
+    """(pointer, bytes) of an L2 prefetch hint: the first l2_next_bytes bytes of the device tensor l2_next (all of
+    it by default), or (None, 0)."""
+    if l2_next is None:
+        return None, 0
+    _require_cuda(l2_next)
+    n = l2_next.numel() * l2_next.element_size()
+    return _ptr(l2_next), n if l2_next_bytes is None else min(int(l2_next_bytes), n)
+
+
+def layer_l2_prefetch_bytes(T: int, k: int, E: int, H: int, I: int) -> tuple[int, int]:
+    """The L2 prefetch hints moe_layer_nvfp4 gives: bytes of the gate/up and of the down packed weights
+    (moe_layer_l2_prefetch_bytes)."""
+    g, d = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    lib().moe_layer_l2_prefetch_bytes(T, k, E, H, I, ctypes.byref(g), ctypes.byref(d))
+    return g.value, d.value
+
+
 def quantize_from_amax(x: torch.Tensor, amax_bits: torch.Tensor, layout: int = SF_ROWMAJOR,
                        q: torch.Tensor | None = None, sf: torch.Tensor | None = None, g: torch.Tensor | None = None,
-                       stream=None):
+                       stream=None, l2_next: torch.Tensor | None = None, l2_next_bytes: int | None = None):
     """quantize() with a dynamic global scale from a known amax: amax_bits is a device int32 [1] holding max |x|
-    as BF16 bits (e.g. the amax_out of grouped_gemm)."""
+    as BF16 bits (e.g. the amax_out of grouped_gemm). l2_next / l2_next_bytes: an L2 prefetch hint for the next
+    kernel's constant operand (nvfp4_quantize_from_amax_prefetch); the outputs do not depend on it."""
     _require_cuda(x, amax_bits)
     x = _bits(x)
     rows, K = x.shape
@@ -246,8 +273,10 @@ def quantize_from_amax(x: torch.Tensor, amax_bits: torch.Tensor, layout: int = S
     q = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if q is None else _need(q, rows * K // 2, "q")
     sf = _sf_empty(rows, K, layout, dev) if sf is None else _need(sf, sf_bytes(rows, K, layout), "sf")
     g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else _need(g, 4, "g", torch.float32)
-    _check(lib().nvfp4_quantize_from_amax(_ptr(x), rows, K, _ptr(amax_bits), _ptr(q), _ptr(sf), _ptr(g), layout,
-                                          _stream(stream)), "nvfp4_quantize_from_amax")
+    pf, pf_bytes = _l2_hint(l2_next, l2_next_bytes)
+    _check(lib().nvfp4_quantize_from_amax_prefetch(_ptr(x), rows, K, _ptr(amax_bits), _ptr(q), _ptr(sf), _ptr(g),
+                                                   layout, pf, pf_bytes, _stream(stream)),
+           "nvfp4_quantize_from_amax_prefetch")
     return q, sf, g
 
 
@@ -348,9 +377,11 @@ def permute(topk_ids: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, num_exper
 
 
 def quantize_permute(x: torch.Tensor, topk_ids: torch.Tensor, num_experts: int, ws=None, stream=None,
-                     sf_layout: int = SF_KSTAGE):
+                     sf_layout: int = SF_KSTAGE, l2_next: torch.Tensor | None = None,
+                     l2_next_bytes: int | None = None):
     """quantize(x) then permute of the result in one call (moe_quantize_permute): the same bytes.
-    Returns (Permuted, g) with g the float32 [1] global scale of x."""
+    Returns (Permuted, g) with g the float32 [1] global scale of x. l2_next / l2_next_bytes: an L2 prefetch
+    hint for the next kernel's constant operand (moe_quantize_permute_prefetch)."""
     _require_cuda(x, topk_ids)
     if topk_ids.dtype != torch.int32:
         raise TypeError("topk_ids must be int32")
@@ -375,10 +406,12 @@ def quantize_permute(x: torch.Tensor, topk_ids: torch.Tensor, num_experts: int, 
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     else:
         _need(ws, need, "ws")
-    _check(lib().moe_quantize_permute(_ptr(x), T, H, _ptr(topk_ids), k, num_experts, _ptr(out.q_perm),
-                                      _ptr(out.sf_perm), sf_layout, _ptr(g), _ptr(out.offsets), _ptr(out.perm_src),
-                                      _ptr(out.inv_perm), _ptr(ws), ws.numel(), _stream(stream)),
-           "moe_quantize_permute")
+    pf, pf_bytes = _l2_hint(l2_next, l2_next_bytes)
+    _check(lib().moe_quantize_permute_prefetch(_ptr(x), T, H, _ptr(topk_ids), k, num_experts, _ptr(out.q_perm),
+                                               _ptr(out.sf_perm), sf_layout, _ptr(g), _ptr(out.offsets),
+                                               _ptr(out.perm_src), _ptr(out.inv_perm), _ptr(ws), ws.numel(), pf,
+                                               pf_bytes, _stream(stream)),
+           "moe_quantize_permute_prefetch")
     return out, g
 
 

@@ -196,6 +196,22 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 // lets the next kernel start its prologue; it carries no memory ordering.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// L2 prefetch of [base, base + bytes), split over the CTAs of the grid: worker = cta * blockDim.x + thread of
+// nworkers = ctas * blockDim.x, and the first thread of each CTA issues bulk prefetches (64 KB each) of its
+// CTA's 16-byte-aligned slice. Used to start the next kernel's constant operand (expert weights) streaming
+// into L2 while a short, latency-bound kernel runs (measured on B200, decode layer: 6-11 us less per layer
+// call; one prefetch per 128-byte line from every thread gained 5-8 us).
+__device__ __forceinline__ void l2_prefetch_slice(const uint8_t* base, int64_t bytes, int64_t worker, int64_t nworkers) {
+    if (base == nullptr || bytes <= 0 || threadIdx.x != 0) return;
+    const int64_t ctas = nworkers / blockDim.x, cta = worker / blockDim.x;
+    const int64_t slice = ((bytes + ctas - 1) / ctas + 15) & ~int64_t(15);
+    const int64_t lo = cta * slice, hi = lo + slice < bytes ? lo + slice : bytes;
+    for (int64_t off = lo; off < hi; off += 65536) {
+        const int64_t n = (hi - off < 65536 ? hi - off : 65536) & ~int64_t(15);
+        if (n > 0) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + off), "r"((uint32_t)n) : "memory");
+    }
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -240,8 +240,12 @@ __global__ void __launch_bounds__(kMaxE) permute_small_kernel(const int32_t* __r
 __global__ void __launch_bounds__(kMaxE) quantize_permute_front_kernel(
     const int32_t* __restrict__ ids, int32_t T, int32_t k, int32_t E, int32_t* __restrict__ offsets,
     int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm, uint32_t* status, const uint4* __restrict__ x,
-    int64_t nvec, uint32_t* __restrict__ partial) {
+    int64_t nvec, uint32_t* __restrict__ partial, const uint8_t* __restrict__ pf, int64_t pf_bytes) {
     pdl_launch_dependents();
+    // the next GEMM's first weight tiles (constant: no wait needed) start streaming into L2 while CTA 0 ranks
+    if (blockIdx.x > 0)
+        l2_prefetch_slice(pf, pf_bytes, (int64_t)(blockIdx.x - 1) * blockDim.x + threadIdx.x,
+                          (int64_t)(gridDim.x - 1) * blockDim.x);
     pdl_wait();
     extern __shared__ uint32_t small_sm[];
     if (blockIdx.x == 0) {
@@ -486,7 +490,8 @@ namespace nvfp4 {
 nvfp4_status quantize_permute(const uint16_t* x, int32_t T, int64_t H, const int32_t* topk_ids, int32_t k, int32_t E,
                               uint8_t* q_perm, uint8_t* sf_perm, nvfp4_sf_layout layout, float* g_x,
                               int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm, uint8_t* q_x,
-                              uint8_t* sf_x, void* scratch, size_t scratch_bytes, cudaStream_t s) {
+                              uint8_t* sf_x, void* scratch, size_t scratch_bytes, cudaStream_t s,
+                              const void* l2_next, size_t l2_next_bytes) {
     const int64_t R = (int64_t)T * k;
     const size_t small_smem = 2 * (size_t)E * (size_t)((T + 31) / 32) * sizeof(uint32_t);
     const int64_t nvec = (int64_t)T * H / 8;
@@ -499,7 +504,8 @@ nvfp4_status quantize_permute(const uint16_t* x, int32_t T, int64_t H, const int
         if (parts < 1) parts = 1;
         uint32_t* partial = static_cast<uint32_t*>(scratch);
         launch_pdl(quantize_permute_front_kernel, dim3((unsigned)(1 + parts)), dim3(kMaxE), small_smem, s, topk_ids, T,
-                   k, E, expert_offsets, perm_src, inv_perm, status, reinterpret_cast<const uint4*>(x), nvec, partial);
+                   k, E, expert_offsets, perm_src, inv_perm, status, reinterpret_cast<const uint4*>(x), nvec, partial,
+                   static_cast<const uint8_t*>(l2_next), (int64_t)l2_next_bytes);
         auto kernel = layout == NVFP4_SF_KSTAGE ? quantize_scatter_kernel<true> : quantize_scatter_kernel<false>;
         const int64_t warps = (int64_t)T * ((H / 16 + 31) / 32);
         launch_pdl(kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, reinterpret_cast<const uint4*>(x), T, H, k,
@@ -514,11 +520,12 @@ nvfp4_status quantize_permute(const uint16_t* x, int32_t T, int64_t H, const int
 }
 }  // namespace nvfp4
 
-extern "C" nvfp4_status moe_quantize_permute(const uint16_t* x, int32_t T, int64_t H, const int32_t* topk_ids,
-                                             int32_t k, int32_t E, uint8_t* q_perm, uint8_t* sf_perm,
-                                             nvfp4_sf_layout sf_perm_layout, float* g_x, int32_t* expert_offsets,
-                                             int32_t* perm_src, int32_t* inv_perm, void* ws, size_t ws_bytes,
-                                             nvfp4_stream_t stream) {
+extern "C" nvfp4_status moe_quantize_permute_prefetch(const uint16_t* x, int32_t T, int64_t H,
+                                                      const int32_t* topk_ids, int32_t k, int32_t E, uint8_t* q_perm,
+                                                      uint8_t* sf_perm, nvfp4_sf_layout sf_perm_layout, float* g_x,
+                                                      int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
+                                                      void* ws, size_t ws_bytes, const void* l2_next,
+                                                      size_t l2_next_bytes, nvfp4_stream_t stream) {
     if (!x || !topk_ids || !q_perm || !sf_perm || !g_x || !expert_offsets || !perm_src || !inv_perm)
         return NVFP4_ERR_INVALID_ARG;
     if (sf_perm_layout != NVFP4_SF_ROWMAJOR && sf_perm_layout != NVFP4_SF_KSTAGE) return NVFP4_ERR_INVALID_ARG;
@@ -535,8 +542,19 @@ extern "C" nvfp4_status moe_quantize_permute(const uint16_t* x, int32_t T, int64
     uint8_t* sf_x = q_x + align256((size_t)T * (size_t)H / 2);
     uint8_t* scratch = sf_x + align256((size_t)T * (size_t)H / 16);
     const size_t scratch_bytes = need - (size_t)(scratch - b);
+    if (l2_next == nullptr) l2_next_bytes = 0;
     return quantize_permute(x, T, H, topk_ids, k, E, q_perm, sf_perm, sf_perm_layout, g_x, expert_offsets, perm_src,
-                            inv_perm, q_x, sf_x, scratch, scratch_bytes, reinterpret_cast<cudaStream_t>(stream));
+                            inv_perm, q_x, sf_x, scratch, scratch_bytes, reinterpret_cast<cudaStream_t>(stream),
+                            l2_next, l2_next_bytes);
+}
+
+extern "C" nvfp4_status moe_quantize_permute(const uint16_t* x, int32_t T, int64_t H, const int32_t* topk_ids,
+                                             int32_t k, int32_t E, uint8_t* q_perm, uint8_t* sf_perm,
+                                             nvfp4_sf_layout sf_perm_layout, float* g_x, int32_t* expert_offsets,
+                                             int32_t* perm_src, int32_t* inv_perm, void* ws, size_t ws_bytes,
+                                             nvfp4_stream_t stream) {
+    return moe_quantize_permute_prefetch(x, T, H, topk_ids, k, E, q_perm, sf_perm, sf_perm_layout, g_x,
+                                         expert_offsets, perm_src, inv_perm, ws, ws_bytes, nullptr, 0, stream);
 }
 
 // ---------------------------------------------------------------------------

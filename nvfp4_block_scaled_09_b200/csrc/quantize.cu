@@ -58,8 +58,11 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
                                                             const float* __restrict__ gdec_in,
                                                             const uint32_t* __restrict__ partial, int npartial,
                                                             uint2* __restrict__ q, uint8_t* __restrict__ sf,
-                                                            float* __restrict__ gdec_out) {
+                                                            float* __restrict__ gdec_out, const uint8_t* __restrict__ pf,
+                                                            int64_t pf_bytes) {
     pdl_launch_dependents();
+    // the next GEMM's first weight tiles (constant: no wait needed) start streaming into L2 meanwhile
+    l2_prefetch_slice(pf, pf_bytes, (int64_t)blockIdx.x * blockDim.x + threadIdx.x, (int64_t)gridDim.x * blockDim.x);
     pdl_wait();
     __shared__ float s_genc;
     if (threadIdx.x < 32) {
@@ -116,7 +119,8 @@ static int amax_grid(int64_t nvec) {
 // Second pass: every CTA folds the npartial amax words (BF16 bits) into the tensor amax, then quantises.
 static void launch_quantize(const uint16_t* x, int64_t rows, int64_t K, const float* global_scale_in,
                             const uint32_t* partial, int npartial, uint8_t* q, uint8_t* sf, float* global_scale_out,
-                            nvfp4_sf_layout layout, cudaStream_t s) {
+                            nvfp4_sf_layout layout, cudaStream_t s, const void* l2_next = nullptr,
+                            size_t l2_next_bytes = 0) {
     const int64_t nblk = rows * K / 16;
     int64_t grid_q = (nblk + kThreads - 1) / kThreads;
     const int64_t cap = (int64_t)device_sm_count() * 16;
@@ -126,7 +130,8 @@ static void launch_quantize(const uint16_t* x, int64_t rows, int64_t K, const fl
                   : layout == NVFP4_SF_KSTAGE  ? quantize_kernel<NVFP4_SF_KSTAGE>
                                                : quantize_kernel<NVFP4_SF_ROWMAJOR>;
     launch_pdl(kernel, dim3((int)grid_q), dim3(kThreads), 0, s, reinterpret_cast<const uint4*>(x), rows, K,
-               global_scale_in, partial, npartial, reinterpret_cast<uint2*>(q), sf, global_scale_out);
+               global_scale_in, partial, npartial, reinterpret_cast<uint2*>(q), sf, global_scale_out,
+               static_cast<const uint8_t*>(l2_next), (int64_t)l2_next_bytes);
 }
 
 }  // namespace nvfp4
@@ -168,9 +173,11 @@ extern "C" nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t rows, int64_t 
     return check_launch();
 }
 
-extern "C" nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows, int64_t K, const uint32_t* amax_bits,
-                                                 uint8_t* q, uint8_t* sf, float* global_scale_out,
-                                                 nvfp4_sf_layout layout, nvfp4_stream_t stream) {
+extern "C" nvfp4_status nvfp4_quantize_from_amax_prefetch(const uint16_t* x, int64_t rows, int64_t K,
+                                                          const uint32_t* amax_bits, uint8_t* q, uint8_t* sf,
+                                                          float* global_scale_out, nvfp4_sf_layout layout,
+                                                          const void* l2_next, size_t l2_next_bytes,
+                                                          nvfp4_stream_t stream) {
     if (!x || !q || !sf || !global_scale_out || !amax_bits) return NVFP4_ERR_INVALID_ARG;
     if (rows <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
     if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_MMA_TILED && layout != NVFP4_SF_KSTAGE)
@@ -180,10 +187,18 @@ extern "C" nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows
     if (layout == NVFP4_SF_KSTAGE && K % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(x) || !aligned8(q) || (layout == NVFP4_SF_KSTAGE && !aligned16(sf))) return NVFP4_ERR_MISALIGNED;
     if (((uintptr_t)global_scale_out & 3u) || ((uintptr_t)amax_bits & 3u)) return NVFP4_ERR_MISALIGNED;
+    if (l2_next == nullptr) l2_next_bytes = 0;
     launch_quantize(x, rows, K, nullptr, amax_bits, 1, q, sf, global_scale_out, layout,
-                    reinterpret_cast<cudaStream_t>(stream));
+                    reinterpret_cast<cudaStream_t>(stream), l2_next, l2_next_bytes);
     count_launch();
     return check_launch();
+}
+
+extern "C" nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows, int64_t K, const uint32_t* amax_bits,
+                                                 uint8_t* q, uint8_t* sf, float* global_scale_out,
+                                                 nvfp4_sf_layout layout, nvfp4_stream_t stream) {
+    return nvfp4_quantize_from_amax_prefetch(x, rows, K, amax_bits, q, sf, global_scale_out, layout, nullptr, 0,
+                                             stream);
 }
 
 extern "C" nvfp4_status nvfp4_amax(const uint16_t* x, int64_t rows, int64_t K, uint32_t* amax_bits,

@@ -69,3 +69,25 @@ def test_bad_expert_id_latches_status():
     x = gpu_bf16(workloads.random_bf16_bits((T, H), seed=5))
     nv.quantize_permute(x, torch.from_numpy(ids).cuda(), E)
     assert nv.device_status() == 8   # NVFP4_ERR_DEVICE_INPUT
+
+
+def test_l2_prefetch_hint_changes_no_byte():
+    # moe_quantize_permute_prefetch and nvfp4_quantize_from_amax_prefetch with a 96 MB hint (the decode layer's)
+    # give the bytes of the calls without one; a hint longer than its tensor is clipped to the tensor by the binding
+    T, E, k, H = 512, 256, 8, 6144
+    ids, _ = workloads.routing(T, E, k, "uniform", seed=5)
+    x = gpu_bf16(workloads.random_bf16_bits((T, H), seed=6))
+    idsd = torch.from_numpy(ids).cuda()
+    weights = torch.empty(128 << 20, dtype=torch.uint8, device="cuda")
+    plain, g0 = nv.quantize_permute(x, idsd, E)
+    hinted, g1 = nv.quantize_permute(x, idsd, E, l2_next=weights, l2_next_bytes=96 << 20)
+    h = gpu_bf16(workloads.random_bf16_bits((T * k, 2048), seed=7))
+    amax = nv.amax(h)
+    q0, sf0, gh0 = nv.quantize_from_amax(h, amax, layout=nv.SF_KSTAGE)
+    q1, sf1, gh1 = nv.quantize_from_amax(h, amax, layout=nv.SF_KSTAGE, l2_next=weights, l2_next_bytes=1 << 40)
+    torch.cuda.synchronize()
+    assert nv.device_status() == 0
+    for name in ("q_perm", "sf_perm", "offsets", "perm_src", "inv_perm"):
+        assert torch.equal(getattr(plain, name), getattr(hinted, name)), name
+    assert torch.equal(g0, g1)
+    assert torch.equal(q0, q1) and torch.equal(sf0, sf1) and torch.equal(gh0, gh1)

@@ -165,3 +165,15 @@ def test_binding_rejects_short_or_strided_buffers():
     with pytest.raises(TypeError):
         need(torch.empty(1, dtype=torch.float64), 4, "g", torch.float32)
     assert need(torch.empty((3, 5), dtype=torch.bfloat16), 30, "out", torch.bfloat16).numel() == 15
+
+
+def test_layer_l2_prefetch_hints_follow_the_header_rule(L):
+    # moe_layer_l2_prefetch_bytes: 96 MB of the gate/up and 48 MB of the down weights (or the whole tensor when
+    # smaller) for batches under 32 rows per expert; nothing from 32 rows per expert on. Host arithmetic only.
+    mb = 1 << 20
+    assert nv.layer_l2_prefetch_bytes(512, 8, 256, 6144, 2048) == (96 * mb, 48 * mb)      # decode, 16 rows/expert
+    assert nv.layer_l2_prefetch_bytes(1024, 8, 256, 6144, 2048) == (0, 0)                 # Zipf, 32 rows/expert
+    assert nv.layer_l2_prefetch_bytes(8192, 8, 256, 6144, 2048) == (0, 0)                 # prefill
+    # 4 experts, H = 256, I = 128: w13 = 4 * 256 * (128 + 16) bytes, w2 = 4 * 256 * (64 + 8) bytes
+    assert nv.layer_l2_prefetch_bytes(4, 1, 4, 256, 128) == (4 * 256 * 144, 4 * 256 * 72)
+    assert nv.layer_l2_prefetch_bytes(0, 8, 256, 6144, 2048) == (0, 0)
