@@ -18,9 +18,11 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kColsPerThread = 8;
-// Grid size in CTAs per SM. About 4 CTAs fit on an SM at once (register-bound), so this is several waves of
-// short token walks. Measured on B200 (same box, bit-identical outputs): 3 per SM (one wave, long walks)
-// 191.8 us at 8192 tokens and 17.7 us at 512; 12, 24 and 40 per SM 172-174 us and 12.6 us (24 best).
+// Grid size in CTAs per SM. 4 CTAs fit on an SM at once (the launch bound keeps a thread at 64 registers:
+// without it ptxas took 86-108 and 2 CTAs fit; measured 204 -> 170 us at 8192 tokens, 14.7 -> 12.1 us at 512,
+// same bits), so this is several waves of short token walks. Measured on B200 (same box, bit-identical
+// outputs): 3 per SM (one wave, long walks) 191.8 us at 8192 tokens and 17.7 us at 512; 12, 24 and 40 per SM
+// 172-174 us and 12.6 us (24 best).
 constexpr int kCtasPerSm = 24;
 
 // Each thread owns one 16-byte column group and walks tokens blockIdx.y, + gridDim.y, ... (a grid of
@@ -30,7 +32,7 @@ constexpr int kCtasPerSm = 24;
 // one round of row reads per token (the combine is bound by that latency at decode sizes). A row index past
 // the last row of y is skipped and latched as bad input.
 template <bool kOneGroup>   // k <= 8
-__global__ void __launch_bounds__(kThreads) combine_kernel(const uint16_t* __restrict__ y,
+__global__ void __launch_bounds__(kThreads, 4) combine_kernel(const uint16_t* __restrict__ y,
                                                            const int32_t* __restrict__ inv_perm,
                                                            const float* __restrict__ w, int64_t T, int32_t k,
                                                            int64_t H, uint16_t* __restrict__ out, uint32_t* status) {
