@@ -271,7 +271,7 @@ NVFP4_API nvfp4_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, i
 /*   Shapes: 1 <= E <= 1024, K % 128 == 0, max_rows >= 0; NONE: N % 128 == 0;*/
 /*   SWIGLU: N % 256 == 0 (N / 2 % 128 == 0: the gate and the up rows of an  */
 /*   output column sit in the same TMEM lane of two 128-row weight blocks,  */
-/*   so half-blocks of gate rows are not offered; the survey's N / 2 % 64   */
+/*   so half-blocks of gate rows are not offered: a SwiGLU N / 2 % 64      */
 /*   is narrowed to this). K % 256 == 128 runs a last stage of 128 K-       */
 /*   elements; NONE with N % 256 == 128 a last column tile of 128 rows.     */
 /*   All pointers device, 16-byte aligned. Rows outside every expert's range */
