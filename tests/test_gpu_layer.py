@@ -61,3 +61,9 @@ def test_one_call_layer_equals_call_by_call(name):
     assert torch.equal(out_one.view(torch.int16), out_staged.view(torch.int16))
     assert torch.equal(out_two.view(torch.int16), out_one.view(torch.int16))
     assert torch.isfinite(out_one.float()).all() and out_one.float().abs().max() > 0
+
+
+def test_smoke_entry_point_passes():
+    # __graft_entry__.smoke(): one small layer against the oracle, stage by stage
+    import __graft_entry__
+    __graft_entry__.smoke()
