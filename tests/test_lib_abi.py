@@ -177,3 +177,14 @@ def test_layer_l2_prefetch_hints_follow_the_header_rule(L):
     # 4 experts, H = 256, I = 128: w13 = 4 * 256 * (128 + 16) bytes, w2 = 4 * 256 * (64 + 8) bytes
     assert nv.layer_l2_prefetch_bytes(4, 1, 4, 256, 128) == (4 * 256 * 144, 4 * 256 * 72)
     assert nv.layer_l2_prefetch_bytes(0, 8, 256, 6144, 2048) == (0, 0)
+
+
+def test_prefetch_forms_reject_arguments_like_the_plain_calls(L):
+    # the *_prefetch calls validate exactly as the plain ones, before any CUDA call; a hint is never required
+    p = ctypes.c_void_p(16)
+    assert L.nvfp4_quantize_from_amax_prefetch(None, 4, 32, None, None, None, None, 0, p, 1 << 20, None) == 1
+    assert L.nvfp4_quantize_from_amax_prefetch(p, 4, 32, ctypes.c_void_p(18), p, p, p, 0, p, 64, None) == 2
+    assert L.nvfp4_quantize_from_amax_prefetch(p, 4, 24, p, p, p, p, 0, None, 0, None) == 3     # K % 16 != 0
+    assert L.moe_quantize_permute_prefetch(None, 4, 256, p, 2, 8, p, p, 2, p, p, p, p, p, 1 << 20, p, 64, None) == 1
+    assert L.moe_quantize_permute_prefetch(p, 4, 192, p, 2, 8, p, p, 2, p, p, p, p, p, 1 << 20, None, 0, None) == 3
+    assert L.moe_quantize_permute_prefetch(p, 4, 256, p, 2, 8, p, p, 2, p, p, p, p, None, 0, p, 64, None) == 4
