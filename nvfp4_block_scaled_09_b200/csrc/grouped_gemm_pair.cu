@@ -19,9 +19,10 @@
 // last full tile that ride on it in the configuration with row tails; the scale
 // ring takes the rest of tensor memory), so the epilogue warps first drain it
 // into registers as final BF16 values and hand it back to the MMA warp; staging
-// and storing those values then overlaps the next tile's main loop. Two
-// configurations (Cfg below): row tails, 4 stages and a 3-slot scale ring for
-// several experts; 5 stages and a scale slot per stage for one expert.
+// and storing those values then overlaps the next tile's main loop. Three
+// configurations (Cfg below): row tails, 5 stages and a 3-slot scale ring for up
+// to 256 experts (4 stages beyond); 5 stages and a scale slot per stage for one
+// expert.
 //
 // The kernel is a template on the epilogue mode, the configuration and SwiGLU or plain output, so each
 // instantiation carries only its own epilogue (measured on B200: a runtime SwiGLU switch cost 1-4% on
@@ -69,12 +70,10 @@ constexpr int kCodeBytes = 16384;
 constexpr int kTileSFBytes = 2048;
 constexpr int kOffA = 0;                          // 128 weight rows x 128 B (SwiGLU: gate/up slabs of 16 rows, interleaved)
 constexpr int kOffSFA = kCodeBytes;               // scales of one packed tile (SwiGLU: gate tile's, then up tile's)
-constexpr int kOffB = kOffSFA + 2 * kTileSFBytes;  // this CTA's half of the activation rows
 constexpr int kThreads = 512;                     // warps: 0 loads, 2 MMA, 4-7 + 12-15 epilogue, 8-11 scales
 constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant, alternating 32-token chunks
 constexpr int kChunksPerWarp = kBNMax / 32 / 2;   // 32-token chunks one epilogue warp drains per tile
                                                   // (plus the tail chunk, columns 256-287, on warps 4-7)
-constexpr int kMaxE = 1024;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int kTileRing = 4;                      // work items the even CTA may publish ahead
@@ -82,9 +81,9 @@ constexpr int kTileConsumersPerCta = 13;          // even CTA: MMA warp + 4 scal
                                                   // odd CTA: its producer + 4 scale writers + 8 epilogue warps
 constexpr int kTileConsumers = 2 * kTileConsumersPerCta;
 
-template <int kStagesT, int kTailT>
+template <int kStagesT, int kTailT, int kMaxET, int kStgElemsT, int kFinTokT>
 struct SharedT {
-    alignas(16) uint16_t ostage[kEpiWarps][32 * 32];  // epilogue: one 32-token x 32-column BF16 block per warp
+    alignas(16) uint16_t ostage[kEpiWarps][kStgElemsT];  // epilogue: one 32-token chunk of BF16 outputs per warp
     uint64_t tq_full[kTileRing];  // the even CTA published tq[i] (in this CTA's copy of the ring)
     uint64_t tq_empty[kTileRing]; // even CTA: every consumer warp of both CTAs read entry i
     int32_t tq[kTileRing];        // work item index (>= total: no more work)
@@ -97,23 +96,30 @@ struct SharedT {
     uint32_t tmem_base;
     int abort;
     int32_t total_tiles;
-    int32_t off[kMaxE + 1];
-    int32_t tile_start[kMaxE + 1];
-    int32_t fin_tok[kBNMax + kTailT];   // fused combine: tokens of this tile whose last row this CTA wrote
+    int32_t off[kMaxET + 1];
+    int32_t tile_start[kMaxET + 1];
+    int32_t fin_tok[kFinTokT];    // fused combine: tokens of this tile whose last row this CTA wrote
     uint64_t fin_bar;             // fused combine: this CTA's 8 epilogue warps meet (bounded waits)
 };
 
-// Two configurations of the kernel, chosen per launch:
-// - kTails (grouped GEMMs): an expert's rows past its last full 256-row tile ride on that tile when there
-//   are at most kTailMax = 32 of them (a second MMA of N = 32 into accumulator columns 256-287) instead
-//   of taking a tile of their own, which would stream the whole weight tile again for a few rows. Their
-//   buffers cost a shared-memory stage (4 of 43 KB) and the scales' TMEM ring is 3 slots deep (a slot is
-//   written just before its MMAs, so it needs fewer slots than there are stages).
-// - no tails (one expert, dense): 5 stages of 40 KB, one scale slot per stage.
-template <bool kTails>
+// Three configurations of the kernel, chosen per launch (kConf):
+// 0 (one expert, dense): 5 stages, one TMEM scale slot per stage.
+// 1, 2 (grouped GEMMs): an expert's rows past its last full 256-row tile ride on that tile when there are at
+//   most kTailMax = 32 of them (a second MMA of N = 32 into accumulator columns 256-287) instead of taking a tile
+//   of their own, which would stream the whole weight tile again for a few rows. The tail's accumulator columns
+//   leave TMEM room for a ring of 3 scale slots (a slot is written just before its MMAs, so it needs fewer slots
+//   than there are stages). Configuration 2 (up to 256 experts) holds 5 data stages: its scheduler tables are
+//   sized for 256 experts, and a SwiGLU tile's staging chunk is half a plain one's. Configuration 1 (up to
+//   1024 experts) holds 4. Measured on B200 (prefill, same box): 3 data stages against 4 cost 8% (gate/up) and
+//   6% (down).
+// The scales of the weight tile take 4 KB of a stage with SwiGLU (the gate and the up tile's) and 2 KB without.
+template <int kConf, bool kSw, bool kFin>
 struct Cfg {
+    static constexpr bool kTails = kConf != 0;
     static constexpr int kTailMax = kTails ? 32 : 0;
-    static constexpr int kStages = kTails ? 4 : 5;
+    static constexpr int kStages = kConf == 1 ? 4 : 5;
+    static constexpr int kMaxE = kConf == 2 ? 256 : 1024;        // experts the scheduler tables hold
+    static constexpr int kOffB = kOffSFA + (kSw ? 2 : 1) * kTileSFBytes;  // this CTA's half of the activation rows
     static constexpr int kOffBT = kOffB + (kBNMax / 2) * kRowBytes;       // this CTA's half of the tail rows
     static constexpr int kOffSFB = kOffBT + (kTailMax / 2) * kRowBytes;   // scales of all the tile's rows, 16 B each
     static constexpr int kStageBytes = (kOffSFB + (kBNMax + kTailMax) * 16 + 1023) / 1024 * 1024;
@@ -123,7 +129,8 @@ struct Cfg {
     static constexpr uint32_t kSFSlot = (kTails ? 16 : 12) * kKSteps;
     static constexpr uint32_t kSFTail = 12 * kKSteps;          // tail SFB of K step kc at slot + kSFTail + 4 kc
     static constexpr uint32_t kTmemSFRing = kAccCols;
-    using Shared = SharedT<kStages, kTailMax>;
+    // a staged chunk: 32 tokens x 16 (SwiGLU) or 32 output columns
+    using Shared = SharedT<kStages, kTailMax, kMaxE, 32 * (kSw ? 16 : 32), kFin ? kBNMax + kTailMax : 1>;
     static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Shared);
     static_assert(kTmemSFRing + kSFSlots * kSFSlot <= kTmemCols, "TMEM budget");
     static_assert(kStageBytes % 1024 == 0 && kOffB % 1024 == 0 && kOffBT % 1024 == 0,
@@ -313,12 +320,12 @@ __device__ __forceinline__ void build_schedule(S& sh, const Params& p, int32_t n
 namespace nvfp4 {
 namespace gp {
 
-template <int kEpi, bool kTails, bool kSw>
+template <int kEpi, int kConf, bool kSw>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a_full,
                              const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_wsw,
                              const __grid_constant__ CUtensorMap tm_wsf, const Params p) {
-    using C = Cfg<kTails>;
+    using C = Cfg<kConf, kSw, kEpi == kEpiFinalize>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
@@ -360,6 +367,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // everything above overlaps the previous kernel; global memory only from here on
     pdl_launch_dependents();
     pdl_wait();
+    if (E > C::kMaxE) {   // the launcher picks a configuration whose tables hold E; never taken
+        if (tid == 0) atomicOr(p.ctl.status, kStatusBadInput);
+        return;
+    }
     for (int i = tid; i <= E; i += kThreads) sh.off[i] = __ldg(p.offsets + i);
     __syncthreads();
     build_schedule<C::kTailMax>(sh, p, n_col_tiles);
@@ -437,10 +448,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         bulk_load(sb + kOffA, g_tile + ko, kPackedTileBytes, bar, pol_w);   // codes + scales
                     }
                     if (my_rows == kBNMax / 2) {
-                        tma_load_2d(sb + kOffB, &tm_a_full, kt * kRowBytes, my_row0, bar, pol_a);
+                        tma_load_2d(sb + C::kOffB, &tm_a_full, kt * kRowBytes, my_row0, bar, pol_a);
                     } else {
                         for (int32_t i = 0; i < my_rows / kBoxRows; i++)
-                            tma_load_2d(sb + kOffB + i * kBoxRows * kRowBytes, &tm_a, kt * kRowBytes,
+                            tma_load_2d(sb + C::kOffB + i * kBoxRows * kRowBytes, &tm_a, kt * kRowBytes,
                                         my_row0 + i * kBoxRows, bar, pol_a);
                     }
                     if (C::kTailMax > 0 && t.tail > 0)
@@ -561,7 +572,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         // the tile's 256 columns, and the tail rows into columns 256-287
                         auto mma_step = [&](int kc) {
                             const uint64_t adesc = make_smem_desc(sb + kOffA + kc * 32, 16, 1024, 2);
-                            mma_mxf4nvf4_pair(tmem, adesc, make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2), idesc,
+                            mma_mxf4nvf4_pair(tmem, adesc, make_smem_desc(sb + C::kOffB + kc * 32, 16, 1024, 2), idesc,
                                               sf + 4 * kc, sf + 16 + 8 * kc, (kt | kc) != 0);
                             if (tail)
                                 mma_mxf4nvf4_pair(tmem + kBNMax, adesc, make_smem_desc(sb + C::kOffBT + kc * 32, 16, 1024, 2),
@@ -838,39 +849,48 @@ using namespace nvfp4;
 
 namespace nvfp4 {
 
+// the largest of the instantiated configurations (SwiGLU, plain, fused combine in each of the three)
+template <int kConf>
+static constexpr size_t pair_conf_smem() {
+    constexpr size_t a = gp::Cfg<kConf, true, false>::kSmemBytes, b = gp::Cfg<kConf, false, false>::kSmemBytes,
+                     c = gp::Cfg<kConf, false, true>::kSmemBytes;
+    return a > b ? (a > c ? a : c) : (b > c ? b : c);
+}
 size_t pair_gemm_smem_bytes() {
-    return gp::Cfg<true>::kSmemBytes > gp::Cfg<false>::kSmemBytes ? gp::Cfg<true>::kSmemBytes
-                                                                  : gp::Cfg<false>::kSmemBytes;
+    constexpr size_t c0 = pair_conf_smem<0>(), c1 = pair_conf_smem<1>(), c2 = pair_conf_smem<2>();
+    return c0 > c1 ? (c0 > c2 ? c0 : c2) : (c1 > c2 ? c1 : c2);
 }
 int pair_gemm_tokens_max() { return gp::kBNMax; }
 int pair_gemm_store_cols(int swiglu) { return swiglu ? 16 : 32; }  // 32 tokens x this many BF16 columns
 
 // The shared-memory opt-in of one instantiation, once per device (thread-safe).
-template <int kEpi, bool kTails, bool kSw>
+template <int kEpi, int kConf, bool kSw>
 static bool pair_kernel_configured(int dev) {
     static std::once_flag once[64];
     static bool ok[64] = {};
     std::call_once(once[dev], [&] {
-        ok[dev] = cudaFuncSetAttribute(gp::grouped_gemm_pair_kernel<kEpi, kTails, kSw>,
+        ok[dev] = cudaFuncSetAttribute(gp::grouped_gemm_pair_kernel<kEpi, kConf, kSw>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)gp::Cfg<kTails>::kSmemBytes) == cudaSuccess;
+                                       (int)gp::Cfg<kConf, kSw, kEpi == kEpiFinalize>::kSmemBytes) == cudaSuccess;
     });
     return ok[dev];
 }
 
 // As many pairs as can be resident at once (the persistent grid), once per device and configuration.
-template <bool kTails>
+template <int kConf>
 static nvfp4_status pair_grid(int dev, int& grid) {
     static std::once_flag once[64];
     static int grid_for[64] = {};
     static nvfp4_status set_result[64] = {};
     std::call_once(once[dev], [&] {
         set_result[dev] = NVFP4_ERR_CUDA;
-        if (!pair_kernel_configured<kEpiPlain, kTails, false>(dev)) return;
+        // the SwiGLU instantiation: the configuration's largest shared memory but for the fused combine's
+        // table, and every instantiation fits one CTA per SM
+        if (!pair_kernel_configured<kEpiPlain, kConf, true>(dev)) return;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)device_sm_count() / 2 * 2);
         cfg.blockDim = dim3(gp::kThreads);
-        cfg.dynamicSmemBytes = gp::Cfg<kTails>::kSmemBytes;
+        cfg.dynamicSmemBytes = gp::Cfg<kConf, true, false>::kSmemBytes;
         cudaLaunchAttribute attr;
         attr.id = cudaLaunchAttributeClusterDimension;
         attr.val.clusterDim.x = 2;
@@ -879,7 +899,7 @@ static nvfp4_status pair_grid(int dev, int& grid) {
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, gp::grouped_gemm_pair_kernel<kEpiPlain, kTails, false>, &cfg) !=
+        if (cudaOccupancyMaxActiveClusters(&clusters, gp::grouped_gemm_pair_kernel<kEpiPlain, kConf, true>, &cfg) !=
                 cudaSuccess ||
             clusters <= 0) {
             set_result[dev] = NVFP4_ERR_SMEM_BUDGET;
@@ -892,38 +912,38 @@ static nvfp4_status pair_grid(int dev, int& grid) {
     return set_result[dev];
 }
 
-template <bool kTails>
+template <int kConf>
 static nvfp4_status launch_pair_config(int dev, const CUtensorMap& tm_a, const CUtensorMap& tm_a_full,
                                        const CUtensorMap& tm_out, const CUtensorMap& tm_wsw, const CUtensorMap& tm_wsf,
                                        const gp::Params& prm, cudaStream_t s) {
     int grid = 0;
-    const nvfp4_status st = pair_grid<kTails>(dev, grid);
+    const nvfp4_status st = pair_grid<kConf>(dev, grid);
     if (st != NVFP4_OK) return st;
-    const size_t smem = gp::Cfg<kTails>::kSmemBytes;
-    // every instantiation has the plain one's resources (same shared memory, threads and cluster shape)
-    // quantised h is SWIGLU only, the fused combine NONE only (the caller checked)
+    // every instantiation runs one CTA per SM in clusters of two; quantised h is SWIGLU only, the fused
+    // combine NONE only (the caller checked)
     if (prm.qo.q != nullptr) {
-        if (!pair_kernel_configured<kEpiQuant, kTails, true>(dev)) return NVFP4_ERR_CUDA;
-        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiQuant, kTails, true>, dim3(grid), dim3(gp::kThreads), smem, s,
-                   tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+        if (!pair_kernel_configured<kEpiQuant, kConf, true>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiQuant, kConf, true>, dim3(grid), dim3(gp::kThreads),
+                   gp::Cfg<kConf, true, false>::kSmemBytes, s, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
     } else if (prm.fin.out != nullptr) {
-        if (!pair_kernel_configured<kEpiFinalize, kTails, false>(dev)) return NVFP4_ERR_CUDA;
-        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiFinalize, kTails, false>, dim3(grid), dim3(gp::kThreads), smem,
-                   s, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+        if (!pair_kernel_configured<kEpiFinalize, kConf, false>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiFinalize, kConf, false>, dim3(grid), dim3(gp::kThreads),
+                   gp::Cfg<kConf, false, true>::kSmemBytes, s, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
     } else if (prm.swiglu) {
-        if (!pair_kernel_configured<kEpiPlain, kTails, true>(dev)) return NVFP4_ERR_CUDA;
-        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain, kTails, true>, dim3(grid), dim3(gp::kThreads), smem, s,
-                   tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+        if (!pair_kernel_configured<kEpiPlain, kConf, true>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain, kConf, true>, dim3(grid), dim3(gp::kThreads),
+                   gp::Cfg<kConf, true, false>::kSmemBytes, s, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
     } else {
-        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain, kTails, false>, dim3(grid), dim3(gp::kThreads), smem, s,
-                   tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
+        if (!pair_kernel_configured<kEpiPlain, kConf, false>(dev)) return NVFP4_ERR_CUDA;
+        launch_pdl(gp::grouped_gemm_pair_kernel<kEpiPlain, kConf, false>, dim3(grid), dim3(gp::kThreads),
+                   gp::Cfg<kConf, false, false>::kSmemBytes, s, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm);
     }
     return NVFP4_OK;
 }
 
 // Launches the pair kernel; the caller validated every argument (same contract as the one-SM kernel).
-// Several experts: the configuration that lets up to 32 rows past a full tile ride on it; one expert
-// (a dense GEMM): the deeper pipeline without that.
+// Several experts: a configuration that lets up to 32 rows past a full tile ride on it; one expert (a dense
+// GEMM): the configuration without that and with a scale slot per stage.
 nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_a_full,
                                       const CUtensorMap& tm_out, const CUtensorMap& tm_wsw,
                                       const CUtensorMap& tm_wsf, const uint8_t* a_sf,
@@ -953,8 +973,11 @@ nvfp4_status launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap
     prm.ctl.status = status;
     prm.ctl.timeout_ns = wait_timeout_ns();
     prm.ctl.flags = debug_flags();
-    const nvfp4_status st = E > 1 ? launch_pair_config<true>(dev, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm, s)
-                                  : launch_pair_config<false>(dev, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm, s);
+    // one expert: no row tails; up to 256 experts: row tails and 5 data stages; more: row tails and 4
+    const nvfp4_status st =
+        E == 1     ? launch_pair_config<0>(dev, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm, s)
+        : E <= 256 ? launch_pair_config<2>(dev, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm, s)
+                   : launch_pair_config<1>(dev, tm_a, tm_a_full, tm_out, tm_wsw, tm_wsf, prm, s);
     if (st != NVFP4_OK) return st;
     count_launch();
     return check_launch();
