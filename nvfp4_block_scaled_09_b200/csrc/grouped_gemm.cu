@@ -74,6 +74,7 @@ constexpr int kABlockBytes = kBM * kRowBytes;    // 16 KB
 constexpr int kSFAtomBytes = 512;                // 128 rows x 4 scales
 constexpr int kSFStageBytes = kKSteps * kSFAtomBytes;
 constexpr int kPackedTileBytes = kABlockBytes + kSFStageBytes;  // one packed weight tile (codes + scales)
+static_assert(kPackedTileBytes % 1024 == 0, "weight tiles keep the 128-byte swizzle's 1024-byte alignment");
 // Stage layout: [A0 codes | A0 scales][A1 codes | A1 scales][B codes][B scales]
 constexpr int kOffA0 = 0;
 constexpr int kOffSFA0 = kABlockBytes;
@@ -414,11 +415,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) {
                     const uint32_t sb = smem_u32(stages + (size_t)stage * kStageBytes);
                     const uint32_t sf = tmem + kTmemSFRing + stage * kTmemSFSlot;
+                    // the stage's first descriptors; a K-step is 32 bytes on and a weight tile kPackedTileBytes on,
+                    // added in the address field (bits 0-13 hold address / 16, below 2^14 in shared memory)
+                    const uint64_t b0 = make_smem_desc(sb + kOffB, 16, 1024, 2);
+                    const uint64_t a0 = make_smem_desc(sb, 16, 1024, 2);
+                    const uint32_t acc0 = kt != 0 ? 1u : 0u;
                     auto mma_step = [&](int kc, int a) {
-                        const uint64_t bdesc = make_smem_desc(sb + kOffB + kc * 32, 16, 1024, 2);
-                        const uint64_t adesc = make_smem_desc(sb + a * kPackedTileBytes + kc * 32, 16, 1024, 2);
-                        mma_mxf4nvf4(tmem + abuf * (kNumA * kAccCols) + a * kAccCols, adesc, bdesc, idesc,
-                                     sf + a * 4 * kKSteps + 4 * kc, sf + kNumA * 4 * kKSteps + 4 * kc, (kt | kc) != 0);
+                        mma_mxf4nvf4(tmem + abuf * (kNumA * kAccCols) + a * kAccCols,
+                                     a0 + (uint64_t)(a * (kPackedTileBytes >> 4) + 2 * kc), b0 + 2 * kc, idesc,
+                                     sf + a * 4 * kKSteps + 4 * kc, sf + kNumA * 4 * kKSteps + 4 * kc, kc != 0 ? 1u : acc0);
                     };
                     if (n_a == kNumA && (kt != ksteps_total - 1 || last_ksteps == kKSteps)) {
 #pragma unroll
