@@ -35,6 +35,7 @@ headline workload; it is a slow baseline, not a target.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import subprocess
@@ -855,7 +856,9 @@ def main(argv=None):
     import torch
     import torch.distributed as dist
     if world > 1:
-        dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank))
+        # a short bound on every collective: a rank that stops ends the others' next barrier with an error
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local_rank),
+                                timeout=datetime.timedelta(seconds=300))
     from nvfp4_block_scaled_09_b200 import build as nvbuild
     nvbuild.build()
     import nvfp4_block_scaled_09_b200 as nv

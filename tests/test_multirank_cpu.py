@@ -2,6 +2,7 @@
 (max over ranks), every rank draws its own replica inputs, and the reference arm
 under torchrun prints exactly one JSON line from rank 0 while the other ranks
 exit 0 without work."""
+import datetime
 import json
 import os
 import socket
@@ -28,7 +29,7 @@ def _rank_main(rank, world, port, out_q):
     sys.path.insert(0, ROOT)
     import bench
     import workloads
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         m = bench.max_over_ranks(1.5 + rank, world, "cpu")
         ids, _ = workloads.routing(64, 16, 4, "uniform", bench.replica_seed(0, rank))
