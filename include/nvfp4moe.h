@@ -146,8 +146,11 @@ NVFP4_API nvfp4_status nvfp4_quantize_from_amax(const uint16_t* x, int64_t rows,
 /* nvfp4_quantize_from_amax_prefetch: the same, and while it runs it pulls  */
 /* the first l2_next_bytes bytes at l2_next (device memory that no kernel   */
 /* in flight writes, e.g. the next GEMM's packed expert weights, taken by   */
-/* its schedule in address order) into L2 with plain prefetches. A hint: the */
+/* its schedule in address order) into L2: bulk L2 prefetches of 64 KB from */
+/* one thread per CTA (the kernel lasts until they land). A hint: the       */
 /* outputs do not depend on it; l2_next NULL or 0 bytes prefetches nothing. */
+/* Otherwise l2_next is 16-byte aligned (else NVFP4_ERR_MISALIGNED) and the */
+/* whole range lies inside one device allocation (not checked).             */
 NVFP4_API nvfp4_status nvfp4_quantize_from_amax_prefetch(const uint16_t* x, int64_t rows, int64_t K,
                                                const uint32_t* amax_bits, uint8_t* q, uint8_t* sf,
                                                float* global_scale_out, nvfp4_sf_layout layout,
@@ -205,7 +208,8 @@ NVFP4_API nvfp4_status moe_quantize_permute(const uint16_t* x, int32_t T, int64_
                                   int32_t* perm_src, int32_t* inv_perm, void* ws, size_t ws_bytes,
                                   nvfp4_stream_t stream);
 /* moe_quantize_permute_prefetch: the same, with the L2 prefetch hint of     */
-/* nvfp4_quantize_from_amax_prefetch (issued by the two-kernel path only).  */
+/* nvfp4_quantize_from_amax_prefetch and its rules (issued by the           */
+/* two-kernel path only).                                                   */
 NVFP4_API nvfp4_status moe_quantize_permute_prefetch(const uint16_t* x, int32_t T, int64_t H,
                                            const int32_t* topk_ids, int32_t k, int32_t E, uint8_t* q_perm,
                                            uint8_t* sf_perm, nvfp4_sf_layout sf_perm_layout, float* g_x,

@@ -534,6 +534,8 @@ extern "C" nvfp4_status moe_quantize_permute_prefetch(const uint16_t* x, int32_t
     if (!aligned16(x) || !aligned16(topk_ids) || !aligned16(q_perm) || !aligned16(sf_perm) ||
         !aligned16(expert_offsets) || !aligned16(perm_src) || !aligned16(inv_perm) || ((uintptr_t)g_x & 3u))
         return NVFP4_ERR_MISALIGNED;
+    if (l2_next == nullptr) l2_next_bytes = 0;
+    if (l2_next_bytes != 0 && !aligned16(l2_next)) return NVFP4_ERR_MISALIGNED;   // bulk prefetches start on 16 B
     const size_t need = moe_quantize_permute_workspace_size(T, k, E, H);
     if (!ws || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
     if (!aligned16(ws)) return NVFP4_ERR_MISALIGNED;
@@ -542,7 +544,6 @@ extern "C" nvfp4_status moe_quantize_permute_prefetch(const uint16_t* x, int32_t
     uint8_t* sf_x = q_x + align256((size_t)T * (size_t)H / 2);
     uint8_t* scratch = sf_x + align256((size_t)T * (size_t)H / 16);
     const size_t scratch_bytes = need - (size_t)(scratch - b);
-    if (l2_next == nullptr) l2_next_bytes = 0;
     return quantize_permute(x, T, H, topk_ids, k, E, q_perm, sf_perm, sf_perm_layout, g_x, expert_offsets, perm_src,
                             inv_perm, q_x, sf_x, scratch, scratch_bytes, reinterpret_cast<cudaStream_t>(stream),
                             l2_next, l2_next_bytes);

@@ -188,6 +188,7 @@ extern "C" nvfp4_status nvfp4_quantize_from_amax_prefetch(const uint16_t* x, int
     if (!aligned16(x) || !aligned8(q) || (layout == NVFP4_SF_KSTAGE && !aligned16(sf))) return NVFP4_ERR_MISALIGNED;
     if (((uintptr_t)global_scale_out & 3u) || ((uintptr_t)amax_bits & 3u)) return NVFP4_ERR_MISALIGNED;
     if (l2_next == nullptr) l2_next_bytes = 0;
+    if (l2_next_bytes != 0 && !aligned16(l2_next)) return NVFP4_ERR_MISALIGNED;   // bulk prefetches start on 16 B
     launch_quantize(x, rows, K, nullptr, amax_bits, 1, q, sf, global_scale_out, layout,
                     reinterpret_cast<cudaStream_t>(stream), l2_next, l2_next_bytes);
     count_launch();

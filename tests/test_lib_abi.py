@@ -188,3 +188,7 @@ def test_prefetch_forms_reject_arguments_like_the_plain_calls(L):
     assert L.moe_quantize_permute_prefetch(None, 4, 256, p, 2, 8, p, p, 2, p, p, p, p, p, 1 << 20, p, 64, None) == 1
     assert L.moe_quantize_permute_prefetch(p, 4, 192, p, 2, 8, p, p, 2, p, p, p, p, p, 1 << 20, None, 0, None) == 3
     assert L.moe_quantize_permute_prefetch(p, 4, 256, p, 2, 8, p, p, 2, p, p, p, p, None, 0, p, 64, None) == 4
+    # an unaligned hint is refused before any CUDA call (bulk prefetches start on 16 bytes); without bytes it is ignored
+    odd = ctypes.c_void_p(24)
+    assert L.nvfp4_quantize_from_amax_prefetch(p, 4, 32, p, p, p, p, 0, odd, 64, None) == 2
+    assert L.moe_quantize_permute_prefetch(p, 4, 256, p, 2, 8, p, p, 2, p, p, p, p, p, 1 << 20, odd, 64, None) == 2
