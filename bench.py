@@ -280,13 +280,20 @@ def parallelism(world):
     return f"replicas x{world} (no data-path collective)" if world > 1 else "single GPU"
 
 
+def moe_weight_bytes(cfg):
+    """Packed FP4 codes and E4M3 scales of every expert's gate/up [2I, H] and down [H, I] weights."""
+    H, I = cfg["H"], cfg["I"]
+    return cfg["E"] * (2 * I * (H // 2 + H // 16) + H * (I // 2 + I // 16))
+
+
 def moe_config_dict(name, cfg, counts, world, resized=False):
     return {"workload": name if not resized else f"{name} resized to T={cfg['T']} E={cfg['E']}",
             "tokens": cfg["T"], "hidden": cfg["H"], "intermediate": cfg["I"], "experts": cfg["E"],
             "top_k": cfg["k"], "routing": cfg["routing"],
             "rows_per_expert": {"min": int(counts.min()), "mean": float(counts.mean()), "max": int(counts.max()),
                                 "empty": int(np.sum(counts == 0))},
-            "l2": "no flush: every step streams all expert weights (5.4 GB) through HBM, far above L2",
+            "l2": f"no flush: every step streams all expert weights ({moe_weight_bytes(cfg) / 1e9:.1f} GB) through HBM, "
+                  "far above L2",
             "parallelism": parallelism(world)}
 
 
