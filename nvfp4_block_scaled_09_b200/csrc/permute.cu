@@ -347,7 +347,15 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(const uint4* __rest
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
     const uint4* qs = q + (int64_t)(ok ? src : 0) * qvec;
     uint4* qd = q_perm + p * qvec;
-    for (int64_t i = lane; i < qvec; i += 32) qd[i] = ok ? __ldg(qs + i) : zero;
+    // four 16-byte pieces per lane in flight before their stores
+    for (int64_t i0 = lane; i0 < qvec; i0 += 4 * 32) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) v[u] = (ok && i0 + 32 * u < qvec) ? __ldg(qs + i0 + 32 * u) : zero;
+#pragma unroll
+        for (int u = 0; u < 4; u++)
+            if (i0 + 32 * u < qvec) qd[i0 + 32 * u] = v[u];
+    }
     if (!kHalf) {
         const uint4* ss = sf + (int64_t)(ok ? src : 0) * sfvec;
         for (int64_t i = lane; i < sfvec; i += 32) {
